@@ -1,0 +1,155 @@
+"""Python front end of the CPU oracle (``sla_oracle.c``).
+
+TEST INFRASTRUCTURE ONLY: the test suite, the smoke check and the benchmark's
+CPU-baseline leg are the only users.  The product path never imports this.
+
+The C file is compiled here with gcc (``-O2 -fopenmp``, IEEE double, no
+fast-math) into ``oracle/liboracle.so``; numpy marshals the buffers.
+Functions:
+
+* :func:`route`        -- pooled, projected top-k block routing (SLA2 router)
+* :func:`sla_forward`  -- sparse branch + ReLU linear branch + alpha combine
+* :func:`pisa_forward` -- PISA exact-or-approximate zero-order forward
+
+Inputs may be torch tensors (bf16 / fp32 / int32, on the CPU) or numpy arrays
+(bf16 given as uint16 bit patterns).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "sla_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle shared library (idempotent)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp.%d" % os.getpid()
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared",
+                               "-Wall", "-Wno-unknown-pragmas", _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB)
+            P = ctypes.c_void_p
+            I = ctypes.c_int
+            L = ctypes.c_int64
+            D = ctypes.c_double
+            lib.oracle_route.argtypes = [I] * 7 + [P] * 6 + [I]
+            lib.oracle_route.restype = I
+            lib.oracle_sla_forward.argtypes = [I] * 7 + [D] + [P] * 5 + [L, P, P, P, P, I]
+            lib.oracle_sla_forward.restype = I
+            lib.oracle_pisa_forward.argtypes = [I] * 7 + [D] + [P] * 4 + [L, P, P, I]
+            lib.oracle_pisa_forward.restype = I
+            lib.oracle_max_threads.argtypes = []
+            lib.oracle_max_threads.restype = I
+            _lib = lib
+    return _lib
+
+
+def max_threads() -> int:
+    return _load().oracle_max_threads()
+
+
+def _bf16_bits(x) -> np.ndarray:
+    """bf16 tensor / uint16 array -> contiguous uint16 numpy array."""
+    if hasattr(x, "view") and hasattr(x, "dtype") and str(x.dtype) == "torch.bfloat16":
+        import torch  # noqa: F401  (only for the dtype view)
+        return np.ascontiguousarray(x.detach().cpu().contiguous().view(torch.int16).numpy()
+                                    .view(np.uint16))
+    a = np.asarray(x)
+    assert a.dtype == np.uint16, "bf16 inputs must be torch.bfloat16 or uint16 bit patterns"
+    return np.ascontiguousarray(a)
+
+
+def _np(x, dtype):
+    if x is None:
+        return None
+    if hasattr(x, "detach"):
+        x = x.detach().cpu().contiguous().numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=dtype))
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _check(rc, name):
+    if rc != 0:
+        raise ValueError("%s: oracle rejected the arguments (code %d)" % (name, rc))
+
+
+def route(q, k, w_q, w_k, Bq, Bk, topk, threads=0):
+    """Returns (lut int32 [B,H,N/Bq,topk] ascending, gap float64 [B,H,N/Bq])."""
+    qb, kb = _bf16_bits(q), _bf16_bits(k)
+    B, H, N, d = qb.shape
+    wq, wk = _np(w_q, np.float32), _np(w_k, np.float32)
+    lut = np.zeros((B, H, N // Bq, topk), dtype=np.int32)
+    gap = np.zeros((B, H, N // Bq), dtype=np.float64)
+    rc = _load().oracle_route(B, H, N, d, Bq, Bk, topk, _ptr(qb), _ptr(kb), _ptr(wq), _ptr(wk),
+                              _ptr(lut), _ptr(gap), threads)
+    _check(rc, "route")
+    return lut, gap
+
+
+def _rows(rows, B, H, N):
+    if rows is None:
+        return None, -1
+    r = _np(rows, np.int64).reshape(-1)
+    return r, r.size
+
+
+def sla_forward(q, k, v, alpha, lut, Bq, Bk, sm_scale=0.0, rows=None, branches=False,
+                threads=0):
+    """SLA2 forward on a given LUT.  rows=None: every row, returns [B,H,N,d];
+    else flat row indices, returns [len(rows), d].  branches=True also returns
+    the sparse-branch and linear-branch outputs."""
+    qb, kb, vb = _bf16_bits(q), _bf16_bits(k), _bf16_bits(v)
+    B, H, N, d = qb.shape
+    al = _np(alpha, np.float32)
+    lt = _np(lut, np.int32)
+    topk = lt.shape[-1]
+    r, nr = _rows(rows, B, H, N)
+    n = B * H * N if r is None else nr
+    out = np.zeros((n, d), dtype=np.float64)
+    os_ = np.zeros((n, d), dtype=np.float64) if branches else None
+    ol_ = np.zeros((n, d), dtype=np.float64) if branches else None
+    rc = _load().oracle_sla_forward(B, H, N, d, Bq, Bk, topk, float(sm_scale), _ptr(qb), _ptr(kb),
+                                    _ptr(vb), _ptr(al), _ptr(lt), nr, _ptr(r), _ptr(out),
+                                    _ptr(os_), _ptr(ol_), threads)
+    _check(rc, "sla_forward")
+    shape = (B, H, N, d) if r is None else (n, d)
+    if branches:
+        return out.reshape(shape), os_.reshape(shape), ol_.reshape(shape)
+    return out.reshape(shape)
+
+
+def pisa_forward(q, k, v, lut, Bq, Bk, sm_scale=0.0, rows=None, threads=0):
+    """PISA zero-order exact-or-approximate forward on a given LUT."""
+    qb, kb, vb = _bf16_bits(q), _bf16_bits(k), _bf16_bits(v)
+    B, H, N, d = qb.shape
+    lt = _np(lut, np.int32)
+    topk = lt.shape[-1]
+    r, nr = _rows(rows, B, H, N)
+    n = B * H * N if r is None else nr
+    out = np.zeros((n, d), dtype=np.float64)
+    rc = _load().oracle_pisa_forward(B, H, N, d, Bq, Bk, topk, float(sm_scale), _ptr(qb),
+                                     _ptr(kb), _ptr(vb), _ptr(lt), nr, _ptr(r), _ptr(out),
+                                     threads)
+    _check(rc, "pisa_forward")
+    return out.reshape((B, H, N, d) if r is None else (n, d))

@@ -1,0 +1,383 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix.
+
+Each pin uses something other than the oracle itself: a library routine for
+a special case (torch's scaled-dot-product attention in fp64, torch.topk),
+the pairwise O(N^2) form of linear attention (a different association from
+the oracle's per-block sums), brute force on tiny inputs (full sort of an
+explicit score matrix), closed forms and invariants.  Chosen so that a
+dropped term, a wrong sign or index, a transposed operand, a wrong block
+multiplicity or a mean-for-sum slip fails at least one of them.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+from oracle import oracle as orc
+
+pytestmark = pytest.mark.filterwarnings("ignore")
+
+
+def f64(x):
+    return x.to(torch.float64)
+
+
+def dense_sdpa(q, k, v, mask=None, scale=None):
+    """Textbook softmax attention (torch library routine, fp64)."""
+    d = q.shape[-1]
+    return torch.nn.functional.scaled_dot_product_attention(
+        f64(q), f64(k), f64(v), attn_mask=mask,
+        scale=scale if scale else 1.0 / math.sqrt(d)).numpy()
+
+
+def block_mask(lut, N, Bq, Bk):
+    """Token-level boolean mask [B,H,N,N] (True = attend) from a block LUT."""
+    B, H, Nq, k = lut.shape
+    Nk = N // Bk
+    m = np.zeros((B, H, Nq, Nk), dtype=bool)
+    for b in range(B):
+        for h in range(H):
+            for i in range(Nq):
+                m[b, h, i, lut[b, h, i]] = True
+    m = np.repeat(np.repeat(m, Bq, axis=2), Bk, axis=3)
+    return torch.from_numpy(m)
+
+
+def random_lut(B, H, Nq, Nk, k, seed):
+    rng = np.random.default_rng(seed)
+    lut = np.zeros((B, H, Nq, k), dtype=np.int32)
+    for b in range(B):
+        for h in range(H):
+            for i in range(Nq):
+                lut[b, h, i] = np.sort(rng.choice(Nk, size=k, replace=False))
+    return lut
+
+
+def full_lut(B, H, Nq, Nk):
+    return np.broadcast_to(np.arange(Nk, dtype=np.int32), (B, H, Nq, Nk)).copy()
+
+
+# ------------------------------------------------------------------ router
+
+@pytest.mark.parametrize("N,d,Bq,Bk,k,use_w,seed", [
+    (256, 64, 64, 64, 2, True, 1),
+    (256, 32, 32, 16, 5, True, 2),
+    (192, 16, 64, 32, 3, False, 3),
+    (256, 64, 128, 64, 1, True, 4),
+    (128, 8, 16, 16, 7, True, 5),
+])
+def test_router_brute_force(N, d, Bq, Bk, k, use_w, seed):
+    """Brute force on tiny inputs: explicit pooled score matrix, full sort."""
+    inp = W.gaussian_inputs(2, 2, N, d, seed, use_w=use_w)
+    lut, gap = orc.route(inp["q"], inp["k"], inp["w_q"], inp["w_k"], Bq, Bk, k)
+    q = f64(inp["q"]).numpy()
+    kk = f64(inp["k"]).numpy()
+    Nq, Nk = N // Bq, N // Bk
+    qbar = q.reshape(2, 2, Nq, Bq, d).mean(axis=3)
+    kbar = kk.reshape(2, 2, Nk, Bk, d).mean(axis=3)
+    if use_w:
+        qbar = qbar @ f64(inp["w_q"]).numpy()
+        kbar = kbar @ f64(inp["w_k"]).numpy()
+    s = qbar @ np.swapaxes(kbar, -1, -2)
+    for b in range(2):
+        for h in range(2):
+            for i in range(Nq):
+                order = np.lexsort((np.arange(Nk), -s[b, h, i]))
+                assert np.array_equal(lut[b, h, i], np.sort(order[:k]))
+                srt = s[b, h, i][order]
+                assert gap[b, h, i] == pytest.approx(srt[k - 1] - srt[k], rel=1e-9, abs=1e-12)
+
+
+def test_router_textbook_topk():
+    """Bq = Bk = 1 and no projection: per-row top-k of Q K^T (torch.topk)."""
+    inp = W.gaussian_inputs(1, 3, 64, 16, 11, use_w=False)
+    lut, _ = orc.route(inp["q"], inp["k"], None, None, 1, 1, 9)
+    s = f64(inp["q"]) @ f64(inp["k"]).transpose(-1, -2)
+    ref = torch.topk(s, 9, dim=-1).indices.sort(dim=-1).values.numpy()
+    assert np.array_equal(lut, ref)
+
+
+def test_router_block_permutation():
+    """Permuting the KV blocks permutes the selected set."""
+    N, d, Bq, Bk, k = 256, 32, 32, 32, 3
+    inp = W.gaussian_inputs(1, 2, N, d, 12)
+    lut, _ = orc.route(inp["q"], inp["k"], inp["w_q"], inp["w_k"], Bq, Bk, k)
+    Nk = N // Bk
+    perm = np.random.default_rng(0).permutation(Nk)           # new block j' = old block perm[j']
+    kp = inp["k"].reshape(1, 2, Nk, Bk, d)[:, :, torch.from_numpy(perm)].reshape(1, 2, N, d)
+    lutp, _ = orc.route(inp["q"], kp.contiguous(), inp["w_q"], inp["w_k"], Bq, Bk, k)
+    inv = np.argsort(perm)
+    for h in range(2):
+        for i in range(N // Bq):
+            assert np.array_equal(lutp[0, h, i], np.sort(inv[lut[0, h, i]]))
+
+
+def test_router_projection_identity_and_scale():
+    N, d, Bq, Bk, k = 256, 32, 64, 32, 3
+    inp = W.gaussian_inputs(1, 2, N, d, 13)
+    eye = torch.eye(d)
+    a, ga = orc.route(inp["q"], inp["k"], None, None, Bq, Bk, k)
+    b, gb = orc.route(inp["q"], inp["k"], eye, eye, Bq, Bk, k)
+    assert np.array_equal(a, b)
+    np.testing.assert_allclose(ga, gb, rtol=1e-12)
+    c, gc = orc.route(inp["q"], inp["k"], 2.0 * inp["w_q"], 0.5 * inp["w_k"], Bq, Bk, k)
+    d_, gd = orc.route(inp["q"], inp["k"], inp["w_q"], inp["w_k"], Bq, Bk, k)
+    assert np.array_equal(c, d_)
+    np.testing.assert_allclose(gc, gd, rtol=1e-12)
+    e, ge = orc.route(inp["q"], inp["k"], 4.0 * inp["w_q"], inp["w_k"], Bq, Bk, k)
+    assert np.array_equal(e, d_)
+    np.testing.assert_allclose(ge, 4.0 * gd, rtol=1e-12)
+
+
+def test_router_extreme_k():
+    N, d = 256, 16
+    inp = W.gaussian_inputs(1, 1, N, d, 14)
+    lut0, g0 = orc.route(inp["q"], inp["k"], inp["w_q"], inp["w_k"], 64, 32, 0)
+    assert lut0.shape == (1, 1, 4, 0) and np.all(np.isinf(g0))
+    lutn, gn = orc.route(inp["q"], inp["k"], inp["w_q"], inp["w_k"], 64, 32, 8)
+    assert np.array_equal(lutn, full_lut(1, 1, 4, 8)) and np.all(np.isinf(gn))
+
+
+def test_router_rejects_bad_shapes():
+    inp = W.gaussian_inputs(1, 1, 256, 16, 15)
+    with pytest.raises(ValueError):
+        orc.route(inp["q"], inp["k"], None, None, 96, 32, 1)      # N % Bq != 0
+    with pytest.raises(ValueError):
+        orc.route(inp["q"], inp["k"], None, None, 64, 32, 9)      # k > Nk
+
+
+# --------------------------------------------------------- sparse branch
+
+@pytest.mark.parametrize("N,d,Bq,Bk", [(256, 64, 64, 64), (256, 32, 128, 32), (192, 16, 32, 64)])
+def test_sparse_all_selected_is_dense_attention(N, d, Bq, Bk):
+    """k = Nk, alpha = 1: the sparse branch is full softmax attention."""
+    inp = W.gaussian_inputs(1, 2, N, d, 21)
+    alpha = torch.ones(1, 2, N)
+    lut = full_lut(1, 2, N // Bq, N // Bk)
+    out = orc.sla_forward(inp["q"], inp["k"], inp["v"], alpha, lut, Bq, Bk)
+    ref = dense_sdpa(inp["q"], inp["k"], inp["v"])
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-11)
+
+
+@pytest.mark.parametrize("scale", [0.0, 0.37])
+def test_sparse_partial_is_masked_attention(scale):
+    """alpha = 1: block-masked softmax attention, renormalised over the kept
+    blocks (torch SDPA with a boolean mask)."""
+    N, d, Bq, Bk, k = 256, 32, 64, 32, 3
+    inp = W.gaussian_inputs(2, 2, N, d, 22)
+    alpha = torch.ones(2, 2, N)
+    lut = random_lut(2, 2, N // Bq, N // Bk, k, 5)
+    out = orc.sla_forward(inp["q"], inp["k"], inp["v"], alpha, lut, Bq, Bk, sm_scale=scale)
+    ref = dense_sdpa(inp["q"], inp["k"], inp["v"], block_mask(lut, N, Bq, Bk),
+                     scale=scale if scale else None)
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-11)
+
+
+def test_sparse_empty_selection_is_zero():
+    N, d = 128, 16
+    inp = W.gaussian_inputs(1, 1, N, d, 23)
+    lut = np.zeros((1, 1, 2, 0), dtype=np.int32)
+    out = orc.sla_forward(inp["q"], inp["k"], inp["v"], torch.ones(1, 1, N), lut, 64, 32)
+    assert np.all(out == 0.0)
+
+
+def test_sparse_shift_invariance():
+    """Adding one vector u to every key shifts each row's logits by q.u: the
+    sparse branch is unchanged.  Keys and u are multiples of 1/8 so k + u is
+    exact in bf16."""
+    N, d, Bq, Bk, k = 128, 16, 32, 32, 2
+    g = torch.Generator().manual_seed(3)
+    q = (torch.randint(-8, 9, (1, 1, N, d), generator=g) / 8).to(torch.bfloat16)
+    kk = (torch.randint(-8, 9, (1, 1, N, d), generator=g) / 8).to(torch.bfloat16)
+    v = torch.randn(1, 1, N, d, generator=g).to(torch.bfloat16)
+    u = (torch.randint(-8, 9, (d,), generator=g) / 8)
+    ku = (kk.float() + u).to(torch.bfloat16)
+    assert torch.equal(ku.float(), kk.float() + u)
+    lut = random_lut(1, 1, N // Bq, N // Bk, k, 7)
+    ones = torch.ones(1, 1, N)
+    a = orc.sla_forward(q, kk, v, ones, lut, Bq, Bk)
+    b = orc.sla_forward(q, ku, v, ones, lut, Bq, Bk)
+    np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+
+
+# --------------------------------------------------------- linear branch
+
+def pairwise_linear(q, k, v, keep=None):
+    """Textbook ReLU linear attention in its O(N^2) pairwise form:
+    sum_n (phi(q).phi(k_n)) v_n / sum_n phi(q).phi(k_n); 0 if the denominator
+    is not positive.  keep: boolean [.., N, N] of pairs that take part."""
+    a = np.maximum(f64(q).numpy(), 0) @ np.swapaxes(np.maximum(f64(k).numpy(), 0), -1, -2)
+    if keep is not None:
+        a = a * keep
+    num = a @ f64(v).numpy()
+    den = a.sum(-1, keepdims=True)
+    with np.errstate(invalid="ignore", divide="ignore"):
+        return np.where(den > 0, num / np.where(den > 0, den, 1), 0.0)
+
+
+def test_linear_no_selection_is_pairwise_linear_attention():
+    N, d, Bq, Bk = 256, 32, 64, 32
+    inp = W.gaussian_inputs(1, 2, N, d, 31)
+    lut = np.zeros((1, 2, N // Bq, 0), dtype=np.int32)
+    out = orc.sla_forward(inp["q"], inp["k"], inp["v"], torch.zeros(1, 2, N), lut, Bq, Bk)
+    ref = pairwise_linear(inp["q"], inp["k"], inp["v"])
+    np.testing.assert_allclose(out, ref, rtol=1e-10, atol=1e-12)
+
+
+def test_linear_covers_only_unselected_blocks():
+    N, d, Bq, Bk, k = 256, 32, 64, 32, 3
+    inp = W.gaussian_inputs(1, 2, N, d, 32)
+    lut = random_lut(1, 2, N // Bq, N // Bk, k, 9)
+    out = orc.sla_forward(inp["q"], inp["k"], inp["v"], torch.zeros(1, 2, N), lut, Bq, Bk)
+    keep = ~block_mask(lut, N, Bq, Bk).numpy()
+    ref = pairwise_linear(inp["q"], inp["k"], inp["v"], keep)
+    np.testing.assert_allclose(out, ref, rtol=1e-10, atol=1e-12)
+
+
+def test_linear_scale_invariance():
+    """phi = ReLU is positively homogeneous: scaling q or k by 2^e > 0 leaves
+    the linear branch unchanged (power-of-two scales are exact in bf16)."""
+    N, d, Bq, Bk, k = 256, 32, 64, 32, 2
+    inp = W.gaussian_inputs(1, 1, N, d, 33)
+    lut = random_lut(1, 1, N // Bq, N // Bk, k, 3)
+    zero = torch.zeros(1, 1, N)
+    a = orc.sla_forward(inp["q"], inp["k"], inp["v"], zero, lut, Bq, Bk)
+    b = orc.sla_forward(inp["q"] * 4, inp["k"] * 0.5, inp["v"], zero, lut, Bq, Bk)
+    np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-14)
+
+
+def test_linear_nonpositive_denominator_gives_zero():
+    N, d, Bq, Bk = 128, 16, 64, 32
+    inp = W.gaussian_inputs(1, 1, N, d, 34)
+    qneg = -inp["q"].abs()
+    lut = random_lut(1, 1, N // Bq, N // Bk, 1, 1)
+    out = orc.sla_forward(qneg, inp["k"], inp["v"], torch.zeros(1, 1, N), lut, Bq, Bk)
+    assert np.all(out == 0.0)
+
+
+# ---------------------------------------------------------------- combine
+
+def test_combine_is_affine_in_alpha():
+    N, d, Bq, Bk, k = 256, 32, 64, 32, 3
+    inp = W.gaussian_inputs(1, 2, N, d, 41)
+    lut = random_lut(1, 2, N // Bq, N // Bk, k, 4)
+    out, os_, ol = orc.sla_forward(inp["q"], inp["k"], inp["v"], inp["alpha"], lut, Bq, Bk,
+                                   branches=True)
+    one = orc.sla_forward(inp["q"], inp["k"], inp["v"], torch.ones(1, 2, N), lut, Bq, Bk)
+    zero = orc.sla_forward(inp["q"], inp["k"], inp["v"], torch.zeros(1, 2, N), lut, Bq, Bk)
+    np.testing.assert_allclose(os_, one, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(ol, zero, rtol=0, atol=1e-13)
+    a = inp["alpha"].double().numpy()[..., None]
+    np.testing.assert_allclose(out, a * one + (1 - a) * zero, rtol=0, atol=1e-12)
+
+
+def test_sla_brute_force_matrix_form():
+    """The whole forward in explicit N x N matrix form on a tiny case."""
+    N, d, Bq, Bk, k = 256, 16, 64, 32, 3
+    inp = W.gaussian_inputs(1, 2, N, d, 42)
+    lut = random_lut(1, 2, N // Bq, N // Bk, k, 8)
+    out = orc.sla_forward(inp["q"], inp["k"], inp["v"], inp["alpha"], lut, Bq, Bk)
+    m = block_mask(lut, N, Bq, Bk).numpy()
+    q, kk, v = (f64(inp[x]).numpy() for x in "qkv")
+    logits = (q @ np.swapaxes(kk, -1, -2)) / math.sqrt(d)
+    logits = np.where(m, logits, -np.inf)
+    p = np.exp(logits - logits.max(-1, keepdims=True))
+    os_ = (p / p.sum(-1, keepdims=True)) @ v
+    a = np.maximum(q, 0) @ np.swapaxes(np.maximum(kk, 0), -1, -2) * (~m)
+    ol = (a @ v) / a.sum(-1, keepdims=True)
+    al = inp["alpha"].double().numpy()[..., None]
+    np.testing.assert_allclose(out, al * os_ + (1 - al) * ol, rtol=0, atol=1e-11)
+
+
+def test_row_sampling_matches_full_output():
+    N, d, Bq, Bk, k = 256, 32, 128, 64, 2
+    inp = W.gaussian_inputs(2, 2, N, d, 43)
+    lut = random_lut(2, 2, N // Bq, N // Bk, k, 2)
+    full = orc.sla_forward(inp["q"], inp["k"], inp["v"], inp["alpha"], lut, Bq, Bk)
+    rows = np.array([1000, 3, 517, 1023, 64, 65])
+    part = orc.sla_forward(inp["q"], inp["k"], inp["v"], inp["alpha"], lut, Bq, Bk, rows=rows)
+    np.testing.assert_array_equal(part, full.reshape(-1, d)[rows])
+    pp = orc.pisa_forward(inp["q"], inp["k"], inp["v"], lut, Bq, Bk, rows=rows)
+    pf = orc.pisa_forward(inp["q"], inp["k"], inp["v"], lut, Bq, Bk)
+    np.testing.assert_array_equal(pp, pf.reshape(-1, d)[rows])
+
+
+def test_oracle_rejects_invalid_lut():
+    N, d = 128, 16
+    inp = W.gaussian_inputs(1, 1, N, d, 44)
+    bad = np.array([[[[0, 0], [1, 2]]]], dtype=np.int32)            # duplicate
+    with pytest.raises(ValueError):
+        orc.sla_forward(inp["q"], inp["k"], inp["v"], inp["alpha"], bad, 64, 32)
+    bad = np.array([[[[0, 4], [1, 2]]]], dtype=np.int32)            # out of range
+    with pytest.raises(ValueError):
+        orc.pisa_forward(inp["q"], inp["k"], inp["v"], bad, 64, 32)
+
+
+# ------------------------------------------------------------------- PISA
+
+def test_pisa_all_exact_is_dense_attention():
+    N, d, B_ = 256, 32, 64
+    inp = W.gaussian_inputs(1, 2, N, d, 51)
+    out = orc.pisa_forward(inp["q"], inp["k"], inp["v"], full_lut(1, 2, N // B_, N // B_), B_, B_)
+    np.testing.assert_allclose(out, dense_sdpa(inp["q"], inp["k"], inp["v"]), rtol=0, atol=1e-11)
+
+
+def block_constant_keys(B, H, N, d, Bk, seed):
+    g = torch.Generator().manual_seed(seed)
+    kb = torch.randn(B, H, N // Bk, 1, d, generator=g).to(torch.bfloat16)
+    return kb.expand(B, H, N // Bk, Bk, d).reshape(B, H, N, d).contiguous()
+
+
+@pytest.mark.parametrize("k", [0, 1, 3, 4])
+def test_pisa_zero_order_exact_for_block_constant_keys(k):
+    """If every key of a block equals its centroid, the zero-order term is
+    the exact block contribution: PISA equals dense attention for any k."""
+    N, d, B_ = 256, 32, 32
+    inp = W.gaussian_inputs(1, 2, N, d, 52)
+    kc = block_constant_keys(1, 2, N, d, B_, 9)
+    lut = random_lut(1, 2, N // B_, N // B_, k, 10 + k)
+    out = orc.pisa_forward(inp["q"], kc, inp["v"], lut, B_, B_)
+    np.testing.assert_allclose(out, dense_sdpa(inp["q"], kc, inp["v"]), rtol=0, atol=1e-11)
+
+
+def test_pisa_no_exact_block_closed_form():
+    """k = 0 with block-constant keys: softmax over the centroids, each with
+    multiplicity Bk, applied to the block mean values."""
+    N, d, B_ = 256, 16, 64
+    inp = W.gaussian_inputs(1, 1, N, d, 53)
+    kc = block_constant_keys(1, 1, N, d, B_, 11)
+    lut = np.zeros((1, 1, N // B_, 0), dtype=np.int32)
+    out = orc.pisa_forward(inp["q"], kc, inp["v"], lut, B_, B_)
+    q = f64(inp["q"]).numpy()[0, 0]
+    cent = f64(kc).numpy()[0, 0, ::B_]                           # [Nk, d]
+    vmean = f64(inp["v"]).numpy()[0, 0].reshape(N // B_, B_, d).mean(1)
+    c = q @ cent.T / math.sqrt(d)
+    w = np.exp(c - c.max(-1, keepdims=True))
+    ref = (w @ vmean) / w.sum(-1, keepdims=True)
+    np.testing.assert_allclose(out[0, 0], ref, rtol=0, atol=1e-12)
+
+
+def test_pisa_zero_order_error_is_first_order():
+    """Keys = centroid + eps * delta (delta zero-mean within each block): the
+    zero-order approximation error against dense attention is O(eps), so
+    halving eps halves it.  All values are exact in bf16."""
+    N, d, B_, k = 256, 16, 32, 2
+    g = torch.Generator().manual_seed(5)
+    base = (torch.randint(-6, 7, (1, 1, N // B_, 1, d), generator=g) / 8.0)
+    base = base.expand(1, 1, N // B_, B_, d).reshape(1, 1, N, d)
+    sign = torch.randint(0, 2, (1, 1, N // B_, B_ // 2, d), generator=g) * 2.0 - 1.0
+    delta = torch.cat([sign, -sign], 3).reshape(1, 1, N, d)      # zero mean per block
+    q = (torch.randint(-8, 9, (1, 1, N, d), generator=g) / 4.0).to(torch.bfloat16)
+    v = torch.randn(1, 1, N, d, generator=g).to(torch.bfloat16)
+    lut = random_lut(1, 1, N // B_, N // B_, k, 12)
+    errs = []
+    for e in (2.0 ** -4, 2.0 ** -5, 2.0 ** -6):
+        kk = (base + e * delta).to(torch.bfloat16)
+        assert torch.equal(kk.double(), (base + e * delta).double())
+        out = orc.pisa_forward(q, kk, v, lut, B_, B_)
+        errs.append(np.abs(out - dense_sdpa(q, kk, v)).max())
+    assert errs[0] > errs[1] > errs[2] > 0
+    for a, b in zip(errs, errs[1:]):
+        assert 1.6 < a / b < 2.5, errs
