@@ -1,0 +1,352 @@
+"""Benchmark of the hybrid sparse-linear attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one sla_forward call in LUT_COMPUTE mode (router: pooling,
+projection, fp64 score + top-k; K/V pre-pass; sparse branch + linear branch
++ alpha combine) over one batch of the workload's synthetic inputs, already
+resident in HBM.  Default workload: SLA2 bf16, B=1 H=12 N=32768 d=128,
+Bq=128 Bk=64, keep 52 of 512 KV blocks (90% sparse), bf16 output.
+
+Printed (rank 0, one JSON line): dense-equivalent TFLOPS (4 B H N^2 d / t) as
+`value`, ms per call, the end-to-end number through the same C ABI with host
+buffers (host->device copies of the inputs and the device->host copy of the
+output inside the timed region), the attention kernel's roofline (live CUDA
+events around each launch on its stream), the CPU oracle's throughput on a
+bounded sample, clocks sampled during the timed region and the launch count.
+
+Multi-GPU (torchrun): every rank runs its own copy of the workload (the heads
+of different problems are independent; no collective on the data path):
+weak scaling, value = all ranks' work / the slowest rank's time.
+
+--impl reference times the CPU oracle (the only reference this method has)
+on the host cores, on a bounded sample of the same workload, per step.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads as W  # noqa: E402
+
+METRIC = "SLA fwd ms/call & dense-equiv TFLOPS (N=32768,H=12,d=128,90% sparse)"
+UNIT = "TFLOPS (dense-equivalent)"
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d.get("hbm_gbs", 6650.0), "bf16_tflops": d.get("bf16_tflops", 1590.0),
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", 1400.0), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# --------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, ValueError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------- oracle (CPU)
+def oracle_sample(w, inp, n_rows=256, seed=11):
+    """Time the CPU oracle on a bounded sample: the full router plus the forward
+    of n_rows seeded rows from two heads.  Returns (dense-equivalent TFLOPS,
+    seconds, threads, description)."""
+    from oracle import oracle as orc
+    threads = len(os.sched_getaffinity(0))
+    t0 = time.perf_counter()
+    lut, _ = orc.route(inp["q"], inp["k"], inp["w_q"], inp["w_k"], w.Bq, w.Bk, w.topk,
+                       threads=threads)
+    t_route = time.perf_counter() - t0
+    rows = W.sample_rows(w.B, w.H, w.N, n_rows, seed, heads=[0, w.B * w.H - 1]).numpy()
+    t0 = time.perf_counter()
+    if w.mode == "pisa":
+        orc.pisa_forward(inp["q"], inp["k"], inp["v"], lut, w.Bq, w.Bk, rows=rows, threads=threads)
+    else:
+        orc.sla_forward(inp["q"], inp["k"], inp["v"], inp["alpha"], lut, w.Bq, w.Bk, rows=rows,
+                        threads=threads)
+    t_fwd = time.perf_counter() - t0
+    total_rows = w.B * w.H * w.N
+    frac = len(rows) / total_rows
+    # time attributed to the sample: its share of the router + the sampled forward
+    t = t_route * frac + t_fwd
+    flops = 4.0 * len(rows) * w.N * w.d
+    desc = ("router on all %d heads (%.2fs, charged pro rata) + forward of %d rows from 2 heads "
+            "(%.2fs, incl. the per-head linear-branch block statistics)" % (
+                w.B * w.H, t_route, len(rows), t_fwd))
+    return flops / t / 1e12, t_route + t_fwd, threads, desc
+
+
+def run_reference(args, w, rank):
+    """--impl reference: the CPU oracle as the reference arm."""
+    if rank != 0:
+        return
+    inp = W.make_inputs(w)
+    for _ in range(args.warmup if args.warmup < 1 else 1):
+        oracle_sample(w, inp, n_rows=32)
+    vals, secs = [], []
+    for _ in range(args.steps):
+        v, s, threads, desc = oracle_sample(w, inp, n_rows=64)
+        vals.append(v)
+        secs.append(s)
+    value = statistics.median(vals)
+    ms_per_call = w.dense_equiv_flops() / (value * 1e12) * 1e3
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_per_call, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "Bq": w.Bq,
+                       "Bk": w.Bk, "topk": w.topk},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------- our arm
+def run_ours(args, w, rank, world, local_rank):
+    import block_sparse_linear_proj_b200 as S
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    inp = W.make_inputs(w)
+    g = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
+    p = S.params(w.B, w.H, w.N, w.d, w.Bq, w.Bk, w.topk, sparse_dtype=w.sparse_dtype)
+    ws = S.workspace(p, device=dev)
+    lut = torch.empty((w.B, w.H, w.Nq, w.topk), dtype=torch.int32, device=dev)
+    out = torch.empty_like(g["q"])
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        if w.mode == "pisa":
+            S.sla_pisa_forward(p, g["q"], g["k"], g["v"], None, None, lut, out, ws, stream)
+        else:
+            S.sla_forward(p, g["q"], g["k"], g["v"], g["alpha"], g["w_q"], g["w_k"], lut, out,
+                          ws, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if S.sla_check_device_status(stream) != 0:
+        raise RuntimeError("device status set during warm-up")
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    # ---- timed region (device-resident inputs)
+    clocks = ClockSampler(local_rank)
+    S.sla_profile_read()                       # drop anything recorded earlier
+    barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    time.sleep(0.3)
+    S.sla_profile_enable(True)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    S.sla_profile_enable(False)
+    clk = clocks.stop()
+    barrier()
+    ms_total = e0.elapsed_time(e1)
+    prof = S.sla_profile_read()
+    if world > 1:
+        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_per_call = ms_total / args.steps
+    value = world * w.dense_equiv_flops() / (ms_per_call * 1e-3) / 1e12
+    launches = sum(c for (_, c) in prof.values())
+
+    # ---- end-to-end through the C ABI with host buffers
+    hosts = {k: (v.pin_memory() if v is not None else None) for k, v in inp.items()}
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in hosts.values() if v is not None)
+    d2h = out_h.numel() * out_h.element_size()
+    e2e_steps = max(3, min(args.steps, 20))
+
+    def e2e_step():
+        for k, v in hosts.items():
+            if v is not None:
+                g[k].copy_(v, non_blocking=True)
+        step()
+        out_h.copy_(out, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    f0 = torch.cuda.Event(enable_timing=True)
+    f1 = torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    f1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = f0.elapsed_time(f1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * w.dense_equiv_flops() / (e2e_ms * 1e-3) / 1e12
+    if S.sla_check_device_status(stream) != 0:
+        raise RuntimeError("device status set during the benchmark")
+
+    if rank != 0:
+        return
+    # ---- roofline of the dominant kernel (attention) and the others
+    pairs = w.B * w.H * w.Nq * w.topk
+    attn_ms, attn_n = prof["attn"]
+    attn_avg = attn_ms / max(attn_n, 1)
+    exec_flops = 4.0 * pairs * w.Bq * w.Bk * w.d
+    g_flops = 2.0 * pairs * w.Bk * w.d * w.d if w.mode == "sla" else 0.0
+    achieved = exec_flops / (attn_avg * 1e-3) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    kv_ms, kv_n = prof["kv_stats"]
+    kv_avg = kv_ms / max(kv_n, 1)
+    kv_bytes = w.B * w.H * w.N * w.d * 2 * 3      # read K and V, write the fp16 copy of V
+    pool_ms, pool_n = prof["pool"]
+    pool_avg = pool_ms / max(pool_n, 1)
+    pool_bytes = w.B * w.H * w.N * w.d * 2        # read Q
+    total_prof = sum(m for (m, _) in prof.values())
+    kernels = {k: {"ms_per_call": m / max(c, 1), "launches": c,
+                   "share": (m / total_prof if total_prof else None)} for k, (m, c) in prof.items() if c}
+    kernels["kv_stats"]["hbm"] = {"achieved_gbs": kv_bytes / (kv_avg * 1e-3) / 1e9,
+                                  "peak_gbs": peaks["hbm_gbs"],
+                                  "frac": kv_bytes / (kv_avg * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+    kernels["pool"]["hbm"] = {"achieved_gbs": pool_bytes / (pool_avg * 1e-3) / 1e9,
+                              "peak_gbs": peaks["hbm_gbs"],
+                              "frac": pool_bytes / (pool_avg * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+    kernels["attn"]["with_linear_G_tflops"] = (exec_flops + g_flops) / (attn_avg * 1e-3) / 1e12
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        v, secs, threads, desc = oracle_sample(w, inp)
+        cpu = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc,
+               "seconds": secs}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_call, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded video-latent generator, no model weights)",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "Bq": w.Bq,
+                   "Bk": w.Bk, "topk": w.topk, "global_batch": w.B * world, "seq_len": w.N,
+                   "parallelism": "replicas%d" % world, "l2": "inputs exceed L2 (302 MB > 126 MB)",
+                   "out_dtype": "bf16", "lut_mode": "compute"},
+        "ms_per_call": ms_per_call,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None, "kernel": "attn",
+                     "peak_source": peaks["source"] + " bf16 sustained",
+                     "algorithmic": "4*Bq*Bk*d per (query block, selected block) pair, %d pairs" % pairs},
+        "kernels": kernels,
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_call": e2e_ms},
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="sla2_bf16", choices=list(W.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    w = W.WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, w, rank)
+        return
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,270 @@
+// kv_stats.cuh -- one streaming pass over K and V (HBM-bound) that produces
+// every per-KV-block statistic the forward needs:
+//   * router:  Kbar_j = mean of the block's keys (fp64, stored [bh][c][j]);
+//   * linear branch ([SALAD] ReLU kernel, block form): z_j = sum phi(k_n)
+//     (fp32 [bh][j][c]) and a per-chunk partial of H = phi(K)^T V (fp32 d x d),
+//     reduced over chunks by h_reduce_kernel in a fixed order;
+//   * PISA precompute ("Pre-calcolo" of the PISA page): the block centroid
+//     kbar_j (bf16) and the value mean vbar_j = (sum_n v_n)/Bk (fp16), both
+//     [bh][j][c], the operands of the zero-order pseudo-tiles;
+//   * an fp16 copy of V, the B operand of the attention kernel's P.V product
+//     (the conversion from bf16 is exact inside the fp16 range; values outside
+//     it are flagged).
+// phi(K)^T V uses warp-level bf16 tensor-core MMA (m16n8k16) with fp32
+// accumulation; K and V tiles of 64 tokens stream through a 3-stage cp.async
+// ring with an XOR swizzle so ldmatrix reads are conflict-free.
+#pragma once
+#include "common.cuh"
+
+namespace sla {
+
+constexpr int kKvTok = 64;     // tokens per KV block (Bk)
+constexpr int kKvStages = 3;
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1,
+                                              uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4],
+                                               uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t relu_bf16x2(uint32_t x) {
+    __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&x);
+    h = __hmax2(h, __floats2bfloat162_rn(0.f, 0.f));
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Byte offset of element (row n, col c) in a [64][D] bf16 tile whose 16-byte
+// chunks are XOR-swizzled by (n & 7).
+template <int D>
+__device__ __forceinline__ uint32_t kv_off(int n, int c) {
+    return static_cast<uint32_t>(n * D * 2 + ((((c >> 3) ^ (n & 7))) << 4) + (c & 7) * 2);
+}
+
+struct KvStatsArgs {
+    const __nv_bfloat16* k;     // [BH][N][D]
+    const __nv_bfloat16* v;     // [BH][N][D] (may be null when only kbarT is wanted)
+    int N, Nk, blocks_per_chunk, nchunk;
+    double* kbarT;              // [BH][D][Nk]           (null: skip)
+    float* zj;                  // [BH][Nk][D]           (null: skip)
+    float* hpart;               // [BH][nchunk][D][D]    (null: skip the MMA)
+    __nv_bfloat16* kc;          // [BH][Nk][D] centroids (null: skip)
+    __half* vbar;               // [BH][Nk][D] value means (null: skip)
+    __half* v16;                // [BH][N][D] fp16 copy of V (null: skip)
+};
+
+// grid (nchunk, BH), 256 threads.
+template <int D>
+__global__ void __launch_bounds__(256, 2) kv_stats_kernel(KvStatsArgs a) {
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    constexpr int TILE = kKvTok * D * 2;               // bytes of one K or V tile
+    unsigned char* ring = smem_raw;                    // [stages][K tile | V tile]
+    double* kpart = reinterpret_cast<double*>(smem_raw + kKvStages * 2 * TILE);   // [256]
+    float* zpart = reinterpret_cast<float*>(kpart + 256);                          // [256]
+    float* vpart = zpart + 256;                                                    // [256]
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const long long bh = blockIdx.y;
+    const int chunk = blockIdx.x;
+    const int jb0 = chunk * a.blocks_per_chunk;
+    const int nblk = min(a.blocks_per_chunk, a.Nk - jb0);
+    if (nblk <= 0) return;
+    const bool want_v = a.v != nullptr;
+    const __nv_bfloat16* kh = a.k + bh * static_cast<long long>(a.N) * D;
+    const __nv_bfloat16* vh = want_v ? a.v + bh * static_cast<long long>(a.N) * D : nullptr;
+
+    auto load_block = [&](int blk, int stage) {
+        unsigned char* kd = ring + stage * 2 * TILE;
+        unsigned char* vd = kd + TILE;
+        const long long row0 = static_cast<long long>(jb0 + blk) * kKvTok;
+        constexpr int CPR = D / 8;                      // 16-byte chunks per row
+        for (int q = tid; q < kKvTok * CPR; q += 256) {
+            const int n = q / CPR, u = q % CPR;
+            const uint32_t off = kv_off<D>(n, u * 8);
+            cp_async16(kd + off, kh + (row0 + n) * D + u * 8);
+            if (want_v) cp_async16(vd + off, vh + (row0 + n) * D + u * 8);
+        }
+    };
+
+    // MMA tiling of the D x D partial: 8 warps, warp tile (D/4) x (D/2).
+    constexpr int WM = D / 4, WN = D / 2;
+    constexpr int MT = WM / 16, NT = WN / 8;
+    const int m0 = (warp & 3) * WM, n0 = (warp >> 2) * WN;
+    float acc[MT][NT][4];
+#pragma unroll
+    for (int i = 0; i < MT; ++i)
+#pragma unroll
+        for (int j = 0; j < NT; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.f;
+    const bool do_mma = a.hpart != nullptr;
+
+#pragma unroll
+    for (int s = 0; s < kKvStages - 1; ++s) {
+        if (s < nblk) load_block(s, s);
+        cp_async_commit();
+    }
+
+    constexpr int HALVES = 256 / D;                 // row groups for the column sums
+    constexpr int RPH = kKvTok / HALVES;
+    const int col = tid % D, half = tid / D;
+
+    for (int blk = 0; blk < nblk; ++blk) {
+        const int stage = blk % kKvStages;
+        cp_async_wait<kKvStages - 2>();
+        __syncthreads();
+        {   // prefetch the block kKvStages-1 ahead into the stage freed last iteration
+            const int nb = blk + kKvStages - 1;
+            if (nb < nblk) load_block(nb, nb % kKvStages);
+            cp_async_commit();
+        }
+        const unsigned char* kt = ring + stage * 2 * TILE;
+        const unsigned char* vt = kt + TILE;
+        const uint32_t kt_s = smem_u32(kt), vt_s = smem_u32(vt);
+
+        // column statistics of this block
+        {
+            double ks = 0.0;
+            float zs = 0.f, vs = 0.f, kmax = 0.f;
+            for (int n = half * RPH; n < (half + 1) * RPH; ++n) {
+                const float kv = __bfloat162float(
+                    *reinterpret_cast<const __nv_bfloat16*>(kt + kv_off<D>(n, col)));
+                ks += static_cast<double>(kv);
+                zs += fmaxf(kv, 0.f);
+                kmax = fmaxf(kmax, fabsf(kv));
+                if (want_v)
+                    vs += __bfloat162float(
+                        *reinterpret_cast<const __nv_bfloat16*>(vt + kv_off<D>(n, col)));
+            }
+            kpart[tid] = ks;
+            zpart[tid] = zs;
+            vpart[tid] = vs;
+            if (a.v16 && !(kmax < 65504.f)) report(kStatusRange);
+        }
+        // fp16 copy of the V tile (coalesced 16-byte stores)
+        if (a.v16) {
+            constexpr int CPR = D / 8;
+            const long long row0 = static_cast<long long>(jb0 + blk) * kKvTok;
+            __half* vo = a.v16 + bh * static_cast<long long>(a.N) * D;
+            bool bad = false;
+            for (int q = tid; q < kKvTok * CPR; q += 256) {
+                const int n = q / CPR, u = q % CPR;
+                const uint4 x = *reinterpret_cast<const uint4*>(vt + kv_off<D>(n, u * 8));
+                const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+                uint32_t h[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float lo = bf16lo(w[e]), hi = bf16hi(w[e]);
+                    bad |= !(fabsf(lo) < 65504.f) || !(fabsf(hi) < 65504.f);
+                    h[e] = pack_half2(lo, hi);
+                }
+                *reinterpret_cast<uint4*>(vo + (row0 + n) * D + u * 8) = make_uint4(h[0], h[1], h[2], h[3]);
+            }
+            if (bad) report(kStatusRange);
+        }
+
+        if (do_mma) {
+#pragma unroll
+            for (int k0 = 0; k0 < kKvTok; k0 += 16) {
+                uint32_t afr[MT][4];
+#pragma unroll
+                for (int i = 0; i < MT; ++i) {
+                    // A = phi(K)^T: matrices (n k0..+7 | k0+8..+15) x (c m..m+7 | m+8..m+15)
+                    const int n = k0 + (lane & 7) + ((lane >> 4) << 3);
+                    const int c = m0 + i * 16 + (((lane >> 3) & 1) << 3);
+                    ldsm_x4_trans(kt_s + kv_off<D>(n, c), afr[i][0], afr[i][1], afr[i][2],
+                                  afr[i][3]);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) afr[i][e] = relu_bf16x2(afr[i][e]);
+                }
+#pragma unroll
+                for (int j = 0; j < NT; j += 2) {
+                    const int n = k0 + (lane & 7) + (((lane >> 3) & 1) << 3);
+                    const int e = n0 + j * 8 + ((lane >> 4) << 3);
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4_trans(vt_s + kv_off<D>(n, e), b0, b1, b2, b3);
+#pragma unroll
+                    for (int i = 0; i < MT; ++i) {
+                        mma_bf16_16816(acc[i][j], afr[i], b0, b1);
+                        mma_bf16_16816(acc[i][j + 1], afr[i], b2, b3);
+                    }
+                }
+            }
+        }
+        __syncthreads();
+        if (tid < D) {
+            double ks = 0.0;
+            float zs = 0.f, vs = 0.f;
+#pragma unroll
+            for (int h = 0; h < HALVES; ++h) {
+                ks += kpart[h * D + tid];
+                zs += zpart[h * D + tid];
+                vs += vpart[h * D + tid];
+            }
+            const int j = jb0 + blk;
+            const double kmean = ks * (1.0 / kKvTok);
+            if (a.kbarT) a.kbarT[(bh * D + tid) * a.Nk + j] = kmean;
+            if (a.zj) a.zj[(bh * a.Nk + j) * D + tid] = zs;
+            if (a.kc) a.kc[(bh * a.Nk + j) * D + tid] = __float2bfloat16_rn(static_cast<float>(kmean));
+            if (a.vbar) a.vbar[(bh * a.Nk + j) * D + tid] = __float2half_rn(vs * (1.f / kKvTok));
+        }
+    }
+    cp_async_wait<0>();
+
+    if (do_mma) {
+        float* hp = a.hpart + (bh * a.nchunk + chunk) * static_cast<long long>(D) * D;
+        const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+        for (int i = 0; i < MT; ++i)
+#pragma unroll
+            for (int j = 0; j < NT; ++j) {
+                const int r = m0 + i * 16 + g, c = n0 + j * 8 + 2 * t;
+                *reinterpret_cast<float2*>(hp + r * D + c) = make_float2(acc[i][j][0], acc[i][j][1]);
+                *reinterpret_cast<float2*>(hp + (r + 8) * D + c) =
+                    make_float2(acc[i][j][2], acc[i][j][3]);
+            }
+    }
+}
+
+// H[bh] = sum over chunks of hpart (fixed order), Z[bh] = sum_j z_j.
+// grid (D*D/256 + 1, BH), 256 threads; the last x-block reduces Z.
+template <int D>
+__global__ void __launch_bounds__(256) h_reduce_kernel(const float* __restrict__ hpart,
+                                                       const float* __restrict__ zj, int nchunk,
+                                                       int Nk, float* __restrict__ hsum,
+                                                       float* __restrict__ zsum) {
+    const long long bh = blockIdx.y;
+    constexpr int NHB = D * D / 256;
+    if (blockIdx.x < NHB) {
+        const int idx = blockIdx.x * 256 + threadIdx.x;
+        const float* src = hpart + bh * nchunk * static_cast<long long>(D) * D + idx;
+        float s = 0.f;
+        for (int c = 0; c < nchunk; ++c) s += src[static_cast<long long>(c) * D * D];
+        hsum[bh * D * D + idx] = s;
+    } else if (threadIdx.x < D) {
+        const float* src = zj + bh * static_cast<long long>(Nk) * D + threadIdx.x;
+        float s = 0.f;
+        for (int j = 0; j < Nk; ++j) s += src[static_cast<long long>(j) * D];
+        zsum[bh * D + threadIdx.x] = s;
+    }
+}
+
+}  // namespace sla

@@ -1,0 +1,481 @@
+// sla_api.cu -- host side of the C ABI declared in include/sla.h: argument
+// validation, workspace carving, TMA descriptor encoding and kernel launches.
+// All device code lives in the included .cuh files (one translation unit, so
+// the device status word needs no relocatable device code).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/sla.h"
+#include "attn.cuh"
+#include "common.cuh"
+#include "kv_stats.cuh"
+#include "router.cuh"
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+// ------------------------------------------------------------- validation
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+sla_status_t check_params(const sla_params_t* p) {
+    if (!p) return SLA_ERR_INVALID_ARG;
+    if (p->B <= 0 || p->H <= 0 || p->N <= 0 || p->d <= 0 || p->Bq <= 0 || p->Bk <= 0 ||
+        p->topk < 0)
+        return SLA_ERR_INVALID_ARG;
+    if (p->N % p->Bq != 0 || p->N % p->Bk != 0) return SLA_ERR_INVALID_ARG;
+    if (p->topk > p->N / p->Bk) return SLA_ERR_INVALID_ARG;
+    if (p->sparse_dtype != SLA_SPARSE_BF16 && p->sparse_dtype != SLA_SPARSE_FP8_E4M3)
+        return SLA_ERR_INVALID_ARG;
+    if (p->lut_mode != SLA_LUT_COMPUTE && p->lut_mode != SLA_LUT_GIVEN) return SLA_ERR_INVALID_ARG;
+    if (p->out_dtype != SLA_OUT_BF16 && p->out_dtype != SLA_OUT_FP32) return SLA_ERR_INVALID_ARG;
+    if (!(std::isfinite(p->sm_scale))) return SLA_ERR_INVALID_ARG;
+    if (p->d != 64 && p->d != 128) return SLA_ERR_UNSUPPORTED;
+    if (p->Bq != 64 && p->Bq != 128) return SLA_ERR_UNSUPPORTED;
+    if (p->Bk != 64) return SLA_ERR_UNSUPPORTED;
+    if (p->N / p->Bk > 8192) return SLA_ERR_UNSUPPORTED;
+    const long long bh = static_cast<long long>(p->B) * p->H;
+    if (bh > 65535) return SLA_ERR_UNSUPPORTED;
+    if (bh * p->N > 0x7fffffffLL) return SLA_ERR_UNSUPPORTED;
+    return SLA_OK;
+}
+
+sla_status_t check_tensor(const void* t, size_t align) {
+    if (!t) return SLA_ERR_INVALID_ARG;
+    if (!aligned(t, align)) return SLA_ERR_INVALID_ARG;
+    return SLA_OK;
+}
+
+// ------------------------------------------------------------- workspace
+struct Ws {
+    size_t qbar, kbarT, m, lut, zj, hpart, hsum, zsum, kc, vbar, v16, total;
+    int nchunk, bpc;
+};
+
+Ws layout(const sla_params_t* p) {
+    Ws w{};
+    const size_t BH = static_cast<size_t>(p->B) * p->H;
+    const size_t d = p->d, Nq = p->N / p->Bq, Nk = p->N / p->Bk;
+    // K/V pre-pass chunking: ~4 waves of CTAs over the heads, >= 8 blocks per chunk
+    const long long target = std::max<long long>(1, 592 / static_cast<long long>(BH));
+    w.bpc = std::max<int>(8, static_cast<int>((Nk + target - 1) / target));
+    w.nchunk = static_cast<int>((Nk + w.bpc - 1) / w.bpc);
+    size_t off = 0;
+    auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes); return o; };
+    w.qbar = take(BH * Nq * d * 8);
+    w.kbarT = take(BH * Nk * d * 8);
+    w.m = take(d * d * 8);
+    w.lut = take(BH * Nq * static_cast<size_t>(p->topk) * 4 + 4);
+    w.zj = take(BH * Nk * d * 4);
+    w.hpart = take(BH * static_cast<size_t>(w.nchunk) * d * d * 4);
+    w.hsum = take(BH * d * d * 4);
+    w.zsum = take(BH * d * 4);
+    w.kc = take(BH * Nk * d * 2);
+    w.vbar = take(BH * Nk * d * 2);
+    w.v16 = take(BH * static_cast<size_t>(p->N) * d * 2);
+    w.total = off;
+    return w;
+}
+
+sla_status_t check_ws(const sla_params_t* p, void* ws, size_t ws_bytes, Ws& w) {
+    w = layout(p);
+    if (!ws || !aligned(ws, kAlign) || ws_bytes < w.total) return SLA_ERR_WORKSPACE;
+    return SLA_OK;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) { return reinterpret_cast<T*>(static_cast<char*>(ws) + off); }
+
+// ------------------------------------------------------------- TMA maps
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                              const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                              const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                              CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn encode_fn() {
+    static EncodeFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeFn>(f);
+    });
+    return fn;
+}
+
+// 2-D map of 16-bit elements over [rows, d] (d innermost), box [64 columns,
+// box_rows], 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, long long rows, int d, int box_rows,
+              CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
+    EncodeFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
+    cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+unsigned long long wait_limit_ns() {
+    const char* s = std::getenv("SLA_DEBUG_WAIT_LIMIT_NS");
+    if (s && *s) {
+        const unsigned long long v = std::strtoull(s, nullptr, 10);
+        if (v > 0) return v;
+    }
+    return 2000000000ull;
+}
+
+bool check_after_call() {
+    const char* s = std::getenv("SLA_CHECK");
+    return s && *s && *s != '0';
+}
+
+sla_status_t launch_status() {
+    return cudaGetLastError() == cudaSuccess ? SLA_OK : SLA_ERR_CUDA;
+}
+
+// ------------------------------------------------------------- tracing
+struct Profiler {
+    std::mutex mu;
+    bool on = false;
+    struct Rec { int kind; cudaEvent_t a, b; };
+    std::vector<Rec> recs;
+    std::vector<cudaEvent_t> pool;
+    cudaEvent_t get() {
+        if (!pool.empty()) { cudaEvent_t e = pool.back(); pool.pop_back(); return e; }
+        cudaEvent_t e = nullptr;
+        cudaEventCreate(&e);
+        return e;
+    }
+};
+Profiler& prof() { static Profiler p; return p; }
+
+// Brackets one launch with events when tracing is on.
+struct Span {
+    int kind; cudaStream_t st; cudaEvent_t a = nullptr, b = nullptr;
+    Span(int k, cudaStream_t s) : kind(k), st(s) {
+        Profiler& P = prof();
+        std::lock_guard<std::mutex> g(P.mu);
+        if (!P.on) return;
+        a = P.get(); b = P.get();
+        if (a) cudaEventRecord(a, st);
+    }
+    ~Span() {
+        if (!a || !b) return;
+        cudaEventRecord(b, st);
+        Profiler& P = prof();
+        std::lock_guard<std::mutex> g(P.mu);
+        P.recs.push_back({kind, a, b});
+    }
+};
+
+// ------------------------------------------------------------- launchers
+int grid_blocks(long long n, int per_sm) {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    long long cap = static_cast<long long>(sms) * per_sm;
+    return static_cast<int>(std::max<long long>(1, std::min(n, cap)));
+}
+
+void launch_pool(const void* x, int rows, long long nblk_total, int nblk_per_head, int d,
+                 int out_mode, double* out, cudaStream_t st) {
+    const int grid = grid_blocks(nblk_total, 8);
+    const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+    Span sp(SLA_KERNEL_POOL, st);
+    if (d == 128)
+        sla::pool_mean_kernel<128><<<grid, 256, 0, st>>>(xb, rows, nblk_total, nblk_per_head, out_mode, out);
+    else
+        sla::pool_mean_kernel<64><<<grid, 256, 0, st>>>(xb, rows, nblk_total, nblk_per_head, out_mode, out);
+}
+
+template <int R, int D>
+sla_status_t launch_score_r(const double* qbar, const double* kbarT, const double* m, int BH,
+                            int Nq, int Nk, int topk, int32_t* lut, cudaStream_t st) {
+    const size_t smem = static_cast<size_t>(D) * R * 8 + 8 * 256 * 4 +
+                        static_cast<size_t>(R) * std::max(Nk, D) * 8;
+    auto kern = sla::score_topk_kernel<R, D>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+        return SLA_ERR_CUDA;
+    dim3 grid((Nq + R - 1) / R, BH);
+    Span sp(SLA_KERNEL_SCORE_TOPK, st);
+    kern<<<grid, 256, smem, st>>>(qbar, kbarT, m, Nq, Nk, topk, lut);
+    return launch_status();
+}
+
+template <int D>
+sla_status_t launch_score(const double* qbar, const double* kbarT, const double* m, int BH,
+                          int Nq, int Nk, int topk, int32_t* lut, cudaStream_t st) {
+    const size_t budget = 200 * 1024;
+    auto need = [&](int R) {
+        return static_cast<size_t>(D) * R * 8 + 8 * 256 * 4 + static_cast<size_t>(R) * std::max(Nk, D) * 8;
+    };
+    if (need(16) <= budget) return launch_score_r<16, D>(qbar, kbarT, m, BH, Nq, Nk, topk, lut, st);
+    if (need(8) <= budget) return launch_score_r<8, D>(qbar, kbarT, m, BH, Nq, Nk, topk, lut, st);
+    if (need(4) <= budget) return launch_score_r<4, D>(qbar, kbarT, m, BH, Nq, Nk, topk, lut, st);
+    return launch_score_r<2, D>(qbar, kbarT, m, BH, Nq, Nk, topk, lut, st);
+}
+
+// Router: Q/K pooling (unless already pooled), W folding, fp64 score + top-k.
+sla_status_t run_router(const sla_params_t* p, const void* q, const void* k, const float* w_q,
+                        const float* w_k, int32_t* lut, void* ws, const Ws& w, bool pool_k,
+                        cudaStream_t st) {
+    const int BH = p->B * p->H, Nq = p->N / p->Bq, Nk = p->N / p->Bk, d = p->d;
+    double* qbar = at<double>(ws, w.qbar);
+    double* kbarT = at<double>(ws, w.kbarT);
+    launch_pool(q, p->Bq, static_cast<long long>(BH) * Nq, Nq, d, 0, qbar, st);
+    if (pool_k) launch_pool(k, p->Bk, static_cast<long long>(BH) * Nk, Nk, d, 1, kbarT, st);
+    const double* m = nullptr;
+    if (w_q || w_k) {
+        Span sp(SLA_KERNEL_FOLD_W, st);
+        sla::fold_w_kernel<<<d, 128, 0, st>>>(w_q, w_k, d, at<double>(ws, w.m));
+        m = at<double>(ws, w.m);
+    }
+    if (launch_status() != SLA_OK) return SLA_ERR_CUDA;
+    if (d == 128) return launch_score<128>(qbar, kbarT, m, BH, Nq, Nk, p->topk, lut, st);
+    return launch_score<64>(qbar, kbarT, m, BH, Nq, Nk, p->topk, lut, st);
+}
+
+template <int D>
+sla_status_t launch_kv(const sla_params_t* p, const void* k, const void* v, void* ws, const Ws& w,
+                       bool want_kbar, bool sla_stats, bool pisa_stats, cudaStream_t st) {
+    const int BH = p->B * p->H, Nk = p->N / p->Bk;
+    sla::KvStatsArgs a{};
+    a.k = static_cast<const __nv_bfloat16*>(k);
+    a.v = static_cast<const __nv_bfloat16*>(v);
+    a.N = p->N;
+    a.Nk = Nk;
+    a.blocks_per_chunk = w.bpc;
+    a.nchunk = w.nchunk;
+    a.kbarT = want_kbar ? at<double>(ws, w.kbarT) : nullptr;
+    a.zj = sla_stats ? at<float>(ws, w.zj) : nullptr;
+    a.hpart = sla_stats ? at<float>(ws, w.hpart) : nullptr;
+    a.kc = pisa_stats ? at<__nv_bfloat16>(ws, w.kc) : nullptr;
+    a.vbar = pisa_stats ? at<__half>(ws, w.vbar) : nullptr;
+    a.v16 = at<__half>(ws, w.v16);
+    const size_t smem = sla::kKvStages * 2 * 64 * D * 2 + 256 * 8 + 2 * 256 * 4;
+    auto kern = sla::kv_stats_kernel<D>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+        return SLA_ERR_CUDA;
+    {
+        Span sp(SLA_KERNEL_KV_STATS, st);
+        kern<<<dim3(w.nchunk, BH), 256, smem, st>>>(a);
+    }
+    if (sla_stats) {
+        constexpr int NHB = D * D / 256;
+        Span sp(SLA_KERNEL_H_REDUCE, st);
+        sla::h_reduce_kernel<D><<<dim3(NHB + 1, BH), 256, 0, st>>>(
+            at<float>(ws, w.hpart), at<float>(ws, w.zj), w.nchunk, Nk, at<float>(ws, w.hsum),
+            at<float>(ws, w.zsum));
+    }
+    return launch_status();
+}
+
+template <int D, bool PISA>
+sla_status_t launch_attn(const sla_params_t* p, const void* q, const void* k, const void* v,
+                         const float* alpha, const int32_t* lut, void* out, void* ws, const Ws& w,
+                         cudaStream_t st) {
+    using L = sla::AttnLayout<D>;
+    const int BH = p->B * p->H, Nq = p->N / p->Bq, Nk = p->N / p->Bk;
+    CUtensorMap mq, mk, mv, mkc, mvc;
+    const long long rows = static_cast<long long>(BH) * p->N;
+    (void)v;   // the P.V product reads the fp16 copy of V made by the K/V pre-pass
+    if (!make_map(&mq, q, rows, D, 128) || !make_map(&mk, k, rows, D, 64) ||
+        !make_map(&mv, at<void>(ws, w.v16), rows, D, 64, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+        return SLA_ERR_CUDA;
+    if (PISA) {
+        if (!make_map(&mkc, at<void>(ws, w.kc), static_cast<long long>(BH) * Nk, D, 64) ||
+            !make_map(&mvc, at<void>(ws, w.vbar), static_cast<long long>(BH) * Nk, D, 64,
+                      CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+            return SLA_ERR_CUDA;
+    } else {
+        mkc = mk;
+        mvc = mv;
+    }
+    sla::AttnArgs a{};
+    a.N = p->N;
+    a.Nq = Nq;
+    a.Nk = Nk;
+    a.Bq = p->Bq;
+    a.topk = p->topk;
+    a.tiles_per_head = (p->N + 127) / 128;
+    const float tau = p->sm_scale > 0.f ? p->sm_scale : 1.0f / std::sqrt(static_cast<float>(D));
+    a.scale_log2 = tau * 1.4426950408889634f;
+    a.log2_bk = std::log2(static_cast<float>(p->Bk));
+    a.lut = lut;
+    a.alpha = alpha;
+    a.hsum = PISA ? nullptr : at<float>(ws, w.hsum);
+    a.zsum = PISA ? nullptr : at<float>(ws, w.zsum);
+    a.zj = PISA ? nullptr : at<float>(ws, w.zj);
+    a.out = out;
+    a.out_f32 = p->out_dtype == SLA_OUT_FP32 ? 1 : 0;
+    a.wait_ns = wait_limit_ns();
+    const int GR = 128 / p->Bq;
+    const int nwords = (Nk + 15) / 16;
+    const size_t sched_cap = static_cast<size_t>(std::min(Nk, GR * std::max(p->topk, 1)));
+    const size_t smem = 1024 + L::OFF_MISC + 256 + 2 * D * 4 + ((nwords + 3) & ~3) * 4 + sched_cap * 4;
+    auto kern = sla::attn_kernel<D, PISA>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+        return SLA_ERR_CUDA;
+    Span sp(SLA_KERNEL_ATTN, st);
+    kern<<<BH * a.tiles_per_head, 256, smem, st>>>(mq, mk, mv, mkc, mvc, a);
+    return launch_status();
+}
+
+sla_status_t finish(sla_status_t s, cudaStream_t st) {
+    if (s != SLA_OK) return s;
+    if (check_after_call()) return sla_check_device_status(st);
+    return SLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t sla_workspace_size(const sla_params_t* p) {
+    if (check_params(p) != SLA_OK) return 0;
+    return layout(p).total;
+}
+
+const char* sla_status_string(sla_status_t s) {
+    switch (s) {
+        case SLA_OK: return "ok";
+        case SLA_ERR_INVALID_ARG: return "invalid argument";
+        case SLA_ERR_UNSUPPORTED: return "unsupported shape or mode";
+        case SLA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        case SLA_ERR_CUDA: return "CUDA call or kernel launch failed";
+        case SLA_ERR_TIMEOUT: return "a kernel's bounded wait ran out";
+        case SLA_ERR_DEVICE_CHECK: return "a kernel found invalid data (LUT entry)";
+    }
+    return "unknown status";
+}
+
+int32_t sla_version(void) { return 100; }
+
+sla_status_t sla_profile_enable(int32_t on) {
+    Profiler& P = prof();
+    std::lock_guard<std::mutex> g(P.mu);
+    P.on = on != 0;
+    return SLA_OK;
+}
+
+sla_status_t sla_profile_read(double* ms_total, int64_t* launches) {
+    Profiler& P = prof();
+    std::lock_guard<std::mutex> g(P.mu);
+    sla_status_t rc = SLA_OK;
+    for (int k = 0; k < SLA_KERNEL_KINDS; ++k) {
+        if (ms_total) ms_total[k] = 0.0;
+        if (launches) launches[k] = 0;
+    }
+    for (auto& r : P.recs) {
+        float ms = 0.f;
+        if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess)
+            rc = SLA_ERR_CUDA;
+        if (ms_total) ms_total[r.kind] += ms;
+        if (launches) launches[r.kind] += 1;
+        P.pool.push_back(r.a);
+        P.pool.push_back(r.b);
+    }
+    P.recs.clear();
+    return rc;
+}
+
+sla_status_t sla_check_device_status(sla_stream_t stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return SLA_ERR_CUDA;
+    unsigned v = 0u;
+    if (cudaMemcpyFromSymbol(&v, sla::g_status, sizeof v) != cudaSuccess) return SLA_ERR_CUDA;
+    if (v) {
+        const unsigned zero = 0u;
+        if (cudaMemcpyToSymbol(sla::g_status, &zero, sizeof zero) != cudaSuccess) return SLA_ERR_CUDA;
+    }
+    if (v & sla::kStatusTimeout) return SLA_ERR_TIMEOUT;
+    if (v & (sla::kStatusBadData | sla::kStatusRange)) return SLA_ERR_DEVICE_CHECK;
+    return SLA_OK;
+}
+
+sla_status_t sla_route(const sla_params_t* p, const void* q, const void* k, const float* w_q,
+                       const float* w_k, int32_t* lut, void* workspace, size_t ws_bytes,
+                       sla_stream_t stream) {
+    sla_status_t s = check_params(p);
+    if (s != SLA_OK) return s;
+    if ((s = check_tensor(q, 16)) || (s = check_tensor(k, 16))) return s;
+    if (p->topk > 0 && (s = check_tensor(lut, 4))) return s;
+    if ((w_q && !aligned(w_q, 4)) || (w_k && !aligned(w_k, 4))) return SLA_ERR_INVALID_ARG;
+    Ws w;
+    if ((s = check_ws(p, workspace, ws_bytes, w))) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return finish(run_router(p, q, k, w_q, w_k, lut, workspace, w, true, st), st);
+}
+
+sla_status_t sla_forward(const sla_params_t* p, const void* q, const void* k, const void* v,
+                         const float* alpha, const float* w_q, const float* w_k, int32_t* lut,
+                         void* out, void* workspace, size_t ws_bytes, sla_stream_t stream) {
+    sla_status_t s = check_params(p);
+    if (s != SLA_OK) return s;
+    if ((s = check_tensor(q, 16)) || (s = check_tensor(k, 16)) || (s = check_tensor(v, 16)) ||
+        (s = check_tensor(out, 16)) || (s = check_tensor(alpha, 4)))
+        return s;
+    if ((w_q && !aligned(w_q, 4)) || (w_k && !aligned(w_k, 4))) return SLA_ERR_INVALID_ARG;
+    if (p->lut_mode == SLA_LUT_GIVEN && !lut && p->topk > 0) return SLA_ERR_INVALID_ARG;
+    if (lut && !aligned(lut, 4)) return SLA_ERR_INVALID_ARG;
+    if (p->sparse_dtype == SLA_SPARSE_FP8_E4M3 && (p->d != 128 || p->Bq != 128))
+        return SLA_ERR_UNSUPPORTED;
+    Ws w;
+    if ((s = check_ws(p, workspace, ws_bytes, w))) return s;
+    if (p->sparse_dtype == SLA_SPARSE_FP8_E4M3) return SLA_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const bool compute = p->lut_mode == SLA_LUT_COMPUTE;
+    int32_t* lut_use = (compute && !lut) ? at<int32_t>(workspace, w.lut) : lut;
+    s = p->d == 128 ? launch_kv<128>(p, k, v, workspace, w, compute, true, false, st)
+                    : launch_kv<64>(p, k, v, workspace, w, compute, true, false, st);
+    if (s != SLA_OK) return s;
+    if (compute && (s = run_router(p, q, k, w_q, w_k, lut_use, workspace, w, false, st))) return s;
+    s = p->d == 128 ? launch_attn<128, false>(p, q, k, v, alpha, lut_use, out, workspace, w, st)
+                    : launch_attn<64, false>(p, q, k, v, alpha, lut_use, out, workspace, w, st);
+    return finish(s, st);
+}
+
+sla_status_t sla_pisa_forward(const sla_params_t* p, const void* q, const void* k, const void* v,
+                              const float* w_q, const float* w_k, int32_t* lut, void* out,
+                              void* workspace, size_t ws_bytes, sla_stream_t stream) {
+    sla_status_t s = check_params(p);
+    if (s != SLA_OK) return s;
+    if ((s = check_tensor(q, 16)) || (s = check_tensor(k, 16)) || (s = check_tensor(v, 16)) ||
+        (s = check_tensor(out, 16)))
+        return s;
+    if ((w_q && !aligned(w_q, 4)) || (w_k && !aligned(w_k, 4))) return SLA_ERR_INVALID_ARG;
+    if (p->lut_mode == SLA_LUT_GIVEN && !lut && p->topk > 0) return SLA_ERR_INVALID_ARG;
+    if (lut && !aligned(lut, 4)) return SLA_ERR_INVALID_ARG;
+    if (p->Bq != p->Bk || p->sparse_dtype != SLA_SPARSE_BF16) return SLA_ERR_UNSUPPORTED;
+    Ws w;
+    if ((s = check_ws(p, workspace, ws_bytes, w))) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const bool compute = p->lut_mode == SLA_LUT_COMPUTE;
+    int32_t* lut_use = (compute && !lut) ? at<int32_t>(workspace, w.lut) : lut;
+    s = p->d == 128 ? launch_kv<128>(p, k, v, workspace, w, compute, false, true, st)
+                    : launch_kv<64>(p, k, v, workspace, w, compute, false, true, st);
+    if (s != SLA_OK) return s;
+    if (compute && (s = run_router(p, q, k, w_q, w_k, lut_use, workspace, w, false, st))) return s;
+    s = p->d == 128 ? launch_attn<128, true>(p, q, k, v, nullptr, lut_use, out, workspace, w, st)
+                    : launch_attn<64, true>(p, q, k, v, nullptr, lut_use, out, workspace, w, st);
+    return finish(s, st);
+}
+
+}  // extern "C"

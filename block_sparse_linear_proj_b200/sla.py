@@ -1,0 +1,208 @@
+"""Thin ctypes binding of the C ABI in ``include/sla.h``.
+
+Argument marshalling only: tensors are checked for device, dtype and layout
+and passed as raw device pointers together with the current CUDA stream;
+every step of the computation runs in the library's kernels.  There is no
+fallback: if ``libsla.so`` is missing or no CUDA device is present, the calls
+raise.
+
+The same names as the C functions: :func:`sla_route`, :func:`sla_forward`,
+:func:`sla_pisa_forward`, :func:`sla_workspace_size`,
+:func:`sla_check_device_status`.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsla.so")
+
+SLA_OK = 0
+SLA_ERR_INVALID_ARG = 1
+SLA_ERR_UNSUPPORTED = 2
+SLA_ERR_WORKSPACE = 3
+SLA_ERR_CUDA = 4
+SLA_ERR_TIMEOUT = 5
+SLA_ERR_DEVICE_CHECK = 6
+
+SLA_SPARSE_BF16 = 0
+SLA_SPARSE_FP8_E4M3 = 1
+SLA_LUT_COMPUTE = 0
+SLA_LUT_GIVEN = 1
+SLA_OUT_BF16 = 0
+SLA_OUT_FP32 = 1
+
+EXPORTED = ("sla_workspace_size", "sla_route", "sla_forward", "sla_pisa_forward",
+            "sla_status_string", "sla_check_device_status", "sla_version",
+            "sla_profile_enable", "sla_profile_read")
+KERNEL_KINDS = ("pool", "kv_stats", "h_reduce", "fold_w", "score_topk", "attn")
+
+
+class SlaParams(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("N", ctypes.c_int32),
+                ("d", ctypes.c_int32), ("Bq", ctypes.c_int32), ("Bk", ctypes.c_int32),
+                ("topk", ctypes.c_int32), ("sm_scale", ctypes.c_float),
+                ("sparse_dtype", ctypes.c_int32), ("lut_mode", ctypes.c_int32),
+                ("out_dtype", ctypes.c_int32)]
+
+
+class SlaError(RuntimeError):
+    def __init__(self, code, where):
+        self.code = code
+        super().__init__("%s: %s (status %d)" % (where, status_string(code), code))
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def load():
+    """Load libsla.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise ImportError("libsla.so not built: run python -m block_sparse_linear_proj_b200.build")
+            lib = ctypes.CDLL(LIB_PATH)
+            P = ctypes.c_void_p
+            PP = ctypes.POINTER(SlaParams)
+            lib.sla_workspace_size.argtypes = [PP]
+            lib.sla_workspace_size.restype = ctypes.c_size_t
+            lib.sla_route.argtypes = [PP, P, P, P, P, P, P, ctypes.c_size_t, P]
+            lib.sla_route.restype = ctypes.c_int
+            lib.sla_forward.argtypes = [PP, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+            lib.sla_forward.restype = ctypes.c_int
+            lib.sla_pisa_forward.argtypes = [PP, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+            lib.sla_pisa_forward.restype = ctypes.c_int
+            lib.sla_status_string.argtypes = [ctypes.c_int]
+            lib.sla_status_string.restype = ctypes.c_char_p
+            lib.sla_check_device_status.argtypes = [P]
+            lib.sla_check_device_status.restype = ctypes.c_int
+            lib.sla_version.argtypes = []
+            lib.sla_version.restype = ctypes.c_int32
+            lib.sla_profile_enable.argtypes = [ctypes.c_int32]
+            lib.sla_profile_enable.restype = ctypes.c_int
+            lib.sla_profile_read.argtypes = [P, P]
+            lib.sla_profile_read.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return load().sla_status_string(int(code)).decode()
+
+
+def params(B, H, N, d, Bq, Bk, topk, sm_scale=0.0, sparse_dtype=SLA_SPARSE_BF16,
+           lut_mode=SLA_LUT_COMPUTE, out_dtype=SLA_OUT_BF16) -> SlaParams:
+    return SlaParams(B, H, N, d, Bq, Bk, topk, float(sm_scale), sparse_dtype, lut_mode,
+                     out_dtype)
+
+
+def out_torch_dtype(p: SlaParams):
+    return torch.float32 if p.out_dtype == SLA_OUT_FP32 else torch.bfloat16
+
+
+def _ptr(t):
+    if t is None or t.numel() == 0:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensor must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _check(t, dtype, shape, name):
+    if t.dtype != dtype:
+        raise TypeError("%s: expected %s, got %s" % (name, dtype, t.dtype))
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError("%s: expected shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def sla_workspace_size(p: SlaParams) -> int:
+    return int(load().sla_workspace_size(ctypes.byref(p)))
+
+
+def workspace(p: SlaParams, device=None) -> torch.Tensor:
+    """A workspace tensor large enough for every call with these parameters."""
+    n = sla_workspace_size(p)
+    if n == 0:
+        raise SlaError(SLA_ERR_INVALID_ARG, "sla_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def _raise(code, where):
+    if code != SLA_OK:
+        raise SlaError(code, where)
+
+
+def sla_route(p, q, k, w_q, w_k, lut, ws, stream=None):
+    """Writes the top-k block LUT [B,H,N/Bq,topk] (int32, ascending) into ``lut``."""
+    B, H, N, d = p.B, p.H, p.N, p.d
+    _check(q, torch.bfloat16, (B, H, N, d), "q")
+    _check(k, torch.bfloat16, (B, H, N, d), "k")
+    _check(lut, torch.int32, (B, H, N // p.Bq, p.topk), "lut")
+    rc = load().sla_route(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(w_q), _ptr(w_k), _ptr(lut),
+                          _ptr(ws), ws.numel(), _stream(stream))
+    _raise(rc, "sla_route")
+    return lut
+
+
+def sla_forward(p, q, k, v, alpha, w_q, w_k, lut, out, ws, stream=None):
+    """SLA2 forward into ``out`` [B,H,N,d] bf16.  ``lut`` is written (LUT_COMPUTE,
+    may be None) or read (LUT_GIVEN)."""
+    B, H, N, d = p.B, p.H, p.N, p.d
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check(t, torch.bfloat16, (B, H, N, d), name)
+    _check(out, out_torch_dtype(p), (B, H, N, d), "out")
+    _check(alpha, torch.float32, (B, H, N), "alpha")
+    if lut is not None:
+        _check(lut, torch.int32, (B, H, N // p.Bq, p.topk), "lut")
+    rc = load().sla_forward(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(w_q),
+                            _ptr(w_k), _ptr(lut), _ptr(out), _ptr(ws), ws.numel(),
+                            _stream(stream))
+    _raise(rc, "sla_forward")
+    return out
+
+
+def sla_pisa_forward(p, q, k, v, w_q, w_k, lut, out, ws, stream=None):
+    """PISA zero-order exact-or-approximate forward into ``out``."""
+    B, H, N, d = p.B, p.H, p.N, p.d
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check(t, torch.bfloat16, (B, H, N, d), name)
+    _check(out, out_torch_dtype(p), (B, H, N, d), "out")
+    if lut is not None:
+        _check(lut, torch.int32, (B, H, N // p.Bq, p.topk), "lut")
+    rc = load().sla_pisa_forward(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(w_q),
+                                 _ptr(w_k), _ptr(lut), _ptr(out), _ptr(ws), ws.numel(),
+                                 _stream(stream))
+    _raise(rc, "sla_pisa_forward")
+    return out
+
+
+def sla_check_device_status(stream=None) -> int:
+    return int(load().sla_check_device_status(_stream(stream)))
+
+
+def sla_profile_enable(on: bool = True) -> None:
+    _raise(load().sla_profile_enable(1 if on else 0), "sla_profile_enable")
+
+
+def sla_profile_read():
+    """{kernel kind: (total ms, launches)} since the last read (synchronises)."""
+    n = len(KERNEL_KINDS)
+    ms = (ctypes.c_double * n)()
+    cnt = (ctypes.c_int64 * n)()
+    _raise(load().sla_profile_read(ctypes.cast(ms, ctypes.c_void_p), ctypes.cast(cnt, ctypes.c_void_p)),
+           "sla_profile_read")
+    return {KERNEL_KINDS[i]: (ms[i], cnt[i]) for i in range(n)}

@@ -1,0 +1,174 @@
+/*
+ * sla.h -- C ABI of the B200 (sm_100a) hybrid sparse-linear attention library.
+ *
+ * Forward pass of hybrid sparse-linear attention for video diffusion
+ * transformers, as described by
+ *   [SLA2]  "SLA2: Sparse-Linear Attention with Learnable Routing and QAT"
+ *           (gist.science summary of arXiv 2602.12675, Italian and Arabic pages)
+ *   [SALAD] "SALAD: Achieve High-Sparsity Attention via Efficient Linear
+ *           Attention Tuning for Video Diffusion Transformer" (2601.16515)
+ *   [PISA]  "PISA - Piecewise Sparse Attention per Efficient Diffusion
+ *           Transformers" (2602.01077)
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Tensors are dense, row-major, d innermost:
+ *      q, k, v      : bf16  [B, H, N, d]            (device memory)
+ *      out          : bf16 or fp32 [B, H, N, d]     (device memory, see out_dtype)
+ *      alpha        : fp32  [B, H, N]               (device memory)
+ *      w_q, w_k     : fp32  [d, d], x . W, shared by all heads; NULL = identity
+ *      lut          : int32 [B, H, N/Bq, topk]      (device memory)
+ *  - Every pointer is a DEVICE pointer owned by the caller; q, k, v, out are
+ *    aligned to 16 bytes, alpha, w_q, w_k, lut to 4 bytes.  lut may be NULL
+ *    when topk == 0.  The library allocates no device memory: scratch is the caller's
+ *    `workspace`, of at least sla_workspace_size() bytes, 256-byte aligned.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream).  Arguments are validated on the host before anything is
+ *    enqueued; on any error nothing is launched.
+ *  - Errors are returned, never thrown.  Kernel-side checks (an out-of-range
+ *    or repeated entry in a caller-given LUT, a bounded wait that ran out)
+ *    set a device status word that sla_check_device_status() reads.
+ *  - Numerics: products on the tensor cores with fp32 accumulation; the
+ *    softmax weights P and the values V enter the P.V product as fp16 (V is
+ *    converted once per call; |v| and |k| must stay below 65504, else the
+ *    kernels flag SLA_ERR_DEVICE_CHECK); the router runs in fp64.
+ *  - Supported shapes: d in {64, 128}; Bq in {64, 128}; Bk = 64;
+ *    N % Bq == 0 and N % Bk == 0 (padding tokens are the caller's job);
+ *    0 <= topk <= N/Bk; N/Bk <= 8192; B*H <= 65535.
+ *    The FP8 sparse branch needs d = 128 and Bq = 128.
+ *    PISA needs Bq == Bk.
+ */
+#ifndef SLA_B200_H
+#define SLA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void *sla_stream_t; /* a cudaStream_t */
+
+typedef enum {
+    SLA_OK = 0,
+    SLA_ERR_INVALID_ARG = 1,   /* NULL/misaligned pointer, inconsistent sizes */
+    SLA_ERR_UNSUPPORTED = 2,   /* valid, but outside the shapes listed above  */
+    SLA_ERR_WORKSPACE = 3,     /* workspace NULL, misaligned or too small     */
+    SLA_ERR_CUDA = 4,          /* a CUDA runtime/driver call or launch failed */
+    SLA_ERR_TIMEOUT = 5,       /* a kernel's bounded wait ran out             */
+    SLA_ERR_DEVICE_CHECK = 6   /* a kernel found invalid data (e.g. LUT entry)*/
+} sla_status_t;
+
+typedef enum { SLA_SPARSE_BF16 = 0, SLA_SPARSE_FP8_E4M3 = 1 } sla_sparse_dtype_t;
+typedef enum { SLA_LUT_COMPUTE = 0, SLA_LUT_GIVEN = 1 } sla_lut_mode_t;
+typedef enum { SLA_OUT_BF16 = 0, SLA_OUT_FP32 = 1 } sla_out_dtype_t;
+
+typedef struct sla_params {
+    int32_t B, H, N, d;      /* batch, heads, tokens, head dim                  */
+    int32_t Bq, Bk;          /* query / key-value block sizes (tokens)          */
+    int32_t topk;            /* KV blocks kept per query block                  */
+    float sm_scale;          /* softmax scale tau; <= 0 means 1/sqrt(d)         */
+    int32_t sparse_dtype;    /* sla_sparse_dtype_t: operand type of the sparse
+                                branch's tensor-core products                   */
+    int32_t lut_mode;        /* sla_lut_mode_t                                  */
+    int32_t out_dtype;       /* sla_out_dtype_t: element type of `out`          */
+} sla_params_t;
+
+/* Bytes of device workspace that sla_route, sla_forward and sla_pisa_forward
+ * need for these parameters (the maximum over the three).  Returns 0 if the
+ * parameters are invalid. */
+size_t sla_workspace_size(const sla_params_t *p);
+
+/*
+ * sla_route -- the learnable router of [SLA2] sec. 2.B ("Router
+ * Apprendibile"; Arabic page sec. 2.b) at inference:
+ *   1. mean-pool Q over blocks of Bq adjacent tokens and K over blocks of Bk;
+ *   2. project: Qt = Qbar . w_q, Kt = Kbar . w_k (NULL = no projection);
+ *   3. compressed block score s_ij = Qt_i . Kt_j (V is not used);
+ *   4. hard top-k per query block i: the topk largest s_ij, ties broken
+ *      toward the lower j, written to lut[b,h,i,:] in ascending j.
+ * Pooling, projection and score are computed in fp64, so the LUT matches an
+ * exact-arithmetic selection except where two scores lie within ~1e-12.
+ * Ignores p->lut_mode, p->sm_scale and p->sparse_dtype.
+ */
+sla_status_t sla_route(const sla_params_t *p, const void *q, const void *k,
+                       const float *w_q, const float *w_k, int32_t *lut,
+                       void *workspace, size_t ws_bytes, sla_stream_t stream);
+
+/*
+ * sla_forward -- SLA2 hybrid forward ([SLA2] sec. 2.A):
+ *   O = alpha (.) O_s + (1 - alpha) (.) O_l
+ * O_s: softmax attention of each query over the tokens of its query block's
+ *      selected KV blocks only, renormalised over them (0 if topk == 0);
+ * O_l: ReLU-feature linear attention ([SALAD] sec. 2, phi = ReLU) over the
+ *      tokens of the blocks NOT selected:
+ *      phi(q) (sum_{j not in S} h_j) / (phi(q) . sum_{j not in S} z_j),
+ *      h_j = phi(K_j)^T V_j, z_j = phi(K_j)^T 1; 0 if the denominator <= 0.
+ * lut: LUT_COMPUTE -> routing as in sla_route (w_q, w_k used) and the LUT is
+ *      written to `lut` (which may be NULL); LUT_GIVEN -> `lut` is read and
+ *      must hold topk distinct entries in [0, N/Bk) per row (any order);
+ *      invalid entries are skipped and flagged SLA_ERR_DEVICE_CHECK.
+ * sparse_dtype FP8_E4M3: Q, K, V are quantised to e4m3 with one absmax
+ *      scale per 64-token block and P to e4m3 per tile ([SLA2] sec. 2.C:
+ *      low-bit Q, K, P, V in the sparse branch); the linear branch stays
+ *      bf16/fp32.
+ */
+sla_status_t sla_forward(const sla_params_t *p, const void *q, const void *k, const void *v,
+                         const float *alpha, const float *w_q, const float *w_k,
+                         int32_t *lut, void *out,
+                         void *workspace, size_t ws_bytes, sla_stream_t stream);
+
+/*
+ * sla_pisa_forward -- PISA exact-or-approximate attention ([PISA] sec. 2,
+ * "Algoritmo Core"), zero-order mode:
+ *   o_t = N_t / D_t,
+ *   N_t = sum_{j in S} sum_n e^{tau q.k_jn - m} v_jn + sum_{j not in S} e^{tau q.kbar_j - m} sum_n v_jn
+ *   D_t = sum_{j in S} sum_n e^{tau q.k_jn - m}      + sum_{j not in S} Bk e^{tau q.kbar_j - m}
+ * with kbar_j the mean key (centroid) of block j; both sums share one
+ * online-softmax maximum m.  S comes from the router (LUT_COMPUTE; pass
+ * w_q = w_k = NULL for PISA's plain pooled score) or from `lut` (LUT_GIVEN).
+ * Requires Bq == Bk and sparse_dtype = BF16.
+ */
+sla_status_t sla_pisa_forward(const sla_params_t *p, const void *q, const void *k,
+                              const void *v, const float *w_q, const float *w_k,
+                              int32_t *lut, void *out,
+                              void *workspace, size_t ws_bytes, sla_stream_t stream);
+
+/* Static text for a status code. */
+const char *sla_status_string(sla_status_t s);
+
+/* Synchronises `stream`, then reads and clears the device status word of the
+ * current device: SLA_OK, SLA_ERR_TIMEOUT or SLA_ERR_DEVICE_CHECK (or
+ * SLA_ERR_CUDA if the synchronisation itself failed). */
+sla_status_t sla_check_device_status(sla_stream_t stream);
+
+/*
+ * Kernel tracing.  While enabled, every kernel the library launches is
+ * bracketed by a pair of CUDA events recorded on its own stream (no device
+ * cost; about a microsecond of host time per launch).  sla_profile_read()
+ * synchronises those events and returns, per kernel kind, the summed device
+ * time in milliseconds and the number of launches since the last read; it
+ * then forgets them.  Host-side state only; guarded by a mutex.
+ */
+typedef enum {
+    SLA_KERNEL_POOL = 0,        /* mean pooling of Q (and K in sla_route)      */
+    SLA_KERNEL_KV_STATS = 1,    /* K/V pre-pass                                 */
+    SLA_KERNEL_H_REDUCE = 2,    /* reduction of the per-chunk H partials       */
+    SLA_KERNEL_FOLD_W = 3,      /* W_q W_k^T                                    */
+    SLA_KERNEL_SCORE_TOPK = 4,  /* fp64 block score + top-k                     */
+    SLA_KERNEL_ATTN = 5,        /* sparse / PISA attention + fused epilogue     */
+    SLA_KERNEL_KINDS = 6
+} sla_kernel_kind_t;
+
+sla_status_t sla_profile_enable(int32_t on);
+/* ms_total and launches: arrays of SLA_KERNEL_KINDS entries (either may be NULL). */
+sla_status_t sla_profile_read(double *ms_total, int64_t *launches);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int32_t sla_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SLA_B200_H */

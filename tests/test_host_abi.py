@@ -1,0 +1,117 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every function the header declares, and rejects bad arguments before
+anything is enqueued (so no call here touches a device)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from block_sparse_linear_proj_b200 import build as B
+from block_sparse_linear_proj_b200 import sla as S
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return S.load()
+
+
+def header_functions():
+    txt = open(os.path.join(ROOT, "include", "sla.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(sla_[a-z_]+)\s*\(", txt)))
+
+
+def test_header_declares_the_calls():
+    fns = header_functions()
+    for name in ("sla_route", "sla_forward", "sla_pisa_forward", "sla_workspace_size",
+                 "sla_status_string", "sla_check_device_status"):
+        assert name in fns
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in header_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        assert S.status_string(code)
+    assert lib.sla_version() >= 100
+
+
+FAKE = ctypes.c_void_p(1 << 20)        # aligned, never dereferenced: validation fails first
+
+
+def call_route(p, q=FAKE, k=FAKE, lut=FAKE, ws=FAKE, ws_bytes=1 << 40):
+    return S.load().sla_route(ctypes.byref(p), q, k, None, None, lut, ws, ws_bytes, None)
+
+
+def call_forward(p, q=FAKE, k=FAKE, v=FAKE, alpha=FAKE, lut=FAKE, out=FAKE, ws=FAKE,
+                 ws_bytes=1 << 40):
+    return S.load().sla_forward(ctypes.byref(p), q, k, v, alpha, None, None, lut, out, ws,
+                                ws_bytes, None)
+
+
+def call_pisa(p, ws_bytes=1 << 40, lut=FAKE):
+    return S.load().sla_pisa_forward(ctypes.byref(p), FAKE, FAKE, FAKE, None, None, lut, FAKE,
+                                     FAKE, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(N=1000), S.SLA_ERR_INVALID_ARG),            # N % Bq != 0
+    (dict(topk=17), S.SLA_ERR_INVALID_ARG),           # topk > Nk
+    (dict(topk=-1), S.SLA_ERR_INVALID_ARG),
+    (dict(B=0), S.SLA_ERR_INVALID_ARG),
+    (dict(d=96), S.SLA_ERR_UNSUPPORTED),
+    (dict(Bq=32), S.SLA_ERR_UNSUPPORTED),
+    (dict(Bk=128, N=1024, topk=2), S.SLA_ERR_UNSUPPORTED),
+    (dict(sparse_dtype=7), S.SLA_ERR_INVALID_ARG),
+    (dict(lut_mode=3), S.SLA_ERR_INVALID_ARG),
+])
+def test_parameter_validation(lib, kw, code):
+    base = dict(B=1, H=2, N=1024, d=64, Bq=64, Bk=64, topk=4)
+    base.update(kw)
+    extra = {k: base.pop(k) for k in ("sparse_dtype", "lut_mode") if k in base}
+    p = S.params(**base, **extra)
+    assert call_route(p) == code
+    assert call_forward(p) == code
+    assert lib.sla_workspace_size(ctypes.byref(p)) == 0
+
+
+def test_pointer_validation(lib):
+    p = S.params(1, 2, 1024, 64, 64, 64, 4)
+    assert call_route(p, q=None) == S.SLA_ERR_INVALID_ARG
+    assert call_route(p, k=ctypes.c_void_p((1 << 20) + 2)) == S.SLA_ERR_INVALID_ARG
+    assert call_forward(p, v=None) == S.SLA_ERR_INVALID_ARG
+    assert call_forward(p, alpha=None) == S.SLA_ERR_INVALID_ARG
+    assert call_forward(p, out=ctypes.c_void_p((1 << 20) + 8)) == S.SLA_ERR_INVALID_ARG
+    pg = S.params(1, 2, 1024, 64, 64, 64, 4, lut_mode=S.SLA_LUT_GIVEN)
+    assert call_forward(pg, lut=None) == S.SLA_ERR_INVALID_ARG
+
+
+def test_workspace_validation(lib):
+    p = S.params(1, 2, 1024, 64, 64, 64, 4)
+    need = lib.sla_workspace_size(ctypes.byref(p))
+    assert need > 0
+    assert call_route(p, ws_bytes=need - 1) == S.SLA_ERR_WORKSPACE
+    assert call_route(p, ws=None) == S.SLA_ERR_WORKSPACE
+    assert call_route(p, ws=ctypes.c_void_p((1 << 20) + 128)) == S.SLA_ERR_WORKSPACE
+    assert call_forward(p, ws_bytes=need - 1) == S.SLA_ERR_WORKSPACE
+
+
+def test_mode_restrictions(lib):
+    # PISA needs Bq == Bk and the bf16 sparse branch
+    assert call_pisa(S.params(1, 2, 1024, 64, 128, 64, 4)) == S.SLA_ERR_UNSUPPORTED
+    assert call_pisa(S.params(1, 2, 1024, 64, 64, 64, 4, sparse_dtype=1)) == S.SLA_ERR_UNSUPPORTED
+    # the FP8 sparse branch needs d = 128 and Bq = 128
+    assert call_forward(S.params(1, 2, 1024, 64, 64, 64, 4, sparse_dtype=1)) == S.SLA_ERR_UNSUPPORTED
+
+
+def test_workspace_size_grows_with_problem(lib):
+    small = S.params(1, 2, 1024, 64, 64, 64, 4)
+    big = S.params(1, 12, 32768, 128, 128, 64, 52)
+    assert lib.sla_workspace_size(ctypes.byref(big)) > lib.sla_workspace_size(ctypes.byref(small))
