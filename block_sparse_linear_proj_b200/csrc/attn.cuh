@@ -39,7 +39,7 @@ struct AttnArgs {
     float log2_bk;                 // log2(Bk), PISA pseudo-tile bias
     const int32_t* lut;            // [BH][Nq][topk]
     const float* alpha;            // [BH][N]        (SLA)
-    const float* hsum;             // [BH][D][D]     (SLA)
+    const float* hsum;             // [BH][D][D]     (SLA), transposed: H^T[e][c]
     const float* zsum;             // [BH][D]        (SLA)
     const float* zj;               // [BH][Nk][D]    (SLA)
     void* out;                     // [BH][N][D] bf16 or fp32
@@ -256,7 +256,6 @@ __global__ void __launch_bounds__(256, 1)
             auto issue_pv = [&](int e) -> bool {
                 const int s = e % kStages, b = e & 1, u = e >> 1;
                 if (!mbar_wait(&p_full[b], u & 1, abort_flag, lim)) return false;
-                if (SLA && !mbar_wait(&k_relu[s], (e / kStages) & 1, abort_flag, lim)) return false;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
@@ -264,7 +263,10 @@ __global__ void __launch_bounds__(256, 1)
                     const uint64_t bd = sdesc(sV(s) + kk * 2048, L::KBOX, 1024, kSwizzle128B);
                     umma_f16_ss(tmem + COL_O, ad, bd, ID_PV, (e > 0 || kk > 0) ? 1u : 0u);
                 }
+                umma_commit(&p_empty[b]);
                 if (SLA) {
+                    if (!mbar_wait(&k_relu[s], (e / kStages) & 1, abort_flag, lim)) return false;
+                    tc_fence_after();
                     const int bits = (sched[e] >> 16) & 3;
                     for (int g = 0; g < 2; ++g) {
                         if (!((bits >> g) & 1)) continue;
@@ -280,7 +282,6 @@ __global__ void __launch_bounds__(256, 1)
                     }
                 }
                 umma_commit(&kv_empty[s]);
-                umma_commit(&p_empty[b]);
                 return true;
             };
             for (int e = 0; ok && e < n_total; ++e) {
@@ -346,13 +347,14 @@ __global__ void __launch_bounds__(256, 1)
                 constexpr int PER = L::KT / 16 / 64;     // uint4 per thread
 #pragma unroll
                 for (int x = 0; x < PER; ++x) {
-                    // phi(k) = max(k, 0), bf16 -> fp16 (exact inside the fp16 range)
-                    uint4 v = kp[t * PER + x];
+                    // phi(k) = max(k, 0), bf16 -> fp16 (exact inside the fp16 range);
+                    // consecutive threads touch consecutive 16-byte chunks (no bank conflicts)
+                    uint4 v = kp[x * 64 + t];
                     v.x = pack_half2(fmaxf(bf16lo(v.x), 0.f), fmaxf(bf16hi(v.x), 0.f));
                     v.y = pack_half2(fmaxf(bf16lo(v.y), 0.f), fmaxf(bf16hi(v.y), 0.f));
                     v.z = pack_half2(fmaxf(bf16lo(v.z), 0.f), fmaxf(bf16hi(v.z), 0.f));
                     v.w = pack_half2(fmaxf(bf16lo(v.w), 0.f), fmaxf(bf16hi(v.w), 0.f));
-                    kp[t * PER + x] = v;
+                    kp[x * 64 + t] = v;
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -503,7 +505,8 @@ __global__ void __launch_bounds__(256, 1)
             // (1) B_g = H - G_g (row c = r of the d x d matrices), bf16 hi + lo,
             //     MN-major 128-byte-swizzled boxes of 64 columns
             if (fin && r < D) {
-                const float* hrow = a.hsum + (static_cast<long long>(bh) * D + r) * D;
+                // H is stored transposed per head, H^T[e][c]: lane r reads column r, coalesced
+                const float* hcol = a.hsum + static_cast<long long>(bh) * D * D + r;
                 for (int gg = 0; gg < n_groups; ++gg) {
                     unsigned char* bhi = smem + L::OFF_STAGE + (2 * gg) * L::BBUF;
                     unsigned char* blo = bhi + L::BBUF;
@@ -521,8 +524,8 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll
                             for (int y = 0; y < 4; ++y) {
                                 const int cc = c + 8 * x + 2 * y;
-                                const float v0 = hrow[cc] - (gs ? __uint_as_float(gv[8 * x + 2 * y]) : 0.f);
-                                const float v1 = hrow[cc + 1] - (gs ? __uint_as_float(gv[8 * x + 2 * y + 1]) : 0.f);
+                                const float v0 = hcol[cc * D] - (gs ? __uint_as_float(gv[8 * x + 2 * y]) : 0.f);
+                                const float v1 = hcol[(cc + 1) * D] - (gs ? __uint_as_float(gv[8 * x + 2 * y + 1]) : 0.f);
                                 hi4[y] = pack_bf16(v0, v1);
                                 lo4[y] = pack_bf16(v0 - bf16lo(hi4[y]), v1 - bf16hi(hi4[y]));
                             }

@@ -244,7 +244,8 @@ __global__ void __launch_bounds__(256, 2) kv_stats_kernel(KvStatsArgs a) {
     }
 }
 
-// H[bh] = sum over chunks of hpart (fixed order), Z[bh] = sum_j z_j.
+// H[bh] = sum over chunks of hpart (fixed order), stored transposed
+// (hsum[bh][e][c] = H[c][e]); Z[bh] = sum_j z_j.
 // grid (D*D/256 + 1, BH), 256 threads; the last x-block reduces Z.
 template <int D>
 __global__ void __launch_bounds__(256) h_reduce_kernel(const float* __restrict__ hpart,
@@ -258,7 +259,8 @@ __global__ void __launch_bounds__(256) h_reduce_kernel(const float* __restrict__
         const float* src = hpart + bh * nchunk * static_cast<long long>(D) * D + idx;
         float s = 0.f;
         for (int c = 0; c < nchunk; ++c) s += src[static_cast<long long>(c) * D * D];
-        hsum[bh * D * D + idx] = s;
+        const int c = idx / D, e = idx % D;
+        hsum[bh * D * D + e * D + c] = s;
     } else if (threadIdx.x < D) {
         const float* src = zj + bh * static_cast<long long>(Nk) * D + threadIdx.x;
         float s = 0.f;
