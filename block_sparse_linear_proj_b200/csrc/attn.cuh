@@ -1,16 +1,19 @@
 // attn.cuh -- block-sparse attention on sm_100a (tcgen05 + TMEM + TMA).
 //
-// One CTA owns 128 query rows = 128/Bq query blocks ("groups") of one head.
-// It walks the union of its groups' selected KV blocks in ascending order
-// (each entry tagged with the groups that selected it) and, in PISA mode,
-// then the head's centroid pseudo-tiles.  Per entry:
-//   S  = Q K_j^T                        tcgen05.mma M=128 N=64  -> TMEM (2 buffers)
-//   P  = exp2(S*tau*log2e - m)          softmax warps, one row per thread,
+// One CTA owns up to 128 query rows = GR query blocks ("groups") of one head
+// (GR = 128/Bq, except the SLA mode with d = 128, where GR = 1 so that the
+// per-group G accumulators fit in tensor memory).  It walks the union of its
+// groups' selected KV blocks in ascending order (each entry tagged with the
+// groups that selected it) and, in PISA mode, then the head's centroid
+// pseudo-tiles.  Q and P live in tensor memory (A operands of the MMAs), so
+// shared memory only carries the K/V tiles.  Per entry:
+//   S  = Q K_j^T                        tcgen05.mma M=128 N=64, A from TMEM -> TMEM (2 buffers)
+//   P  = 2^(S*tau*log2e - m)            softmax warps, one row per thread,
 //                                       online max with lazy rescale of O;
-//                                       P is stored as fp16
-//   O += P V_j                          tcgen05.mma M=128 N=d   -> TMEM (fp16 V copy)
-//   G_g += phi(K_j)^T V_j  (SLA only)   tcgen05.mma M=128 N=d   -> TMEM, per group;
-//                                       phi(K_j) written in place as fp16
+//                                       packed fp16 exp2, P written to TMEM
+//   O += P V_j                          tcgen05.mma M=128 N=d, A from TMEM (fp16 V copy)
+//   G_g += phi(K_j)^T V_j  (SLA only)   tcgen05.mma M=128 N=d   -> TMEM, per group
+//                                       (fp16 phi(K) copy from the K/V pre-pass)
 // Linear branch (SALAD ReLU kernel; SLA2 combine): after the loop,
 //   O_l = phi(Q) (H - G_g) / (phi(q) . (Z - sum_{j in S_g} z_j))
 // with (H - G_g) split into bf16 hi + lo and multiplied on the tensor core,
@@ -21,20 +24,28 @@
 // e^{q.kbar_j - m} (sum_n v_n) enters N_t and Bk e^{q.kbar_j - m} enters D_t in
 // the same online softmax; out = N_t / D_t.
 //
-// Warp roles (256 threads): w0 TMA producer, w1 MMA issuer (+ TMEM owner),
-// w2-3 phi(K) transform + z sums (SLA), w4-7 softmax and epilogue.
-// Every wait is bounded; a wait that runs out sets the device status word and
-// the CTA unwinds after draining its own TMA loads and MMAs.
+// K tiles and V (+ phi(K)) tiles stream through two separate rings: a K slot is
+// released as soon as S of its block completes, so K loads run several blocks
+// ahead of the P.V / G products.
+// Warp roles (384 threads): w0 TMA producer for both rings, w1 issues S = Q K^T
+// (and owns TMEM), w3 issues P.V, phi(K)^T V and the linear-branch products (two
+// issuers, so one's barrier waits overlap the other's MMAs: an MMA issue blocks
+// until the tensor pipe takes it), w2 the per-group sums of z_j over the
+// selected blocks (SLA), w4-11 softmax
+// and epilogue: two warpgroups, each thread owning one row (its TMEM lane) and
+// one half of the columns (exp2 and P for 32 of the 64 keys of a block; the
+// row maximum is taken over all 64 by both, so no exchange per block).  Every
+// wait is bounded; a wait that runs out sets the device status word and the
+// CTA unwinds after draining its own TMA loads and MMAs.
 #pragma once
 #include "common.cuh"
 
 namespace sla {
 
-constexpr int kStages = 3;
 constexpr float kRescaleLog2 = 8.0f;    // lazy O rescale threshold (log2 units)
 
 struct AttnArgs {
-    int N, Nq, Nk, Bq, topk, tiles_per_head;
+    int N, Nq, Nk, Bq, GR, topk, tiles_per_head;
     float scale_log2;              // tau * log2(e)
     float log2_bk;                 // log2(Bk), PISA pseudo-tile bias
     const int32_t* lut;            // [BH][Nq][topk]
@@ -52,6 +63,43 @@ __device__ __forceinline__ float fast_exp2(float x) {
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
+// 2^x for two fp16 values at once (one MUFU operation).
+__device__ __forceinline__ uint32_t exp2_h2(uint32_t x) {
+    uint32_t y;
+    asm("ex2.approx.f16x2 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+__device__ __forceinline__ uint32_t hadd2_u(uint32_t a, uint32_t b) {
+    __half2 r = __hadd2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+
+// P = 2^(x - m) for the 32 logits sv[OFF .. OFF+31] as 16 packed fp16 pairs;
+// returns their sum.  EXACT: sv holds raw scores (x = s*c), else x itself.
+template <int OFF, bool EXACT>
+__device__ __forceinline__ float softmax_half(const uint32_t (&sv)[64], float c, float m, bool live,
+                                              uint32_t (&pw)[16]) {
+    float ls = 0.f;
+#pragma unroll
+    for (int ch = 0; ch < 4; ++ch) {
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            const int j = OFF + ch * 8 + 2 * x;
+            float x0, x1;
+            if (EXACT) {
+                x0 = fmaf(__uint_as_float(sv[j]), c, -m);
+                x1 = fmaf(__uint_as_float(sv[j + 1]), c, -m);
+            } else {
+                x0 = __uint_as_float(sv[j]) - m;
+                x1 = __uint_as_float(sv[j + 1]) - m;
+            }
+            pw[4 * ch + x] = live ? exp2_h2(pack_half2(x0, x1)) : 0u;
+        }
+        const uint32_t s4 = hadd2_u(hadd2_u(pw[4 * ch], pw[4 * ch + 1]), hadd2_u(pw[4 * ch + 2], pw[4 * ch + 3]));
+        ls += half_lo(s4) + half_hi(s4);
+    }
+    return ls;
+}
 
 // 32 consecutive output values of one row: bf16 (four 16-byte stores) or fp32.
 __device__ __forceinline__ void store_row32(void* out, int f32, long long off, const float (&v)[32]) {
@@ -68,32 +116,46 @@ __device__ __forceinline__ void store_row32(void* out, int f32, long long off, c
     }
 }
 
-template <int D>
+template <int D, bool PISA>
 struct AttnLayout {
+    static constexpr int KS = PISA ? 6 : 4;          // K ring slots
+    static constexpr int VS = PISA ? 6 : 4;          // V (+ phi(K)) ring slots
+    static constexpr int PF = 0;                     // L2 prefetch distance (blocks); 0 = off
     static constexpr int QB = 128 * D * 2;           // Q tile bytes
-    static constexpr int KT = 64 * D * 2;            // K (or V) tile bytes
+    static constexpr int KT = 64 * D * 2;            // one 64-token tile (bf16 or fp16)
+    static constexpr int VT = (PISA ? 1 : 2) * KT;   // V (+ phi(K)) slot
     static constexpr int KBOX = 64 * 128;            // one 64-row x 128-byte box
     static constexpr int QBOX = 128 * 128;           // one 128-row x 128-byte box
-    static constexpr int PT = 128 * 128;             // P tile: 128 rows x 64 bf16
-    static constexpr int OFF_Q = 0;
-    static constexpr int OFF_STAGE = OFF_Q + QB;
-    static constexpr int OFF_P = OFF_STAGE + kStages * 2 * KT;
-    static constexpr int OFF_MISC = OFF_P + 2 * PT;
+    static constexpr int OFF_K = 0;
+    static constexpr int OFF_V = OFF_K + KS * KT;
+    // Q lands in the last two K slots; it moves to TMEM before their first use
+    static constexpr int OFF_Q = OFF_K + (KS - 2) * KT;
+    static constexpr int OFF_MISC = OFF_V + VS * VT;
+    static constexpr int OFF_STAGE = OFF_V;          // epilogue buffers reuse the V ring
+    static_assert(QB == 2 * KT, "Q tile spans two K slots");
     static constexpr int BBUF = D * D * 2;           // one (H - G) hi or lo buffer
     static constexpr int BBOX = D * 128;             // one 64-column box of it
 };
 
+constexpr int kAttnThreads = 384;
+
 template <int D, bool PISA>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(kAttnThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKc,
-                const __grid_constant__ CUtensorMap tmVc, const AttnArgs a) {
-    using L = AttnLayout<D>;
+                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmPhi,
+                const __grid_constant__ CUtensorMap tmKc, const __grid_constant__ CUtensorMap tmVc,
+                const AttnArgs a) {
+    using L = AttnLayout<D, PISA>;
     constexpr bool SLA = !PISA;
     constexpr int NBOX = D / 64;
-    constexpr uint32_t NCOLS = (PISA ? (128 + D) : (128 + 3 * D)) <= 256 ? 256 : 512;
+    constexpr int KS = L::KS, VS = L::VS;
+    // tensor memory columns: S0 | S1 | O | G_0 (| G_1 when d = 64) | Q | P0 | P1
+    constexpr uint32_t NCOLS = 512;
     constexpr uint32_t COL_O = 128;
     constexpr uint32_t COL_G0 = 128 + D;
+    constexpr uint32_t COL_Q = PISA ? 128 + D : (D == 128 ? 128 + 2 * D : 128 + 3 * D);
+    constexpr uint32_t COL_P = COL_Q + D / 2;        // + 32 * b
+    static_assert(COL_P + 64 <= NCOLS, "tensor memory budget");
 
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -103,11 +165,12 @@ __global__ void __launch_bounds__(256, 1)
     // misc region
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_MISC);
     uint64_t* q_full = bars + 0;
-    uint64_t* kv_full = bars + 1;                 // [kStages]
-    uint64_t* kv_empty = kv_full + kStages;       // [kStages]
-    uint64_t* kdone = kv_empty + kStages;         // [kStages]  S_e done -> K_j reusable
-    uint64_t* k_relu = kdone + kStages;           // [kStages]  phi(K_j) written
-    uint64_t* s_full = k_relu + kStages;          // [2]
+    uint64_t* k_full = bars + 1;                  // [KS]
+    uint64_t* k_empty = k_full + KS;              // [KS]
+    uint64_t* v_full = k_empty + KS;              // [VS]
+    uint64_t* v_empty = v_full + VS;              // [VS]
+    uint64_t* q_tmem = v_empty + VS;              // Q copied into TMEM
+    uint64_t* s_full = q_tmem + 1;                // [2]
     uint64_t* s_empty = s_full + 2;               // [2]
     uint64_t* p_full = s_empty + 2;               // [2]
     uint64_t* p_empty = p_full + 2;               // [2]
@@ -115,41 +178,50 @@ __global__ void __launch_bounds__(256, 1)
     uint64_t* epi_ready = final_bar + 1;
     uint64_t* lin_done = epi_ready + 1;
     uint64_t* drain_bar = lin_done + 1;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+    uint64_t* drain2_bar = drain_bar + 1;
+    uint64_t* xl_bar = drain2_bar + 1;            // [4] final row-sum exchange per quarter
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xl_bar + 4);
     int* n_exact_s = reinterpret_cast<int*>(tmem_slot + 1);
     volatile int* abort_flag = n_exact_s + 1;
     int* g_any = n_exact_s + 2;                   // [2] group selected >= 1 block
-    float* zu = reinterpret_cast<float*>(smem + L::OFF_MISC + 256);       // [2][D]
-    uint32_t* mark = reinterpret_cast<uint32_t*>(zu + 2 * D);            // [ceil(Nk/16)]
+    float* zu = reinterpret_cast<float*>(smem + L::OFF_MISC + 384);       // [2][D]
+    float* xl = zu + 2 * D;                                              // [2][128] row-sum halves
+    uint32_t* mark = reinterpret_cast<uint32_t*>(xl + 256);              // [ceil(Nk/16)]
     const int nwords = (a.Nk + 15) >> 4;
     int32_t* sched = reinterpret_cast<int32_t*>(mark + ((nwords + 3) & ~3));
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int bh = blockIdx.x / a.tiles_per_head;
     const int tile = blockIdx.x % a.tiles_per_head;
-    const int GR = 128 / a.Bq;
+    const int GR = a.GR;
     const int qb0 = tile * GR;
+    const int row0 = qb0 * a.Bq;                  // first token of the tile
     const int n_groups = min(GR, a.Nq - qb0);
 
     // ------------------------------------------------------------ set-up
     if (tid == 0) {
         mbar_init(q_full, 1);
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(&kv_full[s], 1);
-            mbar_init(&kv_empty[s], 1);
-            mbar_init(&kdone[s], 1);
-            mbar_init(&k_relu[s], 2);
+        mbar_init(q_tmem, 8);
+        for (int s = 0; s < KS; ++s) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&k_empty[s], 1);
+        }
+        for (int s = 0; s < VS; ++s) {
+            mbar_init(&v_full[s], 1);
+            mbar_init(&v_empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&s_full[b], 1);
-            mbar_init(&s_empty[b], 4);
-            mbar_init(&p_full[b], 4);
+            mbar_init(&s_empty[b], 8);
+            mbar_init(&p_full[b], 8);
             mbar_init(&p_empty[b], 1);
         }
         mbar_init(final_bar, 1);
-        mbar_init(epi_ready, 6);
+        mbar_init(epi_ready, 9);
         mbar_init(lin_done, 1);
         mbar_init(drain_bar, 1);
+        mbar_init(drain2_bar, 1);
+        for (int x = 0; x < 4; ++x) mbar_init(&xl_bar[x], 2);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -157,9 +229,9 @@ __global__ void __launch_bounds__(256, 1)
         tmem_alloc(tmem_slot, NCOLS);
         tmem_relinquish();
     }
-    for (int w = tid; w < nwords; w += 256) mark[w] = 0u;
+    for (int w = tid; w < nwords; w += kAttnThreads) mark[w] = 0u;
     __syncthreads();
-    for (int x = tid; x < n_groups * a.topk; x += 256) {
+    for (int x = tid; x < n_groups * a.topk; x += kAttnThreads) {
         const int g = x / a.topk;
         const int j = a.lut[(static_cast<long long>(bh) * a.Nq + qb0 + g) * a.topk + x % a.topk];
         if (j < 0 || j >= a.Nk) { report(kStatusBadData); continue; }
@@ -169,16 +241,31 @@ __global__ void __launch_bounds__(256, 1)
     }
     __syncthreads();
     if (warp == 0) {
+        // count, then write the selected blocks in ascending order rotated by a
+        // per-tile offset: the CTAs of one head (which run concurrently) then
+        // start their walks at different KV blocks instead of all requesting
+        // the same tiles from L2 at the same moment
         int cnt = 0;
         uint32_t any = 0u;
         const uint32_t lt = (1u << lane) - 1u;
         for (int j0 = 0; j0 < a.Nk; j0 += 32) {
             const int j = j0 + lane;
             const uint32_t bits = j < a.Nk ? (mark[j >> 4] >> (2 * (j & 15))) & 3u : 0u;
-            const uint32_t bal = __ballot_sync(0xffffffffu, bits != 0u);
-            if (bits) sched[cnt + __popc(bal & lt)] = j | static_cast<int>(bits << 16);
-            cnt += __popc(bal);
+            cnt += __popc(__ballot_sync(0xffffffffu, bits != 0u));
             any |= bits;
+        }
+        const int rot = cnt > 0 ? static_cast<int>((static_cast<unsigned>(tile) * 2654435761u >> 7) % cnt) : 0;
+        int pos = 0;
+        for (int j0 = 0; j0 < a.Nk; j0 += 32) {
+            const int j = j0 + lane;
+            const uint32_t bits = j < a.Nk ? (mark[j >> 4] >> (2 * (j & 15))) & 3u : 0u;
+            const uint32_t bal = __ballot_sync(0xffffffffu, bits != 0u);
+            if (bits) {
+                int at = pos + __popc(bal & lt) - rot;
+                if (at < 0) at += cnt;
+                sched[at] = j | static_cast<int>(bits << 16);
+            }
+            pos += __popc(bal);
         }
         any = __reduce_or_sync(0xffffffffu, any);
         if (lane == 0) {
@@ -197,10 +284,9 @@ __global__ void __launch_bounds__(256, 1)
     const unsigned long long lim = a.wait_ns;
     const unsigned long long drain_lim = 4000000000ull;
 
-    const uint32_t sQ = sbase + L::OFF_Q;
-    auto sK = [&](int s) { return sbase + L::OFF_STAGE + s * 2 * L::KT; };
-    auto sV = [&](int s) { return sbase + L::OFF_STAGE + s * 2 * L::KT + L::KT; };
-    auto sP = [&](int b) { return sbase + L::OFF_P + b * L::PT; };
+    auto sK = [&](int s) { return sbase + L::OFF_K + s * L::KT; };
+    auto sV = [&](int s) { return sbase + L::OFF_V + s * L::VT; };
+    auto sPhi = [&](int s) { return sbase + L::OFF_V + s * L::VT + L::KT; };
 
     auto fail = [&]() {
         *abort_flag = 1;
@@ -209,71 +295,130 @@ __global__ void __launch_bounds__(256, 1)
 
     if (warp == 0) {
         // ======================================================== TMA producer
+        // Two rings, one thread: issue whichever pending load is needed first and
+        // has a free slot.  K(e) is consumed by S(e), which runs about two blocks
+        // ahead of P.V(e), so K(kn) goes first while kn <= vn + 2.
         if (lane == 0) {
             prefetch_tmap(&tmQ);
             prefetch_tmap(&tmK);
             prefetch_tmap(&tmV);
-            const int qrow = bh * a.N + tile * 128;
+            if (SLA) prefetch_tmap(&tmPhi);
+            if (PISA) { prefetch_tmap(&tmKc); prefetch_tmap(&tmVc); }
+            const int qrow = bh * a.N + row0;
             mbar_arrive_expect_tx(q_full, L::QB);
             for (int b = 0; b < NBOX; ++b)
                 tma_load_2d(smem + L::OFF_Q + b * L::QBOX, &tmQ, q_full, b * 64, qrow);
-            int issued = 0;
-            for (int e = 0; e < n_total; ++e) {
-                const int s = e % kStages, r = e / kStages;
-                if (!mbar_wait(&kv_empty[s], (r & 1) ^ 1, abort_flag, lim)) { fail(); break; }
-                mbar_arrive_expect_tx(&kv_full[s], 2 * L::KT);
-                unsigned char* kd = smem + L::OFF_STAGE + s * 2 * L::KT;
-                unsigned char* vd = kd + L::KT;
-                if (e < n_exact) {
-                    const int row = bh * a.N + (sched[e] & 0xFFFF) * 64;
-                    for (int b = 0; b < NBOX; ++b) {
-                        tma_load_2d(kd + b * L::KBOX, &tmK, &kv_full[s], b * 64, row);
-                        tma_load_2d(vd + b * L::KBOX, &tmV, &kv_full[s], b * 64, row);
-                    }
-                } else {
-                    const int row = bh * a.Nk + (e - n_exact) * 64;
-                    for (int b = 0; b < NBOX; ++b) {
-                        tma_load_2d(kd + b * L::KBOX, &tmKc, &kv_full[s], b * 64, row);
-                        tma_load_2d(vd + b * L::KBOX, &tmVc, &kv_full[s], b * 64, row);
+            int kn = 0, vn = 0;
+            bool q_moved = false;
+            unsigned long long t0 = globaltimer_ns();
+            uint32_t idle = 0;
+            while (kn < n_total || vn < n_total) {
+                bool did = false;
+                const bool want_k = kn < n_total && (vn >= n_total || kn <= vn + 2);
+                if (want_k) {
+                    const int s = kn % KS, r = kn / KS;
+                    const bool q_ok = !(r == 0 && s >= KS - 2) || q_moved || (q_moved = mbar_ready(q_tmem, 0));
+                    if (q_ok && mbar_ready(&k_empty[s], (r & 1) ^ 1)) {
+                        mbar_arrive_expect_tx(&k_full[s], L::KT);
+                        unsigned char* kd = smem + L::OFF_K + s * L::KT;
+                        if (kn < n_exact) {
+                            const int row = bh * a.N + (sched[kn] & 0xFFFF) * 64;
+                            for (int b = 0; b < NBOX; ++b) tma_load_2d(kd + b * L::KBOX, &tmK, &k_full[s], b * 64, row);
+                        } else {
+                            const int row = bh * a.Nk + (kn - n_exact) * 64;
+                            for (int b = 0; b < NBOX; ++b) tma_load_2d(kd + b * L::KBOX, &tmKc, &k_full[s], b * 64, row);
+                        }
+                        ++kn;
+                        did = true;
                     }
                 }
-                issued = e + 1;
+                if (!did && vn < n_total) {
+                    const int s = vn % VS, r = vn / VS;
+                    if (mbar_ready(&v_empty[s], (r & 1) ^ 1)) {
+                        mbar_arrive_expect_tx(&v_full[s], L::VT);
+                        unsigned char* vd = smem + L::OFF_V + s * L::VT;
+                        unsigned char* pd = vd + L::KT;
+                        if (vn < n_exact) {
+                            const int row = bh * a.N + (sched[vn] & 0xFFFF) * 64;
+                            for (int b = 0; b < NBOX; ++b) {
+                                tma_load_2d(vd + b * L::KBOX, &tmV, &v_full[s], b * 64, row);
+                                if (SLA) tma_load_2d(pd + b * L::KBOX, &tmPhi, &v_full[s], b * 64, row);
+                            }
+                        } else {
+                            const int row = bh * a.Nk + (vn - n_exact) * 64;
+                            for (int b = 0; b < NBOX; ++b) tma_load_2d(vd + b * L::KBOX, &tmVc, &v_full[s], b * 64, row);
+                        }
+                        ++vn;
+                        did = true;
+                    }
+                }
+                if (did) {
+                    idle = 0;
+                    t0 = globaltimer_ns();
+                } else if (++idle >= 64) {
+                    idle = 0;
+                    if (*abort_flag || globaltimer_ns() - t0 > lim) { fail(); break; }
+                }
             }
             // drain: every load this thread issued has landed before the CTA exits
             mbar_wait(q_full, 0, abort_flag, drain_lim);
-            for (int e = max(0, issued - kStages); e < issued; ++e)
-                mbar_wait(&kv_full[e % kStages], (e / kStages) & 1, abort_flag, drain_lim);
+            for (int e = max(0, kn - KS); e < kn; ++e)
+                mbar_wait(&k_full[e % KS], (e / KS) & 1, abort_flag, drain_lim);
+            for (int e = max(0, vn - VS); e < vn; ++e)
+                mbar_wait(&v_full[e % VS], (e / VS) & 1, abort_flag, drain_lim);
         }
     } else if (warp == 1) {
-        // ======================================================== MMA issuer
+        // ======================================================== S = Q K^T issuer
         if (lane == 0) {
             constexpr uint32_t ID_S = idesc_bf16(128, 64, 0, 0);
+            bool ok = mbar_wait(q_tmem, 0, abort_flag, lim);
+            tc_fence_after();
+            for (int e = 0; ok && e < n_total; ++e) {
+                // S(e) needs its K tile and its S buffer back from the softmax of e-2
+                const int s = e % KS, b = e & 1;
+                if (!mbar_wait(&k_full[s], (e / KS) & 1, abort_flag, lim) ||
+                    !mbar_wait(&s_empty[b], ((e >> 1) & 1) ^ 1, abort_flag, lim)) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint64_t bd = sdesc(sK(s) + (kk >> 2) * L::KBOX + (kk & 3) * 32, 16, 1024, kSwizzle128B);
+                    umma_f16_ts(tmem + b * 64, tmem + COL_Q + kk * 8, bd, ID_S, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(&s_full[b]);
+                umma_commit(&k_empty[s]);
+            }
+            if (!ok) fail();
+            // drain: this thread's MMAs complete before TMEM is released
+            umma_commit(drain_bar);
+            mbar_wait(drain_bar, 0, abort_flag, drain_lim);
+        }
+    } else if (warp == 3) {
+        // ======================================================== P.V / G / linear issuer
+        if (lane == 0) {
             constexpr uint32_t ID_PV = idesc_f16(128, D, 0, 1);
             constexpr uint32_t ID_G = idesc_f16(128, D, 1, 1);
-            bool ok = mbar_wait(q_full, 0, abort_flag, lim);
-            tc_fence_after();
+            bool ok = true;
             int g_started[2] = {0, 0};                // accumulate flag of G_g
-            auto issue_pv = [&](int e) -> bool {
-                const int s = e % kStages, b = e & 1, u = e >> 1;
-                if (!mbar_wait(&p_full[b], u & 1, abort_flag, lim)) return false;
+            for (int e = 0; ok && e < n_total; ++e) {
+                const int s = e % VS, b = e & 1, u = e >> 1;
+                if (!mbar_wait(&v_full[s], (e / VS) & 1, abort_flag, lim) ||
+                    !mbar_wait(&p_full[b], u & 1, abort_flag, lim)) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t ad = sdesc(sP(b) + kk * 32, 16, 1024, kSwizzle128B);
                     const uint64_t bd = sdesc(sV(s) + kk * 2048, L::KBOX, 1024, kSwizzle128B);
-                    umma_f16_ss(tmem + COL_O, ad, bd, ID_PV, (e > 0 || kk > 0) ? 1u : 0u);
+                    umma_f16_ts(tmem + COL_O, tmem + COL_P + 32 * b + kk * 8, bd, ID_PV,
+                                (e > 0 || kk > 0) ? 1u : 0u);
                 }
                 umma_commit(&p_empty[b]);
                 if (SLA) {
-                    if (!mbar_wait(&k_relu[s], (e / kStages) & 1, abort_flag, lim)) return false;
-                    tc_fence_after();
                     const int bits = (sched[e] >> 16) & 3;
                     for (int g = 0; g < 2; ++g) {
                         if (!((bits >> g) & 1)) continue;
                         const uint32_t lbo = D == 128 ? L::KBOX : 0;   // D = 64: M rows 64-127 repeat
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk) {
-                            const uint64_t ad = sdesc(sK(s) + kk * 2048, lbo, 1024, kSwizzle128B);
+                            const uint64_t ad = sdesc(sPhi(s) + kk * 2048, lbo, 1024, kSwizzle128B);
                             const uint64_t bd = sdesc(sV(s) + kk * 2048, L::KBOX, 1024, kSwizzle128B);
                             umma_f16_ss(tmem + COL_G0 + g * D, ad, bd, ID_G,
                                         (g_started[g] || kk > 0) ? 1u : 0u);
@@ -281,25 +426,8 @@ __global__ void __launch_bounds__(256, 1)
                         g_started[g] = 1;
                     }
                 }
-                umma_commit(&kv_empty[s]);
-                return true;
-            };
-            for (int e = 0; ok && e < n_total; ++e) {
-                const int s = e % kStages, r = e / kStages, b = e & 1, u = e >> 1;
-                if (!mbar_wait(&kv_full[s], r & 1, abort_flag, lim) ||
-                    !mbar_wait(&s_empty[b], (u & 1) ^ 1, abort_flag, lim)) { ok = false; break; }
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint64_t ad = sdesc(sQ + (kk >> 2) * L::QBOX + (kk & 3) * 32, 16, 1024, kSwizzle128B);
-                    const uint64_t bd = sdesc(sK(s) + (kk >> 2) * L::KBOX + (kk & 3) * 32, 16, 1024, kSwizzle128B);
-                    umma_f16_ss(tmem + b * 64, ad, bd, ID_S, kk > 0 ? 1u : 0u);
-                }
-                umma_commit(&s_full[b]);
-                if (SLA) umma_commit(&kdone[s]);
-                if (e > 0 && !issue_pv(e - 1)) { ok = false; break; }
+                umma_commit(&v_empty[s]);
             }
-            if (ok && n_total > 0 && !issue_pv(n_total - 1)) ok = false;
             if (!ok) fail();
             umma_commit(final_bar);
             if (SLA && ok) {
@@ -312,9 +440,8 @@ __global__ void __launch_bounds__(256, 1)
                             const uint32_t bb = sbase + L::OFF_STAGE + (2 * g + part) * L::BBUF;
 #pragma unroll
                             for (int kk = 0; kk < D / 16; ++kk) {
-                                const uint64_t ad = sdesc(sQ + (kk >> 2) * L::QBOX + (kk & 3) * 32, 16, 1024, kSwizzle128B);
                                 const uint64_t bd = sdesc(bb + kk * 2048, L::BBOX, 1024, kSwizzle128B);
-                                umma_f16_ss(tmem + COL_G0 + g * D, ad, bd, ID_L,
+                                umma_f16_ts(tmem + COL_G0 + g * D, tmem + COL_Q + kk * 8, bd, ID_L,
                                             (part > 0 || kk > 0) ? 1u : 0u);
                             }
                         }
@@ -324,62 +451,40 @@ __global__ void __launch_bounds__(256, 1)
                     fail();
                 }
             }
-            // drain: all MMAs of this CTA complete before TMEM is released
-            umma_commit(drain_bar);
-            mbar_wait(drain_bar, 0, abort_flag, drain_lim);
+            umma_commit(drain2_bar);
+            mbar_wait(drain2_bar, 0, abort_flag, drain_lim);
         }
-    } else if (warp < 4) {
-        // ======================================================== phi(K) transform (SLA)
+    } else if (warp == 2) {
+        // ======================================================== z sums (SLA)
+        // Zu_g = Z - sum_{j in S_g} z_j, the linear-branch denominator vector.
         if (SLA) {
-            const int t = tid - 64;                      // 0..63
-            float zacc[2][D / 64];
-#pragma unroll
-            for (int g = 0; g < 2; ++g)
-#pragma unroll
-                for (int c = 0; c < D / 64; ++c) zacc[g][c] = 0.f;
+            const int t = lane;                          // 0..31, columns t + 32 c
             const float* zjh = a.zj + static_cast<long long>(bh) * a.Nk * D;
-            bool ok = true;
-            for (int e = 0; e < n_exact; ++e) {
-                const int s = e % kStages, r = e / kStages;
-                if (!mbar_wait(&kv_full[s], r & 1, abort_flag, lim) ||
-                    !mbar_wait(&kdone[s], r & 1, abort_flag, lim)) { ok = false; break; }
-                uint4* kp = reinterpret_cast<uint4*>(smem + L::OFF_STAGE + s * 2 * L::KT);
-                constexpr int PER = L::KT / 16 / 64;     // uint4 per thread
-#pragma unroll
-                for (int x = 0; x < PER; ++x) {
-                    // phi(k) = max(k, 0), bf16 -> fp16 (exact inside the fp16 range);
-                    // consecutive threads touch consecutive 16-byte chunks (no bank conflicts)
-                    uint4 v = kp[x * 64 + t];
-                    v.x = pack_half2(fmaxf(bf16lo(v.x), 0.f), fmaxf(bf16hi(v.x), 0.f));
-                    v.y = pack_half2(fmaxf(bf16lo(v.y), 0.f), fmaxf(bf16hi(v.y), 0.f));
-                    v.z = pack_half2(fmaxf(bf16lo(v.z), 0.f), fmaxf(bf16hi(v.z), 0.f));
-                    v.w = pack_half2(fmaxf(bf16lo(v.w), 0.f), fmaxf(bf16hi(v.w), 0.f));
-                    kp[x * 64 + t] = v;
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&k_relu[s]);
-                const int ent = sched[e];
-                const int j = ent & 0xFFFF;
-#pragma unroll
-                for (int g = 0; g < 2; ++g) {
-                    if (!((ent >> (16 + g)) & 1)) continue;
-#pragma unroll
-                    for (int c = 0; c < D / 64; ++c) zacc[g][c] += zjh[static_cast<long long>(j) * D + t + 64 * c];
-                }
-            }
-            if (!ok) fail();
             const float* zs = a.zsum + static_cast<long long>(bh) * D;
+            for (int g = 0; g < 2; ++g) {
+                float acc[D / 32];
 #pragma unroll
-            for (int g = 0; g < 2; ++g)
+                for (int c = 0; c < D / 32; ++c) acc[c] = 0.f;
+                if (g < n_groups) {
+                    const int32_t* row = a.lut + (static_cast<long long>(bh) * a.Nq + qb0 + g) * a.topk;
+#pragma unroll 4
+                    for (int x = 0; x < a.topk; ++x) {
+                        const int j = row[x];
+                        if (j < 0 || j >= a.Nk) continue;
 #pragma unroll
-                for (int c = 0; c < D / 64; ++c) zu[g * D + t + 64 * c] = zs[t + 64 * c] - zacc[g][c];
+                        for (int c = 0; c < D / 32; ++c) acc[c] += __ldg(zjh + static_cast<long long>(j) * D + t + 32 * c);
+                    }
+                }
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) zu[g * D + t + 32 * c] = zs[t + 32 * c] - acc[c];
+            }
             __syncwarp();
             if (lane == 0) mbar_arrive(epi_ready);
         }
     } else {
         // ======================================================== softmax + epilogue
-        const int q4 = warp - 4;
+        const int q4 = warp & 3;                         // TMEM lane quarter
+        const int h = (warp - 4) >> 2;                   // column half (0 or 1)
         const int r = q4 * 32 + lane;                    // row within the tile
         const int g = r / a.Bq;
         const uint32_t tl = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
@@ -387,8 +492,34 @@ __global__ void __launch_bounds__(256, 1)
         auto wwait = [&](uint64_t* bar, uint32_t par) {
             return __all_sync(0xffffffffu, mbar_wait(bar, par, abort_flag, lim) ? 1 : 0) != 0;
         };
-        float m_run = -INFINITY, l_run = 0.f;
-        bool ok = true;
+        const float c = a.scale_log2;
+        float m_run = -INFINITY, l_run = 0.f;          // running max (log2 units), this half's row sum
+        bool ok = wwait(q_full, 0);
+        // Q row r -> TMEM lane r (packed bf16 pairs), the A operand of S = Q K^T;
+        // this half copies Q columns [h*D/2, (h+1)*D/2)
+        if (ok) {
+            if (D == 128) {
+                uint32_t qv[32];
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(smem + L::OFF_Q + h * L::QBOX + sw128(r, ch));
+                    qv[4 * ch] = v.x; qv[4 * ch + 1] = v.y; qv[4 * ch + 2] = v.z; qv[4 * ch + 3] = v.w;
+                }
+                tmem_st32(tl + COL_Q + 32 * h, qv);
+            } else {
+                uint32_t qv[16];
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(smem + L::OFF_Q + sw128(r, 4 * h + ch));
+                    qv[4 * ch] = v.x; qv[4 * ch + 1] = v.y; qv[4 * ch + 2] = v.z; qv[4 * ch + 3] = v.w;
+                }
+                tmem_st16(tl + COL_Q + 16 * h, qv);
+            }
+            tmem_st_wait();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(q_tmem);
         uint32_t sv[64];
         for (int e = 0; e < n_total; ++e) {
             const int b = e & 1, u = e >> 1;
@@ -401,14 +532,16 @@ __global__ void __launch_bounds__(256, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&s_empty[b]);
 
+            // row maximum over all 64 logits (x = s * c, + log2 Bk for centroids;
+            // masked ones are -inf); exp2 only for this half's 32 columns
+            bool act = true;
             float mx = -INFINITY;
             if (e < n_exact) {
-                const bool act = (sched[e] >> (16 + g)) & 1;
+                act = (sched[e] >> (16 + g)) & 1;
+                if (act) {
 #pragma unroll
-                for (int j = 0; j < 64; ++j) {
-                    const float x = act ? __uint_as_float(sv[j]) * a.scale_log2 : -INFINITY;
-                    sv[j] = __float_as_uint(x);
-                    mx = fmaxf(mx, x);
+                    for (int j = 0; j < 64; ++j) mx = fmaxf(mx, __uint_as_float(sv[j]));
+                    mx *= c;
                 }
             } else {
                 const int c0 = (e - n_exact) * 64;
@@ -420,8 +553,7 @@ __global__ void __launch_bounds__(256, 1)
                     for (int jj = 0; jj < 16; ++jj) {
                         const int j = 16 * w + jj;
                         const bool masked = (c0 + j) >= a.Nk || ((mw >> (2 * jj + g)) & 1u);
-                        const float x = masked ? -INFINITY
-                                               : fmaf(__uint_as_float(sv[j]), a.scale_log2, a.log2_bk);
+                        const float x = masked ? -INFINITY : fmaf(__uint_as_float(sv[j]), c, a.log2_bk);
                         sv[j] = __float_as_uint(x);
                         mx = fmaxf(mx, x);
                     }
@@ -433,41 +565,35 @@ __global__ void __launch_bounds__(256, 1)
             const float m_new = need ? mx : m_run;
             const bool rescale_o = need && m_run != -INFINITY;
             if (__any_sync(0xffffffffu, rescale_o)) {
-                // O holds PV_{0..e-1}: wait for PV_{e-1} (its P buffer's release)
+                // O holds PV_{0..e-1}: wait for PV_{e-1} (its P buffer's release);
+                // this half rescales O columns [h*D/2, (h+1)*D/2)
                 if (e > 0 && !wwait(&p_empty[b ^ 1], ((e - 1) >> 1) & 1)) { ok = false; break; }
                 tc_fence_after();
                 const float f = rescale_o ? fast_exp2(m_run - m_new) : 1.f;
 #pragma unroll 1
-                for (int c = 0; c < D; c += 32) {
+                for (int cc = h * (D / 2); cc < (h + 1) * (D / 2); cc += 32) {
                     uint32_t ov[32];
-                    tmem_ld32(tl + COL_O + c, ov);
+                    tmem_ld32(tl + COL_O + cc, ov);
                     tmem_ld_wait();
 #pragma unroll
                     for (int x = 0; x < 32; ++x) ov[x] = __float_as_uint(__uint_as_float(ov[x]) * f);
-                    tmem_st32(tl + COL_O + c, ov);
+                    tmem_st32(tl + COL_O + cc, ov);
                 }
                 tmem_st_wait();
                 l_run *= f;
             }
             m_run = m_new;
-            // P = exp2(x - m), fp16, into P buffer b (row r, 128-byte swizzle)
-            unsigned char* prow = smem + L::OFF_P + b * L::PT;
-            float ls = 0.f;
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-                uint32_t w4[4];
-#pragma unroll
-                for (int x = 0; x < 4; ++x) {
-                    const int j = ch * 8 + 2 * x;
-                    const float p0 = m_run == -INFINITY ? 0.f : fast_exp2(__uint_as_float(sv[j]) - m_run);
-                    const float p1 = m_run == -INFINITY ? 0.f : fast_exp2(__uint_as_float(sv[j + 1]) - m_run);
-                    w4[x] = pack_half2(p0, p1);
-                    ls += half_lo(w4[x]) + half_hi(w4[x]);
-                }
-                *reinterpret_cast<uint4*>(prow + sw128(r, ch)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-            }
+            // P = 2^(x - m) for columns [32h, 32h + 32) as packed fp16 pairs into TMEM
+            const bool live = act && m_run != -INFINITY;
+            uint32_t pw[16];
+            const bool exact = e < n_exact;
+            const float ls = h == 0 ? (exact ? softmax_half<0, true>(sv, c, m_run, live, pw)
+                                             : softmax_half<0, false>(sv, c, m_run, live, pw))
+                                    : (exact ? softmax_half<32, true>(sv, c, m_run, live, pw)
+                                             : softmax_half<32, false>(sv, c, m_run, live, pw));
+            tmem_st16(tl + COL_P + 32 * b + 16 * h, pw);
+            tmem_st_wait();
             l_run += ls;
-            fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_full[b]);
@@ -475,19 +601,27 @@ __global__ void __launch_bounds__(256, 1)
         if (!ok) fail();
 
         // ------------------------------------------------ epilogue
-        const bool fin = ok && wwait(final_bar, 0);
+        // row sum = both halves' sums (exchanged once through shared memory)
+        xl[h * 128 + r] = l_run;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&xl_bar[q4]);
+        const bool xok = wwait(&xl_bar[q4], 0);
+        const float l_tot = xok ? l_run + xl[(h ^ 1) * 128 + r] : 0.f;
+        if (ok && !xok) fail();
+        const bool fin = ok && xok && wwait(final_bar, 0);
         tc_fence_after();
-        const long long grow = static_cast<long long>(bh) * a.N + static_cast<long long>(tile) * 128 + r;
-        const bool row_ok = tile * 128 + r < a.N;
-        const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+        const long long grow = static_cast<long long>(bh) * a.N + row0 + r;
+        const bool row_ok = g < n_groups && row0 + r < a.N;
+        const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
         const bool have_o = n_total > 0;
+        constexpr int HC = D / 2;                        // output columns of this half
         if (PISA) {
             if (fin) {
 #pragma unroll 1
-                for (int c = 0; c < D; c += 32) {
+                for (int cc = h * HC; cc < (h + 1) * HC; cc += 32) {
                     uint32_t ov[32];
                     if (have_o) {
-                        tmem_ld32(tl + COL_O + c, ov);
+                        tmem_ld32(tl + COL_O + cc, ov);
                         tmem_ld_wait();
                     } else {
 #pragma unroll
@@ -497,13 +631,13 @@ __global__ void __launch_bounds__(256, 1)
                         float res[32];
 #pragma unroll
                         for (int x = 0; x < 32; ++x) res[x] = __uint_as_float(ov[x]) * inv_l;
-                        store_row32(a.out, a.out_f32, grow * D + c, res);
+                        store_row32(a.out, a.out_f32, grow * D + cc, res);
                     }
                 }
             }
         } else {
-            // (1) B_g = H - G_g (row c = r of the d x d matrices), bf16 hi + lo,
-            //     MN-major 128-byte-swizzled boxes of 64 columns
+            // (1) B_g = H - G_g (row r of the d x d matrices, this half's columns),
+            //     bf16 hi + lo, MN-major 128-byte-swizzled boxes of 64 columns
             if (fin && r < D) {
                 // H is stored transposed per head, H^T[e][c]: lane r reads column r, coalesced
                 const float* hcol = a.hsum + static_cast<long long>(bh) * D * D + r;
@@ -512,10 +646,10 @@ __global__ void __launch_bounds__(256, 1)
                     unsigned char* blo = bhi + L::BBUF;
                     const bool gs = g_any[gg] != 0;
 #pragma unroll 1
-                    for (int c = 0; c < D; c += 32) {
+                    for (int cc = h * HC; cc < (h + 1) * HC; cc += 32) {
                         uint32_t gv[32];
                         if (gs) {
-                            tmem_ld32(tl + COL_G0 + gg * D + c, gv);
+                            tmem_ld32(tl + COL_G0 + gg * D + cc, gv);
                             tmem_ld_wait();
                         }
 #pragma unroll
@@ -523,65 +657,60 @@ __global__ void __launch_bounds__(256, 1)
                             uint32_t hi4[4], lo4[4];
 #pragma unroll
                             for (int y = 0; y < 4; ++y) {
-                                const int cc = c + 8 * x + 2 * y;
-                                const float v0 = hcol[cc * D] - (gs ? __uint_as_float(gv[8 * x + 2 * y]) : 0.f);
-                                const float v1 = hcol[(cc + 1) * D] - (gs ? __uint_as_float(gv[8 * x + 2 * y + 1]) : 0.f);
+                                const int c2 = cc + 8 * x + 2 * y;
+                                const float v0 = hcol[c2 * D] - (gs ? __uint_as_float(gv[8 * x + 2 * y]) : 0.f);
+                                const float v1 = hcol[(c2 + 1) * D] - (gs ? __uint_as_float(gv[8 * x + 2 * y + 1]) : 0.f);
                                 hi4[y] = pack_bf16(v0, v1);
                                 lo4[y] = pack_bf16(v0 - bf16lo(hi4[y]), v1 - bf16hi(hi4[y]));
                             }
-                            const int cc = c + 8 * x;
-                            const uint32_t off = (cc >> 6) * L::BBOX + sw128(r, (cc & 63) >> 3);
+                            const int c8 = cc + 8 * x;
+                            const uint32_t off = (c8 >> 6) * L::BBOX + sw128(r, (c8 & 63) >> 3);
                             *reinterpret_cast<uint4*>(bhi + off) = make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]);
                             *reinterpret_cast<uint4*>(blo + off) = make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]);
                         }
                     }
                 }
             }
-            // (2) phi(Q) in place (row r of each 64-column box)
-            {
+            // (2) phi(Q) in place in TMEM (the A operand of the linear-branch MMA):
+            //     both halves read the whole row for the denominator, each writes back its half
+            uint32_t phq[D / 2];
+            if (fin) {
 #pragma unroll
                 for (int bx = 0; bx < NBOX; ++bx) {
-#pragma unroll
-                    for (int ch = 0; ch < 8; ++ch) {
-                        uint4* p = reinterpret_cast<uint4*>(smem + L::OFF_Q + bx * L::QBOX + sw128(r, ch));
-                        uint4 v = *p;
-                        v.x = relu_bf16x2_u(v.x); v.y = relu_bf16x2_u(v.y);
-                        v.z = relu_bf16x2_u(v.z); v.w = relu_bf16x2_u(v.w);
-                        *p = v;
-                    }
+                    tmem_ld32(tl + COL_Q + 32 * bx, *reinterpret_cast<uint32_t(*)[32]>(&phq[32 * bx]));
                 }
+                tmem_ld_wait();
+#pragma unroll
+                for (int x = 0; x < D / 2; ++x) phq[x] = relu_bf16x2_u(phq[x]);
+                if (D == 128) {
+                    if (h == 0) tmem_st32(tl + COL_Q, *reinterpret_cast<uint32_t(*)[32]>(&phq[0]));
+                    else tmem_st32(tl + COL_Q + 32, *reinterpret_cast<uint32_t(*)[32]>(&phq[D == 128 ? 32 : 0]));
+                } else {
+                    if (h == 0) tmem_st16(tl + COL_Q, *reinterpret_cast<uint32_t(*)[16]>(&phq[0]));
+                    else tmem_st16(tl + COL_Q + 16, *reinterpret_cast<uint32_t(*)[16]>(&phq[16]));
+                }
+                tmem_st_wait();
             }
-            fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(epi_ready);
-            const bool lin = fin && wwait(epi_ready, 0) &&
-                             wwait(lin_done, 0);
+            const bool lin = fin && wwait(epi_ready, 0) && wwait(lin_done, 0);
             if (fin && !lin) fail();
             tc_fence_after();
             if (lin) {
                 // denominator phi(q) . Zu_g
                 float den = 0.f;
+                const float* z = zu + (g < 2 ? g : 0) * D;
 #pragma unroll
-                for (int bx = 0; bx < NBOX; ++bx)
-#pragma unroll
-                    for (int ch = 0; ch < 8; ++ch) {
-                        const uint4 v = *reinterpret_cast<const uint4*>(smem + L::OFF_Q + bx * L::QBOX + sw128(r, ch));
-                        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-                        const float* z = zu + g * D + bx * 64 + ch * 8;
-#pragma unroll
-                        for (int y = 0; y < 4; ++y) den += bf16lo(w[y]) * z[2 * y] + bf16hi(w[y]) * z[2 * y + 1];
-                    }
+                for (int x = 0; x < D / 2; ++x) den += bf16lo(phq[x]) * z[2 * x] + bf16hi(phq[x]) * z[2 * x + 1];
                 const float inv_den = den > 0.f ? 1.f / den : 0.f;
                 const float al = row_ok ? a.alpha[grow] : 0.f;
                 const uint32_t col_lin = COL_G0 + (g < n_groups ? g : 0) * D;
 #pragma unroll 1
-                for (int c = 0; c < D; c += 32) {
+                for (int cc = h * HC; cc < (h + 1) * HC; cc += 32) {
                     uint32_t ov[32], lv[32];
-                    tmem_ld32(tl + col_lin + c, lv);
-                    if (have_o) {
-                        tmem_ld32(tl + COL_O + c, ov);
-                    }
+                    tmem_ld32(tl + col_lin + cc, lv);
+                    if (have_o) tmem_ld32(tl + COL_O + cc, ov);
                     tmem_ld_wait();
                     if (!have_o) {
 #pragma unroll
@@ -593,7 +722,7 @@ __global__ void __launch_bounds__(256, 1)
                         for (int x = 0; x < 32; ++x)
                             res[x] = al * (__uint_as_float(ov[x]) * inv_l) +
                                      (1.f - al) * (__uint_as_float(lv[x]) * inv_den);
-                        store_row32(a.out, a.out_f32, grow * D + c, res);
+                        store_row32(a.out, a.out_f32, grow * D + cc, res);
                     }
                 }
             }

@@ -7,9 +7,10 @@
 //   * PISA precompute ("Pre-calcolo" of the PISA page): the block centroid
 //     kbar_j (bf16) and the value mean vbar_j = (sum_n v_n)/Bk (fp16), both
 //     [bh][j][c], the operands of the zero-order pseudo-tiles;
-//   * an fp16 copy of V, the B operand of the attention kernel's P.V product
-//     (the conversion from bf16 is exact inside the fp16 range; values outside
-//     it are flagged).
+//   * an fp16 copy of V, the B operand of the attention kernel's P.V product,
+//     and (SLA) phi(K) = max(K, 0) in fp16, the A operand of its phi(K)^T V
+//     product (the conversion from bf16 is exact inside the fp16 range; values
+//     outside it are flagged).
 // phi(K)^T V uses warp-level bf16 tensor-core MMA (m16n8k16) with fp32
 // accumulation; K and V tiles of 64 tokens stream through a 3-stage cp.async
 // ring with an XOR swizzle so ldmatrix reads are conflict-free.
@@ -69,6 +70,7 @@ struct KvStatsArgs {
     __nv_bfloat16* kc;          // [BH][Nk][D] centroids (null: skip)
     __half* vbar;               // [BH][Nk][D] value means (null: skip)
     __half* v16;                // [BH][N][D] fp16 copy of V (null: skip)
+    __half* phik16;             // [BH][N][D] fp16 phi(K) (null: skip)
 };
 
 // grid (nchunk, BH), 256 threads.
@@ -179,6 +181,22 @@ __global__ void __launch_bounds__(256, 2) kv_stats_kernel(KvStatsArgs a) {
                 *reinterpret_cast<uint4*>(vo + (row0 + n) * D + u * 8) = make_uint4(h[0], h[1], h[2], h[3]);
             }
             if (bad) report(kStatusRange);
+        }
+        // fp16 phi(K) = max(K, 0)
+        if (a.phik16) {
+            constexpr int CPR = D / 8;
+            const long long row0 = static_cast<long long>(jb0 + blk) * kKvTok;
+            __half* ko = a.phik16 + bh * static_cast<long long>(a.N) * D;
+            for (int q = tid; q < kKvTok * CPR; q += 256) {
+                const int n = q / CPR, u = q % CPR;
+                const uint4 x = *reinterpret_cast<const uint4*>(kt + kv_off<D>(n, u * 8));
+                const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+                uint32_t h[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    h[e] = pack_half2(fmaxf(bf16lo(w[e]), 0.f), fmaxf(bf16hi(w[e]), 0.f));
+                *reinterpret_cast<uint4*>(ko + (row0 + n) * D + u * 8) = make_uint4(h[0], h[1], h[2], h[3]);
+            }
         }
 
         if (do_mma) {

@@ -55,7 +55,7 @@ sla_status_t check_tensor(const void* t, size_t align) {
 
 // ------------------------------------------------------------- workspace
 struct Ws {
-    size_t qbar, kbarT, m, lut, zj, hpart, hsum, zsum, kc, vbar, v16, total;
+    size_t qbar, kbarT, m, lut, zj, hpart, hsum, zsum, kc, vbar, v16, phik16, total;
     int nchunk, bpc;
 };
 
@@ -80,6 +80,7 @@ Ws layout(const sla_params_t* p) {
     w.kc = take(BH * Nk * d * 2);
     w.vbar = take(BH * Nk * d * 2);
     w.v16 = take(BH * static_cast<size_t>(p->N) * d * 2);
+    w.phik16 = take(BH * static_cast<size_t>(p->N) * d * 2);
     w.total = off;
     return w;
 }
@@ -267,6 +268,7 @@ sla_status_t launch_kv(const sla_params_t* p, const void* k, const void* v, void
     a.kc = pisa_stats ? at<__nv_bfloat16>(ws, w.kc) : nullptr;
     a.vbar = pisa_stats ? at<__half>(ws, w.vbar) : nullptr;
     a.v16 = at<__half>(ws, w.v16);
+    a.phik16 = sla_stats ? at<__half>(ws, w.phik16) : nullptr;
     const size_t smem = sla::kKvStages * 2 * 64 * D * 2 + 256 * 8 + 2 * 256 * 4;
     auto kern = sla::kv_stats_kernel<D>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -290,14 +292,20 @@ template <int D, bool PISA>
 sla_status_t launch_attn(const sla_params_t* p, const void* q, const void* k, const void* v,
                          const float* alpha, const int32_t* lut, void* out, void* ws, const Ws& w,
                          cudaStream_t st) {
-    using L = sla::AttnLayout<D>;
+    using L = sla::AttnLayout<D, PISA>;
     const int BH = p->B * p->H, Nq = p->N / p->Bq, Nk = p->N / p->Bk;
-    CUtensorMap mq, mk, mv, mkc, mvc;
+    CUtensorMap mq, mk, mv, mphi, mkc, mvc;
     const long long rows = static_cast<long long>(BH) * p->N;
     (void)v;   // the P.V product reads the fp16 copy of V made by the K/V pre-pass
     if (!make_map(&mq, q, rows, D, 128) || !make_map(&mk, k, rows, D, 64) ||
         !make_map(&mv, at<void>(ws, w.v16), rows, D, 64, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
         return SLA_ERR_CUDA;
+    if (!PISA) {
+        if (!make_map(&mphi, at<void>(ws, w.phik16), rows, D, 64, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+            return SLA_ERR_CUDA;
+    } else {
+        mphi = mv;
+    }
     if (PISA) {
         if (!make_map(&mkc, at<void>(ws, w.kc), static_cast<long long>(BH) * Nk, D, 64) ||
             !make_map(&mvc, at<void>(ws, w.vbar), static_cast<long long>(BH) * Nk, D, 64,
@@ -312,8 +320,11 @@ sla_status_t launch_attn(const sla_params_t* p, const void* q, const void* k, co
     a.Nq = Nq;
     a.Nk = Nk;
     a.Bq = p->Bq;
+    // query blocks per CTA: 128 rows, except SLA with d = 128 (one block, so the
+    // per-group G accumulator and Q, P fit in the 512 TMEM columns)
+    a.GR = (!PISA && D == 128) ? 1 : 128 / p->Bq;
     a.topk = p->topk;
-    a.tiles_per_head = (p->N + 127) / 128;
+    a.tiles_per_head = (Nq + a.GR - 1) / a.GR;
     const float tau = p->sm_scale > 0.f ? p->sm_scale : 1.0f / std::sqrt(static_cast<float>(D));
     a.scale_log2 = tau * 1.4426950408889634f;
     a.log2_bk = std::log2(static_cast<float>(p->Bk));
@@ -325,16 +336,18 @@ sla_status_t launch_attn(const sla_params_t* p, const void* q, const void* k, co
     a.out = out;
     a.out_f32 = p->out_dtype == SLA_OUT_FP32 ? 1 : 0;
     a.wait_ns = wait_limit_ns();
-    const int GR = 128 / p->Bq;
+    const int GR = a.GR;
     const int nwords = (Nk + 15) / 16;
     const size_t sched_cap = static_cast<size_t>(std::min(Nk, GR * std::max(p->topk, 1)));
-    const size_t smem = 1024 + L::OFF_MISC + 256 + 2 * D * 4 + ((nwords + 3) & ~3) * 4 + sched_cap * 4;
+    const size_t smem = 1024 + L::OFF_MISC + 384 + 2 * D * 4 + 256 * 4 + ((nwords + 3) & ~3) * 4 +
+                        sched_cap * 4;
+    if (smem > 232448) return SLA_ERR_UNSUPPORTED;   // LUT row too long for the shared-memory schedule
     auto kern = sla::attn_kernel<D, PISA>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
         return SLA_ERR_CUDA;
     Span sp(SLA_KERNEL_ATTN, st);
-    kern<<<BH * a.tiles_per_head, 256, smem, st>>>(mq, mk, mv, mkc, mvc, a);
+    kern<<<BH * a.tiles_per_head, sla::kAttnThreads, smem, st>>>(mq, mk, mv, mphi, mkc, mvc, a);
     return launch_status();
 }
 
