@@ -55,6 +55,7 @@ struct AttnArgs {
     const float* zj;               // [BH][Nk][D]    (SLA)
     void* out;                     // [BH][N][D] bf16 or fp32
     int out_f32;
+    int lut_sorted;                // LUT rows strictly ascending and in range (router output)
     unsigned long long wait_ns;
 };
 
@@ -101,18 +102,25 @@ __device__ __forceinline__ float softmax_half(const uint32_t (&sv)[64], float c,
     return ls;
 }
 
-// 32 consecutive output values of one row: bf16 (four 16-byte stores) or fp32.
-__device__ __forceinline__ void store_row32(void* out, int f32, long long off, const float (&v)[32]) {
+// Stage 32 consecutive output values of row r (columns cc .. cc+31) in shared
+// memory for the tensor store: boxes of 128-byte rows (64 bf16 or 32 fp32
+// columns), 128 rows each, 128-byte swizzle.
+__device__ __forceinline__ void stage_row32(unsigned char* stage, int f32, int r, int cc,
+                                            const float (&v)[32]) {
     if (f32) {
-        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + off);
+        unsigned char* box = stage + (cc >> 5) * 16384;
 #pragma unroll
-        for (int x = 0; x < 8; ++x) dst[x] = make_float4(v[4 * x], v[4 * x + 1], v[4 * x + 2], v[4 * x + 3]);
+        for (int x = 0; x < 8; ++x)
+            *reinterpret_cast<float4*>(box + sw128(r, x)) =
+                make_float4(v[4 * x], v[4 * x + 1], v[4 * x + 2], v[4 * x + 3]);
     } else {
-        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + off);
+        unsigned char* box = stage + (cc >> 6) * 16384;
+        const int c0 = (cc & 63) >> 3;
 #pragma unroll
         for (int x = 0; x < 4; ++x)
-            dst[x] = make_uint4(pack_bf16(v[8 * x], v[8 * x + 1]), pack_bf16(v[8 * x + 2], v[8 * x + 3]),
-                                pack_bf16(v[8 * x + 4], v[8 * x + 5]), pack_bf16(v[8 * x + 6], v[8 * x + 7]));
+            *reinterpret_cast<uint4*>(box + sw128(r, c0 + x)) =
+                make_uint4(pack_bf16(v[8 * x], v[8 * x + 1]), pack_bf16(v[8 * x + 2], v[8 * x + 3]),
+                           pack_bf16(v[8 * x + 4], v[8 * x + 5]), pack_bf16(v[8 * x + 6], v[8 * x + 7]));
     }
 }
 
@@ -135,6 +143,9 @@ struct AttnLayout {
     static_assert(QB == 2 * KT, "Q tile spans two K slots");
     static constexpr int BBUF = D * D * 2;           // one (H - G) hi or lo buffer
     static constexpr int BBOX = D * 128;             // one 64-column box of it
+    // output staging for the tensor store, after the (H - G) buffers in the V ring
+    static constexpr int OUT_OFF = OFF_V + (PISA ? 0 : (D == 128 ? 2 : 4) * BBUF);
+    static_assert(OUT_OFF + D * 4 * 128 <= OFF_MISC, "output staging fits in the V ring");
 };
 
 constexpr int kAttnThreads = 384;
@@ -144,7 +155,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmPhi,
                 const __grid_constant__ CUtensorMap tmKc, const __grid_constant__ CUtensorMap tmVc,
-                const AttnArgs a) {
+                const __grid_constant__ CUtensorMap tmOut, const AttnArgs a) {
     using L = AttnLayout<D, PISA>;
     constexpr bool SLA = !PISA;
     constexpr int NBOX = D / 64;
@@ -179,7 +190,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     uint64_t* lin_done = epi_ready + 1;
     uint64_t* drain_bar = lin_done + 1;
     uint64_t* drain2_bar = drain_bar + 1;
-    uint64_t* xl_bar = drain2_bar + 1;            // [4] final row-sum exchange per quarter
+    uint64_t* g_init = drain2_bar + 1;            // G accumulators preloaded with H
+    uint64_t* xl_bar = g_init + 1;                // [4] final row-sum exchange per quarter
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xl_bar + 4);
     int* n_exact_s = reinterpret_cast<int*>(tmem_slot + 1);
     volatile int* abort_flag = n_exact_s + 1;
@@ -221,6 +233,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         mbar_init(lin_done, 1);
         mbar_init(drain_bar, 1);
         mbar_init(drain2_bar, 1);
+        mbar_init(g_init, 8);
         for (int x = 0; x < 4; ++x) mbar_init(&xl_bar[x], 2);
         *abort_flag = 0;
         fence_barrier_init();
@@ -229,6 +242,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tmem_alloc(tmem_slot, NCOLS);
         tmem_relinquish();
     }
+    // Schedule.  Router-made LUT rows are ascending, distinct and in range: with one
+    // group per CTA the row is the schedule.  Otherwise the groups' rows are merged
+    // (and checked) through a per-block bit mask.
+    const bool fast = a.lut_sorted && GR == 1;
+    if (fast) {
+        if (warp == 0) {
+            const int cnt = a.topk;
+            const int rot = cnt > 0 ? static_cast<int>((static_cast<unsigned>(tile) * 2654435761u >> 7) % cnt) : 0;
+            const int32_t* row = a.lut + (static_cast<long long>(bh) * a.Nq + qb0) * a.topk;
+            for (int x = lane; x < cnt; x += 32) {
+                int at = x - rot;
+                if (at < 0) at += cnt;
+                sched[at] = row[x] | (1 << 16);
+            }
+            if (lane == 0) {
+                *n_exact_s = cnt;
+                g_any[0] = cnt > 0;
+                g_any[1] = 0;
+            }
+        }
+    } else {
     for (int w = tid; w < nwords; w += kAttnThreads) mark[w] = 0u;
     __syncthreads();
     for (int x = tid; x < n_groups * a.topk; x += kAttnThreads) {
@@ -273,6 +307,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             g_any[0] = any & 1u;
             g_any[1] = (any >> 1) & 1u;
         }
+    }
     }
     tc_fence_before();
     __syncthreads();
@@ -396,9 +431,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // ======================================================== P.V / G / linear issuer
         if (lane == 0) {
             constexpr uint32_t ID_PV = idesc_f16(128, D, 0, 1);
-            constexpr uint32_t ID_G = idesc_f16(128, D, 1, 1);
+            // G_g starts as H (preloaded by the softmax warps) and accumulates
+            // -phi(K_j)^T V_j, so it ends as H - sum_{j in S_g} h_j
+            constexpr uint32_t ID_G = idesc_f16(128, D, 1, 1, 1);
             bool ok = true;
-            int g_started[2] = {0, 0};                // accumulate flag of G_g
+            bool g_ready = !SLA;
             for (int e = 0; ok && e < n_total; ++e) {
                 const int s = e % VS, b = e & 1, u = e >> 1;
                 if (!mbar_wait(&v_full[s], (e / VS) & 1, abort_flag, lim) ||
@@ -412,6 +449,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 }
                 umma_commit(&p_empty[b]);
                 if (SLA) {
+                    if (!g_ready) {
+                        if (!mbar_wait(g_init, 0, abort_flag, lim)) { ok = false; break; }
+                        tc_fence_after();
+                        g_ready = true;
+                    }
                     const int bits = (sched[e] >> 16) & 3;
                     for (int g = 0; g < 2; ++g) {
                         if (!((bits >> g) & 1)) continue;
@@ -420,10 +462,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         for (int kk = 0; kk < 4; ++kk) {
                             const uint64_t ad = sdesc(sPhi(s) + kk * 2048, lbo, 1024, kSwizzle128B);
                             const uint64_t bd = sdesc(sV(s) + kk * 2048, L::KBOX, 1024, kSwizzle128B);
-                            umma_f16_ss(tmem + COL_G0 + g * D, ad, bd, ID_G,
-                                        (g_started[g] || kk > 0) ? 1u : 0u);
+                            umma_f16_ss(tmem + COL_G0 + g * D, ad, bd, ID_G, 1u);
                         }
-                        g_started[g] = 1;
                     }
                 }
                 umma_commit(&v_empty[s]);
@@ -520,6 +560,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(q_tmem);
+        if (SLA) {
+            // G_g := H (row r = c of the d x d matrix, this half's columns); H is
+            // stored transposed per head, H^T[e][c], so lane r's loads are coalesced
+            if (ok && r < D) {
+                const float* hcol = a.hsum + static_cast<long long>(bh) * D * D + r;
+#pragma unroll 1
+                for (int cc = h * (D / 2); cc < (h + 1) * (D / 2); cc += 32) {
+                    uint32_t hv[32];
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) hv[x] = __float_as_uint(__ldg(hcol + static_cast<long long>(cc + x) * D));
+                    for (int gg = 0; gg < n_groups; ++gg) tmem_st32(tl + COL_G0 + gg * D + cc, hv);
+                }
+                tmem_st_wait();
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(g_init);
+        }
         uint32_t sv[64];
         for (int e = 0; e < n_total; ++e) {
             const int b = e & 1, u = e >> 1;
@@ -627,39 +685,32 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
                         for (int x = 0; x < 32; ++x) ov[x] = 0u;
                     }
-                    if (row_ok) {
-                        float res[32];
+                    float res[32];
 #pragma unroll
-                        for (int x = 0; x < 32; ++x) res[x] = __uint_as_float(ov[x]) * inv_l;
-                        store_row32(a.out, a.out_f32, grow * D + cc, res);
-                    }
+                    for (int x = 0; x < 32; ++x) res[x] = __uint_as_float(ov[x]) * inv_l;
+                    stage_row32(smem + L::OUT_OFF, a.out_f32, r, cc, res);
                 }
             }
         } else {
             // (1) B_g = H - G_g (row r of the d x d matrices, this half's columns),
             //     bf16 hi + lo, MN-major 128-byte-swizzled boxes of 64 columns
             if (fin && r < D) {
-                // H is stored transposed per head, H^T[e][c]: lane r reads column r, coalesced
-                const float* hcol = a.hsum + static_cast<long long>(bh) * D * D + r;
+                // the G_g columns hold H - G_g (row r of the d x d matrix)
                 for (int gg = 0; gg < n_groups; ++gg) {
                     unsigned char* bhi = smem + L::OFF_STAGE + (2 * gg) * L::BBUF;
                     unsigned char* blo = bhi + L::BBUF;
-                    const bool gs = g_any[gg] != 0;
 #pragma unroll 1
                     for (int cc = h * HC; cc < (h + 1) * HC; cc += 32) {
                         uint32_t gv[32];
-                        if (gs) {
-                            tmem_ld32(tl + COL_G0 + gg * D + cc, gv);
-                            tmem_ld_wait();
-                        }
+                        tmem_ld32(tl + COL_G0 + gg * D + cc, gv);
+                        tmem_ld_wait();
 #pragma unroll
                         for (int x = 0; x < 4; ++x) {
                             uint32_t hi4[4], lo4[4];
 #pragma unroll
                             for (int y = 0; y < 4; ++y) {
-                                const int c2 = cc + 8 * x + 2 * y;
-                                const float v0 = hcol[c2 * D] - (gs ? __uint_as_float(gv[8 * x + 2 * y]) : 0.f);
-                                const float v1 = hcol[(c2 + 1) * D] - (gs ? __uint_as_float(gv[8 * x + 2 * y + 1]) : 0.f);
+                                const float v0 = __uint_as_float(gv[8 * x + 2 * y]);
+                                const float v1 = __uint_as_float(gv[8 * x + 2 * y + 1]);
                                 hi4[y] = pack_bf16(v0, v1);
                                 lo4[y] = pack_bf16(v0 - bf16lo(hi4[y]), v1 - bf16hi(hi4[y]));
                             }
@@ -716,16 +767,34 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
                         for (int x = 0; x < 32; ++x) ov[x] = 0u;
                     }
-                    if (row_ok) {
-                        float res[32];
+                    float res[32];
 #pragma unroll
-                        for (int x = 0; x < 32; ++x)
-                            res[x] = al * (__uint_as_float(ov[x]) * inv_l) +
-                                     (1.f - al) * (__uint_as_float(lv[x]) * inv_den);
-                        store_row32(a.out, a.out_f32, grow * D + cc, res);
-                    }
+                    for (int x = 0; x < 32; ++x)
+                        res[x] = al * (__uint_as_float(ov[x]) * inv_l) +
+                                 (1.f - al) * (__uint_as_float(lv[x]) * inv_den);
+                    stage_row32(smem + L::OUT_OFF, a.out_f32, r, cc, res);
                 }
             }
+        }
+    }
+
+    // ------------------------------------------------------------ output store
+    if (warp >= 4) {
+        // all 8 softmax warps have staged their rows; one thread stores the valid
+        // 64-row groups of the tile with the tensor engine
+        fence_proxy_async_smem();
+        named_bar(1, 256);
+        if (warp == 4 && lane == 0 && !*abort_flag) {
+            const int nb = a.out_f32 ? D / 32 : D / 64;
+            const int bc = a.out_f32 ? 32 : 64;
+            for (int k = 0; k < 2; ++k) {
+                if (64 * k >= n_groups * a.Bq || row0 + 64 * k + 64 > a.N) continue;
+                for (int b = 0; b < nb; ++b)
+                    tma_store_2d(&tmOut, smem + L::OUT_OFF + b * 16384 + k * 64 * 128, b * bc,
+                                 bh * a.N + row0 + 64 * k);
+            }
+            tma_store_commit();
+            tma_store_wait_read();
         }
     }
 

@@ -114,15 +114,16 @@ EncodeFn encode_fn() {
     return fn;
 }
 
-// 2-D map of 16-bit elements over [rows, d] (d innermost), box [64 columns,
-// box_rows], 128-byte swizzle.
+// 2-D map over [rows, d] (d innermost), box [128 bytes of columns, box_rows],
+// 128-byte swizzle.
 bool make_map(CUtensorMap* m, const void* base, long long rows, int d, int box_rows,
               CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
     EncodeFn fn = encode_fn();
     if (!fn) return false;
+    const int es = dt == CU_TENSOR_MAP_DATA_TYPE_FLOAT32 ? 4 : 2;
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
-    cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
-    cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * es};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / es), static_cast<cuuint32_t>(box_rows)};
     cuuint32_t estr[2] = {1, 1};
     return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box,
               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -294,9 +295,13 @@ sla_status_t launch_attn(const sla_params_t* p, const void* q, const void* k, co
                          cudaStream_t st) {
     using L = sla::AttnLayout<D, PISA>;
     const int BH = p->B * p->H, Nq = p->N / p->Bq, Nk = p->N / p->Bk;
-    CUtensorMap mq, mk, mv, mphi, mkc, mvc;
+    CUtensorMap mq, mk, mv, mphi, mkc, mvc, mout;
     const long long rows = static_cast<long long>(BH) * p->N;
     (void)v;   // the P.V product reads the fp16 copy of V made by the K/V pre-pass
+    if (!make_map(&mout, out, rows, D, 64,
+                  p->out_dtype == SLA_OUT_FP32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                               : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16))
+        return SLA_ERR_CUDA;
     if (!make_map(&mq, q, rows, D, 128) || !make_map(&mk, k, rows, D, 64) ||
         !make_map(&mv, at<void>(ws, w.v16), rows, D, 64, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
         return SLA_ERR_CUDA;
@@ -335,6 +340,7 @@ sla_status_t launch_attn(const sla_params_t* p, const void* q, const void* k, co
     a.zj = PISA ? nullptr : at<float>(ws, w.zj);
     a.out = out;
     a.out_f32 = p->out_dtype == SLA_OUT_FP32 ? 1 : 0;
+    a.lut_sorted = p->lut_mode == SLA_LUT_COMPUTE ? 1 : 0;
     a.wait_ns = wait_limit_ns();
     const int GR = a.GR;
     const int nwords = (Nk + 15) / 16;
@@ -347,7 +353,7 @@ sla_status_t launch_attn(const sla_params_t* p, const void* q, const void* k, co
                              static_cast<int>(smem)) != cudaSuccess)
         return SLA_ERR_CUDA;
     Span sp(SLA_KERNEL_ATTN, st);
-    kern<<<BH * a.tiles_per_head, sla::kAttnThreads, smem, st>>>(mq, mk, mv, mphi, mkc, mvc, a);
+    kern<<<BH * a.tiles_per_head, sla::kAttnThreads, smem, st>>>(mq, mk, mv, mphi, mkc, mvc, mout, a);
     return launch_status();
 }
 
