@@ -498,3 +498,70 @@ sla_status_t sla_pisa_forward(const sla_params_t* p, const void* q, const void* 
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------ routing without allocation
+// The scratch of sla_route_noalloc lives in this file-scope device array: the
+// module's device memory, reserved on every GPU that loads the library and held
+// until the process exits.  Host code only has a stand-in for the array's name,
+// so its device address is looked up per device with cudaGetSymbolAddress.
+namespace {
+
+constexpr size_t kRouteScratchBytes = static_cast<size_t>(32) << 20;   // 32 MiB
+static __device__ __align__(256) unsigned char g_route_scratch[kRouteScratchBytes];
+
+struct RouteScratch {
+    std::mutex mu;
+    void* ptr[64] = {};
+};
+
+RouteScratch& route_scratch() {
+    static RouteScratch r;
+    return r;
+}
+
+// Device address of g_route_scratch on the current device (looked up once per device).
+sla_status_t route_scratch_ptr(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SLA_ERR_CUDA;
+    RouteScratch& r = route_scratch();
+    std::lock_guard<std::mutex> g(r.mu);
+    if (!r.ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || !p) return SLA_ERR_CUDA;
+        r.ptr[dev] = p;
+    }
+    *out = r.ptr[dev];
+    return SLA_OK;
+}
+
+// Only the router's three scratch regions: pooled Q, pooled K (transposed), W_q W_k^T.
+Ws route_layout(const sla_params_t* p) {
+    Ws w{};
+    const size_t BH = static_cast<size_t>(p->B) * p->H;
+    const size_t d = p->d, Nq = p->N / p->Bq, Nk = p->N / p->Bk;
+    size_t off = 0;
+    auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes); return o; };
+    w.qbar = take(BH * Nq * d * 8);
+    w.kbarT = take(BH * Nk * d * 8);
+    w.m = take(d * d * 8);
+    w.total = off;
+    return w;
+}
+
+}  // namespace
+
+extern "C" sla_status_t sla_route_noalloc(const sla_params_t* p, const void* q, const void* k,
+                                          const float* w_q, const float* w_k, int32_t* lut,
+                                          sla_stream_t stream) {
+    sla_status_t s = check_params(p);
+    if (s != SLA_OK) return s;
+    if ((s = check_tensor(q, 16)) || (s = check_tensor(k, 16))) return s;
+    if (p->topk > 0 && (s = check_tensor(lut, 4))) return s;
+    if ((w_q && !aligned(w_q, 4)) || (w_k && !aligned(w_k, 4))) return SLA_ERR_INVALID_ARG;
+    const Ws w = route_layout(p);
+    if (w.total > kRouteScratchBytes) return SLA_ERR_WORKSPACE;
+    void* scratch = nullptr;
+    if ((s = route_scratch_ptr(&scratch))) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return finish(run_router(p, q, k, w_q, w_k, lut, scratch, w, true, st), st);
+}

@@ -38,7 +38,7 @@ SLA_OUT_FP32 = 1
 
 EXPORTED = ("sla_workspace_size", "sla_route", "sla_forward", "sla_pisa_forward",
             "sla_status_string", "sla_check_device_status", "sla_version",
-            "sla_profile_enable", "sla_profile_read")
+            "sla_profile_enable", "sla_profile_read", "sla_route_noalloc")
 KERNEL_KINDS = ("pool", "kv_stats", "h_reduce", "fold_w", "score_topk", "attn")
 
 
@@ -74,6 +74,8 @@ def load():
             lib.sla_workspace_size.restype = ctypes.c_size_t
             lib.sla_route.argtypes = [PP, P, P, P, P, P, P, ctypes.c_size_t, P]
             lib.sla_route.restype = ctypes.c_int
+            lib.sla_route_noalloc.argtypes = [PP, P, P, P, P, P, P]
+            lib.sla_route_noalloc.restype = ctypes.c_int
             lib.sla_forward.argtypes = [PP, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
             lib.sla_forward.restype = ctypes.c_int
             lib.sla_pisa_forward.argtypes = [PP, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
@@ -155,6 +157,19 @@ def sla_route(p, q, k, w_q, w_k, lut, ws, stream=None):
     rc = load().sla_route(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(w_q), _ptr(w_k), _ptr(lut),
                           _ptr(ws), ws.numel(), _stream(stream))
     _raise(rc, "sla_route")
+    return lut
+
+
+def sla_route_noalloc(p, q, k, w_q, w_k, lut, stream=None):
+    """sla_route without a workspace: scratch comes from the library's built-in
+    32 MiB device array (see include/sla.h)."""
+    B, H, N, d = p.B, p.H, p.N, p.d
+    _check(q, torch.bfloat16, (B, H, N, d), "q")
+    _check(k, torch.bfloat16, (B, H, N, d), "k")
+    _check(lut, torch.int32, (B, H, N // p.Bq, p.topk), "lut")
+    rc = load().sla_route_noalloc(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(w_q), _ptr(w_k),
+                                  _ptr(lut), _stream(stream))
+    _raise(rc, "sla_route_noalloc")
     return lut
 
 

@@ -97,6 +97,27 @@ sla_status_t sla_route(const sla_params_t *p, const void *q, const void *k,
                        void *workspace, size_t ws_bytes, sla_stream_t stream);
 
 /*
+ * sla_route_noalloc -- the same routing as sla_route, for callers that cannot
+ * allocate device memory: for example a plugin running under a host engine that
+ * owns the whole device-memory budget and gives plugins no allocator, or a
+ * serving loop that must never enter an allocator once it is running.  (The
+ * papers have no counterpart; this is an interface convenience.)
+ * It takes no workspace: its scratch is a 32 MiB array built into the library,
+ * which every GPU that loads the library keeps reserved until the process
+ * exits.  Calls whose scratch (8 * B*H * (N/Bq + N/Bk) * d + 8 * d*d bytes,
+ * each part rounded up to 256) exceeds 32 MiB return SLA_ERR_WORKSPACE.
+ * The first call on a device looks up the array's device address for that
+ * device (cudaGetSymbolAddress, with that device current); make that first
+ * call before any stream capture.  All calls share the one array and nothing
+ * in it needs clearing between calls, but calls that overlap on the GPU (on
+ * different streams, or on one device from several threads) race on it.
+ * It allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+ */
+sla_status_t sla_route_noalloc(const sla_params_t *p, const void *q, const void *k,
+                               const float *w_q, const float *w_k, int32_t *lut,
+                               sla_stream_t stream);
+
+/*
  * sla_forward -- SLA2 hybrid forward ([SLA2] sec. 2.A):
  *   O = alpha (.) O_s + (1 - alpha) (.) O_l
  * O_s: softmax attention of each query over the tokens of its query block's
