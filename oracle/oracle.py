@@ -9,6 +9,8 @@ Functions:
 
 * :func:`route`        -- pooled, projected top-k block routing (SLA2 router)
 * :func:`sla_forward`  -- sparse branch + ReLU linear branch + alpha combine
+  (``fp8=True``: the sparse branch on E4M3-quantised Q, K, P, V)
+* :func:`e4m3`         -- the E4M3 conversion (round to nearest even, saturating)
 * :func:`pisa_forward` -- PISA exact-or-approximate zero-order forward
 
 Inputs may be torch tensors (bf16 / fp32 / int32, on the CPU) or numpy arrays
@@ -52,10 +54,12 @@ def _load():
             D = ctypes.c_double
             lib.oracle_route.argtypes = [I] * 7 + [P] * 6 + [I]
             lib.oracle_route.restype = I
-            lib.oracle_sla_forward.argtypes = [I] * 7 + [D] + [P] * 5 + [L, P, P, P, P, I]
+            lib.oracle_sla_forward.argtypes = [I] * 7 + [D] + [P] * 5 + [L, P, P, P, P, I, I]
             lib.oracle_sla_forward.restype = I
             lib.oracle_pisa_forward.argtypes = [I] * 7 + [D] + [P] * 4 + [L, P, P, I]
             lib.oracle_pisa_forward.restype = I
+            lib.oracle_e4m3_array.argtypes = [P, P, L]
+            lib.oracle_e4m3_array.restype = None
             lib.oracle_max_threads.argtypes = []
             lib.oracle_max_threads.restype = I
             _lib = lib
@@ -114,11 +118,20 @@ def _rows(rows, B, H, N):
     return r, r.size
 
 
+def e4m3(x) -> np.ndarray:
+    """E4M3 conversion of float64 values (round to nearest even, saturating)."""
+    a = np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+    out = np.empty_like(a)
+    _load().oracle_e4m3_array(_ptr(a), _ptr(out), a.size)
+    return out
+
+
 def sla_forward(q, k, v, alpha, lut, Bq, Bk, sm_scale=0.0, rows=None, branches=False,
-                threads=0):
+                threads=0, fp8=False):
     """SLA2 forward on a given LUT.  rows=None: every row, returns [B,H,N,d];
     else flat row indices, returns [len(rows), d].  branches=True also returns
-    the sparse-branch and linear-branch outputs."""
+    the sparse-branch and linear-branch outputs.  fp8=True: the sparse branch
+    on E4M3-quantised Q, K, P, V with per-64-token-block scales (Bk = 64)."""
     qb, kb, vb = _bf16_bits(q), _bf16_bits(k), _bf16_bits(v)
     B, H, N, d = qb.shape
     al = _np(alpha, np.float32)
@@ -131,7 +144,7 @@ def sla_forward(q, k, v, alpha, lut, Bq, Bk, sm_scale=0.0, rows=None, branches=F
     ol_ = np.zeros((n, d), dtype=np.float64) if branches else None
     rc = _load().oracle_sla_forward(B, H, N, d, Bq, Bk, topk, float(sm_scale), _ptr(qb), _ptr(kb),
                                     _ptr(vb), _ptr(al), _ptr(lt), nr, _ptr(r), _ptr(out),
-                                    _ptr(os_), _ptr(ol_), threads)
+                                    _ptr(os_), _ptr(ol_), 1 if fp8 else 0, threads)
     _check(rc, "sla_forward")
     shape = (B, H, N, d) if r is None else (n, d)
     if branches:

@@ -24,7 +24,10 @@
  * Parity status: every function here is pinned by the CPU test-suite
  * (dense-attention and pairwise linear-attention special cases, brute-force
  * routing on tiny inputs, block-constant-key exactness of the zero-order
- * term, and its first-order error decay).
+ * term, and its first-order error decay; the E4M3 codec against an
+ * enumeration of the format and a library conversion; the FP8 sparse
+ * branch against the exact forward on inputs whose every quantisation step
+ * is exact, and against the size of error the format implies elsewhere).
  */
 #include <math.h>
 #include <stdint.h>
@@ -73,6 +76,32 @@ static int check_shape(int B, int H, int N, int d, int Bq, int Bk, int topk)
     if (N % Bq || N % Bk) return 0;
     if (topk < 0 || topk > N / Bk) return 0;
     return 1;
+}
+
+/* ------------------------------------------------------------------ */
+/* 8-bit floating point, E4M3 variant (the OCP 8-bit floating-point
+ * specification): 1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits,
+ * no infinities.  Normal values (1 + m/8) 2^(e-7) for e = 1..15, except
+ * e = 15, m = 7, which is NaN: the largest finite magnitude is 448.
+ * Subnormal values (m/8) 2^-6.  Conversion rounds to nearest, ties to even,
+ * and saturates magnitudes beyond 448 to 448. */
+double oracle_e4m3(double x)
+{
+    if (x != x) return x;
+    const double a = fabs(x);
+    if (a >= 448.0) return copysign(448.0, x);
+    if (a == 0.0) return x;
+    int e2;
+    frexp(a, &e2);                 /* a in [2^(e2-1), 2^e2) */
+    int lead = e2 - 1;
+    if (lead < -6) lead = -6;      /* subnormals share the spacing 2^-9 */
+    const double spacing = ldexp(1.0, lead - 3);
+    return copysign(nearbyint(a / spacing) * spacing, x);
+}
+
+void oracle_e4m3_array(const double *in, double *out, int64_t n)
+{
+    for (int64_t a = 0; a < n; ++a) out[a] = oracle_e4m3(in[a]);
 }
 
 /* A LUT row must hold topk distinct block indices in [0, Nk). */
@@ -261,16 +290,43 @@ static rowreq_t *gather_rows(int64_t total, int64_t nrows, const int64_t *rows, 
  *     O_l := 0 when the denominator is <= 0.
  *   Combine ([SLA2-it] sec. 2.A; [SLA2-ar] sec. 2.a):
  *     O = alpha . O_s + (1 - alpha) . O_l.
+ *   fp8 != 0: the sparse branch runs on quantised Q, K, P and V, as the
+ *   forward pass of the low-bit sparse branch does ([SLA2-it] sec. 2.C;
+ *   [SLA2-ar] sec. 2.j, QAT: the forward quantises Q, K, P and V), with E4M3
+ *   and these scale rules (Bk must be 64):
+ *     per 64-token block b of Q, K and V: s_b = max|x| / 448 (1 for an
+ *     all-zero block), x8 = e4m3(x / s_b);
+ *     logits in log2 units x_tn = (q8_t . k8_n) s_q(t) s_k(j) tau log2(e);
+ *     P_tn = 2^(x_tn - M_t) with M_t = ceil(max_n x_tn), l_t = sum_n P_tn;
+ *     Phat_tn = e4m3(P_tn 448 s_v(j) / s_vmax), s_vmax = max over the LUT row;
+ *     O_s(t) = (s_vmax / 448) sum_n Phat_tn v8_n / l_t.
+ *   The linear branch and the combine are not quantised.
  * rows: flat indices (b*H + h)*N + t (NULL = all rows, in order).
  * out, out_s, out_l: [nrows, d] (out_s, out_l may be NULL). */
+
+/* Per-64-token-block absmax scale and E4M3 codes of one head's [N, d] tensor. */
+static void quantise_blocks(const uint16_t *x, int N, int d, double *x8, double *scale)
+{
+    for (int b = 0; b < N / 64; ++b) {
+        double amax = 0.0;
+        for (size_t e = (size_t)b * 64 * d; e < (size_t)(b + 1) * 64 * d; ++e)
+            if (fabs(bf(x[e])) > amax) amax = fabs(bf(x[e]));
+        const double s = amax > 0.0 ? amax / 448.0 : 1.0;
+        scale[b] = s;
+        for (size_t e = (size_t)b * 64 * d; e < (size_t)(b + 1) * 64 * d; ++e)
+            x8[e] = oracle_e4m3(bf(x[e]) / s);
+    }
+}
+
 int oracle_sla_forward(int B, int H, int N, int d, int Bq, int Bk, int topk, double sm_scale,
                        const uint16_t *q, const uint16_t *k, const uint16_t *v,
                        const float *alpha, const int32_t *lut,
                        int64_t nrows, const int64_t *rows,
-                       double *out, double *out_s, double *out_l, int nthreads)
+                       double *out, double *out_s, double *out_l, int fp8, int nthreads)
 {
     if (!check_shape(B, H, N, d, Bq, Bk, topk) || !q || !k || !v || !alpha || !lut || !out)
         return ORC_EINVAL;
+    if (fp8 && Bk != 64) return ORC_EINVAL;
     set_threads(nthreads);
     const int Nq = N / Bq, Nk = N / Bk;
     const double tau = sm_scale > 0.0 ? sm_scale : 1.0 / sqrt((double)d);
@@ -285,7 +341,18 @@ int oracle_sla_forward(int B, int H, int N, int d, int Bq, int Bk, int topk, dou
 
     double *hj = malloc(sizeof(double) * (size_t)Nk * d * d);
     double *zj = malloc(sizeof(double) * (size_t)Nk * d);
-    if (!hj || !zj) { free(req); free(hj); free(zj); return ORC_ENOMEM; }
+    /* FP8: one head's codes and scales */
+    const size_t nq8 = fp8 ? (size_t)N * d : 1, ns8 = fp8 ? (size_t)N / 64 : 1;
+    double *q8 = malloc(sizeof(double) * nq8), *k8 = malloc(sizeof(double) * nq8);
+    double *v8 = malloc(sizeof(double) * nq8);
+    double *sq = malloc(sizeof(double) * ns8), *sk = malloc(sizeof(double) * ns8);
+    double *sv = malloc(sizeof(double) * ns8);
+    if (!hj || !zj || !q8 || !k8 || !v8 || !sq || !sk || !sv) {
+        free(req); free(hj); free(zj);
+        free(q8); free(k8); free(v8); free(sq); free(sk); free(sv);
+        return ORC_ENOMEM;
+    }
+    const double log2e = 1.0 / log(2.0);
     int err = ORC_OK;
 
     int64_t a0 = 0;
@@ -297,6 +364,11 @@ int oracle_sla_forward(int B, int H, int N, int d, int Bq, int Bk, int topk, dou
         const uint16_t *kh = k + (size_t)bh * N * d;
         const uint16_t *vh = v + (size_t)bh * N * d;
         linear_block_stats(kh, vh, Nk, Bk, d, hj, zj);
+        if (fp8) {
+            quantise_blocks(qh, N, d, q8, sq);
+            quantise_blocks(kh, N, d, k8, sk);
+            quantise_blocks(vh, N, d, v8, sv);
+        }
 
         /* distinct query blocks among the requested rows of this head */
         int64_t nblk = 0;
@@ -334,30 +406,59 @@ int oracle_sla_forward(int B, int H, int N, int d, int Bq, int Bk, int topk, dou
                 double *o = out + req[a].slot * d;
                 for (int c = 0; c < d; ++c) qd[c] = bf(qh[(size_t)t * d + c]);
 
-                /* sparse branch: two passes, max then weights */
-                double m = -INFINITY;
-                for (int s = 0; s < topk; ++s) {
-                    for (int r = 0; r < Bk; ++r) {
-                        size_t nn = (size_t)S[s] * Bk + r;
-                        double acc = 0.0;
-                        for (int c = 0; c < d; ++c) acc += qd[c] * bf(kh[nn * d + c]);
-                        logit[s * Bk + r] = tau * acc;
-                        if (tau * acc > m) m = tau * acc;
-                    }
-                }
                 double den_s = 0.0;
                 double os[512];
                 double ol[512];
                 for (int c = 0; c < d; ++c) { os[c] = 0.0; ol[c] = 0.0; }
-                for (int s = 0; s < topk; ++s) {
-                    for (int r = 0; r < Bk; ++r) {
-                        size_t nn = (size_t)S[s] * Bk + r;
-                        double p = exp(logit[s * Bk + r] - m);
-                        den_s += p;
-                        for (int c = 0; c < d; ++c) os[c] += p * bf(vh[nn * d + c]);
+                if (fp8) {
+                    /* quantised sparse branch: log2-unit logits, power-of-two row reference */
+                    double svmax = 0.0, mx = -INFINITY;
+                    for (int s = 0; s < topk; ++s)
+                        if (sv[S[s]] > svmax) svmax = sv[S[s]];
+                    for (int s = 0; s < topk; ++s) {
+                        for (int r = 0; r < Bk; ++r) {
+                            size_t nn = (size_t)S[s] * Bk + r;
+                            double acc = 0.0;
+                            for (int c = 0; c < d; ++c) acc += q8[(size_t)t * d + c] * k8[nn * d + c];
+                            const double x = acc * sq[t / 64] * sk[S[s]] * tau * log2e;
+                            logit[s * Bk + r] = x;
+                            if (x > mx) mx = x;
+                        }
                     }
+                    const double M = ceil(mx);
+                    for (int s = 0; s < topk; ++s) {
+                        const double qf = 448.0 * sv[S[s]] / svmax;
+                        for (int r = 0; r < Bk; ++r) {
+                            size_t nn = (size_t)S[s] * Bk + r;
+                            const double p = exp2(logit[s * Bk + r] - M);
+                            den_s += p;
+                            const double ph = oracle_e4m3(p * qf);
+                            for (int c = 0; c < d; ++c) os[c] += ph * v8[nn * d + c];
+                        }
+                    }
+                    for (int c = 0; c < d; ++c) os[c] = den_s > 0.0 ? os[c] * (svmax / 448.0) / den_s : 0.0;
+                } else {
+                    /* exact sparse branch: two passes, max then weights */
+                    double m = -INFINITY;
+                    for (int s = 0; s < topk; ++s) {
+                        for (int r = 0; r < Bk; ++r) {
+                            size_t nn = (size_t)S[s] * Bk + r;
+                            double acc = 0.0;
+                            for (int c = 0; c < d; ++c) acc += qd[c] * bf(kh[nn * d + c]);
+                            logit[s * Bk + r] = tau * acc;
+                            if (tau * acc > m) m = tau * acc;
+                        }
+                    }
+                    for (int s = 0; s < topk; ++s) {
+                        for (int r = 0; r < Bk; ++r) {
+                            size_t nn = (size_t)S[s] * Bk + r;
+                            double p = exp(logit[s * Bk + r] - m);
+                            den_s += p;
+                            for (int c = 0; c < d; ++c) os[c] += p * bf(vh[nn * d + c]);
+                        }
+                    }
+                    for (int c = 0; c < d; ++c) os[c] = den_s > 0.0 ? os[c] / den_s : 0.0;
                 }
-                for (int c = 0; c < d; ++c) os[c] = den_s > 0.0 ? os[c] / den_s : 0.0;
 
                 /* linear branch over the unselected blocks */
                 double den_l = 0.0;
@@ -383,6 +484,7 @@ int oracle_sla_forward(int B, int H, int N, int d, int Bq, int Bk, int topk, dou
         a0 = a1;
     }
     free(hj); free(zj); free(req);
+    free(q8); free(k8); free(v8); free(sq); free(sk); free(sv);
     return err;
 }
 

@@ -381,3 +381,136 @@ def test_pisa_zero_order_error_is_first_order():
     assert errs[0] > errs[1] > errs[2] > 0
     for a, b in zip(errs, errs[1:]):
         assert 1.6 < a / b < 2.5, errs
+
+
+# ---------------------------------------------------------------- E4M3 and the FP8 mode
+
+def e4m3_decode(code):
+    """Value of one 8-bit E4M3 code, from the format's definition: sign bit,
+    4 exponent bits (bias 7), 3 mantissa bits; exponent field 0 is subnormal;
+    exponent 15 with mantissa 7 is NaN (no infinities)."""
+    s = -1.0 if code & 0x80 else 1.0
+    e = (code >> 3) & 0xF
+    m = code & 0x7
+    if e == 15 and m == 7:
+        return float("nan")
+    if e == 0:
+        return s * (m / 8.0) * 2.0 ** -6
+    return s * (1.0 + m / 8.0) * 2.0 ** (e - 7)
+
+
+def e4m3_table():
+    """Non-negative finite values in code order, with their mantissa parity."""
+    vals = [e4m3_decode(c) for c in range(0x7F)]
+    return np.array(vals), np.array([c & 1 for c in range(0x7F)])
+
+
+def test_e4m3_codes_are_fixed_points_and_ties_go_to_even():
+    vals, odd = e4m3_table()
+    assert vals[-1] == 448.0 and vals[1] == 2.0 ** -9 and vals[8] == 2.0 ** -6
+    assert np.all(np.diff(vals) > 0)
+    both = np.concatenate([vals, -vals[1:]])
+    assert np.array_equal(orc.e4m3(both), both)
+    mids = (vals[:-1] + vals[1:]) / 2
+    want = np.where(odd[:-1] == 0, vals[:-1], vals[1:])
+    assert np.array_equal(orc.e4m3(mids), want)
+    assert np.array_equal(orc.e4m3(-mids), -want)
+    # just off the midpoints: plain nearest
+    assert np.array_equal(orc.e4m3(mids * (1 - 1e-9)), vals[:-1])
+    assert np.array_equal(orc.e4m3(mids * (1 + 1e-9)), vals[1:])
+
+
+def test_e4m3_saturates_and_underflows():
+    big = np.array([448.0, 449.0, 463.99, 464.0, 480.0, 1e6, np.inf])
+    assert np.array_equal(orc.e4m3(big), np.full(7, 448.0))
+    assert np.array_equal(orc.e4m3(-big), np.full(7, -448.0))
+    assert np.array_equal(orc.e4m3(np.array([2.0 ** -10, 1e-30, 0.0])), np.zeros(3))
+    assert orc.e4m3(np.array([2.0 ** -10 * 1.0001]))[0] == 2.0 ** -9
+    assert np.isnan(orc.e4m3(np.array([np.nan]))[0])
+
+
+def test_e4m3_matches_library_conversion():
+    """torch's float8_e4m3fn cast (round to nearest even) on values within range."""
+    rng = np.random.default_rng(7)
+    mag = 2.0 ** rng.uniform(-11, math.log2(448), 200000)
+    x = mag * rng.choice([-1.0, 1.0], mag.size)
+    lib = torch.from_numpy(x).to(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(orc.e4m3(x), lib)
+
+
+def exact_fp8_inputs(seed):
+    """Inputs on which every FP8 quantisation step is exact: block absmaxes are
+    448 * 2^-r (so each scale is a power of two), every entry divided by its
+    block scale is an E4M3 value, and with sm_scale = ln 2 the logits in log2
+    units are small integers, so each P = 2^(integer) times a power-of-two
+    factor is an E4M3 value too.  Q, K and V use different scales per
+    64-token block (two Q scale blocks inside one 128-token query block)."""
+    rng = np.random.default_rng(seed)
+    B, H, N, d = 1, 2, 512, 128
+    q = np.zeros((B, H, N, d))
+    k = np.zeros((B, H, N, d))
+    v = np.zeros((B, H, N, d))
+    vals, _ = e4m3_table()
+    for b in range(B):
+        for h in range(H):
+            for blk in range(N // 64):
+                rq, rk, rv = rng.integers(7, 9), rng.integers(7, 9), rng.integers(6, 10)
+                for t in range(blk * 64, blk * 64 + 64):
+                    cq = rng.choice(np.arange(2, d), 2, replace=False)
+                    q[b, h, t, cq] = rng.choice([-1.0, 1.0], 2) * (rng.choice([1.0, 2.0], 2) if rq == 7 else 1.0)
+                    ck = rng.choice(np.arange(2, d), 3, replace=False)
+                    k[b, h, t, ck] = rng.choice([-1.0, 1.0], 3)
+                    v[b, h, t] = rng.choice(vals[1:], d) * rng.choice([-1.0, 1.0], d) * 2.0 ** -rv
+                # block absmax: column 0 of Q and column 1 of K never meet a nonzero
+                q[b, h, blk * 64, 0] = 448.0 * 2.0 ** -rq
+                k[b, h, blk * 64, 1] = 448.0 * 2.0 ** -rk
+                v[b, h, blk * 64, 5] = 448.0 * 2.0 ** -rv
+    to = lambda x: torch.from_numpy(x).to(torch.bfloat16)
+    qt, kt, vt = to(q), to(k), to(v)
+    for a, x in ((qt, q), (kt, k), (vt, v)):
+        assert np.array_equal(a.double().numpy(), x), "construction must be exact in bf16"
+    alpha = torch.from_numpy(rng.uniform(0, 1, (B, H, N))).float()
+    return qt, kt, vt, alpha
+
+
+@pytest.mark.parametrize("topk", [1, 3, 8])
+def test_fp8_mode_is_exact_when_every_quantisation_is_exact(topk):
+    q, k, v, alpha = exact_fp8_inputs(11 + topk)
+    Bq, Bk = 128, 64
+    lut, _ = orc.route(q, k, None, None, Bq, Bk, topk)
+    ln2 = math.log(2.0)
+    o8, s8, l8 = orc.sla_forward(q, k, v, alpha, lut, Bq, Bk, sm_scale=ln2, branches=True, fp8=True)
+    o, s, l = orc.sla_forward(q, k, v, alpha, lut, Bq, Bk, sm_scale=ln2, branches=True)
+    scale = np.abs(s).max()
+    assert scale > 0
+    assert np.abs(s8 - s).max() <= 1e-12 * scale
+    assert np.array_equal(l8, l)
+    assert np.abs(o8 - o).max() <= 1e-12 * scale
+    # the case is not degenerate: within a query block's selected keys the
+    # logits (log2 units) span several powers of two
+    qd, kd = q.double().numpy()[0, 0], k.double().numpy()[0, 0]
+    keys = np.concatenate([np.arange(j * Bk, (j + 1) * Bk) for j in lut[0, 0, 1]])
+    spread = np.ptp(qd[Bq:2 * Bq] @ kd[keys].T, axis=1)
+    assert spread.max() >= 3
+
+
+def test_fp8_mode_error_has_the_size_the_format_implies():
+    """On Gaussian inputs the quantised branch differs from the exact one by
+    a few percent (E4M3 keeps 3 mantissa bits): nonzero, and far from gross."""
+    inp = W.gaussian_inputs(1, 2, 1024, 128, 77)
+    lut, _ = orc.route(inp["q"], inp["k"], inp["w_q"], inp["w_k"], 128, 64, 6)
+    _, s8, l8 = orc.sla_forward(inp["q"], inp["k"], inp["v"], inp["alpha"], lut, 128, 64,
+                                branches=True, fp8=True)
+    _, s, l = orc.sla_forward(inp["q"], inp["k"], inp["v"], inp["alpha"], lut, 128, 64, branches=True)
+    assert np.array_equal(l8, l)
+    rel = np.abs(s8 - s).mean() / np.abs(s).mean()
+    assert 0.005 < rel < 0.1, rel
+    cos = (s8 * s).sum() / np.sqrt((s8 * s8).sum() * (s * s).sum())
+    assert cos > 0.99
+
+
+def test_fp8_mode_requires_64_token_blocks():
+    inp = W.gaussian_inputs(1, 1, 256, 64, 5)
+    lut, _ = orc.route(inp["q"], inp["k"], None, None, 64, 32, 2)
+    with pytest.raises(ValueError):
+        orc.sla_forward(inp["q"], inp["k"], inp["v"], inp["alpha"], lut, 64, 32, fp8=True)
