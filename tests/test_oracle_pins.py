@@ -438,13 +438,16 @@ def test_e4m3_matches_library_conversion():
     assert np.array_equal(orc.e4m3(x), lib)
 
 
-def exact_fp8_inputs(seed):
+def exact_fp8_inputs(seed, v_fifths=False):
     """Inputs on which every FP8 quantisation step is exact: block absmaxes are
     448 * 2^-r (so each scale is a power of two), every entry divided by its
     block scale is an E4M3 value, and with sm_scale = ln 2 the logits in log2
     units are small integers, so each P = 2^(integer) times a power-of-two
     factor is an E4M3 value too.  Q, K and V use different scales per
-    64-token block (two Q scale blocks inside one 128-token query block)."""
+    64-token block (two Q scale blocks inside one 128-token query block).
+    v_fifths: V blocks take absmax 448 * f * 2^-r with f in {1, 5/8}; every
+    step except the rounding of P stays exact, and P * 448 s_v,j / s_v,max
+    is then a power of two times 448 f_j / f_max, never an E4M3 tie."""
     rng = np.random.default_rng(seed)
     B, H, N, d = 1, 2, 512, 128
     q = np.zeros((B, H, N, d))
@@ -455,16 +458,17 @@ def exact_fp8_inputs(seed):
         for h in range(H):
             for blk in range(N // 64):
                 rq, rk, rv = rng.integers(7, 9), rng.integers(7, 9), rng.integers(6, 10)
+                fv = rng.choice([1.0, 0.625]) if v_fifths else 1.0
                 for t in range(blk * 64, blk * 64 + 64):
-                    cq = rng.choice(np.arange(2, d), 2, replace=False)
+                    cq = rng.choice(np.arange(2, 10), 2, replace=False)
                     q[b, h, t, cq] = rng.choice([-1.0, 1.0], 2) * (rng.choice([1.0, 2.0], 2) if rq == 7 else 1.0)
-                    ck = rng.choice(np.arange(2, d), 3, replace=False)
+                    ck = rng.choice(np.arange(2, 10), 3, replace=False)
                     k[b, h, t, ck] = rng.choice([-1.0, 1.0], 3)
-                    v[b, h, t] = rng.choice(vals[1:], d) * rng.choice([-1.0, 1.0], d) * 2.0 ** -rv
+                    v[b, h, t] = rng.choice(vals[1:], d) * rng.choice([-1.0, 1.0], d) * fv * 2.0 ** -rv
                 # block absmax: column 0 of Q and column 1 of K never meet a nonzero
                 q[b, h, blk * 64, 0] = 448.0 * 2.0 ** -rq
                 k[b, h, blk * 64, 1] = 448.0 * 2.0 ** -rk
-                v[b, h, blk * 64, 5] = 448.0 * 2.0 ** -rv
+                v[b, h, blk * 64, 5] = 448.0 * fv * 2.0 ** -rv
     to = lambda x: torch.from_numpy(x).to(torch.bfloat16)
     qt, kt, vt = to(q), to(k), to(v)
     for a, x in ((qt, q), (kt, k), (vt, v)):
@@ -492,6 +496,41 @@ def test_fp8_mode_is_exact_when_every_quantisation_is_exact(topk):
     keys = np.concatenate([np.arange(j * Bk, (j + 1) * Bk) for j in lut[0, 0, 1]])
     spread = np.ptp(qd[Bq:2 * Bq] @ kd[keys].T, axis=1)
     assert spread.max() >= 3
+
+
+@pytest.mark.parametrize("topk", [2, 5])
+def test_fp8_p_rounding_matches_library_codec_on_known_weights(topk):
+    """Only the rounding of P is inexact here: every P is a power of two, so
+    block j's quantised weights are its exact weights times
+    gamma_j = e4m3(448 rho_j) / (448 rho_j), rho_j = s_v,j / s_v,max, with the
+    row sum taken over the unquantised P.  The sparse branch must equal fp64
+    softmax attention over the selected blocks with V_j scaled by gamma_j
+    (E4M3 rounding from torch's float8_e4m3fn cast)."""
+    q, k, v, alpha = exact_fp8_inputs(40 + topk, v_fifths=True)
+    Bq, Bk = 128, 64
+    B, H, N, d = q.shape
+    lut, _ = orc.route(q, k, None, None, Bq, Bk, topk)
+    ln2 = math.log(2.0)
+    _, s8, _ = orc.sla_forward(q, k, v, alpha, lut, Bq, Bk, sm_scale=ln2, branches=True, fp8=True)
+    qd, kd, vd = f64(q), f64(k), f64(v)
+    s_v = vd.reshape(B, H, N // 64, 64 * d).abs().amax(-1) / 448.0
+    want = torch.zeros(B, H, N, d, dtype=torch.float64)
+    nontrivial = 0
+    for b in range(B):
+        for h in range(H):
+            for i in range(N // Bq):
+                sel = torch.as_tensor(lut[b, h, i], dtype=torch.long)
+                rho = s_v[b, h, sel] / s_v[b, h, sel].max()
+                gamma = (448.0 * rho).to(torch.float8_e4m3fn).double() / (448.0 * rho)
+                nontrivial += int((gamma != 1).sum())
+                keys = torch.cat([torch.arange(j * Bk, (j + 1) * Bk) for j in sel.tolist()])
+                vj = vd[b, h, keys] * gamma.repeat_interleave(Bk)[:, None]
+                rows = slice(i * Bq, (i + 1) * Bq)
+                w = torch.softmax(ln2 * qd[b, h, rows] @ kd[b, h, keys].T, dim=-1)
+                want[b, h, rows] = w @ vj
+    assert nontrivial > 0
+    want = want.numpy()
+    assert np.abs(s8 - want).max() <= 1e-12 * np.abs(want).max()
 
 
 def test_fp8_mode_error_has_the_size_the_format_implies():
