@@ -295,7 +295,7 @@ static rowreq_t *gather_rows(int64_t total, int64_t nrows, const int64_t *rows, 
  *   [SLA2-ar] sec. 2.j, QAT: the forward quantises Q, K, P and V), with E4M3
  *   and these scale rules (Bk must be 64):
  *     per 64-token block b of Q, K and V: s_b = max|x| / 448 (1 for an
- *     all-zero block), x8 = e4m3(x / s_b);
+ *     all-zero block), x8 = e4m3(x / s_b), s_b and x / s_b in fp32;
  *     logits in log2 units x_tn = (q8_t . k8_n) s_q(t) s_k(j) tau log2(e);
  *     P_tn = 2^(x_tn - M_t) with M_t = ceil(max_n x_tn), l_t = sum_n P_tn;
  *     Phat_tn = e4m3(P_tn 448 s_v(j) / s_vmax), s_vmax = max over the LUT row;
@@ -304,17 +304,23 @@ static rowreq_t *gather_rows(int64_t total, int64_t nrows, const int64_t *rows, 
  * rows: flat indices (b*H + h)*N + t (NULL = all rows, in order).
  * out, out_s, out_l: [nrows, d] (out_s, out_l may be NULL). */
 
-/* Per-64-token-block absmax scale and E4M3 codes of one head's [N, d] tensor. */
+/* Per-64-token-block absmax scale and E4M3 codes of one head's [N, d] tensor.
+ * The scale and the quotient that picks each code are single-precision IEEE
+ * operations (correctly rounded), the precision the GPU path decides its codes
+ * in; the pages fix no precision for them, and deciding a code in another
+ * precision flips it whenever the quotient falls on a rounding midpoint. */
 static void quantise_blocks(const uint16_t *x, int N, int d, double *x8, double *scale)
 {
     for (int b = 0; b < N / 64; ++b) {
-        double amax = 0.0;
+        float amax = 0.0f;
         for (size_t e = (size_t)b * 64 * d; e < (size_t)(b + 1) * 64 * d; ++e)
-            if (fabs(bf(x[e])) > amax) amax = fabs(bf(x[e]));
-        const double s = amax > 0.0 ? amax / 448.0 : 1.0;
-        scale[b] = s;
-        for (size_t e = (size_t)b * 64 * d; e < (size_t)(b + 1) * 64 * d; ++e)
-            x8[e] = oracle_e4m3(bf(x[e]) / s);
+            if (fabsf((float)bf(x[e])) > amax) amax = fabsf((float)bf(x[e]));
+        const float s = amax > 0.0f ? amax / 448.0f : 1.0f;
+        scale[b] = (double)s;
+        for (size_t e = (size_t)b * 64 * d; e < (size_t)(b + 1) * 64 * d; ++e) {
+            const float quotient = (float)bf(x[e]) / s;
+            x8[e] = oracle_e4m3((double)quotient);
+        }
     }
 }
 
