@@ -44,6 +44,21 @@ namespace sla {
 
 constexpr float kRescaleLog2 = 8.0f;    // lazy O rescale threshold (log2 units)
 
+enum : int { kModeSla = 0, kModePisa = 1, kModeSlaFp8 = 2 };
+
+// Tensor maps of one launch (see the host for shapes, boxes and swizzles).
+struct AttnMaps {
+    CUtensorMap q;      // bf16 Q [BH*N, d], box 64 x 128 rows
+    CUtensorMap k;      // K tiles: bf16 K (box 64 x 64) or, FP8, e4m3 K (box 128 B x 64)
+    CUtensorMap v;      // fp16 V copy, box 64 x 64
+    CUtensorMap phi;    // fp16 phi(K), box 64 x 64
+    CUtensorMap kc;     // PISA centroids (bf16 [BH*Nk, d])
+    CUtensorMap vc;     // PISA value means (fp16 [BH*Nk, d])
+    CUtensorMap out;    // output, box 128 B x 64 rows
+    CUtensorMap q8;     // FP8: e4m3 Q, box 128 B x 128 rows
+    CUtensorMap v8t;    // FP8: e4m3 V^T per block [BH*Nk*d, 64], box 64 B x d, 64-byte swizzle
+};
+
 struct AttnArgs {
     int N, Nq, Nk, Bq, GR, topk, tiles_per_head;
     float scale_log2;              // tau * log2(e)
@@ -56,6 +71,10 @@ struct AttnArgs {
     void* out;                     // [BH][N][D] bf16 or fp32
     int out_f32;
     int lut_sorted;                // LUT rows strictly ascending and in range (router output)
+    int sched_cap;                 // capacity of the shared-memory schedule
+    const float* sq;               // FP8: [BH][N/64] Q block scales
+    const float* sk;               // FP8: [BH][Nk]  K block scales
+    const float* sv;               // FP8: [BH][Nk]  V block scales
     unsigned long long wait_ns;
 };
 
@@ -102,6 +121,25 @@ __device__ __forceinline__ float softmax_half(const uint32_t (&sv)[64], float c,
     return ls;
 }
 
+// FP8 P for the 32 logits sv[OFF .. OFF+31] (raw scores, x = s*ce): fp32 exp2,
+// quantised as e4m3(P * qf) four per 32-bit word; returns the fp32 sum of P.
+template <int OFF>
+__device__ __forceinline__ float softmax_half_e4m3(const uint32_t (&sv)[64], float ce, float m, bool live,
+                                                   float qf, uint32_t (&p8)[8]) {
+    float ls = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+        float p[4];
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            p[x] = live ? fast_exp2(fmaf(__uint_as_float(sv[OFF + 4 * w + x]), ce, -m)) : 0.f;
+            ls += p[x];
+        }
+        p8[w] = pack_e4m3x4(p[0] * qf, p[1] * qf, p[2] * qf, p[3] * qf);
+    }
+    return ls;
+}
+
 // Stage 32 consecutive output values of row r (columns cc .. cc+31) in shared
 // memory for the tensor store: boxes of 128-byte rows (64 bf16 or 32 fp32
 // columns), 128 rows each, 128-byte swizzle.
@@ -124,25 +162,33 @@ __device__ __forceinline__ void stage_row32(unsigned char* stage, int f32, int r
     }
 }
 
-template <int D, bool PISA>
+template <int D, int MODE>
 struct AttnLayout {
-    static constexpr int KS = PISA ? 6 : 4;          // K ring slots
-    static constexpr int VS = PISA ? 6 : 4;          // V (+ phi(K)) ring slots
-    static constexpr int PF = 0;                     // L2 prefetch distance (blocks); 0 = off
-    static constexpr int QB = 128 * D * 2;           // Q tile bytes
-    static constexpr int KT = 64 * D * 2;            // one 64-token tile (bf16 or fp16)
-    static constexpr int VT = (PISA ? 1 : 2) * KT;   // V (+ phi(K)) slot
-    static constexpr int KBOX = 64 * 128;            // one 64-row x 128-byte box
-    static constexpr int QBOX = 128 * 128;           // one 128-row x 128-byte box
+    static constexpr bool PISA = MODE == kModePisa, FP8 = MODE == kModeSlaFp8;
+    static constexpr int KS = (PISA || FP8) ? 6 : 4;  // K ring slots
+    static constexpr int VS = PISA ? 6 : 4;           // V ring slots
+    static constexpr int PF = 0;                      // L2 prefetch distance (blocks); 0 = off
+    static constexpr int T16 = 64 * D * 2;            // one 64-token tile of 16-bit values
+    static constexpr int QB = 128 * D * (FP8 ? 3 : 2);   // (e4m3 Q +) bf16 Q
+    static constexpr int KT = 64 * D * (FP8 ? 1 : 2);    // one K tile
+    // V slot: [P.V operand | fp16 phi(K) | fp16 V (FP8: the G operand)]
+    static constexpr int V_PV = 0;
+    static constexpr int V_PHI = FP8 ? 64 * D : T16;
+    static constexpr int V_V16 = FP8 ? 64 * D + T16 : 0;
+    static constexpr int VT = PISA ? T16 : (FP8 ? 64 * D + 2 * T16 : 2 * T16);
+    static constexpr int KBOX = 64 * 128;             // one 64-row x 128-byte box
+    static constexpr int QBOX = 128 * 128;            // one 128-row x 128-byte box
     static constexpr int OFF_K = 0;
     static constexpr int OFF_V = OFF_K + KS * KT;
-    // Q lands in the last two K slots; it moves to TMEM before their first use
-    static constexpr int OFF_Q = OFF_K + (KS - 2) * KT;
+    // Q lands in the last QSLOTS K slots; it moves to TMEM before their first use
+    static constexpr int QSLOTS = QB / KT;
+    static_assert(QB % KT == 0 && QSLOTS <= KS, "Q tiles alias whole K slots");
+    static constexpr int OFF_Q = OFF_K + (KS - QSLOTS) * KT;
+    static constexpr int OFF_QB = OFF_Q + (FP8 ? 128 * D : 0);   // bf16 Q
     static constexpr int OFF_MISC = OFF_V + VS * VT;
-    static constexpr int OFF_STAGE = OFF_V;          // epilogue buffers reuse the V ring
-    static_assert(QB == 2 * KT, "Q tile spans two K slots");
-    static constexpr int BBUF = D * D * 2;           // one (H - G) hi or lo buffer
-    static constexpr int BBOX = D * 128;             // one 64-column box of it
+    static constexpr int OFF_STAGE = OFF_V;           // epilogue buffers reuse the V ring
+    static constexpr int BBUF = D * D * 2;            // one (H - G) hi or lo buffer
+    static constexpr int BBOX = D * 128;              // one 64-column box of it
     // output staging for the tensor store, after the (H - G) buffers in the V ring
     static constexpr int OUT_OFF = OFF_V + (PISA ? 0 : (D == 128 ? 2 : 4) * BBUF);
     static_assert(OUT_OFF + D * 4 * 128 <= OFF_MISC, "output staging fits in the V ring");
@@ -150,23 +196,24 @@ struct AttnLayout {
 
 constexpr int kAttnThreads = 384;
 
-template <int D, bool PISA>
+template <int D, int MODE>
 __global__ void __launch_bounds__(kAttnThreads, 1)
-    attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmPhi,
-                const __grid_constant__ CUtensorMap tmKc, const __grid_constant__ CUtensorMap tmVc,
-                const __grid_constant__ CUtensorMap tmOut, const AttnArgs a) {
-    using L = AttnLayout<D, PISA>;
+    attn_kernel(const __grid_constant__ AttnMaps tm, const AttnArgs a) {
+    using L = AttnLayout<D, MODE>;
+    constexpr bool PISA = L::PISA, FP8 = L::FP8;
     constexpr bool SLA = !PISA;
     constexpr int NBOX = D / 64;
     constexpr int KS = L::KS, VS = L::VS;
-    // tensor memory columns: S0 | S1 | O | G_0 (| G_1 when d = 64) | Q | P0 | P1
+    // tensor memory columns: S0 | S1 | O | G_0 (| G_1 when d = 64) | Q | P0 | P1 (| bf16 Q)
+    // Q and P are packed 16-bit pairs (e4m3 quads in FP8 mode)
     constexpr uint32_t NCOLS = 512;
     constexpr uint32_t COL_O = 128;
     constexpr uint32_t COL_G0 = 128 + D;
     constexpr uint32_t COL_Q = PISA ? 128 + D : (D == 128 ? 128 + 2 * D : 128 + 3 * D);
-    constexpr uint32_t COL_P = COL_Q + D / 2;        // + 32 * b
-    static_assert(COL_P + 64 <= NCOLS, "tensor memory budget");
+    constexpr uint32_t PCOLS = FP8 ? 16 : 32;        // one P buffer
+    constexpr uint32_t COL_P = COL_Q + (FP8 ? D / 4 : D / 2);   // + PCOLS * b
+    constexpr uint32_t COL_QB = FP8 ? COL_P + 2 * PCOLS : COL_Q; // bf16 Q (linear branch)
+    static_assert((FP8 ? COL_QB + D / 2 : COL_P + 2 * PCOLS) <= NCOLS, "tensor memory budget");
 
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -201,6 +248,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     uint32_t* mark = reinterpret_cast<uint32_t*>(xl + 256);              // [ceil(Nk/16)]
     const int nwords = (a.Nk + 15) >> 4;
     int32_t* sched = reinterpret_cast<int32_t*>(mark + ((nwords + 3) & ~3));
+    float* ent_sk = reinterpret_cast<float*>(sched + a.sched_cap);       // FP8: per-entry K scale
+    float* ent_sv = ent_sk + a.sched_cap;                                // FP8: per-entry V scale
+    float* svmax_s = reinterpret_cast<float*>(g_any + 2);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int bh = blockIdx.x / a.tiles_per_head;
@@ -309,6 +359,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
     }
     }
+    if (FP8 && warp == 0) {
+        // per-entry K and V scales; the V scales' maximum fixes the P quantisation
+        __syncwarp();
+        const int cnt = *n_exact_s;
+        float vm = 0.f;
+        for (int e = lane; e < cnt; e += 32) {
+            const int j = sched[e] & 0xFFFF;
+            ent_sk[e] = a.sk[static_cast<long long>(bh) * a.Nk + j];
+            ent_sv[e] = a.sv[static_cast<long long>(bh) * a.Nk + j];
+            vm = fmaxf(vm, ent_sv[e]);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) vm = fmaxf(vm, __shfl_xor_sync(0xffffffffu, vm, o));
+        if (lane == 0) *svmax_s = vm > 0.f ? vm : 1.f;
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -321,7 +386,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
     auto sK = [&](int s) { return sbase + L::OFF_K + s * L::KT; };
     auto sV = [&](int s) { return sbase + L::OFF_V + s * L::VT; };
-    auto sPhi = [&](int s) { return sbase + L::OFF_V + s * L::VT + L::KT; };
+    auto sPhi = [&](int s) { return sbase + L::OFF_V + s * L::VT + L::V_PHI; };
+    auto sV16 = [&](int s) { return sbase + L::OFF_V + s * L::VT + L::V_V16; };
 
     auto fail = [&]() {
         *abort_flag = 1;
@@ -334,15 +400,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // has a free slot.  K(e) is consumed by S(e), which runs about two blocks
         // ahead of P.V(e), so K(kn) goes first while kn <= vn + 2.
         if (lane == 0) {
-            prefetch_tmap(&tmQ);
-            prefetch_tmap(&tmK);
-            prefetch_tmap(&tmV);
-            if (SLA) prefetch_tmap(&tmPhi);
-            if (PISA) { prefetch_tmap(&tmKc); prefetch_tmap(&tmVc); }
+            prefetch_tmap(&tm.q);
+            prefetch_tmap(&tm.k);
+            prefetch_tmap(&tm.v);
+            if (SLA) prefetch_tmap(&tm.phi);
+            if (PISA) { prefetch_tmap(&tm.kc); prefetch_tmap(&tm.vc); }
+            if (FP8) { prefetch_tmap(&tm.q8); prefetch_tmap(&tm.v8t); }
             const int qrow = bh * a.N + row0;
             mbar_arrive_expect_tx(q_full, L::QB);
+            if (FP8) tma_load_2d(smem + L::OFF_Q, &tm.q8, q_full, 0, qrow);
             for (int b = 0; b < NBOX; ++b)
-                tma_load_2d(smem + L::OFF_Q + b * L::QBOX, &tmQ, q_full, b * 64, qrow);
+                tma_load_2d(smem + L::OFF_QB + b * L::QBOX, &tm.q, q_full, b * 64, qrow);
             int kn = 0, vn = 0;
             bool q_moved = false;
             unsigned long long t0 = globaltimer_ns();
@@ -352,16 +420,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 const bool want_k = kn < n_total && (vn >= n_total || kn <= vn + 2);
                 if (want_k) {
                     const int s = kn % KS, r = kn / KS;
-                    const bool q_ok = !(r == 0 && s >= KS - 2) || q_moved || (q_moved = mbar_ready(q_tmem, 0));
+                    const bool q_ok = !(r == 0 && s >= KS - L::QSLOTS) || q_moved || (q_moved = mbar_ready(q_tmem, 0));
                     if (q_ok && mbar_ready(&k_empty[s], (r & 1) ^ 1)) {
                         mbar_arrive_expect_tx(&k_full[s], L::KT);
                         unsigned char* kd = smem + L::OFF_K + s * L::KT;
                         if (kn < n_exact) {
                             const int row = bh * a.N + (sched[kn] & 0xFFFF) * 64;
-                            for (int b = 0; b < NBOX; ++b) tma_load_2d(kd + b * L::KBOX, &tmK, &k_full[s], b * 64, row);
+                            if (FP8) tma_load_2d(kd, &tm.k, &k_full[s], 0, row);
+                            else for (int b = 0; b < NBOX; ++b) tma_load_2d(kd + b * L::KBOX, &tm.k, &k_full[s], b * 64, row);
                         } else {
                             const int row = bh * a.Nk + (kn - n_exact) * 64;
-                            for (int b = 0; b < NBOX; ++b) tma_load_2d(kd + b * L::KBOX, &tmKc, &k_full[s], b * 64, row);
+                            for (int b = 0; b < NBOX; ++b) tma_load_2d(kd + b * L::KBOX, &tm.kc, &k_full[s], b * 64, row);
                         }
                         ++kn;
                         did = true;
@@ -372,16 +441,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     if (mbar_ready(&v_empty[s], (r & 1) ^ 1)) {
                         mbar_arrive_expect_tx(&v_full[s], L::VT);
                         unsigned char* vd = smem + L::OFF_V + s * L::VT;
-                        unsigned char* pd = vd + L::KT;
                         if (vn < n_exact) {
-                            const int row = bh * a.N + (sched[vn] & 0xFFFF) * 64;
+                            const int j = sched[vn] & 0xFFFF;
+                            const int row = bh * a.N + j * 64;
+                            if (FP8) tma_load_2d(vd + L::V_PV, &tm.v8t, &v_full[s], 0, (bh * a.Nk + j) * D);
                             for (int b = 0; b < NBOX; ++b) {
-                                tma_load_2d(vd + b * L::KBOX, &tmV, &v_full[s], b * 64, row);
-                                if (SLA) tma_load_2d(pd + b * L::KBOX, &tmPhi, &v_full[s], b * 64, row);
+                                if (SLA) tma_load_2d(vd + L::V_PHI + b * L::KBOX, &tm.phi, &v_full[s], b * 64, row);
+                                tma_load_2d(vd + (FP8 ? L::V_V16 : L::V_PV) + b * L::KBOX, &tm.v, &v_full[s], b * 64, row);
                             }
                         } else {
                             const int row = bh * a.Nk + (vn - n_exact) * 64;
-                            for (int b = 0; b < NBOX; ++b) tma_load_2d(vd + b * L::KBOX, &tmVc, &v_full[s], b * 64, row);
+                            for (int b = 0; b < NBOX; ++b) tma_load_2d(vd + b * L::KBOX, &tm.vc, &v_full[s], b * 64, row);
                         }
                         ++vn;
                         did = true;
@@ -405,7 +475,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     } else if (warp == 1) {
         // ======================================================== S = Q K^T issuer
         if (lane == 0) {
-            constexpr uint32_t ID_S = idesc_bf16(128, 64, 0, 0);
+            constexpr uint32_t ID_S = FP8 ? idesc_e4m3(128, 64) : idesc_bf16(128, 64, 0, 0);
             bool ok = mbar_wait(q_tmem, 0, abort_flag, lim);
             tc_fence_after();
             for (int e = 0; ok && e < n_total; ++e) {
@@ -414,10 +484,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 if (!mbar_wait(&k_full[s], (e / KS) & 1, abort_flag, lim) ||
                     !mbar_wait(&s_empty[b], ((e >> 1) & 1) ^ 1, abort_flag, lim)) { ok = false; break; }
                 tc_fence_after();
+                if (FP8) {
+                    // e4m3: 32 elements (32 bytes) of K per instruction
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint64_t bd = sdesc(sK(s) + (kk >> 2) * L::KBOX + (kk & 3) * 32, 16, 1024, kSwizzle128B);
-                    umma_f16_ts(tmem + b * 64, tmem + COL_Q + kk * 8, bd, ID_S, kk > 0 ? 1u : 0u);
+                    for (int kk = 0; kk < D / 32; ++kk) {
+                        const uint64_t bd = sdesc(sK(s) + kk * 32, 16, 1024, kSwizzle128B);
+                        umma_f8_ts(tmem + b * 64, tmem + COL_Q + kk * 8, bd, ID_S, kk > 0 ? 1u : 0u);
+                    }
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint64_t bd = sdesc(sK(s) + (kk >> 2) * L::KBOX + (kk & 3) * 32, 16, 1024, kSwizzle128B);
+                        umma_f16_ts(tmem + b * 64, tmem + COL_Q + kk * 8, bd, ID_S, kk > 0 ? 1u : 0u);
+                    }
                 }
                 umma_commit(&s_full[b]);
                 umma_commit(&k_empty[s]);
@@ -430,7 +509,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     } else if (warp == 3) {
         // ======================================================== P.V / G / linear issuer
         if (lane == 0) {
-            constexpr uint32_t ID_PV = idesc_f16(128, D, 0, 1);
+            constexpr uint32_t ID_PV = FP8 ? idesc_e4m3(128, D) : idesc_f16(128, D, 0, 1);
             // G_g starts as H (preloaded by the softmax warps) and accumulates
             // -phi(K_j)^T V_j, so it ends as H - sum_{j in S_g} h_j
             constexpr uint32_t ID_G = idesc_f16(128, D, 1, 1, 1);
@@ -441,11 +520,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 if (!mbar_wait(&v_full[s], (e / VS) & 1, abort_flag, lim) ||
                     !mbar_wait(&p_full[b], u & 1, abort_flag, lim)) { ok = false; break; }
                 tc_fence_after();
+                if (FP8) {
+                    // B = V^T (e4m3, K-major: 64 tokens = 64 bytes per row, 64-byte swizzle)
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t bd = sdesc(sV(s) + kk * 2048, L::KBOX, 1024, kSwizzle128B);
-                    umma_f16_ts(tmem + COL_O, tmem + COL_P + 32 * b + kk * 8, bd, ID_PV,
-                                (e > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < 2; ++kk) {
+                        const uint64_t bd = sdesc(sV(s) + kk * 32, 16, 512, kSwizzle64B);
+                        umma_f8_ts(tmem + COL_O, tmem + COL_P + PCOLS * b + kk * 8, bd, ID_PV,
+                                   (e > 0 || kk > 0) ? 1u : 0u);
+                    }
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t bd = sdesc(sV(s) + kk * 2048, L::KBOX, 1024, kSwizzle128B);
+                        umma_f16_ts(tmem + COL_O, tmem + COL_P + PCOLS * b + kk * 8, bd, ID_PV,
+                                    (e > 0 || kk > 0) ? 1u : 0u);
+                    }
                 }
                 umma_commit(&p_empty[b]);
                 if (SLA) {
@@ -461,7 +550,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk) {
                             const uint64_t ad = sdesc(sPhi(s) + kk * 2048, lbo, 1024, kSwizzle128B);
-                            const uint64_t bd = sdesc(sV(s) + kk * 2048, L::KBOX, 1024, kSwizzle128B);
+                            const uint64_t bd = sdesc(sV16(s) + kk * 2048, L::KBOX, 1024, kSwizzle128B);
                             umma_f16_ss(tmem + COL_G0 + g * D, ad, bd, ID_G, 1u);
                         }
                     }
@@ -481,7 +570,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
                             for (int kk = 0; kk < D / 16; ++kk) {
                                 const uint64_t bd = sdesc(bb + kk * 2048, L::BBOX, 1024, kSwizzle128B);
-                                umma_f16_ts(tmem + COL_G0 + g * D, tmem + COL_Q + kk * 8, bd, ID_L,
+                                umma_f16_ts(tmem + COL_G0 + g * D, tmem + COL_QB + kk * 8, bd, ID_L,
                                             (part > 0 || kk > 0) ? 1u : 0u);
                             }
                         }
@@ -536,16 +625,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         float m_run = -INFINITY, l_run = 0.f;          // running max (log2 units), this half's row sum
         bool ok = wwait(q_full, 0);
         // Q row r -> TMEM lane r (packed bf16 pairs), the A operand of S = Q K^T;
-        // this half copies Q columns [h*D/2, (h+1)*D/2)
+        // this half copies Q columns [h*D/2, (h+1)*D/2).  FP8: the e4m3 row (four
+        // per column) for S, and the bf16 row for the linear branch.
         if (ok) {
+            if (FP8) {
+                uint32_t q8[16];
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(smem + L::OFF_Q + sw128(r, 4 * h + ch));
+                    q8[4 * ch] = v.x; q8[4 * ch + 1] = v.y; q8[4 * ch + 2] = v.z; q8[4 * ch + 3] = v.w;
+                }
+                tmem_st16(tl + COL_Q + 16 * h, q8);
+            }
             if (D == 128) {
                 uint32_t qv[32];
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch) {
-                    const uint4 v = *reinterpret_cast<const uint4*>(smem + L::OFF_Q + h * L::QBOX + sw128(r, ch));
+                    const uint4 v = *reinterpret_cast<const uint4*>(smem + L::OFF_QB + h * L::QBOX + sw128(r, ch));
                     qv[4 * ch] = v.x; qv[4 * ch + 1] = v.y; qv[4 * ch + 2] = v.z; qv[4 * ch + 3] = v.w;
                 }
-                tmem_st32(tl + COL_Q + 32 * h, qv);
+                tmem_st32(tl + COL_QB + 32 * h, qv);
             } else {
                 uint32_t qv[16];
 #pragma unroll
@@ -578,6 +677,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(g_init);
         }
+        // FP8: this row's Q block scale and the tile's P quantisation reference
+        const float sq = FP8 ? a.sq[(static_cast<long long>(bh) * a.N + row0 + r) / 64] : 1.f;
+        const float svmax = FP8 ? *svmax_s : 1.f;
         uint32_t sv[64];
         for (int e = 0; e < n_total; ++e) {
             const int b = e & 1, u = e >> 1;
@@ -594,12 +696,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             // masked ones are -inf); exp2 only for this half's 32 columns
             bool act = true;
             float mx = -INFINITY;
+            // logit scale of this block (FP8: times the Q and K block scales)
+            const float ce = FP8 ? c * sq * ent_sk[e] : c;
             if (e < n_exact) {
                 act = (sched[e] >> (16 + g)) & 1;
                 if (act) {
 #pragma unroll
                     for (int j = 0; j < 64; ++j) mx = fmaxf(mx, __uint_as_float(sv[j]));
-                    mx *= c;
+                    mx *= ce;
                 }
             } else {
                 const int c0 = (e - n_exact) * 64;
@@ -619,15 +723,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             }
             // P buffer b is free once PV_{e-2} completed
             if (!wwait(&p_empty[b], (u & 1) ^ 1)) { ok = false; break; }
-            const bool need = mx > m_run + kRescaleLog2;
-            const float m_new = need ? mx : m_run;
+            // lazy rescale (P <= 2^8).  FP8: the reference is the power of two at or
+            // above the running maximum, so P <= 1 and every rescale is an exact
+            // power of two (it commutes with the e4m3 rounding of earlier P)
+            const bool need = mx > m_run + (FP8 ? 0.f : kRescaleLog2);
+            const float m_new = need ? (FP8 ? ceilf(mx) : mx) : m_run;
             const bool rescale_o = need && m_run != -INFINITY;
             if (__any_sync(0xffffffffu, rescale_o)) {
                 // O holds PV_{0..e-1}: wait for PV_{e-1} (its P buffer's release);
                 // this half rescales O columns [h*D/2, (h+1)*D/2)
                 if (e > 0 && !wwait(&p_empty[b ^ 1], ((e - 1) >> 1) & 1)) { ok = false; break; }
                 tc_fence_after();
-                const float f = rescale_o ? fast_exp2(m_run - m_new) : 1.f;
+                const float f = rescale_o ? (FP8 ? exp2_int(m_run - m_new) : fast_exp2(m_run - m_new)) : 1.f;
 #pragma unroll 1
                 for (int cc = h * (D / 2); cc < (h + 1) * (D / 2); cc += 32) {
                     uint32_t ov[32];
@@ -641,15 +748,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 l_run *= f;
             }
             m_run = m_new;
-            // P = 2^(x - m) for columns [32h, 32h + 32) as packed fp16 pairs into TMEM
+            // P = 2^(x - m) for columns [32h, 32h + 32) into TMEM: packed fp16 pairs,
+            // or (FP8) e4m3 quads of P * 448 * s_v,j / s_v,max with the row sum from fp32 P
             const bool live = act && m_run != -INFINITY;
-            uint32_t pw[16];
-            const bool exact = e < n_exact;
-            const float ls = h == 0 ? (exact ? softmax_half<0, true>(sv, c, m_run, live, pw)
-                                             : softmax_half<0, false>(sv, c, m_run, live, pw))
-                                    : (exact ? softmax_half<32, true>(sv, c, m_run, live, pw)
-                                             : softmax_half<32, false>(sv, c, m_run, live, pw));
-            tmem_st16(tl + COL_P + 32 * b + 16 * h, pw);
+            float ls;
+            if (FP8) {
+                uint32_t p8[8];
+                const float qf = 448.f * ent_sv[e] / svmax;
+                ls = h == 0 ? softmax_half_e4m3<0>(sv, ce, m_run, live, qf, p8)
+                            : softmax_half_e4m3<32>(sv, ce, m_run, live, qf, p8);
+                tmem_st8(tl + COL_P + PCOLS * b + 8 * h, p8);
+            } else {
+                uint32_t pw[16];
+                const bool exact = e < n_exact;
+                ls = h == 0 ? (exact ? softmax_half<0, true>(sv, c, m_run, live, pw)
+                                     : softmax_half<0, false>(sv, c, m_run, live, pw))
+                            : (exact ? softmax_half<32, true>(sv, c, m_run, live, pw)
+                                     : softmax_half<32, false>(sv, c, m_run, live, pw));
+                tmem_st16(tl + COL_P + PCOLS * b + 16 * h, pw);
+            }
             tmem_st_wait();
             l_run += ls;
             tc_fence_before();
@@ -670,7 +787,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tc_fence_after();
         const long long grow = static_cast<long long>(bh) * a.N + row0 + r;
         const bool row_ok = g < n_groups && row0 + r < a.N;
-        const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
+        // FP8: O accumulated P * 448 * s_v,j / s_v,max times V / s_v,j
+        const float inv_l = l_tot > 0.f ? (FP8 ? svmax / 448.f : 1.f) / l_tot : 0.f;
         const bool have_o = n_total > 0;
         constexpr int HC = D / 2;                        // output columns of this half
         if (PISA) {
@@ -728,17 +846,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             if (fin) {
 #pragma unroll
                 for (int bx = 0; bx < NBOX; ++bx) {
-                    tmem_ld32(tl + COL_Q + 32 * bx, *reinterpret_cast<uint32_t(*)[32]>(&phq[32 * bx]));
+                    tmem_ld32(tl + COL_QB + 32 * bx, *reinterpret_cast<uint32_t(*)[32]>(&phq[32 * bx]));
                 }
                 tmem_ld_wait();
 #pragma unroll
                 for (int x = 0; x < D / 2; ++x) phq[x] = relu_bf16x2_u(phq[x]);
                 if (D == 128) {
-                    if (h == 0) tmem_st32(tl + COL_Q, *reinterpret_cast<uint32_t(*)[32]>(&phq[0]));
-                    else tmem_st32(tl + COL_Q + 32, *reinterpret_cast<uint32_t(*)[32]>(&phq[D == 128 ? 32 : 0]));
+                    if (h == 0) tmem_st32(tl + COL_QB, *reinterpret_cast<uint32_t(*)[32]>(&phq[0]));
+                    else tmem_st32(tl + COL_QB + 32, *reinterpret_cast<uint32_t(*)[32]>(&phq[D == 128 ? 32 : 0]));
                 } else {
-                    if (h == 0) tmem_st16(tl + COL_Q, *reinterpret_cast<uint32_t(*)[16]>(&phq[0]));
-                    else tmem_st16(tl + COL_Q + 16, *reinterpret_cast<uint32_t(*)[16]>(&phq[16]));
+                    if (h == 0) tmem_st16(tl + COL_QB, *reinterpret_cast<uint32_t(*)[16]>(&phq[0]));
+                    else tmem_st16(tl + COL_QB + 16, *reinterpret_cast<uint32_t(*)[16]>(&phq[16]));
                 }
                 tmem_st_wait();
             }
@@ -785,12 +903,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         fence_proxy_async_smem();
         named_bar(1, 256);
         if (warp == 4 && lane == 0 && !*abort_flag) {
+            const CUtensorMap* tmOut = &tm.out;
             const int nb = a.out_f32 ? D / 32 : D / 64;
             const int bc = a.out_f32 ? 32 : 64;
             for (int k = 0; k < 2; ++k) {
                 if (64 * k >= n_groups * a.Bq || row0 + 64 * k + 64 > a.N) continue;
                 for (int b = 0; b < nb; ++b)
-                    tma_store_2d(&tmOut, smem + L::OUT_OFF + b * 16384 + k * 64 * 128, b * bc,
+                    tma_store_2d(tmOut, smem + L::OUT_OFF + b * 16384 + k * 64 * 128, b * bc,
                                  bh * a.N + row0 + 64 * k);
             }
             tma_store_commit();

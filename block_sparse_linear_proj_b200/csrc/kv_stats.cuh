@@ -71,6 +71,12 @@ struct KvStatsArgs {
     __half* vbar;               // [BH][Nk][D] value means (null: skip)
     __half* v16;                // [BH][N][D] fp16 copy of V (null: skip)
     __half* phik16;             // [BH][N][D] fp16 phi(K) (null: skip)
+    // FP8 sparse branch (null: skip): e4m3 K [BH][N][D] and V transposed per
+    // 64-token block [BH][Nk][D][64], one absmax scale per block (absmax / 448)
+    uint8_t* k8;
+    uint8_t* v8t;
+    float* sk;                  // [BH][Nk]
+    float* sv;                  // [BH][Nk]
 };
 
 // grid (nchunk, BH), 256 threads.
@@ -82,6 +88,7 @@ __global__ void __launch_bounds__(256, 2) kv_stats_kernel(KvStatsArgs a) {
     double* kpart = reinterpret_cast<double*>(smem_raw + kKvStages * 2 * TILE);   // [256]
     float* zpart = reinterpret_cast<float*>(kpart + 256);                          // [256]
     float* vpart = zpart + 256;                                                    // [256]
+    float* amax = vpart + 256;                                                     // [2][8]
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const long long bh = blockIdx.y;
@@ -160,6 +167,19 @@ __global__ void __launch_bounds__(256, 2) kv_stats_kernel(KvStatsArgs a) {
             zpart[tid] = zs;
             vpart[tid] = vs;
             if (a.v16 && !(kmax < 65504.f)) report(kStatusRange);
+            if (a.k8) {
+                // per-block absmax of K and V (warp max, then 8 partials in smem)
+                float vmax = 0.f;
+                for (int n = half * RPH; n < (half + 1) * RPH; ++n)
+                    vmax = fmaxf(vmax, fabsf(__bfloat162float(
+                        *reinterpret_cast<const __nv_bfloat16*>(vt + kv_off<D>(n, col)))));
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    kmax = fmaxf(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+                    vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+                }
+                if (lane == 0) { amax[warp] = kmax; amax[8 + warp] = vmax; }
+            }
         }
         // fp16 copy of the V tile (coalesced 16-byte stores)
         if (a.v16) {
@@ -181,6 +201,42 @@ __global__ void __launch_bounds__(256, 2) kv_stats_kernel(KvStatsArgs a) {
                 *reinterpret_cast<uint4*>(vo + (row0 + n) * D + u * 8) = make_uint4(h[0], h[1], h[2], h[3]);
             }
             if (bad) report(kStatusRange);
+        }
+        // e4m3 K (row-major) and V (transposed per block) with one scale per block
+        if (a.k8) {
+            __syncthreads();
+            float km = 0.f, vm = 0.f;
+#pragma unroll
+            for (int w = 0; w < 8; ++w) { km = fmaxf(km, amax[w]); vm = fmaxf(vm, amax[8 + w]); }
+            // codes are picked by the correctly rounded quotient x / s (not x * (1/s),
+            // which lands on the other side of a rounding midpoint now and then)
+            const float s_k = km > 0.f ? km / 448.f : 1.f, s_v = vm > 0.f ? vm / 448.f : 1.f;
+            const int j = jb0 + blk;
+            if (tid == 0) {
+                a.sk[bh * a.Nk + j] = s_k;
+                a.sv[bh * a.Nk + j] = s_v;
+            }
+            constexpr int CPR = D / 8;
+            const long long row0 = static_cast<long long>(j) * kKvTok;
+            uint8_t* ko = a.k8 + bh * static_cast<long long>(a.N) * D;
+            for (int q = tid; q < kKvTok * CPR; q += 256) {
+                const int n = q / CPR, u = q % CPR;
+                const uint4 x = *reinterpret_cast<const uint4*>(kt + kv_off<D>(n, u * 8));
+                const uint32_t w0 = pack_e4m3x4(bf16lo(x.x) / s_k, bf16hi(x.x) / s_k, bf16lo(x.y) / s_k, bf16hi(x.y) / s_k);
+                const uint32_t w1 = pack_e4m3x4(bf16lo(x.z) / s_k, bf16hi(x.z) / s_k, bf16lo(x.w) / s_k, bf16hi(x.w) / s_k);
+                *reinterpret_cast<uint2*>(ko + (row0 + n) * D + u * 8) = make_uint2(w0, w1);
+            }
+            // V^T: row c of the block holds the 64 tokens of feature c
+            uint8_t* vo = a.v8t + (bh * a.Nk + j) * static_cast<long long>(D) * kKvTok;
+            for (int q = tid; q < D * (kKvTok / 8); q += 256) {
+                const int c = q % D, n0 = (q / D) * 8;
+                float f[8];
+#pragma unroll
+                for (int t = 0; t < 8; ++t)
+                    f[t] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(vt + kv_off<D>(n0 + t, c))) / s_v;
+                *reinterpret_cast<uint2*>(vo + c * kKvTok + n0) =
+                    make_uint2(pack_e4m3x4(f[0], f[1], f[2], f[3]), pack_e4m3x4(f[4], f[5], f[6], f[7]));
+            }
         }
         // fp16 phi(K) = max(K, 0)
         if (a.phik16) {
@@ -284,6 +340,45 @@ __global__ void __launch_bounds__(256) h_reduce_kernel(const float* __restrict__
         float s = 0.f;
         for (int j = 0; j < Nk; ++j) s += src[static_cast<long long>(j) * D];
         zsum[bh * D + threadIdx.x] = s;
+    }
+}
+
+// e4m3 Q with one absmax scale per 64-token block (absmax / 448).
+// Grid-stride over the BH*N/64 blocks; 256 threads, 64 x D tile in registers.
+template <int D>
+__global__ void __launch_bounds__(256) quant_q_kernel(const __nv_bfloat16* __restrict__ q,
+                                                      long long nblk, uint8_t* __restrict__ q8,
+                                                      float* __restrict__ sq) {
+    constexpr int VEC = 64 * D / 8 / 256;          // uint4 per thread
+    __shared__ float part[8];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (long long blk = blockIdx.x; blk < nblk; blk += gridDim.x) {
+        const uint4* src = reinterpret_cast<const uint4*>(q + blk * 64 * D);
+        uint4 x[VEC];
+        float m = 0.f;
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) {
+            x[i] = __ldg(src + i * 256 + tid);
+            const uint32_t w[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) m = fmaxf(m, fmaxf(fabsf(bf16lo(w[e])), fabsf(bf16hi(w[e]))));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == 0) part[warp] = m;
+        __syncthreads();
+        float am = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) am = fmaxf(am, part[w]);
+        const float s = am > 0.f ? am / 448.f : 1.f;   // codes from the rounded quotient x / s
+        if (tid == 0) sq[blk] = s;
+        uint2* dst = reinterpret_cast<uint2*>(q8 + blk * 64 * D);
+#pragma unroll
+        for (int i = 0; i < VEC; ++i)
+            dst[i * 256 + tid] = make_uint2(
+                pack_e4m3x4(bf16lo(x[i].x) / s, bf16hi(x[i].x) / s, bf16lo(x[i].y) / s, bf16hi(x[i].y) / s),
+                pack_e4m3x4(bf16lo(x[i].z) / s, bf16hi(x[i].z) / s, bf16lo(x[i].w) / s, bf16hi(x[i].w) / s));
+        __syncthreads();
     }
 }
 

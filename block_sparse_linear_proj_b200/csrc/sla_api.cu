@@ -55,7 +55,9 @@ sla_status_t check_tensor(const void* t, size_t align) {
 
 // ------------------------------------------------------------- workspace
 struct Ws {
-    size_t qbar, kbarT, m, lut, zj, hpart, hsum, zsum, kc, vbar, v16, phik16, total;
+    size_t qbar, kbarT, m, lut, zj, hpart, hsum, zsum, kc, vbar, v16, phik16;
+    size_t q8, k8, v8t, sq, sk, sv;       // FP8 sparse branch
+    size_t total;
     int nchunk, bpc;
 };
 
@@ -81,6 +83,14 @@ Ws layout(const sla_params_t* p) {
     w.vbar = take(BH * Nk * d * 2);
     w.v16 = take(BH * static_cast<size_t>(p->N) * d * 2);
     w.phik16 = take(BH * static_cast<size_t>(p->N) * d * 2);
+    if (p->sparse_dtype == SLA_SPARSE_FP8_E4M3) {
+        w.q8 = take(BH * static_cast<size_t>(p->N) * d);
+        w.k8 = take(BH * static_cast<size_t>(p->N) * d);
+        w.v8t = take(BH * static_cast<size_t>(p->N) * d);
+        w.sq = take(BH * static_cast<size_t>(p->N) / 64 * 4);
+        w.sk = take(BH * Nk * 4);
+        w.sv = take(BH * Nk * 4);
+    }
     w.total = off;
     return w;
 }
@@ -114,19 +124,20 @@ EncodeFn encode_fn() {
     return fn;
 }
 
-// 2-D map over [rows, d] (d innermost), box [128 bytes of columns, box_rows],
-// 128-byte swizzle.
+// 2-D map over [rows, d] (d innermost), box [box_bytes of columns, box_rows]
+// (128 bytes, 128-byte swizzle, unless given).
 bool make_map(CUtensorMap* m, const void* base, long long rows, int d, int box_rows,
-              CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
+              CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, int box_bytes = 128,
+              CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B) {
     EncodeFn fn = encode_fn();
     if (!fn) return false;
-    const int es = dt == CU_TENSOR_MAP_DATA_TYPE_FLOAT32 ? 4 : 2;
+    const int es = dt == CU_TENSOR_MAP_DATA_TYPE_FLOAT32 ? 4 : (dt == CU_TENSOR_MAP_DATA_TYPE_UINT8 ? 1 : 2);
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * es};
-    cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / es), static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(box_bytes / es), static_cast<cuuint32_t>(box_rows)};
     cuuint32_t estr[2] = {1, 1};
     return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box,
-              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -254,7 +265,8 @@ sla_status_t run_router(const sla_params_t* p, const void* q, const void* k, con
 
 template <int D>
 sla_status_t launch_kv(const sla_params_t* p, const void* k, const void* v, void* ws, const Ws& w,
-                       bool want_kbar, bool sla_stats, bool pisa_stats, cudaStream_t st) {
+                       bool want_kbar, bool sla_stats, bool pisa_stats, cudaStream_t st,
+                       bool fp8 = false) {
     const int BH = p->B * p->H, Nk = p->N / p->Bk;
     sla::KvStatsArgs a{};
     a.k = static_cast<const __nv_bfloat16*>(k);
@@ -270,7 +282,11 @@ sla_status_t launch_kv(const sla_params_t* p, const void* k, const void* v, void
     a.vbar = pisa_stats ? at<__half>(ws, w.vbar) : nullptr;
     a.v16 = at<__half>(ws, w.v16);
     a.phik16 = sla_stats ? at<__half>(ws, w.phik16) : nullptr;
-    const size_t smem = sla::kKvStages * 2 * 64 * D * 2 + 256 * 8 + 2 * 256 * 4;
+    a.k8 = fp8 ? at<uint8_t>(ws, w.k8) : nullptr;
+    a.v8t = fp8 ? at<uint8_t>(ws, w.v8t) : nullptr;
+    a.sk = fp8 ? at<float>(ws, w.sk) : nullptr;
+    a.sv = fp8 ? at<float>(ws, w.sv) : nullptr;
+    const size_t smem = sla::kKvStages * 2 * 64 * D * 2 + 256 * 8 + 2 * 256 * 4 + 16 * 4;
     auto kern = sla::kv_stats_kernel<D>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
@@ -289,36 +305,39 @@ sla_status_t launch_kv(const sla_params_t* p, const void* k, const void* v, void
     return launch_status();
 }
 
-template <int D, bool PISA>
+template <int D, int MODE>
 sla_status_t launch_attn(const sla_params_t* p, const void* q, const void* k, const void* v,
                          const float* alpha, const int32_t* lut, void* out, void* ws, const Ws& w,
                          cudaStream_t st) {
-    using L = sla::AttnLayout<D, PISA>;
+    using L = sla::AttnLayout<D, MODE>;
+    constexpr bool PISA = MODE == sla::kModePisa, FP8 = MODE == sla::kModeSlaFp8;
     const int BH = p->B * p->H, Nq = p->N / p->Bq, Nk = p->N / p->Bk;
-    CUtensorMap mq, mk, mv, mphi, mkc, mvc, mout;
+    sla::AttnMaps tm;
+    std::memset(&tm, 0, sizeof tm);
     const long long rows = static_cast<long long>(BH) * p->N;
-    (void)v;   // the P.V product reads the fp16 copy of V made by the K/V pre-pass
-    if (!make_map(&mout, out, rows, D, 64,
+    constexpr auto F16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    constexpr auto U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    (void)v;   // the P.V product reads the fp16 (or e4m3) copy of V made by the K/V pre-pass
+    if (!make_map(&tm.out, out, rows, D, 64,
                   p->out_dtype == SLA_OUT_FP32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
-                                               : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16))
+                                               : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) ||
+        !make_map(&tm.q, q, rows, D, 128) ||
+        !make_map(&tm.v, at<void>(ws, w.v16), rows, D, 64, F16))
         return SLA_ERR_CUDA;
-    if (!make_map(&mq, q, rows, D, 128) || !make_map(&mk, k, rows, D, 64) ||
-        !make_map(&mv, at<void>(ws, w.v16), rows, D, 64, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
-        return SLA_ERR_CUDA;
-    if (!PISA) {
-        if (!make_map(&mphi, at<void>(ws, w.phik16), rows, D, 64, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+    if (FP8) {
+        if (!make_map(&tm.k, at<void>(ws, w.k8), rows, D, 64, U8) ||
+            !make_map(&tm.q8, at<void>(ws, w.q8), rows, D, 128, U8) ||
+            !make_map(&tm.v8t, at<void>(ws, w.v8t), static_cast<long long>(BH) * Nk * D, 64, D, U8, 64,
+                      CU_TENSOR_MAP_SWIZZLE_64B))
             return SLA_ERR_CUDA;
-    } else {
-        mphi = mv;
+    } else if (!make_map(&tm.k, k, rows, D, 64)) {
+        return SLA_ERR_CUDA;
     }
+    if (!PISA && !make_map(&tm.phi, at<void>(ws, w.phik16), rows, D, 64, F16)) return SLA_ERR_CUDA;
     if (PISA) {
-        if (!make_map(&mkc, at<void>(ws, w.kc), static_cast<long long>(BH) * Nk, D, 64) ||
-            !make_map(&mvc, at<void>(ws, w.vbar), static_cast<long long>(BH) * Nk, D, 64,
-                      CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+        if (!make_map(&tm.kc, at<void>(ws, w.kc), static_cast<long long>(BH) * Nk, D, 64) ||
+            !make_map(&tm.vc, at<void>(ws, w.vbar), static_cast<long long>(BH) * Nk, D, 64, F16))
             return SLA_ERR_CUDA;
-    } else {
-        mkc = mk;
-        mvc = mv;
     }
     sla::AttnArgs a{};
     a.N = p->N;
@@ -341,19 +360,23 @@ sla_status_t launch_attn(const sla_params_t* p, const void* q, const void* k, co
     a.out = out;
     a.out_f32 = p->out_dtype == SLA_OUT_FP32 ? 1 : 0;
     a.lut_sorted = p->lut_mode == SLA_LUT_COMPUTE ? 1 : 0;
+    a.sq = FP8 ? at<float>(ws, w.sq) : nullptr;
+    a.sk = FP8 ? at<float>(ws, w.sk) : nullptr;
+    a.sv = FP8 ? at<float>(ws, w.sv) : nullptr;
     a.wait_ns = wait_limit_ns();
     const int GR = a.GR;
     const int nwords = (Nk + 15) / 16;
-    const size_t sched_cap = static_cast<size_t>(std::min(Nk, GR * std::max(p->topk, 1)));
+    const int sched_cap = std::max(4, (std::min(Nk, GR * std::max(p->topk, 1)) + 3) & ~3);
+    a.sched_cap = sched_cap;
     const size_t smem = 1024 + L::OFF_MISC + 384 + 2 * D * 4 + 256 * 4 + ((nwords + 3) & ~3) * 4 +
-                        sched_cap * 4;
+                        static_cast<size_t>(sched_cap) * 4 * 3;
     if (smem > 232448) return SLA_ERR_UNSUPPORTED;   // LUT row too long for the shared-memory schedule
-    auto kern = sla::attn_kernel<D, PISA>;
+    auto kern = sla::attn_kernel<D, MODE>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
         return SLA_ERR_CUDA;
     Span sp(SLA_KERNEL_ATTN, st);
-    kern<<<BH * a.tiles_per_head, sla::kAttnThreads, smem, st>>>(mq, mk, mv, mphi, mkc, mvc, mout, a);
+    kern<<<BH * a.tiles_per_head, sla::kAttnThreads, smem, st>>>(tm, a);
     return launch_status();
 }
 
@@ -458,16 +481,27 @@ sla_status_t sla_forward(const sla_params_t* p, const void* q, const void* k, co
         return SLA_ERR_UNSUPPORTED;
     Ws w;
     if ((s = check_ws(p, workspace, ws_bytes, w))) return s;
-    if (p->sparse_dtype == SLA_SPARSE_FP8_E4M3) return SLA_ERR_UNSUPPORTED;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const bool compute = p->lut_mode == SLA_LUT_COMPUTE;
+    const bool fp8 = p->sparse_dtype == SLA_SPARSE_FP8_E4M3;
     int32_t* lut_use = (compute && !lut) ? at<int32_t>(workspace, w.lut) : lut;
-    s = p->d == 128 ? launch_kv<128>(p, k, v, workspace, w, compute, true, false, st)
+    s = p->d == 128 ? launch_kv<128>(p, k, v, workspace, w, compute, true, false, st, fp8)
                     : launch_kv<64>(p, k, v, workspace, w, compute, true, false, st);
     if (s != SLA_OK) return s;
+    if (fp8) {
+        const long long nblk = static_cast<long long>(p->B) * p->H * p->N / 64;
+        Span sp(SLA_KERNEL_POOL, st);
+        sla::quant_q_kernel<128><<<grid_blocks(nblk, 8), 256, 0, st>>>(
+            static_cast<const __nv_bfloat16*>(q), nblk, at<uint8_t>(workspace, w.q8),
+            at<float>(workspace, w.sq));
+        if (launch_status() != SLA_OK) return SLA_ERR_CUDA;
+    }
     if (compute && (s = run_router(p, q, k, w_q, w_k, lut_use, workspace, w, false, st))) return s;
-    s = p->d == 128 ? launch_attn<128, false>(p, q, k, v, alpha, lut_use, out, workspace, w, st)
-                    : launch_attn<64, false>(p, q, k, v, alpha, lut_use, out, workspace, w, st);
+    if (fp8)
+        s = launch_attn<128, sla::kModeSlaFp8>(p, q, k, v, alpha, lut_use, out, workspace, w, st);
+    else
+        s = p->d == 128 ? launch_attn<128, sla::kModeSla>(p, q, k, v, alpha, lut_use, out, workspace, w, st)
+                        : launch_attn<64, sla::kModeSla>(p, q, k, v, alpha, lut_use, out, workspace, w, st);
     return finish(s, st);
 }
 
@@ -492,8 +526,8 @@ sla_status_t sla_pisa_forward(const sla_params_t* p, const void* q, const void* 
                     : launch_kv<64>(p, k, v, workspace, w, compute, false, true, st);
     if (s != SLA_OK) return s;
     if (compute && (s = run_router(p, q, k, w_q, w_k, lut_use, workspace, w, false, st))) return s;
-    s = p->d == 128 ? launch_attn<128, true>(p, q, k, v, nullptr, lut_use, out, workspace, w, st)
-                    : launch_attn<64, true>(p, q, k, v, nullptr, lut_use, out, workspace, w, st);
+    s = p->d == 128 ? launch_attn<128, sla::kModePisa>(p, q, k, v, nullptr, lut_use, out, workspace, w, st)
+                    : launch_attn<64, sla::kModePisa>(p, q, k, v, nullptr, lut_use, out, workspace, w, st);
     return finish(s, st);
 }
 
