@@ -114,62 +114,140 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------- oracle (CPU)
-def oracle_sample(w, inp, n_rows=256, seed=11):
-    """Time the CPU oracle on a bounded sample: the full router plus the forward
-    of n_rows seeded rows from two heads.  Returns (dense-equivalent TFLOPS,
-    seconds, threads, description)."""
+def _oracle_forward(w, inp, heads, rows, threads):
+    """Router, then forward, of the oracle on the given heads (all their rows
+    when rows is None).  Returns (route seconds, forward seconds)."""
     from oracle import oracle as orc
-    threads = len(os.sched_getaffinity(0))
+    hs = slice(heads[0], heads[-1] + 1)
+    q, k, v = inp["q"][:, hs], inp["k"][:, hs], inp["v"][:, hs]
     t0 = time.perf_counter()
-    lut, _ = orc.route(inp["q"], inp["k"], inp["w_q"], inp["w_k"], w.Bq, w.Bk, w.topk,
-                       threads=threads)
-    t_route = time.perf_counter() - t0
-    rows = W.sample_rows(w.B, w.H, w.N, n_rows, seed, heads=[0, w.B * w.H - 1]).numpy()
-    t0 = time.perf_counter()
+    lut, _ = orc.route(q, k, inp["w_q"], inp["w_k"], w.Bq, w.Bk, w.topk, threads=threads)
+    t1 = time.perf_counter()
     if w.mode == "pisa":
-        orc.pisa_forward(inp["q"], inp["k"], inp["v"], lut, w.Bq, w.Bk, rows=rows, threads=threads)
+        orc.pisa_forward(q, k, v, lut, w.Bq, w.Bk, rows=rows, threads=threads)
     else:
-        orc.sla_forward(inp["q"], inp["k"], inp["v"], inp["alpha"], lut, w.Bq, w.Bk, rows=rows,
-                        threads=threads)
-    t_fwd = time.perf_counter() - t0
-    total_rows = w.B * w.H * w.N
-    frac = len(rows) / total_rows
-    # time attributed to the sample: its share of the router + the sampled forward
-    t = t_route * frac + t_fwd
+        orc.sla_forward(q, k, v, inp["alpha"][:, hs], lut, w.Bq, w.Bk, rows=rows, threads=threads,
+                        fp8=w.sparse_dtype == W.SPARSE_FP8_E4M3)
+    return t1 - t0, time.perf_counter() - t1
+
+
+def oracle_heads(w, inp, budget_s=10.0):
+    """The oracle on whole heads (every row), one head after another until
+    budget_s has been spent (at least one head).  Returns (dense-equivalent
+    TFLOPS, seconds, threads, description)."""
+    threads = len(os.sched_getaffinity(0))
+    t_route = t_fwd = 0.0
+    done = 0
+    for h in range(w.H):
+        r, f = _oracle_forward(w, inp, [h], None, threads)
+        t_route += r
+        t_fwd += f
+        done += w.B                       # head h of every batch entry
+        if t_route + t_fwd >= budget_s:
+            break
+    t = t_route + t_fwd
+    flops = 4.0 * done * w.N * w.N * w.d
+    desc = ("%d of %d heads, every row: router %.2fs + forward %.2fs (the forward includes each "
+            "head's linear-branch block statistics)" % (done, w.B * w.H, t_route, t_fwd))
+    return flops / t / 1e12, t, threads, desc
+
+
+def oracle_rows(w, inp, head, n_rows, seed):
+    """One reference-arm step: the oracle's router on one head and the forward of
+    n_rows seeded rows of it (the head's linear-branch block statistics included)."""
+    threads = len(os.sched_getaffinity(0))
+    rng = np.random.default_rng(seed)
+    rows = np.sort(rng.choice(w.N, size=min(n_rows, w.N), replace=False)).astype(np.int64)
+    r, f = _oracle_forward(w, inp, [head], rows, threads)
     flops = 4.0 * len(rows) * w.N * w.d
-    desc = ("router on all %d heads (%.2fs, charged pro rata) + forward of %d rows from 2 heads "
-            "(%.2fs, incl. the per-head linear-branch block statistics)" % (
-                w.B * w.H, t_route, len(rows), t_fwd))
-    return flops / t / 1e12, t_route + t_fwd, threads, desc
+    return flops / (r + f) / 1e12, r + f, threads
 
 
 def run_reference(args, w, rank):
-    """--impl reference: the CPU oracle as the reference arm."""
+    """--impl reference: the CPU oracle as the reference arm (rank 0 only)."""
     if rank != 0:
         return
     inp = W.make_inputs(w)
-    for _ in range(args.warmup if args.warmup < 1 else 1):
-        oracle_sample(w, inp, n_rows=32)
-    vals, secs = [], []
-    for _ in range(args.steps):
-        v, s, threads, desc = oracle_sample(w, inp, n_rows=64)
+    # per-step sample sized so warm-up + steps stay within a few minutes
+    n_rows = int(max(64, min(1024, 1024 * 150 // max(1, args.steps + args.warmup))))
+    nh = w.H
+    for i in range(args.warmup):
+        oracle_rows(w, inp, i % nh, n_rows, 1000 + i)
+    vals = []
+    threads = 0
+    t_all = 0.0
+    for i in range(args.steps):
+        v, t, threads = oracle_rows(w, inp, i % nh, n_rows, i)
         vals.append(v)
-        secs.append(s)
+        t_all += t
     value = statistics.median(vals)
     ms_per_call = w.dense_equiv_flops() / (value * 1e12) * 1e3
+    desc = ("per step: router on one head + forward of %d seeded rows of it (heads in turn), "
+            "%.2fs per step on average" % (n_rows, t_all / max(1, args.steps)))
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms_per_call, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "Bq": w.Bq,
-                       "Bk": w.Bk, "topk": w.topk},
+            "config": config_of(w, 1),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                              "sample": desc},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
+def config_of(w, world):
+    in_bytes = 3 * w.B * w.H * w.N * w.d * 2
+    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "Bq": w.Bq, "Bk": w.Bk,
+            "topk": w.topk, "mode": w.mode,
+            "sparse_dtype": "e4m3" if w.sparse_dtype == W.SPARSE_FP8_E4M3 else "bf16",
+            "global_batch": w.B * world, "seq_len": w.N, "parallelism": "replicas%d" % world,
+            "l2": "inputs exceed L2 (%d MB of Q, K, V > 126 MB)" % (in_bytes // 10**6)
+                  if in_bytes > 126 * 10**6 else "inputs fit in L2",
+            "out_dtype": "bf16", "lut_mode": "compute"}
+
+
+def ncu_traffic(w):
+    """DRAM bytes per attention launch from the committed ncu summary of this
+    workload, if the attention kernel's source is unchanged since (its sha256
+    is recorded there); else None."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "attn_kernel_%s.md" % w.name)
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    with open(path) as f:
+        for ln in f:
+            if ":" in ln and ln.startswith("- "):
+                k, v = ln[2:].split(":", 1)
+                fields[k.strip()] = v.strip().strip("`")
+    h = hashlib.sha256()
+    for name in ("attn.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "block_sparse_linear_proj_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    if fields.get("kernel_source_sha256") != h.hexdigest():
+        return None
+    try:
+        return float(fields["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
 # ------------------------------------------------------------------- our arm
+def max_over_ranks(x, world, device):
+    """The slowest rank's figure (every rank takes part; all get the result)."""
+    if world == 1:
+        return x
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(w, world, ms_per_call):
+    """Weak scaling: every rank runs one copy of the workload; the job's
+    throughput is all copies' dense-equivalent FLOPs over the slowest time."""
+    return world * w.dense_equiv_flops() / (ms_per_call * 1e-3) / 1e12
+
+
 def run_ours(args, w, rank, world, local_rank):
     import block_sparse_linear_proj_b200 as S
     dev = torch.device("cuda", local_rank)
@@ -220,12 +298,9 @@ def run_ours(args, w, rank, world, local_rank):
     barrier()
     ms_total = e0.elapsed_time(e1)
     prof = S.sla_profile_read()
-    if world > 1:
-        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(ms_total, world, dev)
     ms_per_call = ms_total / args.steps
-    value = world * w.dense_equiv_flops() / (ms_per_call * 1e-3) / 1e12
+    value = whole_job_value(w, world, ms_per_call)
     launches = sum(c for (_, c) in prof.values())
 
     # ---- end-to-end through the C ABI with host buffers
@@ -253,11 +328,8 @@ def run_ours(args, w, rank, world, local_rank):
     f1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = f0.elapsed_time(f1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * w.dense_equiv_flops() / (e2e_ms * 1e-3) / 1e12
+    e2e_ms = max_over_ranks(e2e_ms, world, dev)
+    e2e_value = whole_job_value(w, world, e2e_ms)
     if S.sla_check_device_status(stream) != 0:
         raise RuntimeError("device status set during the benchmark")
 
@@ -270,7 +342,10 @@ def run_ours(args, w, rank, world, local_rank):
     exec_flops = 4.0 * pairs * w.Bq * w.Bk * w.d
     g_flops = 2.0 * pairs * w.Bk * w.d * w.d if w.mode == "sla" else 0.0
     achieved = exec_flops / (attn_avg * 1e-3) / 1e12
-    peak = peaks["bf16_tflops_sustained"]
+    fp8 = w.sparse_dtype == W.SPARSE_FP8_E4M3
+    # the attention kernel runs back to back for the whole timed region: the
+    # sustained peak; FP8 takes the bf16 figure times the nominal ratio (2)
+    peak = peaks["bf16_tflops_sustained"] * (2.0 if fp8 else 1.0)
     kv_ms, kv_n = prof["kv_stats"]
     kv_avg = kv_ms / max(kv_n, 1)
     kv_bytes = w.B * w.H * w.N * w.d * 2 * 3      # read K and V, write the fp16 copy of V
@@ -290,23 +365,21 @@ def run_ours(args, w, rank, world, local_rank):
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        v, secs, threads, desc = oracle_sample(w, inp)
+        v, secs, threads, desc = oracle_heads(w, inp)
         cpu = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc,
                "seconds": secs}
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_call, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if fp8 else "bf16",
         "data": "synthetic (seeded video-latent generator, no model weights)",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "Bq": w.Bq,
-                   "Bk": w.Bk, "topk": w.topk, "global_batch": w.B * world, "seq_len": w.N,
-                   "parallelism": "replicas%d" % world, "l2": "inputs exceed L2 (302 MB > 126 MB)",
-                   "out_dtype": "bf16", "lut_mode": "compute"},
+        "config": config_of(w, world),
         "ms_per_call": ms_per_call,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": None, "kernel": "attn",
-                     "peak_source": peaks["source"] + " bf16 sustained",
+                     "frac": achieved / peak, "traffic": ncu_traffic(w), "kernel": "attn",
+                     "peak_source": peaks["source"] + (" bf16 sustained x 2 (fp8)" if fp8
+                                                       else " bf16 sustained"),
                      "algorithmic": "4*Bq*Bk*d per (query block, selected block) pair, %d pairs" % pairs},
         "kernels": kernels,
         "cpu_baseline": cpu,

@@ -408,7 +408,7 @@ const char* sla_status_string(sla_status_t s) {
     return "unknown status";
 }
 
-int32_t sla_version(void) { return 100; }
+int32_t sla_version(void) { return 200; }
 
 sla_status_t sla_profile_enable(int32_t on) {
     Profiler& P = prof();
@@ -490,7 +490,7 @@ sla_status_t sla_forward(const sla_params_t* p, const void* q, const void* k, co
     if (s != SLA_OK) return s;
     if (fp8) {
         const long long nblk = static_cast<long long>(p->B) * p->H * p->N / 64;
-        Span sp(SLA_KERNEL_POOL, st);
+        Span sp(SLA_KERNEL_QUANT_Q, st);
         sla::quant_q_kernel<128><<<grid_blocks(nblk, 8), 256, 0, st>>>(
             static_cast<const __nv_bfloat16*>(q), nblk, at<uint8_t>(workspace, w.q8),
             at<float>(workspace, w.sq));

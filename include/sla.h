@@ -179,7 +179,8 @@ typedef enum {
     SLA_KERNEL_FOLD_W = 3,      /* W_q W_k^T                                    */
     SLA_KERNEL_SCORE_TOPK = 4,  /* fp64 block score + top-k                     */
     SLA_KERNEL_ATTN = 5,        /* sparse / PISA attention + fused epilogue     */
-    SLA_KERNEL_KINDS = 6
+    SLA_KERNEL_QUANT_Q = 6,     /* e4m3 quantisation of Q (FP8 sparse branch)   */
+    SLA_KERNEL_KINDS = 7
 } sla_kernel_kind_t;
 
 sla_status_t sla_profile_enable(int32_t on);
