@@ -348,7 +348,10 @@ def run_ours(args, w, rank, world, local_rank):
     peak = peaks["bf16_tflops_sustained"] * (2.0 if fp8 else 1.0)
     kv_ms, kv_n = prof["kv_stats"]
     kv_avg = kv_ms / max(kv_n, 1)
-    kv_bytes = w.B * w.H * w.N * w.d * 2 * 3      # read K and V, write the fp16 copy of V
+    # read K and V (bf16); write fp16 V and fp16 phi(K) (SLA), the centroids (PISA),
+    # and e4m3 K and V (FP8)
+    tok = w.B * w.H * w.N * w.d
+    kv_bytes = tok * 2 * 2 + (tok * 2 * 2 if w.mode == "sla" else tok * 2) + (tok * 2 if fp8 else 0)
     pool_ms, pool_n = prof["pool"]
     pool_avg = pool_ms / max(pool_n, 1)
     pool_bytes = w.B * w.H * w.N * w.d * 2        # read Q
