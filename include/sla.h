@@ -130,10 +130,17 @@ sla_status_t sla_route_noalloc(const sla_params_t *p, const void *q, const void 
  *      written to `lut` (which may be NULL); LUT_GIVEN -> `lut` is read and
  *      must hold topk distinct entries in [0, N/Bk) per row (any order);
  *      invalid entries are skipped and flagged SLA_ERR_DEVICE_CHECK.
- * sparse_dtype FP8_E4M3: Q, K, V are quantised to e4m3 with one absmax
- *      scale per 64-token block and P to e4m3 per tile ([SLA2] sec. 2.C:
- *      low-bit Q, K, P, V in the sparse branch); the linear branch stays
- *      bf16/fp32.
+ * sparse_dtype FP8_E4M3 (needs d = 128, Bq = 128): the sparse branch runs on
+ *      e4m3 Q, K, P and V ([SLA2] sec. 2.C; Arabic page sec. 2.j: the forward
+ *      quantises Q, K, P and V).  Q, K, V: one scale per 64-token block,
+ *      s = fl32(absmax / 448) (1 for an all-zero block), code = e4m3 of the
+ *      rounded fp32 quotient x / s (round to nearest even, saturating).
+ *      Logits use the e4m3 Q.K product times s_q s_k.  P is taken against the
+ *      power of two at or above the running row maximum and quantised per
+ *      64-key tile as e4m3(P * 448 s_v,j / s_v,max), s_v,max the largest V
+ *      scale of the query block's LUT row; O is dequantised by s_v,max / 448
+ *      and divided by the row sum of the unquantised P.  The linear branch
+ *      and the combine stay bf16/fp32.
  */
 sla_status_t sla_forward(const sla_params_t *p, const void *q, const void *k, const void *v,
                          const float *alpha, const float *w_q, const float *w_k,
