@@ -687,6 +687,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             tc_fence_after();
             tmem_ld32(tl + b * 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
             tmem_ld32(tl + b * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+            // P buffer b is free once PV_{e-2} completed: test it while S is in flight
+            const bool pe_ready = mbar_ready(&p_empty[b], (u & 1) ^ 1);
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
@@ -700,11 +702,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const float ce = FP8 ? c * sq * ent_sk[e] : c;
             if (e < n_exact) {
                 act = (sched[e] >> (16 + g)) & 1;
-                if (act) {
-#pragma unroll
-                    for (int j = 0; j < 64; ++j) mx = fmaxf(mx, __uint_as_float(sv[j]));
-                    mx *= ce;
-                }
+                if (act) mx = max64_bits(sv) * ce;
             } else {
                 const int c0 = (e - n_exact) * 64;
 #pragma unroll
@@ -721,8 +719,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     }
                 }
             }
-            // P buffer b is free once PV_{e-2} completed
-            if (!wwait(&p_empty[b], (u & 1) ^ 1)) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, pe_ready) && !wwait(&p_empty[b], (u & 1) ^ 1)) { ok = false; break; }
             // lazy rescale (P <= 2^8).  FP8: the reference is the power of two at or
             // above the running maximum, so P <= 1 and every rescale is an exact
             // power of two (it commutes with the e4m3 rounding of earlier P)

@@ -320,6 +320,31 @@ __device__ __forceinline__ float half_hi(uint32_t w) {
 }
 
 // Two fp32 -> two e4m3 (round to nearest even, saturating to +-448), low byte = lo.
+// max(a, b, c) in one instruction (the three-input form of sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// Maximum of 64 floats held as bit patterns: eight independent three-input
+// chains, then a two-level tree (depth 6 instead of a 63-long chain).
+__device__ __forceinline__ float max64_bits(const uint32_t (&v)[64]) {
+    float a[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        a[i] = fmax3(__uint_as_float(v[i]), __uint_as_float(v[8 + i]), __uint_as_float(v[16 + i]));
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        a[i] = fmax3(a[i], __uint_as_float(v[24 + i]), __uint_as_float(v[32 + i]));
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        a[i] = fmax3(a[i], __uint_as_float(v[40 + i]), __uint_as_float(v[48 + i]));
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a[i] = fmaxf(a[i], __uint_as_float(v[56 + i]));
+    return fmax3(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
+}
+
 // 2^k for an integral k <= 0, exactly (0 below the normal range).
 __device__ __forceinline__ float exp2_int(float k) {
     const int e = 127 + static_cast<int>(k);
