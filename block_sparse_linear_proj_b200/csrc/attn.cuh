@@ -165,11 +165,9 @@ __device__ __forceinline__ void stage_row32(unsigned char* stage, int f32, int r
 template <int D, int MODE>
 struct AttnLayout {
     static constexpr bool PISA = MODE == kModePisa, FP8 = MODE == kModeSlaFp8;
-    static constexpr int KS = (PISA || FP8) ? 6 : 4;  // K ring slots
-    static constexpr int VS = PISA ? 6 : 4;           // V ring slots
-    static constexpr int PF = 0;                      // L2 prefetch distance (blocks); 0 = off
+    static constexpr int KS = PISA ? (D == 128 ? 5 : 6) : (FP8 ? 6 : 4);   // K ring slots
+    static constexpr int VS = PISA ? (D == 128 ? 5 : 6) : (D == 128 ? 3 : 4);  // V ring slots
     static constexpr int T16 = 64 * D * 2;            // one 64-token tile of 16-bit values
-    static constexpr int QB = 128 * D * (FP8 ? 3 : 2);   // (e4m3 Q +) bf16 Q
     static constexpr int KT = 64 * D * (FP8 ? 1 : 2);    // one K tile
     // V slot: [P.V operand | fp16 phi(K) | fp16 V (FP8: the G operand)]
     static constexpr int V_PV = 0;
@@ -180,18 +178,17 @@ struct AttnLayout {
     static constexpr int QBOX = 128 * 128;            // one 128-row x 128-byte box
     static constexpr int OFF_K = 0;
     static constexpr int OFF_V = OFF_K + KS * KT;
-    // Q lands in the last QSLOTS K slots; it moves to TMEM before their first use
-    static constexpr int QSLOTS = QB / KT;
-    static_assert(QB % KT == 0 && QSLOTS <= KS, "Q tiles alias whole K slots");
-    static constexpr int OFF_Q = OFF_K + (KS - QSLOTS) * KT;
-    static constexpr int OFF_QB = OFF_Q + (FP8 ? 128 * D : 0);   // bf16 Q
-    static constexpr int OFF_MISC = OFF_V + VS * VT;
-    static constexpr int OFF_STAGE = OFF_V;           // epilogue buffers reuse the V ring
+    // the query tile stays in shared memory for the whole CTA: e4m3 Q (FP8), bf16 Q
+    static constexpr int OFF_Q8 = OFF_V + VS * VT;
+    static constexpr int OFF_Q = OFF_Q8 + (FP8 ? 128 * D : 0);
+    static constexpr int QB = 128 * D * (FP8 ? 3 : 2);   // bytes of the query-tile load
+    static constexpr int OFF_MISC = OFF_Q + 128 * D * 2;
+    static constexpr int GRMAX = D == 128 ? 1 : 2;    // query blocks per CTA (SLA mode)
     static constexpr int BBUF = D * D * 2;            // one (H - G) hi or lo buffer
     static constexpr int BBOX = D * 128;              // one 64-column box of it
-    // output staging for the tensor store, after the (H - G) buffers in the V ring
-    static constexpr int OUT_OFF = OFF_V + (PISA ? 0 : (D == 128 ? 2 : 4) * BBUF);
-    static_assert(OUT_OFF + D * 4 * 128 <= OFF_MISC, "output staging fits in the V ring");
+    // epilogue buffers reuse the rings: (H - G) hi/lo, then the output staging
+    static constexpr int OUT_OFF = OFF_K + (PISA ? 0 : 2 * GRMAX * BBUF);
+    static_assert(OUT_OFF + D * 4 * 128 <= OFF_Q8, "epilogue buffers fit in the K/V rings");
 };
 
 constexpr int kAttnThreads = 384;
@@ -204,16 +201,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     constexpr bool SLA = !PISA;
     constexpr int NBOX = D / 64;
     constexpr int KS = L::KS, VS = L::VS;
-    // tensor memory columns: S0 | S1 | O | G_0 (| G_1 when d = 64) | Q | P0 | P1 (| bf16 Q)
-    // Q and P are packed 16-bit pairs (e4m3 quads in FP8 mode)
+    // tensor memory columns: S_0 | S_1 | O_0 | O_1 | G_0 (| G_1 when d = 64).
+    // P(e) is written over the first columns of its S buffer (packed fp16 pairs,
+    // or e4m3 quads in FP8 mode).
     constexpr uint32_t NCOLS = 512;
-    constexpr uint32_t COL_O = 128;
-    constexpr uint32_t COL_G0 = 128 + D;
-    constexpr uint32_t COL_Q = PISA ? 128 + D : (D == 128 ? 128 + 2 * D : 128 + 3 * D);
-    constexpr uint32_t PCOLS = FP8 ? 16 : 32;        // one P buffer
-    constexpr uint32_t COL_P = COL_Q + (FP8 ? D / 4 : D / 2);   // + PCOLS * b
-    constexpr uint32_t COL_QB = FP8 ? COL_P + 2 * PCOLS : COL_Q; // bf16 Q (linear branch)
-    static_assert((FP8 ? COL_QB + D / 2 : COL_P + 2 * PCOLS) <= NCOLS, "tensor memory budget");
+    constexpr uint32_t COL_O = 128;                   // + h * D
+    constexpr uint32_t COL_G0 = 128 + 2 * D;          // + g * D
+    static_assert(PISA || COL_G0 + L::GRMAX * D <= NCOLS, "tensor memory budget");
 
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -227,30 +221,30 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     uint64_t* k_empty = k_full + KS;              // [KS]
     uint64_t* v_full = k_empty + KS;              // [VS]
     uint64_t* v_empty = v_full + VS;              // [VS]
-    uint64_t* q_tmem = v_empty + VS;              // Q copied into TMEM
-    uint64_t* s_full = q_tmem + 1;                // [2]
-    uint64_t* s_empty = s_full + 2;               // [2]
-    uint64_t* p_full = s_empty + 2;               // [2]
-    uint64_t* p_empty = p_full + 2;               // [2]
-    uint64_t* final_bar = p_empty + 2;
+    uint64_t* s_full = v_empty + VS;              // [2] S(e) in buffer e & 1
+    uint64_t* p_full = s_full + 2;                // [2] P(e) written (4 warps)
+    uint64_t* pv_done = p_full + 2;               // [2] P.V(e) complete: buffer free, O_{e&1} current
+    uint64_t* final_bar = pv_done + 2;
     uint64_t* epi_ready = final_bar + 1;
     uint64_t* lin_done = epi_ready + 1;
     uint64_t* drain_bar = lin_done + 1;
     uint64_t* drain2_bar = drain_bar + 1;
     uint64_t* g_init = drain2_bar + 1;            // G accumulators preloaded with H
-    uint64_t* xl_bar = g_init + 1;                // [4] final row-sum exchange per quarter
+    uint64_t* xl_bar = g_init + 1;                // [4] exchanges between the two warpgroups
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xl_bar + 4);
     int* n_exact_s = reinterpret_cast<int*>(tmem_slot + 1);
     volatile int* abort_flag = n_exact_s + 1;
     int* g_any = n_exact_s + 2;                   // [2] group selected >= 1 block
+    float* svmax_s = reinterpret_cast<float*>(g_any + 2);
     float* zu = reinterpret_cast<float*>(smem + L::OFF_MISC + 384);       // [2][D]
-    float* xl = zu + 2 * D;                                              // [2][128] row-sum halves
-    uint32_t* mark = reinterpret_cast<uint32_t*>(xl + 256);              // [ceil(Nk/16)]
+    float* xm = zu + 2 * D;                                              // [2][128] row maxima
+    float* xl = xm + 256;                                                // [2][128] row sums
+    float* xd = xl + 256;                                                // [2][128] denominators
+    uint32_t* mark = reinterpret_cast<uint32_t*>(xd + 256);              // [ceil(Nk/16)]
     const int nwords = (a.Nk + 15) >> 4;
     int32_t* sched = reinterpret_cast<int32_t*>(mark + ((nwords + 3) & ~3));
     float* ent_sk = reinterpret_cast<float*>(sched + a.sched_cap);       // FP8: per-entry K scale
     float* ent_sv = ent_sk + a.sched_cap;                                // FP8: per-entry V scale
-    float* svmax_s = reinterpret_cast<float*>(g_any + 2);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int bh = blockIdx.x / a.tiles_per_head;
@@ -263,7 +257,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // ------------------------------------------------------------ set-up
     if (tid == 0) {
         mbar_init(q_full, 1);
-        mbar_init(q_tmem, 8);
         for (int s = 0; s < KS; ++s) {
             mbar_init(&k_full[s], 1);
             mbar_init(&k_empty[s], 1);
@@ -274,9 +267,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&s_full[b], 1);
-            mbar_init(&s_empty[b], 8);
-            mbar_init(&p_full[b], 8);
-            mbar_init(&p_empty[b], 1);
+            mbar_init(&p_full[b], 4);
+            mbar_init(&pv_done[b], 1);
         }
         mbar_init(final_bar, 1);
         mbar_init(epi_ready, 9);
@@ -388,6 +380,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     auto sV = [&](int s) { return sbase + L::OFF_V + s * L::VT; };
     auto sPhi = [&](int s) { return sbase + L::OFF_V + s * L::VT + L::V_PHI; };
     auto sV16 = [&](int s) { return sbase + L::OFF_V + s * L::VT + L::V_V16; };
+    // K-major 128-byte-swizzled descriptor of the query tile (bf16) at K-step kk (16 columns)
+    auto qdesc = [&](int kk) {
+        return sdesc(sbase + L::OFF_Q + (kk >> 2) * L::QBOX + (kk & 3) * 32, 16, 1024, kSwizzle128B);
+    };
 
     auto fail = [&]() {
         *abort_flag = 1;
@@ -408,11 +404,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             if (FP8) { prefetch_tmap(&tm.q8); prefetch_tmap(&tm.v8t); }
             const int qrow = bh * a.N + row0;
             mbar_arrive_expect_tx(q_full, L::QB);
-            if (FP8) tma_load_2d(smem + L::OFF_Q, &tm.q8, q_full, 0, qrow);
+            if (FP8) tma_load_2d(smem + L::OFF_Q8, &tm.q8, q_full, 0, qrow);
             for (int b = 0; b < NBOX; ++b)
-                tma_load_2d(smem + L::OFF_QB + b * L::QBOX, &tm.q, q_full, b * 64, qrow);
+                tma_load_2d(smem + L::OFF_Q + b * L::QBOX, &tm.q, q_full, b * 64, qrow);
             int kn = 0, vn = 0;
-            bool q_moved = false;
             unsigned long long t0 = globaltimer_ns();
             uint32_t idle = 0;
             while (kn < n_total || vn < n_total) {
@@ -420,8 +415,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 const bool want_k = kn < n_total && (vn >= n_total || kn <= vn + 2);
                 if (want_k) {
                     const int s = kn % KS, r = kn / KS;
-                    const bool q_ok = !(r == 0 && s >= KS - L::QSLOTS) || q_moved || (q_moved = mbar_ready(q_tmem, 0));
-                    if (q_ok && mbar_ready(&k_empty[s], (r & 1) ^ 1)) {
+                    if (mbar_ready(&k_empty[s], (r & 1) ^ 1)) {
                         mbar_arrive_expect_tx(&k_full[s], L::KT);
                         unsigned char* kd = smem + L::OFF_K + s * L::KT;
                         if (kn < n_exact) {
@@ -476,26 +470,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // ======================================================== S = Q K^T issuer
         if (lane == 0) {
             constexpr uint32_t ID_S = FP8 ? idesc_e4m3(128, 64) : idesc_bf16(128, 64, 0, 0);
-            bool ok = mbar_wait(q_tmem, 0, abort_flag, lim);
-            tc_fence_after();
+            bool ok = mbar_wait(q_full, 0, abort_flag, lim);
             for (int e = 0; ok && e < n_total; ++e) {
-                // S(e) needs its K tile and its S buffer back from the softmax of e-2
+                // S(e) needs its K tile and its buffer back: P(e-2), written over
+                // S(e-2), has been consumed once P.V(e-2) completed
                 const int s = e % KS, b = e & 1;
                 if (!mbar_wait(&k_full[s], (e / KS) & 1, abort_flag, lim) ||
-                    !mbar_wait(&s_empty[b], ((e >> 1) & 1) ^ 1, abort_flag, lim)) { ok = false; break; }
+                    (e >= 2 && !mbar_wait(&pv_done[b], ((e >> 1) - 1) & 1, abort_flag, lim))) { ok = false; break; }
                 tc_fence_after();
                 if (FP8) {
-                    // e4m3: 32 elements (32 bytes) of K per instruction
+                    // e4m3: 32 elements (32 bytes) per instruction
 #pragma unroll
                     for (int kk = 0; kk < D / 32; ++kk) {
+                        const uint64_t ad = sdesc(sbase + L::OFF_Q8 + kk * 32, 16, 1024, kSwizzle128B);
                         const uint64_t bd = sdesc(sK(s) + kk * 32, 16, 1024, kSwizzle128B);
-                        umma_f8_ts(tmem + b * 64, tmem + COL_Q + kk * 8, bd, ID_S, kk > 0 ? 1u : 0u);
+                        umma_f8_ss(tmem + b * 64, ad, bd, ID_S, kk > 0 ? 1u : 0u);
                     }
                 } else {
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint64_t bd = sdesc(sK(s) + (kk >> 2) * L::KBOX + (kk & 3) * 32, 16, 1024, kSwizzle128B);
-                        umma_f16_ts(tmem + b * 64, tmem + COL_Q + kk * 8, bd, ID_S, kk > 0 ? 1u : 0u);
+                        umma_f16_ss(tmem + b * 64, qdesc(kk), bd, ID_S, kk > 0 ? 1u : 0u);
                     }
                 }
                 umma_commit(&s_full[b]);
@@ -520,23 +515,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 if (!mbar_wait(&v_full[s], (e / VS) & 1, abort_flag, lim) ||
                     !mbar_wait(&p_full[b], u & 1, abort_flag, lim)) { ok = false; break; }
                 tc_fence_after();
+                // O_b += P(e) V_e, P read from the first columns of S buffer b
+                const uint32_t o_col = tmem + COL_O + b * D;
                 if (FP8) {
                     // B = V^T (e4m3, K-major: 64 tokens = 64 bytes per row, 64-byte swizzle)
 #pragma unroll
                     for (int kk = 0; kk < 2; ++kk) {
                         const uint64_t bd = sdesc(sV(s) + kk * 32, 16, 512, kSwizzle64B);
-                        umma_f8_ts(tmem + COL_O, tmem + COL_P + PCOLS * b + kk * 8, bd, ID_PV,
-                                   (e > 0 || kk > 0) ? 1u : 0u);
+                        umma_f8_ts(o_col, tmem + b * 64 + kk * 8, bd, ID_PV, (u > 0 || kk > 0) ? 1u : 0u);
                     }
                 } else {
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
                         const uint64_t bd = sdesc(sV(s) + kk * 2048, L::KBOX, 1024, kSwizzle128B);
-                        umma_f16_ts(tmem + COL_O, tmem + COL_P + PCOLS * b + kk * 8, bd, ID_PV,
-                                    (e > 0 || kk > 0) ? 1u : 0u);
+                        umma_f16_ts(o_col, tmem + b * 64 + kk * 8, bd, ID_PV, (u > 0 || kk > 0) ? 1u : 0u);
                     }
                 }
-                umma_commit(&p_empty[b]);
+                umma_commit(&pv_done[b]);
                 if (SLA) {
                     if (!g_ready) {
                         if (!mbar_wait(g_init, 0, abort_flag, lim)) { ok = false; break; }
@@ -560,17 +555,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             if (!ok) fail();
             umma_commit(final_bar);
             if (SLA && ok) {
-                // linear branch: D_lin_g = phi(Q) (H - G_g), hi + lo, into G_g's columns
+                // linear branch: D_lin_g = phi(Q) (H - G_g), hi + lo, into G_g's columns;
+                // phi(Q) was written over the query tile in shared memory
                 if (mbar_wait(epi_ready, 0, abort_flag, lim)) {
                     tc_fence_after();
                     constexpr uint32_t ID_L = idesc_bf16(128, D, 0, 1);
                     for (int g = 0; g < n_groups; ++g) {
                         for (int part = 0; part < 2; ++part) {
-                            const uint32_t bb = sbase + L::OFF_STAGE + (2 * g + part) * L::BBUF;
+                            const uint32_t bb = sbase + L::OFF_K + (2 * g + part) * L::BBUF;
 #pragma unroll
                             for (int kk = 0; kk < D / 16; ++kk) {
                                 const uint64_t bd = sdesc(bb + kk * 2048, L::BBOX, 1024, kSwizzle128B);
-                                umma_f16_ts(tmem + COL_G0 + g * D, tmem + COL_QB + kk * 8, bd, ID_L,
+                                umma_f16_ss(tmem + COL_G0 + g * D, qdesc(kk), bd, ID_L,
                                             (part > 0 || kk > 0) ? 1u : 0u);
                             }
                         }
@@ -612,8 +608,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
     } else {
         // ======================================================== softmax + epilogue
+        // Warpgroup h takes the entries e with e % 2 == h: S buffer h, O_h and its
+        // own running maximum and row sum, so the two warpgroups work on two
+        // entries at once; their partial results are merged in the epilogue.
         const int q4 = warp & 3;                         // TMEM lane quarter
-        const int h = (warp - 4) >> 2;                   // column half (0 or 1)
+        const int h = (warp - 4) >> 2;                   // warpgroup
         const int r = q4 * 32 + lane;                    // row within the tile
         const int g = r / a.Bq;
         const uint32_t tl = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
@@ -622,47 +621,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             return __all_sync(0xffffffffu, mbar_wait(bar, par, abort_flag, lim) ? 1 : 0) != 0;
         };
         const float c = a.scale_log2;
-        float m_run = -INFINITY, l_run = 0.f;          // running max (log2 units), this half's row sum
-        bool ok = wwait(q_full, 0);
-        // Q row r -> TMEM lane r (packed bf16 pairs), the A operand of S = Q K^T;
-        // this half copies Q columns [h*D/2, (h+1)*D/2).  FP8: the e4m3 row (four
-        // per column) for S, and the bf16 row for the linear branch.
-        if (ok) {
-            if (FP8) {
-                uint32_t q8[16];
-#pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-                    const uint4 v = *reinterpret_cast<const uint4*>(smem + L::OFF_Q + sw128(r, 4 * h + ch));
-                    q8[4 * ch] = v.x; q8[4 * ch + 1] = v.y; q8[4 * ch + 2] = v.z; q8[4 * ch + 3] = v.w;
-                }
-                tmem_st16(tl + COL_Q + 16 * h, q8);
-            }
-            if (D == 128) {
-                uint32_t qv[32];
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    const uint4 v = *reinterpret_cast<const uint4*>(smem + L::OFF_QB + h * L::QBOX + sw128(r, ch));
-                    qv[4 * ch] = v.x; qv[4 * ch + 1] = v.y; qv[4 * ch + 2] = v.z; qv[4 * ch + 3] = v.w;
-                }
-                tmem_st32(tl + COL_QB + 32 * h, qv);
-            } else {
-                uint32_t qv[16];
-#pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-                    const uint4 v = *reinterpret_cast<const uint4*>(smem + L::OFF_Q + sw128(r, 4 * h + ch));
-                    qv[4 * ch] = v.x; qv[4 * ch + 1] = v.y; qv[4 * ch + 2] = v.z; qv[4 * ch + 3] = v.w;
-                }
-                tmem_st16(tl + COL_Q + 16 * h, qv);
-            }
-            tmem_st_wait();
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(q_tmem);
+        float m_run = -INFINITY, l_run = 0.f;          // this warpgroup's running max (log2 units) and sum
+        bool ok = true;
         if (SLA) {
-            // G_g := H (row r = c of the d x d matrix, this half's columns); H is
-            // stored transposed per head, H^T[e][c], so lane r's loads are coalesced
-            if (ok && r < D) {
+            // G_g := H (row r = c of the d x d matrix, this warpgroup's half of the
+            // columns); H is stored transposed per head, H^T[e][c], so lane r's loads
+            // are coalesced
+            if (r < D) {
                 const float* hcol = a.hsum + static_cast<long long>(bh) * D * D + r;
 #pragma unroll 1
                 for (int cc = h * (D / 2); cc < (h + 1) * (D / 2); cc += 32) {
@@ -680,22 +645,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // FP8: this row's Q block scale and the tile's P quantisation reference
         const float sq = FP8 ? a.sq[(static_cast<long long>(bh) * a.N + row0 + r) / 64] : 1.f;
         const float svmax = FP8 ? *svmax_s : 1.f;
+        const uint32_t o_h = COL_O + h * D;
         uint32_t sv[64];
-        for (int e = 0; e < n_total; ++e) {
-            const int b = e & 1, u = e >> 1;
-            if (!wwait(&s_full[b], u & 1)) { ok = false; break; }
+        for (int e = h; e < n_total; e += 2) {
+            const int u = e >> 1;
+            if (!wwait(&s_full[h], u & 1)) { ok = false; break; }
             tc_fence_after();
-            tmem_ld32(tl + b * 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-            tmem_ld32(tl + b * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-            // P buffer b is free once PV_{e-2} completed: test it while S is in flight
-            const bool pe_ready = mbar_ready(&p_empty[b], (u & 1) ^ 1);
+            tmem_ld32(tl + h * 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+            tmem_ld32(tl + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
             tmem_ld_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s_empty[b]);
 
-            // row maximum over all 64 logits (x = s * c, + log2 Bk for centroids;
-            // masked ones are -inf); exp2 only for this half's 32 columns
+            // row maximum over the 64 logits (x = s * c, + log2 Bk for centroids;
+            // masked ones are -inf)
             bool act = true;
             float mx = -INFINITY;
             // logit scale of this block (FP8: times the Q and K block scales)
@@ -719,7 +680,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     }
                 }
             }
-            if (!__all_sync(0xffffffffu, pe_ready) && !wwait(&p_empty[b], (u & 1) ^ 1)) { ok = false; break; }
             // lazy rescale (P <= 2^8).  FP8: the reference is the power of two at or
             // above the running maximum, so P <= 1 and every rescale is an exact
             // power of two (it commutes with the e4m3 rounding of earlier P)
@@ -727,92 +687,100 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const float m_new = need ? (FP8 ? ceilf(mx) : mx) : m_run;
             const bool rescale_o = need && m_run != -INFINITY;
             if (__any_sync(0xffffffffu, rescale_o)) {
-                // O holds PV_{0..e-1}: wait for PV_{e-1} (its P buffer's release);
-                // this half rescales O columns [h*D/2, (h+1)*D/2)
-                if (e > 0 && !wwait(&p_empty[b ^ 1], ((e - 1) >> 1) & 1)) { ok = false; break; }
-                tc_fence_after();
+                // O_h holds P.V of this warpgroup's entries up to e-2, all complete:
+                // S(e) was issued only after P.V(e-2) finished
                 const float f = rescale_o ? (FP8 ? exp2_int(m_run - m_new) : fast_exp2(m_run - m_new)) : 1.f;
 #pragma unroll 1
-                for (int cc = h * (D / 2); cc < (h + 1) * (D / 2); cc += 32) {
+                for (int cc = 0; cc < D; cc += 32) {
                     uint32_t ov[32];
-                    tmem_ld32(tl + COL_O + cc, ov);
+                    tmem_ld32(tl + o_h + cc, ov);
                     tmem_ld_wait();
 #pragma unroll
                     for (int x = 0; x < 32; ++x) ov[x] = __float_as_uint(__uint_as_float(ov[x]) * f);
-                    tmem_st32(tl + COL_O + cc, ov);
+                    tmem_st32(tl + o_h + cc, ov);
                 }
                 tmem_st_wait();
                 l_run *= f;
             }
             m_run = m_new;
-            // P = 2^(x - m) for columns [32h, 32h + 32) into TMEM: packed fp16 pairs,
-            // or (FP8) e4m3 quads of P * 448 * s_v,j / s_v,max with the row sum from fp32 P
+            // P = 2^(x - m) over the 64 keys, written over the first columns of S
+            // buffer h: packed fp16 pairs, or (FP8) e4m3 quads of
+            // P * 448 * s_v,j / s_v,max with the row sum from fp32 P
             const bool live = act && m_run != -INFINITY;
             float ls;
             if (FP8) {
-                uint32_t p8[8];
+                uint32_t p8[16];
                 const float qf = 448.f * ent_sv[e] / svmax;
-                ls = h == 0 ? softmax_half_e4m3<0>(sv, ce, m_run, live, qf, p8)
-                            : softmax_half_e4m3<32>(sv, ce, m_run, live, qf, p8);
-                tmem_st8(tl + COL_P + PCOLS * b + 8 * h, p8);
+                ls = softmax_half_e4m3<0>(sv, ce, m_run, live, qf, *reinterpret_cast<uint32_t(*)[8]>(&p8[0]));
+                ls += softmax_half_e4m3<32>(sv, ce, m_run, live, qf, *reinterpret_cast<uint32_t(*)[8]>(&p8[8]));
+                tmem_st16(tl + h * 64, p8);
             } else {
-                uint32_t pw[16];
+                uint32_t pwa[16], pwb[16];
                 const bool exact = e < n_exact;
-                ls = h == 0 ? (exact ? softmax_half<0, true>(sv, c, m_run, live, pw)
-                                     : softmax_half<0, false>(sv, c, m_run, live, pw))
-                            : (exact ? softmax_half<32, true>(sv, c, m_run, live, pw)
-                                     : softmax_half<32, false>(sv, c, m_run, live, pw));
-                tmem_st16(tl + COL_P + PCOLS * b + 16 * h, pw);
+                ls = exact ? softmax_half<0, true>(sv, c, m_run, live, pwa) : softmax_half<0, false>(sv, c, m_run, live, pwa);
+                tmem_st16(tl + h * 64, pwa);
+                ls += exact ? softmax_half<32, true>(sv, c, m_run, live, pwb) : softmax_half<32, false>(sv, c, m_run, live, pwb);
+                tmem_st16(tl + h * 64 + 16, pwb);
             }
             tmem_st_wait();
             l_run += ls;
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&p_full[b]);
+            if (lane == 0) mbar_arrive(&p_full[h]);
         }
         if (!ok) fail();
 
         // ------------------------------------------------ epilogue
-        // row sum = both halves' sums (exchanged once through shared memory)
+        // merge the two warpgroups' partial softmaxes (exchanged once through shared memory)
+        xm[h * 128 + r] = m_run;
         xl[h * 128 + r] = l_run;
         __syncwarp();
         if (lane == 0) mbar_arrive(&xl_bar[q4]);
         const bool xok = wwait(&xl_bar[q4], 0);
-        const float l_tot = xok ? l_run + xl[(h ^ 1) * 128 + r] : 0.f;
         if (ok && !xok) fail();
+        float f0 = 0.f, f1 = 0.f, l_tot = 0.f;
+        if (xok) {
+            const float m0 = xm[r], m1 = xm[128 + r];
+            const float mm = fmaxf(m0, m1);
+            if (m0 != -INFINITY) f0 = FP8 ? exp2_int(m0 - mm) : fast_exp2(m0 - mm);
+            if (m1 != -INFINITY) f1 = FP8 ? exp2_int(m1 - mm) : fast_exp2(m1 - mm);
+            l_tot = f0 * xl[r] + f1 * xl[128 + r];
+        }
         const bool fin = ok && xok && wwait(final_bar, 0);
+        if (ok && xok && !fin) fail();
         tc_fence_after();
         const long long grow = static_cast<long long>(bh) * a.N + row0 + r;
         const bool row_ok = g < n_groups && row0 + r < a.N;
         // FP8: O accumulated P * 448 * s_v,j / s_v,max times V / s_v,j
         const float inv_l = l_tot > 0.f ? (FP8 ? svmax / 448.f : 1.f) / l_tot : 0.f;
-        const bool have_o = n_total > 0;
-        constexpr int HC = D / 2;                        // output columns of this half
+        const bool have0 = n_total > 0 && f0 != 0.f, have1 = n_total > 1 && f1 != 0.f;
+        constexpr int HC = D / 2;                        // output columns of this warpgroup
+        // sum of the two partial P.V accumulators for 32 columns, scaled by 1/l
+        auto o_sum = [&](int cc, float (&res)[32]) {
+            uint32_t o0[32], o1[32];
+            if (have0) tmem_ld32(tl + COL_O + cc, o0);
+            if (have1) tmem_ld32(tl + COL_O + D + cc, o1);
+            tmem_ld_wait();
+#pragma unroll
+            for (int x = 0; x < 32; ++x)
+                res[x] = ((have0 ? f0 * __uint_as_float(o0[x]) : 0.f) +
+                          (have1 ? f1 * __uint_as_float(o1[x]) : 0.f)) * inv_l;
+        };
         if (PISA) {
             if (fin) {
 #pragma unroll 1
                 for (int cc = h * HC; cc < (h + 1) * HC; cc += 32) {
-                    uint32_t ov[32];
-                    if (have_o) {
-                        tmem_ld32(tl + COL_O + cc, ov);
-                        tmem_ld_wait();
-                    } else {
-#pragma unroll
-                        for (int x = 0; x < 32; ++x) ov[x] = 0u;
-                    }
                     float res[32];
-#pragma unroll
-                    for (int x = 0; x < 32; ++x) res[x] = __uint_as_float(ov[x]) * inv_l;
+                    o_sum(cc, res);
                     stage_row32(smem + L::OUT_OFF, a.out_f32, r, cc, res);
                 }
             }
         } else {
-            // (1) B_g = H - G_g (row r of the d x d matrices, this half's columns),
+            // (1) B_g = H - G_g (row r of the d x d matrices, this warpgroup's columns),
             //     bf16 hi + lo, MN-major 128-byte-swizzled boxes of 64 columns
             if (fin && r < D) {
-                // the G_g columns hold H - G_g (row r of the d x d matrix)
                 for (int gg = 0; gg < n_groups; ++gg) {
-                    unsigned char* bhi = smem + L::OFF_STAGE + (2 * gg) * L::BBUF;
+                    unsigned char* bhi = smem + L::OFF_K + (2 * gg) * L::BBUF;
                     unsigned char* blo = bhi + L::BBUF;
 #pragma unroll 1
                     for (int cc = h * HC; cc < (h + 1) * HC; cc += 32) {
@@ -837,56 +805,51 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     }
                 }
             }
-            // (2) phi(Q) in place in TMEM (the A operand of the linear-branch MMA):
-            //     both halves read the whole row for the denominator, each writes back its half
-            uint32_t phq[D / 2];
+            // (2) phi(Q) over the query tile in shared memory (the A operand of the
+            //     linear-branch product): this warpgroup's half of row r, and its part
+            //     of the denominator phi(q) . Zu_g
+            float den = 0.f;
             if (fin) {
+                const float* z = zu + (g < 2 ? g : 0) * D;
 #pragma unroll
-                for (int bx = 0; bx < NBOX; ++bx) {
-                    tmem_ld32(tl + COL_QB + 32 * bx, *reinterpret_cast<uint32_t(*)[32]>(&phq[32 * bx]));
+                for (int x = 0; x < HC / 8; ++x) {
+                    const int c8 = h * HC + 8 * x;               // first column of this chunk
+                    unsigned char* p = smem + L::OFF_Q + (c8 >> 6) * L::QBOX + sw128(r, (c8 & 63) >> 3);
+                    uint4 v = *reinterpret_cast<const uint4*>(p);
+                    v.x = relu_bf16x2_u(v.x); v.y = relu_bf16x2_u(v.y);
+                    v.z = relu_bf16x2_u(v.z); v.w = relu_bf16x2_u(v.w);
+                    *reinterpret_cast<uint4*>(p) = v;
+                    den += bf16lo(v.x) * z[c8] + bf16hi(v.x) * z[c8 + 1] + bf16lo(v.y) * z[c8 + 2] +
+                           bf16hi(v.y) * z[c8 + 3] + bf16lo(v.z) * z[c8 + 4] + bf16hi(v.z) * z[c8 + 5] +
+                           bf16lo(v.w) * z[c8 + 6] + bf16hi(v.w) * z[c8 + 7];
                 }
-                tmem_ld_wait();
-#pragma unroll
-                for (int x = 0; x < D / 2; ++x) phq[x] = relu_bf16x2_u(phq[x]);
-                if (D == 128) {
-                    if (h == 0) tmem_st32(tl + COL_QB, *reinterpret_cast<uint32_t(*)[32]>(&phq[0]));
-                    else tmem_st32(tl + COL_QB + 32, *reinterpret_cast<uint32_t(*)[32]>(&phq[D == 128 ? 32 : 0]));
-                } else {
-                    if (h == 0) tmem_st16(tl + COL_QB, *reinterpret_cast<uint32_t(*)[16]>(&phq[0]));
-                    else tmem_st16(tl + COL_QB + 16, *reinterpret_cast<uint32_t(*)[16]>(&phq[16]));
-                }
-                tmem_st_wait();
             }
+            xd[h * 128 + r] = den;
+            fence_proxy_async_smem();                      // phi(Q), B_g -> the tensor core
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(epi_ready);
-            const bool lin = fin && wwait(epi_ready, 0) && wwait(lin_done, 0);
+            if (lane == 0) {
+                mbar_arrive(&xl_bar[q4]);
+                mbar_arrive(epi_ready);
+            }
+            const bool dok = wwait(&xl_bar[q4], 1);
+            den = dok ? xd[r] + xd[128 + r] : 0.f;
+            const bool lin = fin && dok && wwait(epi_ready, 0) && wwait(lin_done, 0);
             if (fin && !lin) fail();
             tc_fence_after();
             if (lin) {
-                // denominator phi(q) . Zu_g
-                float den = 0.f;
-                const float* z = zu + (g < 2 ? g : 0) * D;
-#pragma unroll
-                for (int x = 0; x < D / 2; ++x) den += bf16lo(phq[x]) * z[2 * x] + bf16hi(phq[x]) * z[2 * x + 1];
                 const float inv_den = den > 0.f ? 1.f / den : 0.f;
                 const float al = row_ok ? a.alpha[grow] : 0.f;
                 const uint32_t col_lin = COL_G0 + (g < n_groups ? g : 0) * D;
 #pragma unroll 1
                 for (int cc = h * HC; cc < (h + 1) * HC; cc += 32) {
-                    uint32_t ov[32], lv[32];
+                    uint32_t lv[32];
                     tmem_ld32(tl + col_lin + cc, lv);
-                    if (have_o) tmem_ld32(tl + COL_O + cc, ov);
-                    tmem_ld_wait();
-                    if (!have_o) {
-#pragma unroll
-                        for (int x = 0; x < 32; ++x) ov[x] = 0u;
-                    }
                     float res[32];
+                    o_sum(cc, res);
 #pragma unroll
                     for (int x = 0; x < 32; ++x)
-                        res[x] = al * (__uint_as_float(ov[x]) * inv_l) +
-                                 (1.f - al) * (__uint_as_float(lv[x]) * inv_den);
+                        res[x] = al * res[x] + (1.f - al) * (__uint_as_float(lv[x]) * inv_den);
                     stage_row32(smem + L::OUT_OFF, a.out_f32, r, cc, res);
                 }
             }

@@ -368,7 +368,9 @@ sla_status_t launch_attn(const sla_params_t* p, const void* q, const void* k, co
     const int nwords = (Nk + 15) / 16;
     const int sched_cap = std::max(4, (std::min(Nk, GR * std::max(p->topk, 1)) + 3) & ~3);
     a.sched_cap = sched_cap;
-    const size_t smem = 1024 + L::OFF_MISC + 384 + 2 * D * 4 + 256 * 4 + ((nwords + 3) & ~3) * 4 +
+    // misc region: barriers (384 B), zu [2][D], the three [2][128] exchange arrays,
+    // the block mask, the schedule and (FP8) the per-entry scales
+    const size_t smem = 1024 + L::OFF_MISC + 384 + 2 * D * 4 + 3 * 256 * 4 + ((nwords + 3) & ~3) * 4 +
                         static_cast<size_t>(sched_cap) * 4 * 3;
     if (smem > 232448) return SLA_ERR_UNSUPPORTED;   // LUT row too long for the shared-memory schedule
     auto kern = sla::attn_kernel<D, MODE>;
