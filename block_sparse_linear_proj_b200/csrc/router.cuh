@@ -100,7 +100,9 @@ __device__ __forceinline__ unsigned long long order_key(double v) {
 // One CTA: head bh = blockIdx.y, query blocks i0 = blockIdx.x * R ... i0 + R - 1.
 // Shared memory: qhat^T [D][R] fp64, hist [8][256] u32, keys [R][max(Nk, D)] u64
 // (the key area doubles as the [R][D] staging buffer of step 1).
-template <int R, int D>
+// PF: step 2 reads the kbar columns eight feature rows ahead of use (pays off on
+// long rows, where each warp walks several column chunks).
+template <int R, int D, bool PF>
 __global__ void __launch_bounds__(256) score_topk_kernel(const double* __restrict__ qbar,
                                                          const double* __restrict__ kbarT,
                                                          const double* __restrict__ m, int Nq,
@@ -157,18 +159,51 @@ __global__ void __launch_bounds__(256) score_topk_kernel(const double* __restric
         double acc0[R], acc1[R];
 #pragma unroll
         for (int r = 0; r < R; ++r) { acc0[r] = 0.0; acc1[r] = 0.0; }
-#pragma unroll 4
-        for (int c = 0; c < D; ++c) {
-            const double ka = va ? __ldg(kt + static_cast<long long>(c) * Nk + ja) : 0.0;
-            const double kb = vb ? __ldg(kt + static_cast<long long>(c) * Nk + jb) : 0.0;
-            const double2* qrow = reinterpret_cast<const double2*>(qhT + c * R);
+        if (PF) {
+            double ka[8], kb[8];
 #pragma unroll
-            for (int r2 = 0; r2 < R / 2; ++r2) {
-                const double2 qq = qrow[r2];
-                acc0[2 * r2] = fma(qq.x, ka, acc0[2 * r2]);
-                acc1[2 * r2] = fma(qq.x, kb, acc1[2 * r2]);
-                acc0[2 * r2 + 1] = fma(qq.y, ka, acc0[2 * r2 + 1]);
-                acc1[2 * r2 + 1] = fma(qq.y, kb, acc1[2 * r2 + 1]);
+            for (int x = 0; x < 8; ++x) {
+                ka[x] = va ? __ldg(kt + static_cast<long long>(x) * Nk + ja) : 0.0;
+                kb[x] = vb ? __ldg(kt + static_cast<long long>(x) * Nk + jb) : 0.0;
+            }
+#pragma unroll 1
+            for (int c0 = 0; c0 < D; c0 += 8) {
+                double na[8], nb[8];
+                const bool more = c0 + 8 < D;
+#pragma unroll
+                for (int x = 0; x < 8; ++x) {
+                    na[x] = (more && va) ? __ldg(kt + static_cast<long long>(c0 + 8 + x) * Nk + ja) : 0.0;
+                    nb[x] = (more && vb) ? __ldg(kt + static_cast<long long>(c0 + 8 + x) * Nk + jb) : 0.0;
+                }
+#pragma unroll
+                for (int x = 0; x < 8; ++x) {
+                    const double2* qrow = reinterpret_cast<const double2*>(qhT + (c0 + x) * R);
+#pragma unroll
+                    for (int r2 = 0; r2 < R / 2; ++r2) {
+                        const double2 qq = qrow[r2];
+                        acc0[2 * r2] = fma(qq.x, ka[x], acc0[2 * r2]);
+                        acc1[2 * r2] = fma(qq.x, kb[x], acc1[2 * r2]);
+                        acc0[2 * r2 + 1] = fma(qq.y, ka[x], acc0[2 * r2 + 1]);
+                        acc1[2 * r2 + 1] = fma(qq.y, kb[x], acc1[2 * r2 + 1]);
+                    }
+                }
+#pragma unroll
+                for (int x = 0; x < 8; ++x) { ka[x] = na[x]; kb[x] = nb[x]; }
+            }
+        } else {
+#pragma unroll 4
+            for (int c = 0; c < D; ++c) {
+                const double ka = va ? __ldg(kt + static_cast<long long>(c) * Nk + ja) : 0.0;
+                const double kb = vb ? __ldg(kt + static_cast<long long>(c) * Nk + jb) : 0.0;
+                const double2* qrow = reinterpret_cast<const double2*>(qhT + c * R);
+#pragma unroll
+                for (int r2 = 0; r2 < R / 2; ++r2) {
+                    const double2 qq = qrow[r2];
+                    acc0[2 * r2] = fma(qq.x, ka, acc0[2 * r2]);
+                    acc1[2 * r2] = fma(qq.x, kb, acc1[2 * r2]);
+                    acc0[2 * r2 + 1] = fma(qq.y, ka, acc0[2 * r2 + 1]);
+                    acc1[2 * r2 + 1] = fma(qq.y, kb, acc1[2 * r2 + 1]);
+                }
             }
         }
 #pragma unroll

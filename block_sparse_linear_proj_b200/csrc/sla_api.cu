@@ -220,7 +220,8 @@ sla_status_t launch_score_r(const double* qbar, const double* kbarT, const doubl
                             int Nq, int Nk, int topk, int32_t* lut, cudaStream_t st) {
     const size_t smem = static_cast<size_t>(D) * R * 8 + 8 * 256 * 4 +
                         static_cast<size_t>(R) * std::max(Nk, D) * 8;
-    auto kern = sla::score_topk_kernel<R, D>;
+    // read-ahead of the kbar columns pays off once each warp walks several 64-column chunks
+    auto kern = Nk >= 1024 ? sla::score_topk_kernel<R, D, true> : sla::score_topk_kernel<R, D, false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
         return SLA_ERR_CUDA;
