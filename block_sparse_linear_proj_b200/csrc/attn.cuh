@@ -239,7 +239,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     float* zu = reinterpret_cast<float*>(smem + L::OFF_MISC + 384);       // [2][D]
     float* xm = zu + 2 * D;                                              // [2][128] row maxima
     float* xl = xm + 256;                                                // [2][128] row sums
-    float* xd = xl + 256;                                                // [2][128] denominators
+    float* xd = xl + 256;                                                // [128] linear-branch denominators
     uint32_t* mark = reinterpret_cast<uint32_t*>(xd + 256);              // [ceil(Nk/16)]
     const int nwords = (a.Nk + 15) >> 4;
     int32_t* sched = reinterpret_cast<int32_t*>(mark + ((nwords + 3) & ~3));
@@ -279,6 +279,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int x = 0; x < 4; ++x) mbar_init(&xl_bar[x], 2);
         *abort_flag = 0;
         fence_barrier_init();
+        // the query tile does not depend on the schedule: start its load now, so
+        // that it overlaps the set-up below (no role waits on q_full before the
+        // CTA-wide barrier that follows the set-up)
+        prefetch_tmap(&tm.q);
+        if (FP8) prefetch_tmap(&tm.q8);
+        const int qrow = bh * a.N + row0;
+        mbar_arrive_expect_tx(q_full, L::QB);
+        if (FP8) tma_load_2d(smem + L::OFF_Q8, &tm.q8, q_full, 0, qrow);
+        for (int b = 0; b < NBOX; ++b)
+            tma_load_2d(smem + L::OFF_Q + b * L::QBOX, &tm.q, q_full, b * 64, qrow);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, NCOLS);
@@ -396,17 +406,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // has a free slot.  K(e) is consumed by S(e), which runs about two blocks
         // ahead of P.V(e), so K(kn) goes first while kn <= vn + 2.
         if (lane == 0) {
-            prefetch_tmap(&tm.q);
             prefetch_tmap(&tm.k);
             prefetch_tmap(&tm.v);
             if (SLA) prefetch_tmap(&tm.phi);
             if (PISA) { prefetch_tmap(&tm.kc); prefetch_tmap(&tm.vc); }
-            if (FP8) { prefetch_tmap(&tm.q8); prefetch_tmap(&tm.v8t); }
-            const int qrow = bh * a.N + row0;
-            mbar_arrive_expect_tx(q_full, L::QB);
-            if (FP8) tma_load_2d(smem + L::OFF_Q8, &tm.q8, q_full, 0, qrow);
-            for (int b = 0; b < NBOX; ++b)
-                tma_load_2d(smem + L::OFF_Q + b * L::QBOX, &tm.q, q_full, b * 64, qrow);
+            if (FP8) prefetch_tmap(&tm.v8t);
             int kn = 0, vn = 0;
             unsigned long long t0 = globaltimer_ns();
             uint32_t idle = 0;
@@ -604,6 +608,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 for (int c = 0; c < D / 32; ++c) zu[g * D + t + 32 * c] = zs[t + 32 * c] - acc[c];
             }
             __syncwarp();
+            // the linear-branch denominators phi(q_r) . Zu_g(r) of the tile's 128 rows,
+            // from the query tile in shared memory (read only, while the main loop runs)
+            if (__all_sync(0xffffffffu, mbar_wait(q_full, 0, abort_flag, lim) ? 1 : 0)) {
+                for (int rr = lane; rr < 128; rr += 32) {
+                    const float* z = zu + min(rr / a.Bq, 1) * D;
+                    float den = 0.f;
+#pragma unroll 4
+                    for (int x = 0; x < D / 8; ++x) {
+                        const int c8 = 8 * x;
+                        const uint4 v = *reinterpret_cast<const uint4*>(
+                            smem + L::OFF_Q + (c8 >> 6) * L::QBOX + sw128(rr, (c8 & 63) >> 3));
+                        const uint32_t w4[4] = {relu_bf16x2_u(v.x), relu_bf16x2_u(v.y), relu_bf16x2_u(v.z),
+                                                relu_bf16x2_u(v.w)};
+#pragma unroll
+                        for (int y = 0; y < 4; ++y)
+                            den += bf16lo(w4[y]) * z[c8 + 2 * y] + bf16hi(w4[y]) * z[c8 + 2 * y + 1];
+                    }
+                    xd[rr] = den;
+                }
+            }
+            __syncwarp();
             if (lane == 0) mbar_arrive(epi_ready);
         }
     } else {
@@ -646,6 +671,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const float sq = FP8 ? a.sq[(static_cast<long long>(bh) * a.N + row0 + r) / 64] : 1.f;
         const float svmax = FP8 ? *svmax_s : 1.f;
         const uint32_t o_h = COL_O + h * D;
+        // this row's combine weight, read now so its latency is off the epilogue
+        const float al = (SLA && g < n_groups && row0 + r < a.N)
+                             ? a.alpha[static_cast<long long>(bh) * a.N + row0 + r] : 0.f;
         uint32_t sv[64];
         for (int e = h; e < n_total; e += 2) {
             const int u = e >> 1;
@@ -749,8 +777,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const bool fin = ok && xok && wwait(final_bar, 0);
         if (ok && xok && !fin) fail();
         tc_fence_after();
-        const long long grow = static_cast<long long>(bh) * a.N + row0 + r;
-        const bool row_ok = g < n_groups && row0 + r < a.N;
         // FP8: O accumulated P * 448 * s_v,j / s_v,max times V / s_v,j
         const float inv_l = l_tot > 0.f ? (FP8 ? svmax / 448.f : 1.f) / l_tot : 0.f;
         const bool have0 = n_total > 0 && f0 != 0.f, have1 = n_total > 1 && f1 != 0.f;
@@ -806,11 +832,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 }
             }
             // (2) phi(Q) over the query tile in shared memory (the A operand of the
-            //     linear-branch product): this warpgroup's half of row r, and its part
-            //     of the denominator phi(q) . Zu_g
-            float den = 0.f;
+            //     linear-branch product), this warpgroup's half of row r
             if (fin) {
-                const float* z = zu + (g < 2 ? g : 0) * D;
 #pragma unroll
                 for (int x = 0; x < HC / 8; ++x) {
                     const int c8 = h * HC + 8 * x;               // first column of this chunk
@@ -819,38 +842,37 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     v.x = relu_bf16x2_u(v.x); v.y = relu_bf16x2_u(v.y);
                     v.z = relu_bf16x2_u(v.z); v.w = relu_bf16x2_u(v.w);
                     *reinterpret_cast<uint4*>(p) = v;
-                    den += bf16lo(v.x) * z[c8] + bf16hi(v.x) * z[c8 + 1] + bf16lo(v.y) * z[c8 + 2] +
-                           bf16hi(v.y) * z[c8 + 3] + bf16lo(v.z) * z[c8 + 4] + bf16hi(v.z) * z[c8 + 5] +
-                           bf16lo(v.w) * z[c8 + 6] + bf16hi(v.w) * z[c8 + 7];
                 }
             }
-            xd[h * 128 + r] = den;
             fence_proxy_async_smem();                      // phi(Q), B_g -> the tensor core
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&xl_bar[q4]);
-                mbar_arrive(epi_ready);
+            if (lane == 0) mbar_arrive(epi_ready);
+            // (3) the sparse part of the combine while the linear-branch product runs
+            float res[HC];
+            if (fin) {
+#pragma unroll
+                for (int x = 0; x < HC / 32; ++x) o_sum(h * HC + 32 * x, *reinterpret_cast<float(*)[32]>(&res[32 * x]));
             }
-            const bool dok = wwait(&xl_bar[q4], 1);
-            den = dok ? xd[r] + xd[128 + r] : 0.f;
-            const bool lin = fin && dok && wwait(epi_ready, 0) && wwait(lin_done, 0);
+            const bool lin = fin && wwait(epi_ready, 0) && wwait(lin_done, 0);
             if (fin && !lin) fail();
             tc_fence_after();
             if (lin) {
+                // denominator phi(q) . Zu_g, from warp 2 (written before its epi_ready arrival)
+                const float den = xd[r];
                 const float inv_den = den > 0.f ? 1.f / den : 0.f;
-                const float al = row_ok ? a.alpha[grow] : 0.f;
                 const uint32_t col_lin = COL_G0 + (g < n_groups ? g : 0) * D;
-#pragma unroll 1
-                for (int cc = h * HC; cc < (h + 1) * HC; cc += 32) {
+#pragma unroll
+                for (int x = 0; x < HC / 32; ++x) {
+                    const int cc = h * HC + 32 * x;
                     uint32_t lv[32];
                     tmem_ld32(tl + col_lin + cc, lv);
-                    float res[32];
-                    o_sum(cc, res);
+                    tmem_ld_wait();
+                    float out32[32];
 #pragma unroll
-                    for (int x = 0; x < 32; ++x)
-                        res[x] = al * res[x] + (1.f - al) * (__uint_as_float(lv[x]) * inv_den);
-                    stage_row32(smem + L::OUT_OFF, a.out_f32, r, cc, res);
+                    for (int y = 0; y < 32; ++y)
+                        out32[y] = al * res[32 * x + y] + (1.f - al) * (__uint_as_float(lv[y]) * inv_den);
+                    stage_row32(smem + L::OUT_OFF, a.out_f32, r, cc, out32);
                 }
             }
         }
