@@ -76,6 +76,7 @@ struct AttnArgs {
     const float* sk;               // FP8: [BH][Nk]  K block scales
     const float* sv;               // FP8: [BH][Nk]  V block scales
     unsigned long long wait_ns;
+    int debug_stall;               // test hook: load no K/V tiles, so the consumers' waits run out
 };
 
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -412,11 +413,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             if (PISA) { prefetch_tmap(&tm.kc); prefetch_tmap(&tm.vc); }
             if (FP8) prefetch_tmap(&tm.v8t);
             int kn = 0, vn = 0;
+            const int n_load = a.debug_stall ? 0 : n_total;
             unsigned long long t0 = globaltimer_ns();
             uint32_t idle = 0;
-            while (kn < n_total || vn < n_total) {
+            while (kn < n_load || vn < n_load) {
                 bool did = false;
-                const bool want_k = kn < n_total && (vn >= n_total || kn <= vn + 2);
+                const bool want_k = kn < n_load && (vn >= n_load || kn <= vn + 2);
                 if (want_k) {
                     const int s = kn % KS, r = kn / KS;
                     if (mbar_ready(&k_empty[s], (r & 1) ^ 1)) {
@@ -434,7 +436,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         did = true;
                     }
                 }
-                if (!did && vn < n_total) {
+                if (!did && vn < n_load) {
                     const int s = vn % VS, r = vn / VS;
                     if (mbar_ready(&v_empty[s], (r & 1) ^ 1)) {
                         mbar_arrive_expect_tx(&v_full[s], L::VT);

@@ -151,6 +151,15 @@ unsigned long long wait_limit_ns() {
     return 2000000000ull;
 }
 
+// Test hook for failure detection: with SLA_DEBUG_STALL set (and not "0") the
+// attention kernel's loader issues no K/V tile loads, so the consumers' bounded
+// waits run out and the call reports SLA_ERR_TIMEOUT; no access is made that
+// would not be made otherwise.
+bool debug_stall() {
+    const char* s = std::getenv("SLA_DEBUG_STALL");
+    return s && *s && *s != '0';
+}
+
 bool check_after_call() {
     const char* s = std::getenv("SLA_CHECK");
     return s && *s && *s != '0';
@@ -238,7 +247,11 @@ sla_status_t launch_score(const double* qbar, const double* kbarT, const double*
     auto need = [&](int R) {
         return static_cast<size_t>(D) * R * 8 + 8 * 256 * 4 + static_cast<size_t>(R) * std::max(Nk, D) * 8;
     };
-    if (need(16) <= budget) return launch_score_r<16, D>(qbar, kbarT, m, BH, Nq, Nk, topk, lut, st);
+    // 16 query blocks per CTA, unless that leaves fewer than two waves of CTAs on
+    // 148 SMs for short rows (then 8 blocks per CTA spreads the fp64 work wider)
+    const bool few = static_cast<long long>((Nq + 15) / 16) * BH < 2 * 148;
+    if (!(few && Nk < 1024) && need(16) <= budget)
+        return launch_score_r<16, D>(qbar, kbarT, m, BH, Nq, Nk, topk, lut, st);
     if (need(8) <= budget) return launch_score_r<8, D>(qbar, kbarT, m, BH, Nq, Nk, topk, lut, st);
     if (need(4) <= budget) return launch_score_r<4, D>(qbar, kbarT, m, BH, Nq, Nk, topk, lut, st);
     return launch_score_r<2, D>(qbar, kbarT, m, BH, Nq, Nk, topk, lut, st);
@@ -365,6 +378,7 @@ sla_status_t launch_attn(const sla_params_t* p, const void* q, const void* k, co
     a.sk = FP8 ? at<float>(ws, w.sk) : nullptr;
     a.sv = FP8 ? at<float>(ws, w.sv) : nullptr;
     a.wait_ns = wait_limit_ns();
+    a.debug_stall = debug_stall() ? 1 : 0;
     const int GR = a.GR;
     const int nwords = (Nk + 15) / 16;
     const int sched_cap = std::max(4, (std::min(Nk, GR * std::max(p->topk, 1)) + 3) & ~3);
