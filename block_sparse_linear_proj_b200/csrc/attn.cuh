@@ -97,9 +97,15 @@ __device__ __forceinline__ uint32_t hadd2_u(uint32_t a, uint32_t b) {
 
 // P = 2^(x - m) for the 32 logits sv[OFF .. OFF+31] as 16 packed fp16 pairs;
 // returns their sum.  EXACT: sv holds raw scores (x = s*c), else x itself.
-template <int OFF, bool EXACT>
+// Rows with nothing to add (!live) get P = 0.  PACKED forms the arguments two at
+// a time with the packed fp32 FMA and handles !live rows through m = +inf (every
+// P exactly +0); the two forms give identical results, and each is faster in one
+// mode of the kernel (PACKED in the PISA mode).
+template <int OFF, bool EXACT, bool PACKED>
 __device__ __forceinline__ float softmax_half(const uint32_t (&sv)[64], float c, float m, bool live,
                                               uint32_t (&pw)[16]) {
+    const float mp = (PACKED && !live) ? INFINITY : m;
+    const uint64_t c2 = f2pack(EXACT ? c : 1.f, EXACT ? c : 1.f), nm2 = f2pack(-mp, -mp);
     float ls = 0.f;
 #pragma unroll
     for (int ch = 0; ch < 4; ++ch) {
@@ -107,14 +113,19 @@ __device__ __forceinline__ float softmax_half(const uint32_t (&sv)[64], float c,
         for (int x = 0; x < 4; ++x) {
             const int j = OFF + ch * 8 + 2 * x;
             float x0, x1;
-            if (EXACT) {
-                x0 = fmaf(__uint_as_float(sv[j]), c, -m);
-                x1 = fmaf(__uint_as_float(sv[j + 1]), c, -m);
+            if (PACKED) {
+                f2unpack(ffma2(f2pack(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1])), c2, nm2), x0, x1);
+                pw[4 * ch + x] = exp2_h2(pack_half2(x0, x1));
             } else {
-                x0 = __uint_as_float(sv[j]) - m;
-                x1 = __uint_as_float(sv[j + 1]) - m;
+                if (EXACT) {
+                    x0 = fmaf(__uint_as_float(sv[j]), c, -m);
+                    x1 = fmaf(__uint_as_float(sv[j + 1]), c, -m);
+                } else {
+                    x0 = __uint_as_float(sv[j]) - m;
+                    x1 = __uint_as_float(sv[j + 1]) - m;
+                }
+                pw[4 * ch + x] = live ? exp2_h2(pack_half2(x0, x1)) : 0u;
             }
-            pw[4 * ch + x] = live ? exp2_h2(pack_half2(x0, x1)) : 0u;
         }
         const uint32_t s4 = hadd2_u(hadd2_u(pw[4 * ch], pw[4 * ch + 1]), hadd2_u(pw[4 * ch + 2], pw[4 * ch + 3]));
         ls += half_lo(s4) + half_hi(s4);
@@ -606,8 +617,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         for (int c = 0; c < D / 32; ++c) acc[c] += __ldg(zjh + static_cast<long long>(j) * D + t + 32 * c);
                     }
                 }
+                // every block selected: the unselected set is empty and its sum is
+                // exactly zero (so is the linear branch), not the rounding residue
+                // of Z minus all z_j
+                const bool none_left = a.topk >= a.Nk;
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) zu[g * D + t + 32 * c] = zs[t + 32 * c] - acc[c];
+                for (int c = 0; c < D / 32; ++c) zu[g * D + t + 32 * c] = none_left ? 0.f : zs[t + 32 * c] - acc[c];
             }
             __syncwarp();
             // the linear-branch denominators phi(q_r) . Zu_g(r) of the tile's 128 rows,
@@ -747,9 +762,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             } else {
                 uint32_t pwa[16], pwb[16];
                 const bool exact = e < n_exact;
-                ls = exact ? softmax_half<0, true>(sv, c, m_run, live, pwa) : softmax_half<0, false>(sv, c, m_run, live, pwa);
+                ls = exact ? softmax_half<0, true, PISA>(sv, c, m_run, live, pwa)
+                           : softmax_half<0, false, PISA>(sv, c, m_run, live, pwa);
                 tmem_st16(tl + h * 64, pwa);
-                ls += exact ? softmax_half<32, true>(sv, c, m_run, live, pwb) : softmax_half<32, false>(sv, c, m_run, live, pwb);
+                ls += exact ? softmax_half<32, true, PISA>(sv, c, m_run, live, pwb)
+                            : softmax_half<32, false, PISA>(sv, c, m_run, live, pwb);
                 tmem_st16(tl + h * 64 + 16, pwb);
             }
             tmem_st_wait();

@@ -320,6 +320,22 @@ __device__ __forceinline__ float half_hi(uint32_t w) {
 }
 
 // Two fp32 -> two e4m3 (round to nearest even, saturating to +-448), low byte = lo.
+// Packed pairs of fp32 (the f32x2 arithmetic of sm_100: two IEEE round-to-nearest
+// operations in one instruction).
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+
 // max(a, b, c) in one instruction (the three-input form of sm_100).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
     float r;

@@ -320,7 +320,9 @@ __global__ void __launch_bounds__(256, 2) kv_stats_kernel(KvStatsArgs a) {
 
 // H[bh] = sum over chunks of hpart (fixed order), stored transposed
 // (hsum[bh][e][c] = H[c][e]); Z[bh] = sum_j z_j.
-// grid (D*D/256 + 1, BH), 256 threads; the last x-block reduces Z.
+// grid (D*D/256 + 1, BH), 256 threads; the last x-block reduces Z: its eight
+// warps take interleaved blocks j, each thread four columns with independent
+// loads, and the eight partial sums are added in a fixed order.
 template <int D>
 __global__ void __launch_bounds__(256) h_reduce_kernel(const float* __restrict__ hpart,
                                                        const float* __restrict__ zj, int nchunk,
@@ -332,14 +334,32 @@ __global__ void __launch_bounds__(256) h_reduce_kernel(const float* __restrict__
         const int idx = blockIdx.x * 256 + threadIdx.x;
         const float* src = hpart + bh * nchunk * static_cast<long long>(D) * D + idx;
         float s = 0.f;
-        for (int c = 0; c < nchunk; ++c) s += src[static_cast<long long>(c) * D * D];
+#pragma unroll 8
+        for (int c = 0; c < nchunk; ++c) s += __ldg(src + static_cast<long long>(c) * D * D);
         const int c = idx / D, e = idx % D;
         hsum[bh * D * D + e * D + c] = s;
-    } else if (threadIdx.x < D) {
-        const float* src = zj + bh * static_cast<long long>(Nk) * D + threadIdx.x;
-        float s = 0.f;
-        for (int j = 0; j < Nk; ++j) s += src[static_cast<long long>(j) * D];
-        zsum[bh * D + threadIdx.x] = s;
+    } else {
+        __shared__ float zp[8][D];
+        constexpr int CPT = D / 32;                      // columns per thread
+        const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+        const float* src = zj + bh * static_cast<long long>(Nk) * D;
+        float acc[CPT];
+#pragma unroll
+        for (int x = 0; x < CPT; ++x) acc[x] = 0.f;
+#pragma unroll 4
+        for (int j = warp; j < Nk; j += 8) {
+#pragma unroll
+            for (int x = 0; x < CPT; ++x) acc[x] += __ldg(src + static_cast<long long>(j) * D + lane + 32 * x);
+        }
+#pragma unroll
+        for (int x = 0; x < CPT; ++x) zp[warp][lane + 32 * x] = acc[x];
+        __syncthreads();
+        if (threadIdx.x < D) {
+            float t = 0.f;
+#pragma unroll
+            for (int w = 0; w < 8; ++w) t += zp[w][threadIdx.x];
+            zsum[bh * D + threadIdx.x] = t;
+        }
     }
 }
 

@@ -75,9 +75,25 @@ __global__ void fold_w_kernel(const float* __restrict__ wq, const float* __restr
     for (int e = threadIdx.x; e < d; e += blockDim.x) {
         double s;
         if (wq && wk) {
+            // each thread streams its own row of W_k and the broadcast row c of
+            // W_q (16-byte loads when both bases allow it; rows are d*4 bytes
+            // apart, a multiple of 16); the sum runs over t in order
             s = 0.0;
-            for (int t = 0; t < d; ++t)
-                s += static_cast<double>(wq[c * d + t]) * static_cast<double>(wk[e * d + t]);
+            if (((reinterpret_cast<uintptr_t>(wq) | reinterpret_cast<uintptr_t>(wk)) & 15u) == 0) {
+                const float4* a4 = reinterpret_cast<const float4*>(wq + c * d);
+                const float4* b4 = reinterpret_cast<const float4*>(wk + e * d);
+#pragma unroll 8
+                for (int t4 = 0; t4 < d / 4; ++t4) {
+                    const float4 x = __ldg(a4 + t4), y = __ldg(b4 + t4);
+                    s += static_cast<double>(x.x) * static_cast<double>(y.x);
+                    s += static_cast<double>(x.y) * static_cast<double>(y.y);
+                    s += static_cast<double>(x.z) * static_cast<double>(y.z);
+                    s += static_cast<double>(x.w) * static_cast<double>(y.w);
+                }
+            } else {
+                for (int t = 0; t < d; ++t)
+                    s += static_cast<double>(wq[c * d + t]) * static_cast<double>(wk[e * d + t]);
+            }
         } else if (wq) {
             s = static_cast<double>(wq[c * d + e]);
         } else {
