@@ -13,31 +13,35 @@
 namespace sla {
 
 // ------------------------------------------------------------------ pooling
-// One CTA handles pooled blocks blk = blockIdx.x, blockIdx.x + gridDim.x, ...
-// of `rows` consecutive rows of x [nblk_total * rows, d] (bf16, d innermost).
+// One warp per pooled block: blocks blk = warp id, + total warps, ... of `rows`
+// consecutive rows of x [nblk_total * rows, d] (bf16, d innermost).  Lane l
+// reads 16-byte vector l % (d/8) of rows l / (d/8), + 32/(d/8), ... (unrolled,
+// independent loads), sums in fp64, and the lanes holding the same columns
+// are combined by shuffles; no block-level synchronisation.
 // out_mode 0: out[blk][c]  (row-major [BH*nblk, d])
 // out_mode 1: out[bh][c][j] with blk = bh*nblk_per_head + j (transposed per head)
 // The value written is the block mean, sum / rows (rows is a power of two, so
-// the division is exact).
+// the division is exact; fp64 sums of bf16 values are exact for any realistic
+// exponent spread, so the result does not depend on the order of the sum).
 template <int D>
-__global__ void __launch_bounds__(256) pool_mean_kernel(const __nv_bfloat16* __restrict__ x,
+__global__ void __launch_bounds__(256, 4) pool_mean_kernel(const __nv_bfloat16* __restrict__ x,
                                                         int rows, long long nblk_total,
                                                         int nblk_per_head, int out_mode,
                                                         double* __restrict__ out) {
     constexpr int VPR = D / 8;            // 16-byte vectors per row
-    constexpr int RPAR = 256 / VPR;       // rows processed in parallel
-    __shared__ double part[RPAR][D];
-    const int tid = threadIdx.x;
-    const int vec = tid % VPR;
-    const int rg = tid / VPR;
+    constexpr int RPL = 32 / VPR;         // rows covered by one warp-wide load
+    const int lane = threadIdx.x & 31;
+    const int vec = lane % VPR, rsub = lane / VPR;
+    const long long nw = static_cast<long long>(gridDim.x) * 8;
     const double inv = 1.0 / static_cast<double>(rows);
-    for (long long blk = blockIdx.x; blk < nblk_total; blk += gridDim.x) {
+    for (long long blk = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5); blk < nblk_total;
+         blk += nw) {
         const uint4* src = reinterpret_cast<const uint4*>(x + blk * rows * D);
         double acc[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[e] = 0.0;
-#pragma unroll 4
-        for (int r = rg; r < rows; r += RPAR) {
+#pragma unroll 16
+        for (int r = rsub; r < rows; r += RPL) {
             const uint4 u = __ldg(src + static_cast<long long>(r) * VPR + vec);
             const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -47,22 +51,22 @@ __global__ void __launch_bounds__(256) pool_mean_kernel(const __nv_bfloat16* __r
             }
         }
 #pragma unroll
-        for (int e = 0; e < 8; ++e) part[rg][vec * 8 + e] = acc[e];
-        __syncthreads();
-        if (tid < D) {
-            double s = 0.0;
-#pragma unroll 4
-            for (int g = 0; g < RPAR; ++g) s += part[g][tid];
-            s *= inv;
+        for (int o = VPR; o < 32; o <<= 1) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
+        }
+        if (rsub == 0) {
             if (out_mode == 0) {
-                out[blk * D + tid] = s;
+                double2* dst = reinterpret_cast<double2*>(out + blk * D + vec * 8);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) dst[e] = make_double2(acc[2 * e] * inv, acc[2 * e + 1] * inv);
             } else {
                 const long long bh = blk / nblk_per_head;
                 const long long j = blk % nblk_per_head;
-                out[(bh * D + tid) * nblk_per_head + j] = s;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) out[(bh * D + vec * 8 + e) * nblk_per_head + j] = acc[e] * inv;
             }
         }
-        __syncthreads();
     }
 }
 

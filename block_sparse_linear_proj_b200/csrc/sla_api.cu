@@ -215,7 +215,8 @@ int grid_blocks(long long n, int per_sm) {
 
 void launch_pool(const void* x, int rows, long long nblk_total, int nblk_per_head, int d,
                  int out_mode, double* out, cudaStream_t st) {
-    const int grid = grid_blocks(nblk_total, 8);
+    // one warp per pooled block, eight warps per CTA
+    const int grid = grid_blocks((nblk_total + 7) / 8, 8);
     const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
     Span sp(SLA_KERNEL_POOL, st);
     if (d == 128)
