@@ -11,7 +11,8 @@ Functions:
 * :func:`sla_forward`  -- sparse branch + ReLU linear branch + alpha combine
   (``fp8=True``: the sparse branch on E4M3-quantised Q, K, P, V)
 * :func:`e4m3`         -- the E4M3 conversion (round to nearest even, saturating)
-* :func:`pisa_forward` -- PISA exact-or-approximate zero-order forward
+* :func:`pisa_forward` -- PISA exact-or-approximate forward (zero-order terms,
+  optionally the global first-order correction)
 
 Inputs may be torch tensors (bf16 / fp32 / int32, on the CPU) or numpy arrays
 (bf16 given as uint16 bit patterns).
@@ -56,7 +57,7 @@ def _load():
             lib.oracle_route.restype = I
             lib.oracle_sla_forward.argtypes = [I] * 7 + [D] + [P] * 5 + [L, P, P, P, P, I, I]
             lib.oracle_sla_forward.restype = I
-            lib.oracle_pisa_forward.argtypes = [I] * 7 + [D] + [P] * 4 + [L, P, P, I]
+            lib.oracle_pisa_forward.argtypes = [I] * 7 + [D] + [P] * 4 + [L, P, P, I, I]
             lib.oracle_pisa_forward.restype = I
             lib.oracle_e4m3_array.argtypes = [P, P, L]
             lib.oracle_e4m3_array.restype = None
@@ -152,8 +153,9 @@ def sla_forward(q, k, v, alpha, lut, Bq, Bk, sm_scale=0.0, rows=None, branches=F
     return out.reshape(shape)
 
 
-def pisa_forward(q, k, v, lut, Bq, Bk, sm_scale=0.0, rows=None, threads=0):
-    """PISA zero-order exact-or-approximate forward on a given LUT."""
+def pisa_forward(q, k, v, lut, Bq, Bk, sm_scale=0.0, rows=None, threads=0, first_order=False):
+    """PISA exact-or-approximate forward on a given LUT: zero-order terms for the
+    unselected blocks, plus (first_order=True) the global first-order term."""
     qb, kb, vb = _bf16_bits(q), _bf16_bits(k), _bf16_bits(v)
     B, H, N, d = qb.shape
     lt = _np(lut, np.int32)
@@ -163,6 +165,6 @@ def pisa_forward(q, k, v, lut, Bq, Bk, sm_scale=0.0, rows=None, threads=0):
     out = np.zeros((n, d), dtype=np.float64)
     rc = _load().oracle_pisa_forward(B, H, N, d, Bq, Bk, topk, float(sm_scale), _ptr(qb),
                                      _ptr(kb), _ptr(vb), _ptr(lt), nr, _ptr(r), _ptr(out),
-                                     threads)
+                                     1 if first_order else 0, threads)
     _check(rc, "pisa_forward")
     return out.reshape((B, H, N, d) if r is None else (n, d))

@@ -505,11 +505,16 @@ int oracle_sla_forward(int B, int H, int N, int d, int Bq, int Bk, int topk, dou
  * the maximum over all exact and centroid logits.  The D_t term is the sum
  * over the block's Bk keys of the zero-order expansion e^{q kbar}; its
  * first-order part vanishes because sum_n (k_n - kbar) = 0.  The global
- * first-order correction (the third N_t term) is not part of this mode. */
+ * first_order != 0 adds the global first-order correction, the third N_t term:
+ *   + tau (q_t Hbar) sum_{j in U_i} e^{cbar_tj - m},
+ *   Hbar = (1/Nk) sum_j H_j,  H_j = sum_{n in j} (k_n - kbar_j)^T v_n,
+ * the mean of the blocks' first-order matrices (the Taylor term of e^{tau q.k_n}
+ * around kbar_j is tau e^{tau q.kbar_j} q.(k_n - kbar_j)); D_t has no first-order
+ * part. */
 int oracle_pisa_forward(int B, int H, int N, int d, int Bq, int Bk, int topk, double sm_scale,
                         const uint16_t *q, const uint16_t *k, const uint16_t *v,
                         const int32_t *lut, int64_t nrows, const int64_t *rows,
-                        double *out, int nthreads)
+                        double *out, int first_order, int nthreads)
 {
     if (!check_shape(B, H, N, d, Bq, Bk, topk) || !q || !k || !v || !lut || !out)
         return ORC_EINVAL;
@@ -526,7 +531,8 @@ int oracle_pisa_forward(int B, int H, int N, int d, int Bq, int Bk, int topk, do
         if (req[a].row < 0 || req[a].row >= total) { free(req); return ORC_EINVAL; }
     double *kbar = malloc(sizeof(double) * (size_t)Nk * d);
     double *vsum = malloc(sizeof(double) * (size_t)Nk * d);
-    if (!kbar || !vsum) { free(req); free(kbar); free(vsum); return ORC_ENOMEM; }
+    double *hbar = malloc(sizeof(double) * (size_t)d * d);
+    if (!kbar || !vsum || !hbar) { free(req); free(kbar); free(vsum); free(hbar); return ORC_ENOMEM; }
     int err = ORC_OK;
 
     int64_t a0 = 0;
@@ -544,6 +550,20 @@ int oracle_pisa_forward(int B, int H, int N, int d, int Bq, int Bk, int topk, do
                 for (int r = 0; r < Bk; ++r) acc += bf(vh[((size_t)j * Bk + r) * d + c]);
                 vsum[(size_t)j * d + c] = acc;
             }
+        if (first_order) {
+            /* Hbar = (1/Nk) sum_j H_j, H_j = sum_{n in j} (k_n - kbar_j)^T v_n ([PISA]
+             * sec. 2: the mean of the blocks' first-order matrices over all blocks) */
+            memset(hbar, 0, sizeof(double) * (size_t)d * d);
+            for (int j = 0; j < Nk; ++j)
+                for (int r = 0; r < Bk; ++r) {
+                    const size_t nn = (size_t)j * Bk + r;
+                    for (int c = 0; c < d; ++c) {
+                        const double dk = bf(kh[nn * d + c]) - kbar[(size_t)j * d + c];
+                        for (int e = 0; e < d; ++e) hbar[(size_t)c * d + e] += dk * bf(vh[nn * d + e]);
+                    }
+                }
+            for (size_t c = 0; c < (size_t)d * d; ++c) hbar[c] /= (double)Nk;
+        }
 
 #pragma omp parallel for schedule(dynamic, 4)
         for (int64_t a = a0; a < a1; ++a) {
@@ -589,11 +609,22 @@ int oracle_pisa_forward(int B, int H, int N, int d, int Bq, int Bk, int topk, do
                     den += w;
                     for (int c = 0; c < d; ++c) num[c] += w * bf(vh[nn * d + c]);
                 }
+            double wu = 0.0;      /* sum over U of e^{tau q.kbar_j - m} */
             for (int j = 0; j < Nk; ++j) {
                 if (selected[j]) continue;
                 double w = exp(cb[j] - m);
+                wu += w;
                 den += (double)Bk * w;
                 for (int c = 0; c < d; ++c) num[c] += w * vsum[(size_t)j * d + c];
+            }
+            if (first_order && wu > 0.0) {
+                /* global first-order term: tau (q_t Hbar) sum_{j in U} e^{tau q.kbar_j - m}
+                 * (the derivative of e^{tau q.k} at kbar_j is tau e^{tau q.kbar_j} q) */
+                for (int e = 0; e < d; ++e) {
+                    double qh_e = 0.0;
+                    for (int c = 0; c < d; ++c) qh_e += qd[c] * hbar[(size_t)c * d + e];
+                    num[e] += tau * qh_e * wu;
+                }
             }
             for (int c = 0; c < d; ++c) o[c] = num[c] / den;
             free(selected); free(ex); free(cb); free(qd);
@@ -601,6 +632,6 @@ int oracle_pisa_forward(int B, int H, int N, int d, int Bq, int Bk, int topk, do
         if (err) break;
         a0 = a1;
     }
-    free(kbar); free(vsum); free(req);
+    free(kbar); free(vsum); free(hbar); free(req);
     return err;
 }

@@ -553,3 +553,51 @@ def test_fp8_mode_requires_64_token_blocks():
     lut, _ = orc.route(inp["q"], inp["k"], None, None, 64, 32, 2)
     with pytest.raises(ValueError):
         orc.sla_forward(inp["q"], inp["k"], inp["v"], inp["alpha"], lut, 64, 32, fp8=True)
+
+
+# ---------------------------------------------------------------- PISA first-order term
+
+def test_pisa_first_order_vanishes_for_block_constant_keys():
+    """Block-constant keys give H_j = 0, hence Hbar = 0: the first-order mode
+    equals the zero-order mode, which is exact (dense attention)."""
+    N, d, Bq, k = 512, 32, 64, 3
+    g = torch.Generator().manual_seed(17)
+    kb = torch.randn(1, 2, N // 64, 1, d, generator=g)
+    kk = kb.expand(1, 2, N // 64, 64, d).reshape(1, 2, N, d).to(torch.bfloat16)
+    q = torch.randn(1, 2, N, d, generator=g).to(torch.bfloat16)
+    v = torch.randn(1, 2, N, d, generator=g).to(torch.bfloat16)
+    lut = random_lut(1, 2, N // Bq, N // 64, k, 4)
+    a = orc.pisa_forward(q, kk, v, lut, Bq, 64, first_order=True)
+    b = orc.pisa_forward(q, kk, v, lut, Bq, 64)
+    assert np.abs(a - b).max() <= 1e-12 * np.abs(b).max()
+    assert np.abs(a - dense_sdpa(q, kk, v)).max() <= 1e-10
+
+
+def test_pisa_first_order_error_is_second_order():
+    """Keys = centroid + eps * delta with the same zero-mean delta pattern and the
+    same values in every block, so every block's first-order matrix H_j equals
+    Hbar.  Against dense attention the zero-order error is O(eps) (halving eps
+    halves it) and the first-order-corrected error is O(eps^2) (halving eps
+    quarters it), and smaller.  All inputs are exact in bf16."""
+    N, d, B_, k = 256, 16, 32, 2
+    g = torch.Generator().manual_seed(6)
+    base = (torch.randint(-6, 7, (1, 1, N // B_, 1, d), generator=g) / 8.0)
+    base = base.expand(1, 1, N // B_, B_, d).reshape(1, 1, N, d)
+    sign = torch.randint(0, 2, (1, 1, 1, B_ // 2, d), generator=g) * 2.0 - 1.0
+    delta = torch.cat([sign, -sign], 3).expand(1, 1, N // B_, B_, d).reshape(1, 1, N, d)
+    q = (torch.randint(-8, 9, (1, 1, N, d), generator=g) / 4.0).to(torch.bfloat16)
+    vb = torch.randn(1, 1, 1, B_, d, generator=g)
+    v = vb.expand(1, 1, N // B_, B_, d).reshape(1, 1, N, d).to(torch.bfloat16)
+    lut = random_lut(1, 1, N // B_, N // B_, k, 13)
+    e0, e1 = [], []
+    for e in (2.0 ** -4, 2.0 ** -5, 2.0 ** -6):
+        kk = (base + e * delta).to(torch.bfloat16)
+        assert torch.equal(kk.double(), (base + e * delta).double())
+        dense = dense_sdpa(q, kk, v)
+        e0.append(np.abs(orc.pisa_forward(q, kk, v, lut, B_, B_) - dense).max())
+        e1.append(np.abs(orc.pisa_forward(q, kk, v, lut, B_, B_, first_order=True) - dense).max())
+    for a, b in zip(e0, e0[1:]):
+        assert 1.6 < a / b < 2.5, e0
+    for a, b in zip(e1, e1[1:]):
+        assert 3.2 < a / b < 5.0, e1
+    assert all(x1 < 0.5 * x0 for x0, x1 in zip(e0, e1)), (e0, e1)
