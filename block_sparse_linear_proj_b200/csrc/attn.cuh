@@ -77,6 +77,11 @@ struct AttnArgs {
     const float* sv;               // FP8: [BH][Nk]  V block scales
     unsigned long long wait_ns;
     int debug_stall;               // test hook: load no K/V tiles, so the consumers' waits run out
+    // PISA global first-order term: + fo_scale * (sum of the centroid P) * (q . Hsum)
+    // with Hsum = sum_j H_j stored transposed [BH][D][D], fo_scale = tau / (Nk * Bk)
+    int first_order;
+    const float* hbar;
+    float fo_scale;
 };
 
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -198,8 +203,9 @@ struct AttnLayout {
     static constexpr int GRMAX = D == 128 ? 1 : 2;    // query blocks per CTA (SLA mode)
     static constexpr int BBUF = D * D * 2;            // one (H - G) hi or lo buffer
     static constexpr int BBOX = D * 128;              // one 64-column box of it
-    // epilogue buffers reuse the rings: (H - G) hi/lo, then the output staging
-    static constexpr int OUT_OFF = OFF_K + (PISA ? 0 : 2 * GRMAX * BBUF);
+    // epilogue buffers reuse the rings: (H - G) hi/lo (PISA: Hsum hi/lo for the
+    // first-order term), then the output staging
+    static constexpr int OUT_OFF = OFF_K + 2 * (PISA ? 1 : GRMAX) * BBUF;
     static_assert(OUT_OFF + D * 4 * 128 <= OFF_Q8, "epilogue buffers fit in the K/V rings");
 };
 
@@ -571,13 +577,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             }
             if (!ok) fail();
             umma_commit(final_bar);
-            if (SLA && ok) {
-                // linear branch: D_lin_g = phi(Q) (H - G_g), hi + lo, into G_g's columns;
-                // phi(Q) was written over the query tile in shared memory
+            if ((SLA || a.first_order) && ok) {
+                // SLA linear branch: D_lin_g = phi(Q) (H - G_g), hi + lo, into G_g's
+                // columns (phi(Q) was written over the query tile in shared memory).
+                // PISA first-order term: Q Hsum, hi + lo, into the same columns.
                 if (mbar_wait(epi_ready, 0, abort_flag, lim)) {
                     tc_fence_after();
                     constexpr uint32_t ID_L = idesc_bf16(128, D, 0, 1);
-                    for (int g = 0; g < n_groups; ++g) {
+                    for (int g = 0; g < (SLA ? n_groups : 1); ++g) {
                         for (int part = 0; part < 2; ++part) {
                             const uint32_t bb = sbase + L::OFF_K + (2 * g + part) * L::BBUF;
 #pragma unroll
@@ -647,6 +654,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(epi_ready);
+        } else if (a.first_order && lane == 0) {
+            mbar_arrive(epi_ready);
         }
     } else {
         // ======================================================== softmax + epilogue
@@ -664,6 +673,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         };
         const float c = a.scale_log2;
         float m_run = -INFINITY, l_run = 0.f;          // this warpgroup's running max (log2 units) and sum
+        float lc_run = 0.f;                            // PISA: the centroid pseudo-tiles' part of l_run
         bool ok = true;
         if (SLA) {
             // G_g := H (row r = c of the d x d matrix, this warpgroup's half of the
@@ -746,6 +756,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 }
                 tmem_st_wait();
                 l_run *= f;
+                lc_run *= f;
             }
             m_run = m_new;
             // P = 2^(x - m) over the 64 keys, written over the first columns of S
@@ -771,6 +782,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             }
             tmem_st_wait();
             l_run += ls;
+            if (PISA && e >= n_exact) lc_run += ls;
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_full[h]);
@@ -781,6 +793,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // merge the two warpgroups' partial softmaxes (exchanged once through shared memory)
         xm[h * 128 + r] = m_run;
         xl[h * 128 + r] = l_run;
+        if (PISA) xd[h * 128 + r] = lc_run;
         __syncwarp();
         if (lane == 0) mbar_arrive(&xl_bar[q4]);
         const bool xok = wwait(&xl_bar[q4], 0);
@@ -793,6 +806,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             if (m1 != -INFINITY) f1 = FP8 ? exp2_int(m1 - mm) : fast_exp2(m1 - mm);
             l_tot = f0 * xl[r] + f1 * xl[128 + r];
         }
+        // PISA: the centroid part of the row sum (= Bk * sum over U of e^{tau q.kbar_j - m})
+        const float lc_tot = (PISA && xok) ? f0 * xd[r] + f1 * xd[128 + r] : 0.f;
         const bool fin = ok && xok && wwait(final_bar, 0);
         if (ok && xok && !fin) fail();
         tc_fence_after();
@@ -811,7 +826,56 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 res[x] = ((have0 ? f0 * __uint_as_float(o0[x]) : 0.f) +
                           (have1 ? f1 * __uint_as_float(o1[x]) : 0.f)) * inv_l;
         };
-        if (PISA) {
+        if (PISA && a.first_order) {
+            // global first-order term: + tau/(Nk Bk) * lc * (q . Hsum), with q . Hsum
+            // on the tensor core (Hsum as bf16 hi + lo, MN-major boxes like the SLA
+            // linear-branch operand; row r = c of Hsum, this warpgroup's columns)
+            if (fin && r < D) {
+                const float* hcol = a.hbar + static_cast<long long>(bh) * D * D + r;
+                unsigned char* bhi = smem + L::OFF_K;
+                unsigned char* blo = bhi + L::BBUF;
+#pragma unroll 1
+                for (int cc = h * HC; cc < (h + 1) * HC; cc += 8) {
+                    uint32_t hi4[4], lo4[4];
+#pragma unroll
+                    for (int y = 0; y < 4; ++y) {
+                        const float v0 = __ldg(hcol + static_cast<long long>(cc + 2 * y) * D);
+                        const float v1 = __ldg(hcol + static_cast<long long>(cc + 2 * y + 1) * D);
+                        hi4[y] = pack_bf16(v0, v1);
+                        lo4[y] = pack_bf16(v0 - bf16lo(hi4[y]), v1 - bf16hi(hi4[y]));
+                    }
+                    const uint32_t off = (cc >> 6) * L::BBOX + sw128(r, (cc & 63) >> 3);
+                    *reinterpret_cast<uint4*>(bhi + off) = make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]);
+                    *reinterpret_cast<uint4*>(blo + off) = make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]);
+                }
+            }
+            fence_proxy_async_smem();                      // Hsum -> the tensor core
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(epi_ready);
+            float res[HC];
+            if (fin) {
+#pragma unroll
+                for (int x = 0; x < HC / 32; ++x) o_sum(h * HC + 32 * x, *reinterpret_cast<float(*)[32]>(&res[32 * x]));
+            }
+            const bool fo = fin && wwait(epi_ready, 0) && wwait(lin_done, 0);
+            if (fin && !fo) fail();
+            tc_fence_after();
+            if (fo) {
+                const float w1 = a.fo_scale * lc_tot * inv_l;
+#pragma unroll
+                for (int x = 0; x < HC / 32; ++x) {
+                    const int cc = h * HC + 32 * x;
+                    uint32_t fv[32];
+                    tmem_ld32(tl + COL_G0 + cc, fv);
+                    tmem_ld_wait();
+                    float out32[32];
+#pragma unroll
+                    for (int y = 0; y < 32; ++y) out32[y] = res[32 * x + y] + w1 * __uint_as_float(fv[y]);
+                    stage_row32(smem + L::OUT_OFF, a.out_f32, r, cc, out32);
+                }
+            }
+        } else if (PISA) {
             if (fin) {
 #pragma unroll 1
                 for (int cc = h * HC; cc < (h + 1) * HC; cc += 32) {

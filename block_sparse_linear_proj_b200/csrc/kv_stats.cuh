@@ -77,6 +77,9 @@ struct KvStatsArgs {
     uint8_t* v8t;
     float* sk;                  // [BH][Nk]
     float* sv;                  // [BH][Nk]
+    // PISA first-order term: the product uses K centred by its block mean,
+    // (k_n - kbar_j), instead of phi(K), so hpart sums the blocks' H_j
+    int center;
 };
 
 // grid (nchunk, BH), 256 threads.
@@ -255,6 +258,24 @@ __global__ void __launch_bounds__(256, 2) kv_stats_kernel(KvStatsArgs a) {
             }
         }
 
+        // centred keys: this block's column means (from the column statistics
+        // above), for the two feature rows of each A fragment
+        float kb0[MT], kb1[MT];
+        if (a.center) {
+            __syncthreads();
+#pragma unroll
+            for (int i = 0; i < MT; ++i) {
+                const int c0 = m0 + i * 16 + (lane >> 2);
+                double s0 = 0.0, s1 = 0.0;
+#pragma unroll
+                for (int hh = 0; hh < HALVES; ++hh) {
+                    s0 += kpart[hh * D + c0];
+                    s1 += kpart[hh * D + c0 + 8];
+                }
+                kb0[i] = static_cast<float>(s0 * (1.0 / kKvTok));
+                kb1[i] = static_cast<float>(s1 * (1.0 / kKvTok));
+            }
+        }
         if (do_mma) {
 #pragma unroll
             for (int k0 = 0; k0 < kKvTok; k0 += 16) {
@@ -266,8 +287,17 @@ __global__ void __launch_bounds__(256, 2) kv_stats_kernel(KvStatsArgs a) {
                     const int c = m0 + i * 16 + (((lane >> 3) & 1) << 3);
                     ldsm_x4_trans(kt_s + kv_off<D>(n, c), afr[i][0], afr[i][1], afr[i][2],
                                   afr[i][3]);
+                    if (a.center) {
+                        // fragments 0, 2 hold feature row m + g, fragments 1, 3 row m + 8 + g
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) afr[i][e] = relu_bf16x2(afr[i][e]);
+                        for (int e = 0; e < 4; ++e) {
+                            const float kb = (e & 1) ? kb1[i] : kb0[i];
+                            afr[i][e] = pack_bf16(bf16lo(afr[i][e]) - kb, bf16hi(afr[i][e]) - kb);
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) afr[i][e] = relu_bf16x2(afr[i][e]);
+                    }
                 }
 #pragma unroll
                 for (int j = 0; j < NT; j += 2) {
@@ -338,7 +368,7 @@ __global__ void __launch_bounds__(256) h_reduce_kernel(const float* __restrict__
         for (int c = 0; c < nchunk; ++c) s += __ldg(src + static_cast<long long>(c) * D * D);
         const int c = idx / D, e = idx % D;
         hsum[bh * D * D + e * D + c] = s;
-    } else {
+    } else if (zj) {
         __shared__ float zp[8][D];
         constexpr int CPT = D / 32;                      // columns per thread
         const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;

@@ -35,6 +35,7 @@ sla_status_t check_params(const sla_params_t* p) {
     if (p->sparse_dtype != SLA_SPARSE_BF16 && p->sparse_dtype != SLA_SPARSE_FP8_E4M3)
         return SLA_ERR_INVALID_ARG;
     if (p->lut_mode != SLA_LUT_COMPUTE && p->lut_mode != SLA_LUT_GIVEN) return SLA_ERR_INVALID_ARG;
+    if (p->pisa_first_order != 0 && p->pisa_first_order != 1) return SLA_ERR_INVALID_ARG;
     if (p->out_dtype != SLA_OUT_BF16 && p->out_dtype != SLA_OUT_FP32) return SLA_ERR_INVALID_ARG;
     if (!(std::isfinite(p->sm_scale))) return SLA_ERR_INVALID_ARG;
     if (p->d != 64 && p->d != 128) return SLA_ERR_UNSUPPORTED;
@@ -281,7 +282,7 @@ sla_status_t run_router(const sla_params_t* p, const void* q, const void* k, con
 template <int D>
 sla_status_t launch_kv(const sla_params_t* p, const void* k, const void* v, void* ws, const Ws& w,
                        bool want_kbar, bool sla_stats, bool pisa_stats, cudaStream_t st,
-                       bool fp8 = false) {
+                       bool fp8 = false, bool first_order = false) {
     const int BH = p->B * p->H, Nk = p->N / p->Bk;
     sla::KvStatsArgs a{};
     a.k = static_cast<const __nv_bfloat16*>(k);
@@ -292,7 +293,8 @@ sla_status_t launch_kv(const sla_params_t* p, const void* k, const void* v, void
     a.nchunk = w.nchunk;
     a.kbarT = want_kbar ? at<double>(ws, w.kbarT) : nullptr;
     a.zj = sla_stats ? at<float>(ws, w.zj) : nullptr;
-    a.hpart = sla_stats ? at<float>(ws, w.hpart) : nullptr;
+    a.hpart = (sla_stats || first_order) ? at<float>(ws, w.hpart) : nullptr;
+    a.center = first_order ? 1 : 0;
     a.kc = pisa_stats ? at<__nv_bfloat16>(ws, w.kc) : nullptr;
     a.vbar = pisa_stats ? at<__half>(ws, w.vbar) : nullptr;
     a.v16 = at<__half>(ws, w.v16);
@@ -310,12 +312,13 @@ sla_status_t launch_kv(const sla_params_t* p, const void* k, const void* v, void
         Span sp(SLA_KERNEL_KV_STATS, st);
         kern<<<dim3(w.nchunk, BH), 256, smem, st>>>(a);
     }
-    if (sla_stats) {
+    if (sla_stats || first_order) {
+        // H (SLA) or the sum of the blocks' first-order matrices (PISA)
         constexpr int NHB = D * D / 256;
         Span sp(SLA_KERNEL_H_REDUCE, st);
         sla::h_reduce_kernel<D><<<dim3(NHB + 1, BH), 256, 0, st>>>(
-            at<float>(ws, w.hpart), at<float>(ws, w.zj), w.nchunk, Nk, at<float>(ws, w.hsum),
-            at<float>(ws, w.zsum));
+            at<float>(ws, w.hpart), sla_stats ? at<float>(ws, w.zj) : nullptr, w.nchunk, Nk,
+            at<float>(ws, w.hsum), at<float>(ws, w.zsum));
     }
     return launch_status();
 }
@@ -380,6 +383,9 @@ sla_status_t launch_attn(const sla_params_t* p, const void* q, const void* k, co
     a.sv = FP8 ? at<float>(ws, w.sv) : nullptr;
     a.wait_ns = wait_limit_ns();
     a.debug_stall = debug_stall() ? 1 : 0;
+    a.first_order = (PISA && p->pisa_first_order) ? 1 : 0;
+    a.hbar = a.first_order ? at<float>(ws, w.hsum) : nullptr;
+    a.fo_scale = tau / (static_cast<float>(Nk) * static_cast<float>(p->Bk));
     const int GR = a.GR;
     const int nwords = (Nk + 15) / 16;
     const int sched_cap = std::max(4, (std::min(Nk, GR * std::max(p->topk, 1)) + 3) & ~3);
@@ -540,8 +546,9 @@ sla_status_t sla_pisa_forward(const sla_params_t* p, const void* q, const void* 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const bool compute = p->lut_mode == SLA_LUT_COMPUTE;
     int32_t* lut_use = (compute && !lut) ? at<int32_t>(workspace, w.lut) : lut;
-    s = p->d == 128 ? launch_kv<128>(p, k, v, workspace, w, compute, false, true, st)
-                    : launch_kv<64>(p, k, v, workspace, w, compute, false, true, st);
+    const bool fo = p->pisa_first_order != 0;
+    s = p->d == 128 ? launch_kv<128>(p, k, v, workspace, w, compute, false, true, st, false, fo)
+                    : launch_kv<64>(p, k, v, workspace, w, compute, false, true, st, false, fo);
     if (s != SLA_OK) return s;
     if (compute && (s = run_router(p, q, k, w_q, w_k, lut_use, workspace, w, false, st))) return s;
     s = p->d == 128 ? launch_attn<128, sla::kModePisa>(p, q, k, v, nullptr, lut_use, out, workspace, w, st)

@@ -47,7 +47,7 @@ class SlaParams(ctypes.Structure):
                 ("d", ctypes.c_int32), ("Bq", ctypes.c_int32), ("Bk", ctypes.c_int32),
                 ("topk", ctypes.c_int32), ("sm_scale", ctypes.c_float),
                 ("sparse_dtype", ctypes.c_int32), ("lut_mode", ctypes.c_int32),
-                ("out_dtype", ctypes.c_int32)]
+                ("out_dtype", ctypes.c_int32), ("pisa_first_order", ctypes.c_int32)]
 
 
 class SlaError(RuntimeError):
@@ -99,9 +99,9 @@ def status_string(code: int) -> str:
 
 
 def params(B, H, N, d, Bq, Bk, topk, sm_scale=0.0, sparse_dtype=SLA_SPARSE_BF16,
-           lut_mode=SLA_LUT_COMPUTE, out_dtype=SLA_OUT_BF16) -> SlaParams:
+           lut_mode=SLA_LUT_COMPUTE, out_dtype=SLA_OUT_BF16, pisa_first_order=False) -> SlaParams:
     return SlaParams(B, H, N, d, Bq, Bk, topk, float(sm_scale), sparse_dtype, lut_mode,
-                     out_dtype)
+                     out_dtype, 1 if pisa_first_order else 0)
 
 
 def out_torch_dtype(p: SlaParams):

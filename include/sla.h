@@ -73,6 +73,8 @@ typedef struct sla_params {
                                 branch's tensor-core products                   */
     int32_t lut_mode;        /* sla_lut_mode_t                                  */
     int32_t out_dtype;       /* sla_out_dtype_t: element type of `out`          */
+    int32_t pisa_first_order;/* sla_pisa_forward: 1 adds the global first-order
+                                correction term, 0 keeps the zero-order terms  */
 } sla_params_t;
 
 /* Bytes of device workspace that sla_route, sla_forward and sla_pisa_forward
@@ -154,7 +156,12 @@ sla_status_t sla_forward(const sla_params_t *p, const void *q, const void *k, co
  *   N_t = sum_{j in S} sum_n e^{tau q.k_jn - m} v_jn + sum_{j not in S} e^{tau q.kbar_j - m} sum_n v_jn
  *   D_t = sum_{j in S} sum_n e^{tau q.k_jn - m}      + sum_{j not in S} Bk e^{tau q.kbar_j - m}
  * with kbar_j the mean key (centroid) of block j; both sums share one
- * online-softmax maximum m.  S comes from the router (LUT_COMPUTE; pass
+ * online-softmax maximum m.  p->pisa_first_order = 1 adds the global
+ * first-order correction to N_t ([PISA] sec. 2, the third numerator term):
+ *   + tau (q_t Hbar) sum_{j not in S} e^{tau q.kbar_j - m},
+ *   Hbar = (1/Nk) sum_j sum_{n in j} (k_n - kbar_j)^T v_n,
+ * the mean over all blocks of the blocks' first-order matrices (D_t has no
+ * first-order part).  S comes from the router (LUT_COMPUTE; pass
  * w_q = w_k = NULL for PISA's plain pooled score) or from `lut` (LUT_GIVEN).
  * Requires Bq == Bk and sparse_dtype = BF16.
  */
