@@ -124,7 +124,8 @@ def _oracle_forward(w, inp, heads, rows, threads):
     lut, _ = orc.route(q, k, inp["w_q"], inp["w_k"], w.Bq, w.Bk, w.topk, threads=threads)
     t1 = time.perf_counter()
     if w.mode == "pisa":
-        orc.pisa_forward(q, k, v, lut, w.Bq, w.Bk, rows=rows, threads=threads)
+        orc.pisa_forward(q, k, v, lut, w.Bq, w.Bk, rows=rows, threads=threads,
+                         first_order=w.first_order)
     else:
         orc.sla_forward(q, k, v, inp["alpha"][:, hs], lut, w.Bq, w.Bk, rows=rows, threads=threads,
                         fp8=w.sparse_dtype == W.SPARSE_FP8_E4M3)
@@ -198,7 +199,7 @@ def run_reference(args, w, rank):
 def config_of(w, world):
     in_bytes = 3 * w.B * w.H * w.N * w.d * 2
     return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "Bq": w.Bq, "Bk": w.Bk,
-            "topk": w.topk, "mode": w.mode,
+            "topk": w.topk, "mode": w.mode + ("+first_order" if w.first_order else ""),
             "sparse_dtype": "e4m3" if w.sparse_dtype == W.SPARSE_FP8_E4M3 else "bf16",
             "global_batch": w.B * world, "seq_len": w.N, "parallelism": "replicas%d" % world,
             "l2": "inputs exceed L2 (%d MB of Q, K, V > 126 MB)" % (in_bytes // 10**6)
@@ -255,7 +256,8 @@ def run_ours(args, w, rank, world, local_rank):
     peaks = load_peaks()
     inp = W.make_inputs(w)
     g = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
-    p = S.params(w.B, w.H, w.N, w.d, w.Bq, w.Bk, w.topk, sparse_dtype=w.sparse_dtype)
+    p = S.params(w.B, w.H, w.N, w.d, w.Bq, w.Bk, w.topk, sparse_dtype=w.sparse_dtype,
+                 pisa_first_order=w.first_order)
     ws = S.workspace(p, device=dev)
     lut = torch.empty((w.B, w.H, w.Nq, w.topk), dtype=torch.int32, device=dev)
     out = torch.empty_like(g["q"])

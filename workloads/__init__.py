@@ -52,6 +52,7 @@ class Workload:
     grid: Optional[tuple] = None   # (T, Y, X) latent grid for the video generator
     alpha_range: Optional[tuple] = (0.0, 1.0)
     use_w: bool = True
+    first_order: bool = False     # PISA: add the global first-order term
 
     @property
     def Nq(self) -> int:
@@ -84,8 +85,11 @@ WORKLOADS = {
                          SPARSE_FP8_E4M3, "video", 1004, (21, 30, 52), (0.0, 1.0), True),
     "pisa": Workload("pisa", 1, 24, 32768, 128, 64, 64, 77, "pisa", SPARSE_BF16,
                      "video", 1005, (21, 30, 52), None, False),
+    # the PISA workload with the global first-order correction
+    "pisa_fo": Workload("pisa_fo", 1, 24, 32768, 128, 64, 64, 77, "pisa", SPARSE_BF16,
+                        "video", 1005, (21, 30, 52), None, False, True),
 }
-ORDER = ["tiny", "sla2_bf16", "sla2_long", "sla2_fp8", "pisa"]
+ORDER = ["tiny", "sla2_bf16", "sla2_long", "sla2_fp8", "pisa", "pisa_fo"]
 
 
 def _bf16(x: torch.Tensor) -> torch.Tensor:
