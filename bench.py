@@ -207,11 +207,25 @@ def config_of(w, world):
             "out_dtype": "bf16", "lut_mode": "compute"}
 
 
+def kernel_code_hash():
+    """sha256 of the attention kernel's code (attn.cuh + common.cuh) with comments
+    and blank space removed, so that only a change of code invalidates a capture."""
+    import hashlib
+    import re
+    h = hashlib.sha256()
+    for name in ("attn.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "block_sparse_linear_proj_b200", "csrc", name)) as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        h.update(" ".join(text.split()).encode())
+    return h.hexdigest()
+
+
 def ncu_traffic(w):
     """DRAM bytes per attention launch from the committed ncu summary of this
-    workload, if the attention kernel's source is unchanged since (its sha256
-    is recorded there); else None."""
-    import hashlib
+    workload, if the attention kernel's code is unchanged since (its hash is
+    recorded there); else None."""
     path = os.path.join(ROOT, "profiles", "attn_kernel_%s.md" % w.name)
     if not os.path.exists(path):
         return None
@@ -221,11 +235,7 @@ def ncu_traffic(w):
             if ":" in ln and ln.startswith("- "):
                 k, v = ln[2:].split(":", 1)
                 fields[k.strip()] = v.strip().strip("`")
-    h = hashlib.sha256()
-    for name in ("attn.cuh", "common.cuh"):
-        with open(os.path.join(ROOT, "block_sparse_linear_proj_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
-    if fields.get("kernel_source_sha256") != h.hexdigest():
+    if fields.get("kernel_code_sha256") != kernel_code_hash():
         return None
     try:
         return float(fields["dram_bytes_per_launch"])

@@ -3,40 +3,45 @@
 // One CTA owns up to 128 query rows = GR query blocks ("groups") of one head
 // (GR = 128/Bq, except the SLA mode with d = 128, where GR = 1 so that the
 // per-group G accumulators fit in tensor memory).  It walks the union of its
-// groups' selected KV blocks in ascending order (each entry tagged with the
-// groups that selected it) and, in PISA mode, then the head's centroid
-// pseudo-tiles.  Q and P live in tensor memory (A operands of the MMAs), so
-// shared memory only carries the K/V tiles.  Per entry:
-//   S  = Q K_j^T                        tcgen05.mma M=128 N=64, A from TMEM -> TMEM (2 buffers)
-//   P  = 2^(S*tau*log2e - m)            softmax warps, one row per thread,
-//                                       online max with lazy rescale of O;
-//                                       packed fp16 exp2, P written to TMEM
-//   O += P V_j                          tcgen05.mma M=128 N=d, A from TMEM (fp16 V copy)
-//   G_g += phi(K_j)^T V_j  (SLA only)   tcgen05.mma M=128 N=d   -> TMEM, per group
-//                                       (fp16 phi(K) copy from the K/V pre-pass)
+// groups' selected KV blocks (each entry tagged with the groups that selected
+// it; the walk starts at a per-tile rotation of the ascending order) and, in
+// PISA mode, then the head's centroid pseudo-tiles.  The query tile stays in
+// shared memory; tensor memory holds S_0 | S_1 | O_0 | O_1 | G.  Entry e goes
+// to softmax warpgroup h = e % 2, which owns S buffer h, accumulator O_h and
+// its own running maximum and row sum:
+//   S  = Q K_e^T                        tcgen05.mma M=128 N=64, A and B from shared memory
+//   P  = 2^(S*tau*log2e - m_h)          warpgroup h, one row per thread, online max with
+//                                       lazy rescale of O_h; packed fp16 exp2 (e4m3 in
+//                                       FP8 mode), written over the first columns of S_h
+//   O_h += P V_e                        tcgen05.mma M=128 N=d, A (P) from tensor memory
+//   G_g -= phi(K_e)^T V_e  (SLA only)   tcgen05.mma M=128 N=d, per group; G_g starts as H
+// S(e) is issued only after P.V(e-2) has completed (P(e-2) sits in S buffer h),
+// so each softmax step waits on one barrier and O_h needs no extra wait before
+// a rescale.  The epilogue merges the two partial softmaxes per row.
 // Linear branch (SALAD ReLU kernel; SLA2 combine): after the loop,
 //   O_l = phi(Q) (H - G_g) / (phi(q) . (Z - sum_{j in S_g} z_j))
-// with (H - G_g) split into bf16 hi + lo and multiplied on the tensor core,
-// then out = alpha O_s + (1 - alpha) O_l.
+// with (H - G_g) split into bf16 hi + lo and multiplied on the tensor core
+// (phi(Q) formed over the query tile in shared memory), then
+// out = alpha O_s + (1 - alpha) O_l.
 // PISA (zero-order "exact-or-approximate"): a centroid pseudo-tile holds 64
 // block centroids kbar_j and value means vbar_j; its logits get + log2(Bk)
 // (the block multiplicity) and the groups' own selected blocks are masked, so
 // e^{q.kbar_j - m} (sum_n v_n) enters N_t and Bk e^{q.kbar_j - m} enters D_t in
-// the same online softmax; out = N_t / D_t.
+// the same online softmax; out = N_t / D_t.  With the global first-order term,
+// tau (q . Hbar) sum_U e^{q.kbar_j - m} is added to N_t in the epilogue (q . Hbar
+// on the tensor core, the centroid sum tracked next to the row sum).
 //
 // K tiles and V (+ phi(K)) tiles stream through two separate rings: a K slot is
-// released as soon as S of its block completes, so K loads run several blocks
-// ahead of the P.V / G products.
-// Warp roles (384 threads): w0 TMA producer for both rings, w1 issues S = Q K^T
-// (and owns TMEM), w3 issues P.V, phi(K)^T V and the linear-branch products (two
-// issuers, so one's barrier waits overlap the other's MMAs: an MMA issue blocks
-// until the tensor pipe takes it), w2 the per-group sums of z_j over the
-// selected blocks (SLA), w4-11 softmax
-// and epilogue: two warpgroups, each thread owning one row (its TMEM lane) and
-// one half of the columns (exp2 and P for 32 of the 64 keys of a block; the
-// row maximum is taken over all 64 by both, so no exchange per block).  Every
-// wait is bounded; a wait that runs out sets the device status word and the
-// CTA unwinds after draining its own TMA loads and MMAs.
+// released as soon as S of its block completes, so K loads run ahead of the
+// P.V / G products.
+// Warp roles (384 threads): w0 TMA producer for both rings (thread 0 also starts
+// the query-tile load at set-up), w1 issues S = Q K^T (and owns TMEM), w3 issues
+// P.V, the G updates and the epilogue products (two issuers, so one's barrier
+// waits overlap the other's MMAs: an MMA issue blocks until the tensor pipe
+// takes it), w2 the per-group sums of z_j and the linear-branch denominators
+// (SLA), w4-11 the two softmax warpgroups and the epilogue.  Every wait is
+// bounded; a wait that runs out sets the device status word and the CTA
+// unwinds after draining its own TMA loads and MMAs.
 #pragma once
 #include "common.cuh"
 
