@@ -262,7 +262,7 @@ sla_status_t launch_score(const double* qbar, const double* kbarT, const double*
 // Router: Q/K pooling (unless already pooled), W folding, fp64 score + top-k.
 sla_status_t run_router(const sla_params_t* p, const void* q, const void* k, const float* w_q,
                         const float* w_k, int32_t* lut, void* ws, const Ws& w, bool pool_k,
-                        cudaStream_t st) {
+                        cudaStream_t st, cudaEvent_t kbar_ready = nullptr) {
     const int BH = p->B * p->H, Nq = p->N / p->Bq, Nk = p->N / p->Bk, d = p->d;
     double* qbar = at<double>(ws, w.qbar);
     double* kbarT = at<double>(ws, w.kbarT);
@@ -275,6 +275,8 @@ sla_status_t run_router(const sla_params_t* p, const void* q, const void* k, con
         m = at<double>(ws, w.m);
     }
     if (launch_status() != SLA_OK) return SLA_ERR_CUDA;
+    // the pooled K means come from the K/V pre-pass when it runs on the side stream
+    if (kbar_ready && cudaStreamWaitEvent(st, kbar_ready, 0) != cudaSuccess) return SLA_ERR_CUDA;
     if (d == 128) return launch_score<128>(qbar, kbarT, m, BH, Nq, Nk, p->topk, lut, st);
     return launch_score<64>(qbar, kbarT, m, BH, Nq, Nk, p->topk, lut, st);
 }
@@ -282,7 +284,7 @@ sla_status_t run_router(const sla_params_t* p, const void* q, const void* k, con
 template <int D>
 sla_status_t launch_kv(const sla_params_t* p, const void* k, const void* v, void* ws, const Ws& w,
                        bool want_kbar, bool sla_stats, bool pisa_stats, cudaStream_t st,
-                       bool fp8 = false, bool first_order = false) {
+                       bool fp8 = false, bool first_order = false, cudaEvent_t after_stats = nullptr) {
     const int BH = p->B * p->H, Nk = p->N / p->Bk;
     sla::KvStatsArgs a{};
     a.k = static_cast<const __nv_bfloat16*>(k);
@@ -312,6 +314,7 @@ sla_status_t launch_kv(const sla_params_t* p, const void* k, const void* v, void
         Span sp(SLA_KERNEL_KV_STATS, st);
         kern<<<dim3(w.nchunk, BH), 256, smem, st>>>(a);
     }
+    if (after_stats && cudaEventRecord(after_stats, st) != cudaSuccess) return SLA_ERR_CUDA;
     if (sla_stats || first_order) {
         // H (SLA) or the sum of the blocks' first-order matrices (PISA)
         constexpr int NHB = D * D / 256;
@@ -490,6 +493,42 @@ sla_status_t sla_route(const sla_params_t* p, const void* q, const void* k, cons
     return finish(run_router(p, q, k, w_q, w_k, lut, workspace, w, true, st), st);
 }
 
+// ------------------------------------------------------------- side stream
+// The K/V pre-pass does not depend on the router's pooling of Q or on W folding,
+// so a forward call runs it on a side stream of the library (one per device,
+// created on first use) between a fork and two join points on the caller's
+// stream: the router's score kernel waits for the pre-pass (it reads the pooled
+// K means the pre-pass writes), the attention kernel also for h_reduce.  The
+// caller sees ordinary stream order.  The enqueue sequence of a call holds a
+// per-device lock, so concurrent host threads never cross their events.  If the
+// side stream cannot be created, everything runs on the caller's stream.
+struct SideStream {
+    cudaStream_t s = nullptr;
+    cudaEvent_t fork = nullptr, kbar = nullptr, stats = nullptr;
+    bool ok = false;
+    std::mutex lock;
+};
+
+SideStream* side_stream() {
+    static SideStream side[64];
+    static std::mutex create;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    SideStream& x = side[dev];
+    std::lock_guard<std::mutex> g(create);
+    if (!x.ok) {
+        if (cudaStreamCreateWithFlags(&x.s, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+        if (cudaEventCreateWithFlags(&x.fork, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&x.kbar, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&x.stats, cudaEventDisableTiming) != cudaSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        x.ok = true;
+    }
+    return &x;
+}
+
 sla_status_t sla_forward(const sla_params_t* p, const void* q, const void* k, const void* v,
                          const float* alpha, const float* w_q, const float* w_k, int32_t* lut,
                          void* out, void* workspace, size_t ws_bytes, sla_stream_t stream) {
@@ -509,18 +548,34 @@ sla_status_t sla_forward(const sla_params_t* p, const void* q, const void* k, co
     const bool compute = p->lut_mode == SLA_LUT_COMPUTE;
     const bool fp8 = p->sparse_dtype == SLA_SPARSE_FP8_E4M3;
     int32_t* lut_use = (compute && !lut) ? at<int32_t>(workspace, w.lut) : lut;
-    s = p->d == 128 ? launch_kv<128>(p, k, v, workspace, w, compute, true, false, st, fp8)
-                    : launch_kv<64>(p, k, v, workspace, w, compute, true, false, st);
+    SideStream* side = side_stream();
+    std::unique_lock<std::mutex> hold;
+    cudaStream_t sst = st;                         // the pre-pass's stream
+    if (side) {
+        hold = std::unique_lock<std::mutex>(side->lock);
+        if (cudaEventRecord(side->fork, st) != cudaSuccess ||
+            cudaStreamWaitEvent(side->s, side->fork, 0) != cudaSuccess)
+            return SLA_ERR_CUDA;
+        sst = side->s;
+    }
+    s = p->d == 128 ? launch_kv<128>(p, k, v, workspace, w, compute, true, false, sst, fp8, false,
+                                     side ? side->kbar : nullptr)
+                    : launch_kv<64>(p, k, v, workspace, w, compute, true, false, sst, false, false,
+                                    side ? side->kbar : nullptr);
     if (s != SLA_OK) return s;
     if (fp8) {
         const long long nblk = static_cast<long long>(p->B) * p->H * p->N / 64;
-        Span sp(SLA_KERNEL_QUANT_Q, st);
-        sla::quant_q_kernel<128><<<grid_blocks(nblk, 8), 256, 0, st>>>(
+        Span sp(SLA_KERNEL_QUANT_Q, sst);
+        sla::quant_q_kernel<128><<<grid_blocks(nblk, 8), 256, 0, sst>>>(
             static_cast<const __nv_bfloat16*>(q), nblk, at<uint8_t>(workspace, w.q8),
             at<float>(workspace, w.sq));
         if (launch_status() != SLA_OK) return SLA_ERR_CUDA;
     }
-    if (compute && (s = run_router(p, q, k, w_q, w_k, lut_use, workspace, w, false, st))) return s;
+    if (side && cudaEventRecord(side->stats, sst) != cudaSuccess) return SLA_ERR_CUDA;
+    if (compute && (s = run_router(p, q, k, w_q, w_k, lut_use, workspace, w, false, st,
+                                   side ? side->kbar : nullptr)))
+        return s;
+    if (side && cudaStreamWaitEvent(st, side->stats, 0) != cudaSuccess) return SLA_ERR_CUDA;
     if (fp8)
         s = launch_attn<128, sla::kModeSlaFp8>(p, q, k, v, alpha, lut_use, out, workspace, w, st);
     else
@@ -547,10 +602,26 @@ sla_status_t sla_pisa_forward(const sla_params_t* p, const void* q, const void* 
     const bool compute = p->lut_mode == SLA_LUT_COMPUTE;
     int32_t* lut_use = (compute && !lut) ? at<int32_t>(workspace, w.lut) : lut;
     const bool fo = p->pisa_first_order != 0;
-    s = p->d == 128 ? launch_kv<128>(p, k, v, workspace, w, compute, false, true, st, false, fo)
-                    : launch_kv<64>(p, k, v, workspace, w, compute, false, true, st, false, fo);
+    SideStream* side = side_stream();
+    std::unique_lock<std::mutex> hold;
+    cudaStream_t sst = st;                         // the pre-pass's stream
+    if (side) {
+        hold = std::unique_lock<std::mutex>(side->lock);
+        if (cudaEventRecord(side->fork, st) != cudaSuccess ||
+            cudaStreamWaitEvent(side->s, side->fork, 0) != cudaSuccess)
+            return SLA_ERR_CUDA;
+        sst = side->s;
+    }
+    s = p->d == 128 ? launch_kv<128>(p, k, v, workspace, w, compute, false, true, sst, false, fo,
+                                     side ? side->kbar : nullptr)
+                    : launch_kv<64>(p, k, v, workspace, w, compute, false, true, sst, false, fo,
+                                    side ? side->kbar : nullptr);
     if (s != SLA_OK) return s;
-    if (compute && (s = run_router(p, q, k, w_q, w_k, lut_use, workspace, w, false, st))) return s;
+    if (side && cudaEventRecord(side->stats, sst) != cudaSuccess) return SLA_ERR_CUDA;
+    if (compute && (s = run_router(p, q, k, w_q, w_k, lut_use, workspace, w, false, st,
+                                   side ? side->kbar : nullptr)))
+        return s;
+    if (side && cudaStreamWaitEvent(st, side->stats, 0) != cudaSuccess) return SLA_ERR_CUDA;
     s = p->d == 128 ? launch_attn<128, sla::kModePisa>(p, q, k, v, nullptr, lut_use, out, workspace, w, st)
                     : launch_attn<64, sla::kModePisa>(p, q, k, v, nullptr, lut_use, out, workspace, w, st);
     return finish(s, st);
