@@ -24,7 +24,12 @@
  *    `workspace`, of at least sla_workspace_size() bytes, 256-byte aligned.
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
  *    default stream).  Arguments are validated on the host before anything is
- *    enqueued; on any error nothing is launched.
+ *    enqueued; on any error nothing is launched.  sla_forward and
+ *    sla_pisa_forward run their K/V pre-pass on a side stream owned by the
+ *    library (one per device, created with two events on first use; no device
+ *    memory), forked from and joined back into `stream` with events, so work
+ *    the caller enqueues on `stream` afterwards sees every result, and a
+ *    capture of `stream` includes that work.
  *  - Errors are returned, never thrown.  Kernel-side checks (an out-of-range
  *    or repeated entry in a caller-given LUT, a bounded wait that ran out)
  *    set a device status word that sla_check_device_status() reads.
