@@ -11,6 +11,7 @@ Functions:
 * :func:`sla_forward`  -- sparse branch + ReLU linear branch + alpha combine
   (``fp8=True``: the sparse branch on E4M3-quantised Q, K, P, V)
 * :func:`e4m3`         -- the E4M3 conversion (round to nearest even, saturating)
+* :func:`int8`         -- the symmetric 8-bit integer code (nearest, ties to even)
 * :func:`pisa_forward` -- PISA exact-or-approximate forward (zero-order terms,
   optionally the global first-order correction)
 
@@ -61,6 +62,8 @@ def _load():
             lib.oracle_pisa_forward.restype = I
             lib.oracle_e4m3_array.argtypes = [P, P, L]
             lib.oracle_e4m3_array.restype = None
+            lib.oracle_int8_array.argtypes = [P, P, L]
+            lib.oracle_int8_array.restype = None
             lib.oracle_max_threads.argtypes = []
             lib.oracle_max_threads.restype = I
             _lib = lib
@@ -127,12 +130,21 @@ def e4m3(x) -> np.ndarray:
     return out
 
 
+def int8(x) -> np.ndarray:
+    """8-bit integer codes of float64 values (nearest, ties to even, within +-127)."""
+    a = np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+    out = np.empty_like(a)
+    _load().oracle_int8_array(_ptr(a), _ptr(out), a.size)
+    return out
+
+
 def sla_forward(q, k, v, alpha, lut, Bq, Bk, sm_scale=0.0, rows=None, branches=False,
-                threads=0, fp8=False):
+                threads=0, fp8=False, int8=False):
     """SLA2 forward on a given LUT.  rows=None: every row, returns [B,H,N,d];
     else flat row indices, returns [len(rows), d].  branches=True also returns
     the sparse-branch and linear-branch outputs.  fp8=True: the sparse branch
-    on E4M3-quantised Q, K, P, V with per-64-token-block scales (Bk = 64)."""
+    on E4M3-quantised Q, K, P, V with per-64-token-block scales (Bk = 64).
+    int8=True: the same with 8-bit integer Q and K codes (P and V E4M3)."""
     qb, kb, vb = _bf16_bits(q), _bf16_bits(k), _bf16_bits(v)
     B, H, N, d = qb.shape
     al = _np(alpha, np.float32)
@@ -145,7 +157,7 @@ def sla_forward(q, k, v, alpha, lut, Bq, Bk, sm_scale=0.0, rows=None, branches=F
     ol_ = np.zeros((n, d), dtype=np.float64) if branches else None
     rc = _load().oracle_sla_forward(B, H, N, d, Bq, Bk, topk, float(sm_scale), _ptr(qb), _ptr(kb),
                                     _ptr(vb), _ptr(al), _ptr(lt), nr, _ptr(r), _ptr(out),
-                                    _ptr(os_), _ptr(ol_), 1 if fp8 else 0, threads)
+                                    _ptr(os_), _ptr(ol_), 2 if int8 else (1 if fp8 else 0), threads)
     _check(rc, "sla_forward")
     shape = (B, H, N, d) if r is None else (n, d)
     if branches:

@@ -104,6 +104,22 @@ void oracle_e4m3_array(const double *in, double *out, int64_t n)
     for (int64_t a = 0; a < n; ++a) out[a] = oracle_e4m3(in[a]);
 }
 
+/* Symmetric 8-bit integer code: the nearest integer (ties to even), clamped to
+ * [-127, 127]. */
+double oracle_int8(double x)
+{
+    if (x != x) return 0.0;
+    double r = nearbyint(x);
+    if (r > 127.0) r = 127.0;
+    if (r < -127.0) r = -127.0;
+    return r;
+}
+
+void oracle_int8_array(const double *in, double *out, int64_t n)
+{
+    for (int64_t a = 0; a < n; ++a) out[a] = oracle_int8(in[a]);
+}
+
 /* A LUT row must hold topk distinct block indices in [0, Nk). */
 static int lut_row_valid(const int32_t *row, int topk, int Nk)
 {
@@ -301,6 +317,11 @@ static rowreq_t *gather_rows(int64_t total, int64_t nrows, const int64_t *rows, 
  *     Phat_tn = e4m3(P_tn 448 s_v(j) / s_vmax), s_vmax = max over the LUT row;
  *     O_s(t) = (s_vmax / 448) sum_n Phat_tn v8_n / l_t.
  *   The linear branch and the combine are not quantised.
+ *   lowbit = 2 (INT8): as above, but Q and K take 8-bit integer codes,
+ *   s_b = max|x| / 127 and x8 = int8(x / s_b) (nearest, ties to even, within
+ *   +-127), so q8_t . k8_n is an exact integer; P and V keep the E4M3 rules
+ *   (an integer P.V accumulator could not take the online rescale exactly).
+ *   lowbit = 1 is the FP8 mode above; 0 is the unquantised branch.
  * rows: flat indices (b*H + h)*N + t (NULL = all rows, in order).
  * out, out_s, out_l: [nrows, d] (out_s, out_l may be NULL). */
 
@@ -309,17 +330,18 @@ static rowreq_t *gather_rows(int64_t total, int64_t nrows, const int64_t *rows, 
  * operations (correctly rounded), the precision the GPU path decides its codes
  * in; the pages fix no precision for them, and deciding a code in another
  * precision flips it whenever the quotient falls on a rounding midpoint. */
-static void quantise_blocks(const uint16_t *x, int N, int d, double *x8, double *scale)
+static void quantise_blocks(const uint16_t *x, int N, int d, double *x8, double *scale, int int8)
 {
+    const float top = int8 ? 127.0f : 448.0f;
     for (int b = 0; b < N / 64; ++b) {
         float amax = 0.0f;
         for (size_t e = (size_t)b * 64 * d; e < (size_t)(b + 1) * 64 * d; ++e)
             if (fabsf((float)bf(x[e])) > amax) amax = fabsf((float)bf(x[e]));
-        const float s = amax > 0.0f ? amax / 448.0f : 1.0f;
+        const float s = amax > 0.0f ? amax / top : 1.0f;
         scale[b] = (double)s;
         for (size_t e = (size_t)b * 64 * d; e < (size_t)(b + 1) * 64 * d; ++e) {
             const float quotient = (float)bf(x[e]) / s;
-            x8[e] = oracle_e4m3((double)quotient);
+            x8[e] = int8 ? oracle_int8((double)quotient) : oracle_e4m3((double)quotient);
         }
     }
 }
@@ -328,10 +350,12 @@ int oracle_sla_forward(int B, int H, int N, int d, int Bq, int Bk, int topk, dou
                        const uint16_t *q, const uint16_t *k, const uint16_t *v,
                        const float *alpha, const int32_t *lut,
                        int64_t nrows, const int64_t *rows,
-                       double *out, double *out_s, double *out_l, int fp8, int nthreads)
+                       double *out, double *out_s, double *out_l, int lowbit, int nthreads)
 {
     if (!check_shape(B, H, N, d, Bq, Bk, topk) || !q || !k || !v || !alpha || !lut || !out)
         return ORC_EINVAL;
+    if (lowbit < 0 || lowbit > 2) return ORC_EINVAL;
+    const int fp8 = lowbit != 0;                   /* some quantised sparse branch */
     if (fp8 && Bk != 64) return ORC_EINVAL;
     set_threads(nthreads);
     const int Nq = N / Bq, Nk = N / Bk;
@@ -371,9 +395,9 @@ int oracle_sla_forward(int B, int H, int N, int d, int Bq, int Bk, int topk, dou
         const uint16_t *vh = v + (size_t)bh * N * d;
         linear_block_stats(kh, vh, Nk, Bk, d, hj, zj);
         if (fp8) {
-            quantise_blocks(qh, N, d, q8, sq);
-            quantise_blocks(kh, N, d, k8, sk);
-            quantise_blocks(vh, N, d, v8, sv);
+            quantise_blocks(qh, N, d, q8, sq, lowbit == 2);
+            quantise_blocks(kh, N, d, k8, sk, lowbit == 2);
+            quantise_blocks(vh, N, d, v8, sv, 0);
         }
 
         /* distinct query blocks among the requested rows of this head */

@@ -601,3 +601,68 @@ def test_pisa_first_order_error_is_second_order():
     for a, b in zip(e1, e1[1:]):
         assert 3.2 < a / b < 5.0, e1
     assert all(x1 < 0.5 * x0 for x0, x1 in zip(e0, e1)), (e0, e1)
+
+
+# ---------------------------------------------------------------- INT8 Q/K codes
+
+def test_int8_codes_match_library_rounding():
+    """Nearest integer with ties to even (numpy's rint), clamped to +-127."""
+    rng = np.random.default_rng(9)
+    x = np.concatenate([rng.uniform(-140, 140, 100000), np.arange(-130, 131) + 0.5,
+                        np.array([127.4999, 127.5, -127.5, 0.0, -0.5])])
+    assert np.array_equal(orc.int8(x), np.clip(np.rint(x), -127, 127))
+
+
+def exact_int8_inputs(seed):
+    """Q entries are integers times 1/2 with a block absmax of 127/2 (scale 1/2),
+    K entries integers with a block absmax of 127 (scale 1): every code is exact,
+    q . k is an integer times 1/2, and with sm_scale = 2 ln 2 the logits in log2
+    units are integers.  V follows the exact E4M3 construction."""
+    q, k, v, alpha = exact_fp8_inputs(seed)
+    rng = np.random.default_rng(seed + 1000)
+    B, H, N, d = q.shape
+    qn = np.zeros((B, H, N, d))
+    kn = np.zeros((B, H, N, d))
+    for b in range(B):
+        for h in range(H):
+            for blk in range(N // 64):
+                for t in range(blk * 64, blk * 64 + 64):
+                    cq = rng.choice(np.arange(2, 10), 2, replace=False)
+                    qn[b, h, t, cq] = rng.choice([-1.0, 1.0, -2.0, 2.0], 2) * 0.5
+                    ck = rng.choice(np.arange(2, 10), 3, replace=False)
+                    kn[b, h, t, ck] = rng.choice([-1.0, 1.0], 3)
+                qn[b, h, blk * 64, 0] = 63.5
+                kn[b, h, blk * 64, 1] = 127.0
+    to = lambda x: torch.from_numpy(x).to(torch.bfloat16)
+    return to(qn), to(kn), v, alpha
+
+
+@pytest.mark.parametrize("topk", [1, 3, 8])
+def test_int8_mode_is_exact_when_every_quantisation_is_exact(topk):
+    q, k, v, alpha = exact_int8_inputs(21 + topk)
+    Bq, Bk = 128, 64
+    lut, _ = orc.route(q, k, None, None, Bq, Bk, topk)
+    sc = 2.0 * math.log(2.0)
+    o8, s8, l8 = orc.sla_forward(q, k, v, alpha, lut, Bq, Bk, sm_scale=sc, branches=True, int8=True)
+    o, s, l = orc.sla_forward(q, k, v, alpha, lut, Bq, Bk, sm_scale=sc, branches=True)
+    scale = np.abs(s).max()
+    assert np.abs(s8 - s).max() <= 1e-12 * scale
+    assert np.abs(o8 - o).max() <= 1e-12 * scale
+    # not degenerate: the logits of a query block's selected keys span several units
+    qd, kd = q.double().numpy()[0, 0], k.double().numpy()[0, 0]
+    keys = np.concatenate([np.arange(j * Bk, (j + 1) * Bk) for j in lut[0, 0, 1]])
+    assert np.ptp(qd[Bq:2 * Bq] @ kd[keys].T, axis=1).max() >= 2
+
+
+def test_int8_mode_error_is_below_fp8():
+    """Q, K as 8-bit integers keep more precision than E4M3, so on Gaussian inputs
+    the INT8 mode's distance from the exact branch is nonzero and below FP8's."""
+    inp = W.gaussian_inputs(1, 2, 1024, 128, 78)
+    lut, _ = orc.route(inp["q"], inp["k"], inp["w_q"], inp["w_k"], 128, 64, 6)
+    args = (inp["q"], inp["k"], inp["v"], inp["alpha"], lut, 128, 64)
+    _, s, _ = orc.sla_forward(*args, branches=True)
+    _, s8, _ = orc.sla_forward(*args, branches=True, fp8=True)
+    _, si, _ = orc.sla_forward(*args, branches=True, int8=True)
+    e8, ei = np.abs(s8 - s).mean(), np.abs(si - s).mean()
+    assert 0 < ei < 0.8 * e8, (ei, e8)
+    assert not np.array_equal(si, s8)
