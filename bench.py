@@ -128,7 +128,7 @@ def _oracle_forward(w, inp, heads, rows, threads):
                          first_order=w.first_order)
     else:
         orc.sla_forward(q, k, v, inp["alpha"][:, hs], lut, w.Bq, w.Bk, rows=rows, threads=threads,
-                        fp8=w.sparse_dtype == W.SPARSE_FP8_E4M3)
+                        fp8=w.sparse_dtype == W.SPARSE_FP8_E4M3, int8=w.sparse_dtype == W.SPARSE_INT8)
     return t1 - t0, time.perf_counter() - t1
 
 
@@ -196,11 +196,15 @@ def run_reference(args, w, rank):
     print(json.dumps(line), flush=True)
 
 
+# the sparse branch's arithmetic types: S = Q K^T, then P V
+SPARSE_TYPES = {W.SPARSE_BF16: "bf16", W.SPARSE_FP8_E4M3: "e4m3", W.SPARSE_INT8: "s8 QK^T, e4m3 PV"}
+
+
 def config_of(w, world):
     in_bytes = 3 * w.B * w.H * w.N * w.d * 2
     return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "Bq": w.Bq, "Bk": w.Bk,
             "topk": w.topk, "mode": w.mode + ("+first_order" if w.first_order else ""),
-            "sparse_dtype": "e4m3" if w.sparse_dtype == W.SPARSE_FP8_E4M3 else "bf16",
+            "sparse_dtype": SPARSE_TYPES[w.sparse_dtype],
             "global_batch": w.B * world, "seq_len": w.N, "parallelism": "replicas%d" % world,
             "l2": "inputs exceed L2 (%d MB of Q, K, V > 126 MB)" % (in_bytes // 10**6)
                   if in_bytes > 126 * 10**6 else "inputs fit in L2",
@@ -354,14 +358,15 @@ def run_ours(args, w, rank, world, local_rank):
     exec_flops = 4.0 * pairs * w.Bq * w.Bk * w.d
     g_flops = 2.0 * pairs * w.Bk * w.d * w.d if w.mode == "sla" else 0.0
     achieved = exec_flops / (attn_avg * 1e-3) / 1e12
-    fp8 = w.sparse_dtype == W.SPARSE_FP8_E4M3
+    fp8 = w.sparse_dtype in (W.SPARSE_FP8_E4M3, W.SPARSE_INT8)
     # the attention kernel runs back to back for the whole timed region: the
-    # sustained peak; FP8 takes the bf16 figure times the nominal ratio (2)
+    # sustained peak; FP8 and INT8 (both 4.5 P/s dense nominal) take the bf16
+    # figure times the nominal ratio (2)
     peak = peaks["bf16_tflops_sustained"] * (2.0 if fp8 else 1.0)
     kv_ms, kv_n = prof["kv_stats"]
     kv_avg = kv_ms / max(kv_n, 1)
     # read K and V (bf16); write fp16 V and fp16 phi(K) (SLA), the centroids (PISA),
-    # and e4m3 K and V (FP8)
+    # and 8-bit K and V (FP8, INT8)
     tok = w.B * w.H * w.N * w.d
     kv_bytes = tok * 2 * 2 + (tok * 2 * 2 if w.mode == "sla" else tok * 2) + (tok * 2 if fp8 else 0)
     pool_ms, pool_n = prof["pool"]
@@ -387,13 +392,13 @@ def run_ours(args, w, rank, world, local_rank):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_call, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if fp8 else "bf16",
+        "scaling": "weak", "vs_baseline": None, "dtype": SPARSE_TYPES[w.sparse_dtype],
         "data": "synthetic (seeded video-latent generator, no model weights)",
         "config": config_of(w, world),
         "ms_per_call": ms_per_call,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": ncu_traffic(w), "kernel": "attn",
-                     "peak_source": peaks["source"] + (" bf16 sustained x 2 (fp8)" if fp8
+                     "peak_source": peaks["source"] + (" bf16 sustained x 2 (8-bit)" if fp8
                                                        else " bf16 sustained"),
                      "algorithmic": "4*Bq*Bk*d per (query block, selected block) pair, %d pairs" % pairs},
         "kernels": kernels,

@@ -49,7 +49,7 @@ namespace sla {
 
 constexpr float kRescaleLog2 = 8.0f;    // lazy O rescale threshold (log2 units)
 
-enum : int { kModeSla = 0, kModePisa = 1, kModeSlaFp8 = 2 };
+enum : int { kModeSla = 0, kModePisa = 1, kModeSlaFp8 = 2, kModeSlaInt8 = 3 };
 
 // Tensor maps of one launch (see the host for shapes, boxes and swizzles).
 struct AttnMaps {
@@ -186,7 +186,9 @@ __device__ __forceinline__ void stage_row32(unsigned char* stage, int f32, int r
 
 template <int D, int MODE>
 struct AttnLayout {
-    static constexpr bool PISA = MODE == kModePisa, FP8 = MODE == kModeSlaFp8;
+    // INT8 shares every FP8 rule except the Q and K codes and the S product
+    static constexpr bool PISA = MODE == kModePisa, I8 = MODE == kModeSlaInt8;
+    static constexpr bool FP8 = MODE == kModeSlaFp8 || I8;
     static constexpr int KS = PISA ? (D == 128 ? 5 : 6) : (FP8 ? 6 : 4);   // K ring slots
     static constexpr int VS = PISA ? (D == 128 ? 5 : 6) : (D == 128 ? 3 : 4);  // V ring slots
     static constexpr int T16 = 64 * D * 2;            // one 64-token tile of 16-bit values
@@ -220,7 +222,7 @@ template <int D, int MODE>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_kernel(const __grid_constant__ AttnMaps tm, const AttnArgs a) {
     using L = AttnLayout<D, MODE>;
-    constexpr bool PISA = L::PISA, FP8 = L::FP8;
+    constexpr bool PISA = L::PISA, FP8 = L::FP8, I8 = L::I8;
     constexpr bool SLA = !PISA;
     constexpr int NBOX = D / 64;
     constexpr int KS = L::KS, VS = L::VS;
@@ -497,7 +499,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     } else if (warp == 1) {
         // ======================================================== S = Q K^T issuer
         if (lane == 0) {
-            constexpr uint32_t ID_S = FP8 ? idesc_e4m3(128, 64) : idesc_bf16(128, 64, 0, 0);
+            constexpr uint32_t ID_S = I8 ? idesc_s8(128, 64) : FP8 ? idesc_e4m3(128, 64) : idesc_bf16(128, 64, 0, 0);
             bool ok = mbar_wait(q_full, 0, abort_flag, lim);
             for (int e = 0; ok && e < n_total; ++e) {
                 // S(e) needs its K tile and its buffer back: P(e-2), written over
@@ -507,12 +509,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     (e >= 2 && !mbar_wait(&pv_done[b], ((e >> 1) - 1) & 1, abort_flag, lim))) { ok = false; break; }
                 tc_fence_after();
                 if (FP8) {
-                    // e4m3: 32 elements (32 bytes) per instruction
+                    // e4m3 (or s8, exact s32 sums): 32 elements (32 bytes) per instruction
 #pragma unroll
                     for (int kk = 0; kk < D / 32; ++kk) {
                         const uint64_t ad = sdesc(sbase + L::OFF_Q8 + kk * 32, 16, 1024, kSwizzle128B);
                         const uint64_t bd = sdesc(sK(s) + kk * 32, 16, 1024, kSwizzle128B);
-                        umma_f8_ss(tmem + b * 64, ad, bd, ID_S, kk > 0 ? 1u : 0u);
+                        if (I8)
+                            umma_i8_ss(tmem + b * 64, ad, bd, ID_S, kk > 0 ? 1u : 0u);
+                        else
+                            umma_f8_ss(tmem + b * 64, ad, bd, ID_S, kk > 0 ? 1u : 0u);
                     }
                 } else {
 #pragma unroll
@@ -714,6 +719,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             tmem_ld32(tl + h * 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
             tmem_ld32(tl + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
             tmem_ld_wait();
+            if (I8) {
+                // s32 scores, |S| <= 128 * 127^2 < 2^22: exact in fp32
+#pragma unroll
+                for (int j = 0; j < 64; ++j) sv[j] = __float_as_uint(small_int_to_float(sv[j]));
+            }
 
             // row maximum over the 64 logits (x = s * c, + log2 Bk for centroids;
             // masked ones are -inf)

@@ -180,6 +180,15 @@ __device__ __forceinline__ void umma_f8_ss(uint32_t d_tmem, uint64_t a_desc, uin
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// D(tmem) (+)= A(smem) * B(smem), signed 8-bit integer operands, s32 accumulation.
+__device__ __forceinline__ void umma_i8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
 // D(tmem) (+)= A(tmem) * B(smem), e4m3 operands (A packed four per 32-bit column).
 __device__ __forceinline__ void umma_f8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                            uint32_t idesc, uint32_t accumulate) {
@@ -291,6 +300,25 @@ __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int a_mn, int b_m
            (static_cast<uint32_t>(M >> 4) << 24);
 }
 // Instruction descriptor, kind::f8f6f4 with e4m3 A/B (both K-major), fp32 D.
+// kind::i8: D s32 (2), A and B signed 8-bit (1), both K-major.
+__host__ __device__ constexpr uint32_t idesc_s8(int M, int N) {
+    return (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+           (static_cast<uint32_t>(M >> 4) << 24);
+}
+// Four symmetric 8-bit integer codes (nearest, ties to even, within +-127), packed
+// little-endian into a 32-bit word.
+__device__ __forceinline__ uint32_t pack_s8x4(float a, float b, float c, float d) {
+    auto q = [](float x) {
+        const int r = max(-127, min(127, __float2int_rn(x)));
+        return static_cast<uint32_t>(r) & 0xFFu;
+    };
+    return q(a) | (q(b) << 8) | (q(c) << 16) | (q(d) << 24);
+}
+// An integer of magnitude below 2^22 as fp32, exactly: its bits added to those of
+// 1.5 * 2^23, then 1.5 * 2^23 subtracted (integer and fp32 add pipes only).
+__device__ __forceinline__ float small_int_to_float(uint32_t bits) {
+    return __int_as_float(static_cast<int>(bits) + 0x4B400000) - 12582912.0f;
+}
 __host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N) {
     return (1u << 4) | (0u << 7) | (0u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
            (static_cast<uint32_t>(M >> 4) << 24);

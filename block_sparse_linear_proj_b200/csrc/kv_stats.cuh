@@ -80,6 +80,8 @@ struct KvStatsArgs {
     // PISA first-order term: the product uses K centred by its block mean,
     // (k_n - kbar_j), instead of phi(K), so hpart sums the blocks' H_j
     int center;
+    // with k8: symmetric 8-bit integer K codes (absmax / 127) instead of e4m3
+    int k_int8;
 };
 
 // grid (nchunk, BH), 256 threads.
@@ -213,7 +215,8 @@ __global__ void __launch_bounds__(256, 2) kv_stats_kernel(KvStatsArgs a) {
             for (int w = 0; w < 8; ++w) { km = fmaxf(km, amax[w]); vm = fmaxf(vm, amax[8 + w]); }
             // codes are picked by the correctly rounded quotient x / s (not x * (1/s),
             // which lands on the other side of a rounding midpoint now and then)
-            const float s_k = km > 0.f ? km / 448.f : 1.f, s_v = vm > 0.f ? vm / 448.f : 1.f;
+            const float s_k = km > 0.f ? km / (a.k_int8 ? 127.f : 448.f) : 1.f;
+            const float s_v = vm > 0.f ? vm / 448.f : 1.f;
             const int j = jb0 + blk;
             if (tid == 0) {
                 a.sk[bh * a.Nk + j] = s_k;
@@ -225,8 +228,14 @@ __global__ void __launch_bounds__(256, 2) kv_stats_kernel(KvStatsArgs a) {
             for (int q = tid; q < kKvTok * CPR; q += 256) {
                 const int n = q / CPR, u = q % CPR;
                 const uint4 x = *reinterpret_cast<const uint4*>(kt + kv_off<D>(n, u * 8));
-                const uint32_t w0 = pack_e4m3x4(bf16lo(x.x) / s_k, bf16hi(x.x) / s_k, bf16lo(x.y) / s_k, bf16hi(x.y) / s_k);
-                const uint32_t w1 = pack_e4m3x4(bf16lo(x.z) / s_k, bf16hi(x.z) / s_k, bf16lo(x.w) / s_k, bf16hi(x.w) / s_k);
+                uint32_t w0, w1;
+                if (a.k_int8) {
+                    w0 = pack_s8x4(bf16lo(x.x) / s_k, bf16hi(x.x) / s_k, bf16lo(x.y) / s_k, bf16hi(x.y) / s_k);
+                    w1 = pack_s8x4(bf16lo(x.z) / s_k, bf16hi(x.z) / s_k, bf16lo(x.w) / s_k, bf16hi(x.w) / s_k);
+                } else {
+                    w0 = pack_e4m3x4(bf16lo(x.x) / s_k, bf16hi(x.x) / s_k, bf16lo(x.y) / s_k, bf16hi(x.y) / s_k);
+                    w1 = pack_e4m3x4(bf16lo(x.z) / s_k, bf16hi(x.z) / s_k, bf16lo(x.w) / s_k, bf16hi(x.w) / s_k);
+                }
                 *reinterpret_cast<uint2*>(ko + (row0 + n) * D + u * 8) = make_uint2(w0, w1);
             }
             // V^T: row c of the block holds the 64 tokens of feature c
@@ -393,9 +402,10 @@ __global__ void __launch_bounds__(256) h_reduce_kernel(const float* __restrict__
     }
 }
 
-// e4m3 Q with one absmax scale per 64-token block (absmax / 448).
+// e4m3 Q (I8: symmetric 8-bit integer Q) with one absmax scale per 64-token
+// block (absmax / 448, or absmax / 127).
 // Grid-stride over the BH*N/64 blocks; 256 threads, 64 x D tile in registers.
-template <int D>
+template <int D, bool I8>
 __global__ void __launch_bounds__(256) quant_q_kernel(const __nv_bfloat16* __restrict__ q,
                                                       long long nblk, uint8_t* __restrict__ q8,
                                                       float* __restrict__ sq) {
@@ -420,14 +430,18 @@ __global__ void __launch_bounds__(256) quant_q_kernel(const __nv_bfloat16* __res
         float am = 0.f;
 #pragma unroll
         for (int w = 0; w < 8; ++w) am = fmaxf(am, part[w]);
-        const float s = am > 0.f ? am / 448.f : 1.f;   // codes from the rounded quotient x / s
+        // codes from the rounded quotient x / s
+        const float s = am > 0.f ? am / (I8 ? 127.f : 448.f) : 1.f;
         if (tid == 0) sq[blk] = s;
         uint2* dst = reinterpret_cast<uint2*>(q8 + blk * 64 * D);
+        auto pack = [](float a0, float a1, float a2, float a3) {
+            return I8 ? pack_s8x4(a0, a1, a2, a3) : pack_e4m3x4(a0, a1, a2, a3);
+        };
 #pragma unroll
         for (int i = 0; i < VEC; ++i)
             dst[i * 256 + tid] = make_uint2(
-                pack_e4m3x4(bf16lo(x[i].x) / s, bf16hi(x[i].x) / s, bf16lo(x[i].y) / s, bf16hi(x[i].y) / s),
-                pack_e4m3x4(bf16lo(x[i].z) / s, bf16hi(x[i].z) / s, bf16lo(x[i].w) / s, bf16hi(x[i].w) / s));
+                pack(bf16lo(x[i].x) / s, bf16hi(x[i].x) / s, bf16lo(x[i].y) / s, bf16hi(x[i].y) / s),
+                pack(bf16lo(x[i].z) / s, bf16hi(x[i].z) / s, bf16lo(x[i].w) / s, bf16hi(x[i].w) / s));
         __syncthreads();
     }
 }

@@ -32,7 +32,8 @@ sla_status_t check_params(const sla_params_t* p) {
         return SLA_ERR_INVALID_ARG;
     if (p->N % p->Bq != 0 || p->N % p->Bk != 0) return SLA_ERR_INVALID_ARG;
     if (p->topk > p->N / p->Bk) return SLA_ERR_INVALID_ARG;
-    if (p->sparse_dtype != SLA_SPARSE_BF16 && p->sparse_dtype != SLA_SPARSE_FP8_E4M3)
+    if (p->sparse_dtype != SLA_SPARSE_BF16 && p->sparse_dtype != SLA_SPARSE_FP8_E4M3 &&
+        p->sparse_dtype != SLA_SPARSE_INT8)
         return SLA_ERR_INVALID_ARG;
     if (p->lut_mode != SLA_LUT_COMPUTE && p->lut_mode != SLA_LUT_GIVEN) return SLA_ERR_INVALID_ARG;
     if (p->pisa_first_order != 0 && p->pisa_first_order != 1) return SLA_ERR_INVALID_ARG;
@@ -84,7 +85,7 @@ Ws layout(const sla_params_t* p) {
     w.vbar = take(BH * Nk * d * 2);
     w.v16 = take(BH * static_cast<size_t>(p->N) * d * 2);
     w.phik16 = take(BH * static_cast<size_t>(p->N) * d * 2);
-    if (p->sparse_dtype == SLA_SPARSE_FP8_E4M3) {
+    if (p->sparse_dtype != SLA_SPARSE_BF16) {     // 8-bit Q, K, V^T codes and their scales
         w.q8 = take(BH * static_cast<size_t>(p->N) * d);
         w.k8 = take(BH * static_cast<size_t>(p->N) * d);
         w.v8t = take(BH * static_cast<size_t>(p->N) * d);
@@ -284,7 +285,8 @@ sla_status_t run_router(const sla_params_t* p, const void* q, const void* k, con
 template <int D>
 sla_status_t launch_kv(const sla_params_t* p, const void* k, const void* v, void* ws, const Ws& w,
                        bool want_kbar, bool sla_stats, bool pisa_stats, cudaStream_t st,
-                       bool fp8 = false, bool first_order = false, cudaEvent_t after_stats = nullptr) {
+                       bool fp8 = false, bool first_order = false, cudaEvent_t after_stats = nullptr,
+                       bool k_int8 = false) {
     const int BH = p->B * p->H, Nk = p->N / p->Bk;
     sla::KvStatsArgs a{};
     a.k = static_cast<const __nv_bfloat16*>(k);
@@ -305,6 +307,7 @@ sla_status_t launch_kv(const sla_params_t* p, const void* k, const void* v, void
     a.v8t = fp8 ? at<uint8_t>(ws, w.v8t) : nullptr;
     a.sk = fp8 ? at<float>(ws, w.sk) : nullptr;
     a.sv = fp8 ? at<float>(ws, w.sv) : nullptr;
+    a.k_int8 = (fp8 && k_int8) ? 1 : 0;
     const size_t smem = sla::kKvStages * 2 * 64 * D * 2 + 256 * 8 + 2 * 256 * 4 + 16 * 4;
     auto kern = sla::kv_stats_kernel<D>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -331,7 +334,7 @@ sla_status_t launch_attn(const sla_params_t* p, const void* q, const void* k, co
                          const float* alpha, const int32_t* lut, void* out, void* ws, const Ws& w,
                          cudaStream_t st) {
     using L = sla::AttnLayout<D, MODE>;
-    constexpr bool PISA = MODE == sla::kModePisa, FP8 = MODE == sla::kModeSlaFp8;
+    constexpr bool PISA = L::PISA, FP8 = L::FP8;
     const int BH = p->B * p->H, Nq = p->N / p->Bq, Nk = p->N / p->Bk;
     sla::AttnMaps tm;
     std::memset(&tm, 0, sizeof tm);
@@ -540,13 +543,15 @@ sla_status_t sla_forward(const sla_params_t* p, const void* q, const void* k, co
     if ((w_q && !aligned(w_q, 4)) || (w_k && !aligned(w_k, 4))) return SLA_ERR_INVALID_ARG;
     if (p->lut_mode == SLA_LUT_GIVEN && !lut && p->topk > 0) return SLA_ERR_INVALID_ARG;
     if (lut && !aligned(lut, 4)) return SLA_ERR_INVALID_ARG;
-    if (p->sparse_dtype == SLA_SPARSE_FP8_E4M3 && (p->d != 128 || p->Bq != 128))
+    if (p->sparse_dtype != SLA_SPARSE_BF16 && (p->d != 128 || p->Bq != 128))
         return SLA_ERR_UNSUPPORTED;
     Ws w;
     if ((s = check_ws(p, workspace, ws_bytes, w))) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const bool compute = p->lut_mode == SLA_LUT_COMPUTE;
-    const bool fp8 = p->sparse_dtype == SLA_SPARSE_FP8_E4M3;
+    // fp8: the 8-bit sparse branch (e4m3 P and V); int8: with integer Q and K codes
+    const bool int8 = p->sparse_dtype == SLA_SPARSE_INT8;
+    const bool fp8 = p->sparse_dtype == SLA_SPARSE_FP8_E4M3 || int8;
     int32_t* lut_use = (compute && !lut) ? at<int32_t>(workspace, w.lut) : lut;
     SideStream* side = side_stream();
     std::unique_lock<std::mutex> hold;
@@ -559,16 +564,16 @@ sla_status_t sla_forward(const sla_params_t* p, const void* q, const void* k, co
         sst = side->s;
     }
     s = p->d == 128 ? launch_kv<128>(p, k, v, workspace, w, compute, true, false, sst, fp8, false,
-                                     side ? side->kbar : nullptr)
+                                     side ? side->kbar : nullptr, int8)
                     : launch_kv<64>(p, k, v, workspace, w, compute, true, false, sst, false, false,
                                     side ? side->kbar : nullptr);
     if (s != SLA_OK) return s;
     if (fp8) {
         const long long nblk = static_cast<long long>(p->B) * p->H * p->N / 64;
         Span sp(SLA_KERNEL_QUANT_Q, sst);
-        sla::quant_q_kernel<128><<<grid_blocks(nblk, 8), 256, 0, sst>>>(
-            static_cast<const __nv_bfloat16*>(q), nblk, at<uint8_t>(workspace, w.q8),
-            at<float>(workspace, w.sq));
+        auto qk = int8 ? sla::quant_q_kernel<128, true> : sla::quant_q_kernel<128, false>;
+        qk<<<grid_blocks(nblk, 8), 256, 0, sst>>>(static_cast<const __nv_bfloat16*>(q), nblk,
+                                                  at<uint8_t>(workspace, w.q8), at<float>(workspace, w.sq));
         if (launch_status() != SLA_OK) return SLA_ERR_CUDA;
     }
     if (side && cudaEventRecord(side->stats, sst) != cudaSuccess) return SLA_ERR_CUDA;
@@ -576,7 +581,9 @@ sla_status_t sla_forward(const sla_params_t* p, const void* q, const void* k, co
                                    side ? side->kbar : nullptr)))
         return s;
     if (side && cudaStreamWaitEvent(st, side->stats, 0) != cudaSuccess) return SLA_ERR_CUDA;
-    if (fp8)
+    if (int8)
+        s = launch_attn<128, sla::kModeSlaInt8>(p, q, k, v, alpha, lut_use, out, workspace, w, st);
+    else if (fp8)
         s = launch_attn<128, sla::kModeSlaFp8>(p, q, k, v, alpha, lut_use, out, workspace, w, st);
     else
         s = p->d == 128 ? launch_attn<128, sla::kModeSla>(p, q, k, v, alpha, lut_use, out, workspace, w, st)

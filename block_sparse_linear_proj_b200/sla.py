@@ -31,6 +31,7 @@ SLA_ERR_DEVICE_CHECK = 6
 
 SLA_SPARSE_BF16 = 0
 SLA_SPARSE_FP8_E4M3 = 1
+SLA_SPARSE_INT8 = 2
 SLA_LUT_COMPUTE = 0
 SLA_LUT_GIVEN = 1
 SLA_OUT_BF16 = 0

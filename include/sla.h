@@ -65,7 +65,7 @@ typedef enum {
     SLA_ERR_DEVICE_CHECK = 6   /* a kernel found invalid data (e.g. LUT entry)*/
 } sla_status_t;
 
-typedef enum { SLA_SPARSE_BF16 = 0, SLA_SPARSE_FP8_E4M3 = 1 } sla_sparse_dtype_t;
+typedef enum { SLA_SPARSE_BF16 = 0, SLA_SPARSE_FP8_E4M3 = 1, SLA_SPARSE_INT8 = 2 } sla_sparse_dtype_t;
 typedef enum { SLA_LUT_COMPUTE = 0, SLA_LUT_GIVEN = 1 } sla_lut_mode_t;
 typedef enum { SLA_OUT_BF16 = 0, SLA_OUT_FP32 = 1 } sla_out_dtype_t;
 
@@ -148,6 +148,12 @@ sla_status_t sla_route_noalloc(const sla_params_t *p, const void *q, const void 
  *      scale of the query block's LUT row; O is dequantised by s_v,max / 448
  *      and divided by the row sum of the unquantised P.  The linear branch
  *      and the combine stay bf16/fp32.
+ * sparse_dtype INT8 (needs d = 128, Bq = 128): as FP8_E4M3, except that Q and
+ *      K take symmetric 8-bit integer codes (s = fl32(absmax / 127), code =
+ *      the nearest integer to fl32(x / s), ties to even, within +-127), so
+ *      S = Q8 K8^T is an exact integer product (tcgen05 kind::i8, s32
+ *      accumulation) scaled by s_q s_k; P and V keep the e4m3 rules (an
+ *      integer P.V accumulator could not take the online rescale exactly).
  */
 sla_status_t sla_forward(const sla_params_t *p, const void *q, const void *k, const void *v,
                          const float *alpha, const float *w_q, const float *w_k,

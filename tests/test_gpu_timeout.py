@@ -41,13 +41,13 @@ def _run(p, g, lut):
     return S.sla_check_device_status(), out
 
 
-@pytest.mark.parametrize("fp8", [False, True], ids=["bf16", "fp8"])
-def test_wait_expiry_reports_timeout_and_context_survives(fp8):
+@pytest.mark.parametrize("sd", [S.SLA_SPARSE_BF16, S.SLA_SPARSE_FP8_E4M3, S.SLA_SPARSE_INT8],
+                         ids=["bf16", "fp8", "int8"])
+def test_wait_expiry_reports_timeout_and_context_survives(sd):
     B, H, N, d, Bq, k = 1, 2, 2048, 128, 128, 6
     inp = W.gaussian_inputs(B, H, N, d, 91)
     lut, _ = orc.route(inp["q"], inp["k"], inp["w_q"], inp["w_k"], Bq, 64, k)
     g = dev(inp)
-    sd = S.SLA_SPARSE_FP8_E4M3 if fp8 else S.SLA_SPARSE_BF16
     p = params(B, H, N, d, Bq, 64, k, given=True, sparse_dtype=sd)
     old = {k: os.environ.get(k) for k in HOOK}
     os.environ.update(HOOK)
@@ -63,8 +63,9 @@ def test_wait_expiry_reports_timeout_and_context_survives(fp8):
     # the context is intact: the same call with the normal limit is correct
     pf = params(B, H, N, d, Bq, 64, k, given=True, sparse_dtype=sd, f32=True)
     out = gpu_forward(pf, g, lut)
-    ref = orc.sla_forward(inp["q"], inp["k"], inp["v"], inp["alpha"], lut, Bq, 64, fp8=fp8)
-    check(out, ref, pf, (6e-2, 6e-3) if fp8 else (2e-2, 2e-3))
+    ref = orc.sla_forward(inp["q"], inp["k"], inp["v"], inp["alpha"], lut, Bq, 64,
+                          fp8=sd == S.SLA_SPARSE_FP8_E4M3, int8=sd == S.SLA_SPARSE_INT8)
+    check(out, ref, pf, (2e-2, 2e-3) if sd == S.SLA_SPARSE_BF16 else (6e-2, 6e-3))
 
 
 def test_pisa_wait_expiry(stalled_loader):

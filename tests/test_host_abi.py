@@ -70,6 +70,7 @@ def call_pisa(p, ws_bytes=1 << 40, lut=FAKE):
     (dict(Bq=32), S.SLA_ERR_UNSUPPORTED),
     (dict(Bk=128, N=1024, topk=2), S.SLA_ERR_UNSUPPORTED),
     (dict(sparse_dtype=7), S.SLA_ERR_INVALID_ARG),
+    (dict(sparse_dtype=3), S.SLA_ERR_INVALID_ARG),
     (dict(lut_mode=3), S.SLA_ERR_INVALID_ARG),
 ])
 def test_parameter_validation(lib, kw, code):
@@ -107,8 +108,19 @@ def test_mode_restrictions(lib):
     # PISA needs Bq == Bk and the bf16 sparse branch
     assert call_pisa(S.params(1, 2, 1024, 64, 128, 64, 4)) == S.SLA_ERR_UNSUPPORTED
     assert call_pisa(S.params(1, 2, 1024, 64, 64, 64, 4, sparse_dtype=1)) == S.SLA_ERR_UNSUPPORTED
-    # the FP8 sparse branch needs d = 128 and Bq = 128
-    assert call_forward(S.params(1, 2, 1024, 64, 64, 64, 4, sparse_dtype=1)) == S.SLA_ERR_UNSUPPORTED
+    assert call_pisa(S.params(1, 2, 1024, 64, 64, 64, 4, sparse_dtype=S.SLA_SPARSE_INT8)) == \
+        S.SLA_ERR_UNSUPPORTED
+    # the FP8 and INT8 sparse branches need d = 128 and Bq = 128
+    for sd in (S.SLA_SPARSE_FP8_E4M3, S.SLA_SPARSE_INT8):
+        assert call_forward(S.params(1, 2, 1024, 64, 64, 64, 4, sparse_dtype=sd)) == S.SLA_ERR_UNSUPPORTED
+        assert call_forward(S.params(1, 2, 1024, 128, 64, 64, 4, sparse_dtype=sd)) == S.SLA_ERR_UNSUPPORTED
+
+
+def test_int8_workspace_matches_fp8(lib):
+    # both 8-bit branches keep the same code and scale buffers
+    sizes = [lib.sla_workspace_size(ctypes.byref(S.params(1, 4, 4096, 128, 128, 64, 8, sparse_dtype=sd)))
+             for sd in (S.SLA_SPARSE_BF16, S.SLA_SPARSE_FP8_E4M3, S.SLA_SPARSE_INT8)]
+    assert sizes[1] == sizes[2] > sizes[0]
 
 
 def test_workspace_size_grows_with_problem(lib):

@@ -33,6 +33,7 @@ import torch
 
 SPARSE_BF16 = 0
 SPARSE_FP8_E4M3 = 1
+SPARSE_INT8 = 2
 
 
 @dataclasses.dataclass(frozen=True)
@@ -46,7 +47,7 @@ class Workload:
     Bk: int
     topk: int
     mode: str                 # "sla" or "pisa"
-    sparse_dtype: int         # SPARSE_BF16 or SPARSE_FP8_E4M3
+    sparse_dtype: int         # SPARSE_BF16, SPARSE_FP8_E4M3 or SPARSE_INT8
     generator: str            # "gaussian" or "video"
     seed: int
     grid: Optional[tuple] = None   # (T, Y, X) latent grid for the video generator
@@ -72,8 +73,9 @@ class Workload:
         return 4.0 * pairs * self.Bq * self.Bk * self.d
 
 
-# The five workloads: tiny, SLA2 bf16 (21x30x52 grid + 8 pad tokens),
-# long (21x45x80 grid + 176 pad tokens), FP8 sparse branch, PISA.
+# The workloads: tiny, SLA2 bf16 (21x30x52 grid + 8 pad tokens), long (21x45x80
+# grid + 176 pad tokens), the FP8 and INT8 sparse branches (the inputs of the FP8
+# one), PISA and PISA with the first-order term (the inputs of the PISA one).
 WORKLOADS = {
     "tiny": Workload("tiny", 1, 2, 1024, 64, 64, 64, 4, "sla", SPARSE_BF16,
                      "gaussian", 1001, None, (0.2, 0.8), True),
@@ -83,13 +85,15 @@ WORKLOADS = {
                           SPARSE_BF16, "video", 1003, (21, 45, 80), (0.0, 1.0), True),
     "sla2_fp8": Workload("sla2_fp8", 1, 12, 32768, 128, 128, 64, 52, "sla",
                          SPARSE_FP8_E4M3, "video", 1004, (21, 30, 52), (0.0, 1.0), True),
+    "sla2_int8": Workload("sla2_int8", 1, 12, 32768, 128, 128, 64, 52, "sla",
+                          SPARSE_INT8, "video", 1004, (21, 30, 52), (0.0, 1.0), True),
     "pisa": Workload("pisa", 1, 24, 32768, 128, 64, 64, 77, "pisa", SPARSE_BF16,
                      "video", 1005, (21, 30, 52), None, False),
     # the PISA workload with the global first-order correction
     "pisa_fo": Workload("pisa_fo", 1, 24, 32768, 128, 64, 64, 77, "pisa", SPARSE_BF16,
                         "video", 1005, (21, 30, 52), None, False, True),
 }
-ORDER = ["tiny", "sla2_bf16", "sla2_long", "sla2_fp8", "pisa", "pisa_fo"]
+ORDER = ["tiny", "sla2_bf16", "sla2_long", "sla2_fp8", "sla2_int8", "pisa", "pisa_fo"]
 
 
 def _bf16(x: torch.Tensor) -> torch.Tensor:
