@@ -3,10 +3,11 @@
 // blocks of adjacent tokens, the proj_q / proj_k projections, the compressed
 // block score and a hard top-k per query block, emitted as an ascending LUT.
 //
-// Precision: pooling, projection and score run in fp64.  Sums of bf16 values
-// in fp64 are exact for any realistic exponent spread, so the selected set
-// equals an exact-arithmetic selection except where two block scores lie
-// within ~1e-12 of each other.
+// Precision: pooling, projection and score run in fp64 (the products on the
+// fp64 tensor-core MMA).  Sums of bf16 values in fp64 are exact for any
+// realistic exponent spread, so the selected set equals an exact-arithmetic
+// selection except where two block scores lie within ~1e-12 of each other; the
+// top-k itself is an exact selection on the fp64 scores (ties to the lower j).
 #pragma once
 #include "common.cuh"
 
@@ -117,141 +118,194 @@ __device__ __forceinline__ unsigned long long order_key(double v) {
                  : (static_cast<unsigned long long>(b) | 0x8000000000000000ull);
 }
 
+// fp64 tensor-core product D(8x8) += A(8x4) B(4x8), A row-major, B column-major:
+// lane l holds A[l/4][l%4], B[l%4][l/4] and D[l/4][2(l%4)], D[l/4][2(l%4)+1].
+__device__ __forceinline__ void dmma_884(double (&d)[2], double a, double b) {
+    asm("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
+        : "+d"(d[0]), "+d"(d[1])
+        : "d"(a), "d"(b));
+}
+
+__device__ __forceinline__ unsigned long long warp_min_u64(unsigned long long v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = min(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
 // One CTA: head bh = blockIdx.y, query blocks i0 = blockIdx.x * R ... i0 + R - 1.
-// Shared memory: qhat^T [D][R] fp64, hist [8][256] u32, keys [R][max(Nk, D)] u64
-// (the key area doubles as the [R][D] staging buffer of step 1).
-// PF: step 2 reads the kbar columns eight feature rows ahead of use (pays off on
-// long rows, where each warp walks several column chunks).
-template <int R, int D, bool PF>
-__global__ void __launch_bounds__(256) score_topk_kernel(const double* __restrict__ qbar,
+// Both products run on the fp64 MMA (m8n8k4, eight-row tiles; R < 8 pads the tile).
+// Shared memory: qhat [8 MT][D + 4] fp64 (rows padded so that the A-fragment
+// loads spread over the banks), hist [8][256] u32, keys [R][max(Nk, D + 4)] u64
+// (the key area doubles as the staging buffer of the pooled rows in step 1).
+// DEPTH: k-steps of K fragments in flight per warp; MINB: CTAs per SM the
+// register budget is sized for.
+template <int R, int D, int DEPTH, int MINB>
+__global__ void __launch_bounds__(256, MINB) score_topk_kernel(const double* __restrict__ qbar,
                                                          const double* __restrict__ kbarT,
                                                          const double* __restrict__ m, int Nq,
                                                          int Nk, int topk,
                                                          int32_t* __restrict__ lut) {
+    constexpr int MT = R >= 8 ? R / 8 : 1;      // eight-row MMA tiles
+    constexpr int LDQ = D + 4;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    double* qhT = reinterpret_cast<double*>(smem_raw);                        // [D][R]
-    unsigned* hist = reinterpret_cast<unsigned*>(qhT + D * R);                  // [8][256]
+    double* qh = reinterpret_cast<double*>(smem_raw);                              // [8 MT][LDQ]
+    unsigned* hist = reinterpret_cast<unsigned*>(qh + 8 * MT * LDQ);               // [8][256]
     unsigned long long* keys = reinterpret_cast<unsigned long long*>(hist + 8 * 256);
+    const int ldk = max(Nk, LDQ);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = lane >> 2, t = lane & 3;
     const long long bh = blockIdx.y;
     const int i0 = blockIdx.x * R;
     const int nrows = min(R, Nq - i0);
     const double* qb = qbar + (bh * Nq + i0) * D;
     const double* kt = kbarT + bh * D * static_cast<long long>(Nk);
 
-    // 1. qhat = qbar . M (or qbar) for the R rows, stored transposed.
+    // 1. qhat = qbar . M for the R rows (padding rows are zero).  Warp w computes
+    //    output columns [w D/8, (w+1) D/8) for every row.
     {
-        double* qtmp = reinterpret_cast<double*>(keys);   // [R][D] scratch
-        for (int a = tid; a < R * D; a += 256) {
-            const int r = a / D;
-            qtmp[a] = r < nrows ? qb[a] : 0.0;
+        double* stage = m ? reinterpret_cast<double*>(keys) : qh;      // [8 MT][LDQ]
+        for (int a = tid; a < 8 * MT * D; a += 256) {
+            const int r = a / D, c = a % D;
+            stage[r * LDQ + c] = r < nrows ? qb[static_cast<long long>(r) * D + c] : 0.0;
         }
         __syncthreads();
-        constexpr int RG = 256 / D;       // row groups
-        constexpr int RPT = R / RG > 0 ? R / RG : 1;
-        const int e = tid % D;
-        const int g = tid / D;
-        if (g < RG && g * RPT < R) {
-            double acc[RPT];
+        if (m) {
+            constexpr int NT = D / 64;               // 8-column tiles per warp
+            double acc[MT][NT][2];
 #pragma unroll
-            for (int r = 0; r < RPT; ++r) acc[r] = 0.0;
-            if (m) {
-                for (int c = 0; c < D; ++c) {
-                    const double mv = __ldg(m + c * D + e);
+            for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-                    for (int r = 0; r < RPT; ++r) acc[r] += qtmp[(g * RPT + r) * D + c] * mv;
+                for (int nt = 0; nt < NT; ++nt) acc[mt][nt][0] = acc[mt][nt][1] = 0.0;
+            const int n0 = warp * (D / 8);
+            // M fragments in a ring of 2 DEPTH k-steps, refilled right after use
+            constexpr int MD = 2 * DEPTH;
+            double bm[MD][NT];
+            auto load_m = [&](double (&b)[NT], int c0) {
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) b[nt] = __ldg(m + (c0 + t) * D + n0 + nt * 8 + g);
+            };
+#pragma unroll
+            for (int u = 0; u < MD; ++u) load_m(bm[u], u * 4);
+#pragma unroll 1
+            for (int ks = 0; ks < D / 4; ks += MD) {
+#pragma unroll
+                for (int u = 0; u < MD; ++u) {
+                    double a[MT];
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt) a[mt] = stage[(mt * 8 + g) * LDQ + (ks + u) * 4 + t];
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) dmma_884(acc[mt][nt], a[mt], bm[u][nt]);
+                    if (ks + u + MD < D / 4) load_m(bm[u], (ks + u + MD) * 4);
                 }
-            } else {
-#pragma unroll
-                for (int r = 0; r < RPT; ++r) acc[r] = qtmp[(g * RPT + r) * D + e];
             }
 #pragma unroll
-            for (int r = 0; r < RPT; ++r) qhT[e * R + g * RPT + r] = acc[r];
+            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    double* dst = qh + (mt * 8 + g) * LDQ + n0 + nt * 8 + 2 * t;
+                    dst[0] = acc[mt][nt][0];
+                    dst[1] = acc[mt][nt][1];
+                }
+            __syncthreads();
         }
-        __syncthreads();
     }
 
-    // 2. scores s[r][j] = qhat_r . kbar_j, fp64; warp w covers 64 columns at a time.
+    // 2. scores s[r][j] = qhat_r . kbar_j on the fp64 MMA.  Warp w covers 64
+    //    columns (eight 8-column tiles) at a time; a ring of DEPTH k-steps of B
+    //    fragments, each slot refilled DEPTH k-steps ahead right after its use.
     for (int j0 = warp * 64; j0 < Nk; j0 += 8 * 64) {
-        const int ja = j0 + lane, jb = j0 + 32 + lane;
-        const bool va = ja < Nk, vb = jb < Nk;
-        double acc0[R], acc1[R];
+        double acc[MT][8][2];
 #pragma unroll
-        for (int r = 0; r < R; ++r) { acc0[r] = 0.0; acc1[r] = 0.0; }
-        if (PF) {
-            double ka[8], kb[8];
+        for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-            for (int x = 0; x < 8; ++x) {
-                ka[x] = va ? __ldg(kt + static_cast<long long>(x) * Nk + ja) : 0.0;
-                kb[x] = vb ? __ldg(kt + static_cast<long long>(x) * Nk + jb) : 0.0;
-            }
+            for (int nt = 0; nt < 8; ++nt) acc[mt][nt][0] = acc[mt][nt][1] = 0.0;
+        bool live[8];
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) live[nt] = j0 + nt * 8 + g < Nk;
+        const double* kc = kt + j0 + g;
+        auto load = [&](double (&b)[8], int c0) {
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt)
+                b[nt] = live[nt] ? __ldg(kc + static_cast<long long>(c0 + t) * Nk + nt * 8) : 0.0;
+        };
+        static_assert((D / 4) % DEPTH == 0, "ring depth must divide the k-steps");
+        double bq[DEPTH][8];
+#pragma unroll
+        for (int u = 0; u < DEPTH; ++u) load(bq[u], u * 4);
 #pragma unroll 1
-            for (int c0 = 0; c0 < D; c0 += 8) {
-                double na[8], nb[8];
-                const bool more = c0 + 8 < D;
+        for (int ks = 0; ks < D / 4; ks += DEPTH) {
 #pragma unroll
-                for (int x = 0; x < 8; ++x) {
-                    na[x] = (more && va) ? __ldg(kt + static_cast<long long>(c0 + 8 + x) * Nk + ja) : 0.0;
-                    nb[x] = (more && vb) ? __ldg(kt + static_cast<long long>(c0 + 8 + x) * Nk + jb) : 0.0;
-                }
+            for (int u = 0; u < DEPTH; ++u) {
+                double a[MT];
 #pragma unroll
-                for (int x = 0; x < 8; ++x) {
-                    const double2* qrow = reinterpret_cast<const double2*>(qhT + (c0 + x) * R);
+                for (int mt = 0; mt < MT; ++mt) a[mt] = qh[(mt * 8 + g) * LDQ + (ks + u) * 4 + t];
 #pragma unroll
-                    for (int r2 = 0; r2 < R / 2; ++r2) {
-                        const double2 qq = qrow[r2];
-                        acc0[2 * r2] = fma(qq.x, ka[x], acc0[2 * r2]);
-                        acc1[2 * r2] = fma(qq.x, kb[x], acc1[2 * r2]);
-                        acc0[2 * r2 + 1] = fma(qq.y, ka[x], acc0[2 * r2 + 1]);
-                        acc1[2 * r2 + 1] = fma(qq.y, kb[x], acc1[2 * r2 + 1]);
-                    }
-                }
+                for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
-                for (int x = 0; x < 8; ++x) { ka[x] = na[x]; kb[x] = nb[x]; }
-            }
-        } else {
-#pragma unroll 4
-            for (int c = 0; c < D; ++c) {
-                const double ka = va ? __ldg(kt + static_cast<long long>(c) * Nk + ja) : 0.0;
-                const double kb = vb ? __ldg(kt + static_cast<long long>(c) * Nk + jb) : 0.0;
-                const double2* qrow = reinterpret_cast<const double2*>(qhT + c * R);
-#pragma unroll
-                for (int r2 = 0; r2 < R / 2; ++r2) {
-                    const double2 qq = qrow[r2];
-                    acc0[2 * r2] = fma(qq.x, ka, acc0[2 * r2]);
-                    acc1[2 * r2] = fma(qq.x, kb, acc1[2 * r2]);
-                    acc0[2 * r2 + 1] = fma(qq.y, ka, acc0[2 * r2 + 1]);
-                    acc1[2 * r2 + 1] = fma(qq.y, kb, acc1[2 * r2 + 1]);
-                }
+                    for (int mt = 0; mt < MT; ++mt) dmma_884(acc[mt][nt], a[mt], bq[u][nt]);
+                if (ks + u + DEPTH < D / 4) load(bq[u], (ks + u + DEPTH) * 4);
             }
         }
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
-            if (va) keys[static_cast<size_t>(r) * Nk + ja] = order_key(acc0[r]);
-            if (vb) keys[static_cast<size_t>(r) * Nk + jb] = order_key(acc1[r]);
+        for (int mt = 0; mt < MT; ++mt) {
+            const int r = mt * 8 + g;
+            if (r >= R) continue;
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) {
+                const int j = j0 + nt * 8 + 2 * t;
+                if (j < Nk) keys[static_cast<size_t>(r) * ldk + j] = order_key(acc[mt][nt][0]);
+                if (j + 1 < Nk) keys[static_cast<size_t>(r) * ldk + j + 1] = order_key(acc[mt][nt][1]);
+            }
         }
     }
     __syncthreads();
     if (topk <= 0) return;
 
-    // 3. per row: radix-select the topk-th largest key, then emit ascending.
+    // 3. per row (one warp): find the topk-th largest key and emit the selected
+    //    block indices ascending.  The candidates are the keys of an interval
+    //    [klo, khi] (every key above it is taken, rem more are needed from it).
+    //    A pass bins them by (key - klo) >> s, s chosen so that 256 bins cover the
+    //    interval, and keeps the bin holding the rem-th largest: the interval
+    //    shrinks at least 128-fold per pass (at most 10 passes).  It stops when
+    //    that bin's keys are exactly the ones still needed (take every key >= its
+    //    lower bound), or when the interval is one key value (take the rem of
+    //    those keys with the lowest j).
     unsigned* h = hist + warp * 256;
     const unsigned lt_mask = (1u << lane) - 1u;
     for (int r = warp; r < nrows; r += 8) {
-        const unsigned long long* kr = keys + static_cast<size_t>(r) * Nk;
+        const unsigned long long* kr = keys + static_cast<size_t>(r) * ldk;
         int32_t* dst = lut + ((bh * Nq) + i0 + r) * static_cast<long long>(topk);
-        unsigned long long prefix = 0ull, pmask = 0ull;
-        int rem = topk;
+        unsigned long long T = 0ull;      // threshold key
+        int rem = topk;                   // keys equal to T still to take (lowest j first)
+        bool ge = false;                  // take every key >= T
         if (topk < Nk) {
-            for (int shift = 56; shift >= 0; shift -= 8) {
+            unsigned long long klo = ~0ull, khi = 0ull;
+            for (int j = lane; j < Nk; j += 32) {
+                const unsigned long long key = kr[j];
+                klo = min(klo, key);
+                khi = max(khi, key);
+            }
+            klo = warp_min_u64(klo);
+            khi = warp_max_u64(khi);
+            for (int pass = 0; pass < 12 && klo != khi; ++pass) {
+                const unsigned long long span = khi - klo;
+                const int sh = max(64 - __clzll(static_cast<long long>(span)) - 8, 0);
                 for (int b = lane; b < 256; b += 32) h[b] = 0u;
                 __syncwarp();
                 for (int j = lane; j < Nk; j += 32) {
                     const unsigned long long key = kr[j];
-                    if ((key & pmask) == prefix) atomicAdd(&h[(key >> shift) & 255ull], 1u);
+                    if (key >= klo && key <= khi) atomicAdd(&h[static_cast<int>((key - klo) >> sh)], 1u);
                 }
                 __syncwarp();
+                // bins from the top: lane l owns bins 255 - 8l ... 248 - 8l
                 int cnt[8], s = 0;
 #pragma unroll
                 for (int b = 0; b < 8; ++b) { cnt[b] = static_cast<int>(h[255 - 8 * lane - b]); s += cnt[b]; }
@@ -264,36 +318,40 @@ __global__ void __launch_bounds__(256) score_topk_kernel(const double* __restric
                 const int excl = incl - s;
                 const bool mine = excl < rem && rem <= incl;
                 const unsigned bal = __ballot_sync(0xffffffffu, mine);
-                int digit = 0, newrem = 0;
+                int digit = 0, newrem = 0, dcnt = 0;
                 if (mine) {
                     int a = excl;
 #pragma unroll
                     for (int b = 0; b < 8; ++b) {
-                        if (a + cnt[b] >= rem) { digit = 255 - 8 * lane - b; newrem = rem - a; break; }
+                        if (a + cnt[b] >= rem) { digit = 255 - 8 * lane - b; newrem = rem - a; dcnt = cnt[b]; break; }
                         a += cnt[b];
                     }
                 }
                 const int src = bal ? __ffs(bal) - 1 : 0;
                 digit = __shfl_sync(0xffffffffu, digit, src);
-                newrem = __shfl_sync(0xffffffffu, newrem, src);
-                prefix |= static_cast<unsigned long long>(digit) << shift;
-                pmask |= 255ull << shift;
-                rem = newrem;
+                rem = __shfl_sync(0xffffffffu, newrem, src);
+                dcnt = __shfl_sync(0xffffffffu, dcnt, src);
+                const unsigned long long nlo = klo + (static_cast<unsigned long long>(digit) << sh);
+                const unsigned long long width = (1ull << sh) - 1ull;
                 __syncwarp();
+                klo = nlo;
+                if (rem == dcnt) { ge = true; break; }
+                if (khi - nlo > width) khi = nlo + width;   // (no wrap past 2^64)
             }
+            T = klo;
         } else {
-            prefix = 0ull;      // every key is >= 0: take all of them
+            ge = true;                    // every key is taken
             rem = 0;
         }
         int out = 0, eqseen = 0;
         for (int j0 = 0; j0 < Nk; j0 += 32) {
             const int j = j0 + lane;
             const unsigned long long key = j < Nk ? kr[j] : 0ull;
-            const bool gt = j < Nk && (topk >= Nk || key > prefix);
-            const bool eq = j < Nk && topk < Nk && key == prefix;
+            const bool gt = j < Nk && key > T;
+            const bool eq = j < Nk && key == T;
             const unsigned beq = __ballot_sync(0xffffffffu, eq);
             const int eqrank = eqseen + __popc(beq & lt_mask);
-            const bool sel = gt || (eq && eqrank < rem);
+            const bool sel = gt || (eq && (ge || eqrank < rem));
             const unsigned bsel = __ballot_sync(0xffffffffu, sel);
             if (sel) dst[out + __popc(bsel & lt_mask)] = j;
             out += __popc(bsel);

@@ -227,13 +227,19 @@ void launch_pool(const void* x, int rows, long long nblk_total, int nblk_per_hea
         sla::pool_mean_kernel<64><<<grid, 256, 0, st>>>(xb, rows, nblk_total, nblk_per_head, out_mode, out);
 }
 
-template <int R, int D>
+// shared memory of score_topk_kernel<R, D>: qhat tiles, histograms, keys (which
+// also stage the pooled rows)
+size_t score_smem(int R, int D, int Nk) {
+    const size_t mt = R >= 8 ? R / 8 : 1, ldq = D + 4;
+    const size_t ldk = std::max<size_t>(Nk, ldq);
+    return 8 * mt * ldq * 8 + 8 * 256 * 4 + std::max(R * ldk, 8 * mt * ldq) * 8;
+}
+
+template <int R, int D, int DEPTH, int MINB>
 sla_status_t launch_score_r(const double* qbar, const double* kbarT, const double* m, int BH,
                             int Nq, int Nk, int topk, int32_t* lut, cudaStream_t st) {
-    const size_t smem = static_cast<size_t>(D) * R * 8 + 8 * 256 * 4 +
-                        static_cast<size_t>(R) * std::max(Nk, D) * 8;
-    // read-ahead of the kbar columns pays off once each warp walks several 64-column chunks
-    auto kern = Nk >= 1024 ? sla::score_topk_kernel<R, D, true> : sla::score_topk_kernel<R, D, false>;
+    const size_t smem = score_smem(R, D, Nk);
+    auto kern = sla::score_topk_kernel<R, D, DEPTH, MINB>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
         return SLA_ERR_CUDA;
@@ -246,18 +252,18 @@ sla_status_t launch_score_r(const double* qbar, const double* kbarT, const doubl
 template <int D>
 sla_status_t launch_score(const double* qbar, const double* kbarT, const double* m, int BH,
                           int Nq, int Nk, int topk, int32_t* lut, cudaStream_t st) {
-    const size_t budget = 200 * 1024;
-    auto need = [&](int R) {
-        return static_cast<size_t>(D) * R * 8 + 8 * 256 * 4 + static_cast<size_t>(R) * std::max(Nk, D) * 8;
-    };
-    // 16 query blocks per CTA, unless that leaves fewer than two waves of CTAs on
-    // 148 SMs for short rows (then 8 blocks per CTA spreads the fp64 work wider)
-    const bool few = static_cast<long long>((Nq + 15) / 16) * BH < 2 * 148;
-    if (!(few && Nk < 1024) && need(16) <= budget)
-        return launch_score_r<16, D>(qbar, kbarT, m, BH, Nq, Nk, topk, lut, st);
-    if (need(8) <= budget) return launch_score_r<8, D>(qbar, kbarT, m, BH, Nq, Nk, topk, lut, st);
-    if (need(4) <= budget) return launch_score_r<4, D>(qbar, kbarT, m, BH, Nq, Nk, topk, lut, st);
-    return launch_score_r<2, D>(qbar, kbarT, m, BH, Nq, Nk, topk, lut, st);
+    // 16 query blocks per CTA (two 8-row tiles of the fp64 MMA per K fragment).
+    // Where two CTAs fit an SM's shared memory, a two-deep fragment ring keeps
+    // the registers within two CTAs; otherwise one CTA per SM with a four-deep ring.
+    constexpr size_t two = 113 * 1024, one = 200 * 1024;
+    if (score_smem(16, D, Nk) <= two)
+        return launch_score_r<16, D, 2, 2>(qbar, kbarT, m, BH, Nq, Nk, topk, lut, st);
+    if (score_smem(16, D, Nk) <= one)
+        return launch_score_r<16, D, 4, 1>(qbar, kbarT, m, BH, Nq, Nk, topk, lut, st);
+    if (score_smem(8, D, Nk) <= one) return launch_score_r<8, D, 4, 1>(qbar, kbarT, m, BH, Nq, Nk, topk, lut, st);
+    if (score_smem(4, D, Nk) <= one) return launch_score_r<4, D, 4, 1>(qbar, kbarT, m, BH, Nq, Nk, topk, lut, st);
+    if (score_smem(2, D, Nk) > 232448) return SLA_ERR_UNSUPPORTED;   // a score row beyond shared memory
+    return launch_score_r<2, D, 4, 1>(qbar, kbarT, m, BH, Nq, Nk, topk, lut, st);
 }
 
 // Router: Q/K pooling (unless already pooled), W folding, fp64 score + top-k.
@@ -497,11 +503,13 @@ sla_status_t sla_route(const sla_params_t* p, const void* q, const void* k, cons
 }
 
 // ------------------------------------------------------------- side stream
-// The K/V pre-pass does not depend on the router's pooling of Q or on W folding,
-// so a forward call runs it on a side stream of the library (one per device,
-// created on first use) between a fork and two join points on the caller's
-// stream: the router's score kernel waits for the pre-pass (it reads the pooled
-// K means the pre-pass writes), the attention kernel also for h_reduce.  The
+// The K/V pre-pass does not depend on the router's pooling of Q or on W folding, so
+// a forward call runs it on a side stream of the library (one per device, created on
+// first use) between a fork and two join points on the caller's stream: the router's
+// score kernel waits for the pre-pass (it reads the pooled K means the pre-pass
+// writes), the attention kernel also for h_reduce.  (Pooling K a second time on the
+// caller's stream, so that the score could start before the pre-pass ends, was
+// measured slower: the extra read of K competes with the pre-pass for HBM.)  The
 // caller sees ordinary stream order.  The enqueue sequence of a call holds a
 // per-device lock, so concurrent host threads never cross their events.  If the
 // side stream cannot be created, everything runs on the caller's stream.
