@@ -294,14 +294,13 @@ def run_ours(args, w, rank, world, local_rank):
         if world > 1:
             torch.distributed.barrier()
 
-    # ---- timed region (device-resident inputs)
+    # ---- timed region (device-resident inputs), without the per-kernel events
     clocks = ClockSampler(local_rank)
     S.sla_profile_read()                       # drop anything recorded earlier
     barrier()
     torch.cuda.synchronize(dev)
     clocks.start()
     time.sleep(0.3)
-    S.sla_profile_enable(True)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
@@ -309,15 +308,31 @@ def run_ours(args, w, rank, world, local_rank):
         step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    S.sla_profile_enable(False)
     clk = clocks.stop()
     barrier()
-    ms_total = e0.elapsed_time(e1)
-    prof = S.sla_profile_read()
-    ms_total = max_over_ranks(ms_total, world, dev)
+    ms_total = max_over_ranks(e0.elapsed_time(e1), world, dev)
     ms_per_call = ms_total / args.steps
     value = whole_job_value(w, world, ms_per_call)
-    launches = sum(c for (_, c) in prof.values())
+
+    # ---- the same steps again with the library's per-kernel events (a pair of
+    # timing events around every launch, on its own stream), for the kernel
+    # breakdown and the roofline; the events themselves cost time, so this pass
+    # is not the headline
+    barrier()
+    torch.cuda.synchronize(dev)
+    S.sla_profile_enable(True)
+    e2 = torch.cuda.Event(enable_timing=True)
+    e3 = torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    for _ in range(args.steps):
+        step()
+    e3.record(stream)
+    torch.cuda.synchronize(dev)
+    S.sla_profile_enable(False)
+    barrier()
+    prof = S.sla_profile_read()
+    ms_profiled = max_over_ranks(e2.elapsed_time(e3), world, dev) / args.steps
+    launches = sum(c for (_, c) in prof.values())      # the same steps as the timed region
 
     # ---- end-to-end through the C ABI with host buffers
     hosts = {k: (v.pin_memory() if v is not None else None) for k, v in inp.items()}
@@ -396,6 +411,7 @@ def run_ours(args, w, rank, world, local_rank):
         "data": "synthetic (seeded video-latent generator, no model weights)",
         "config": config_of(w, world),
         "ms_per_call": ms_per_call,
+        "ms_per_call_with_kernel_events": ms_profiled,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": ncu_traffic(w), "kernel": "attn",
                      "peak_source": peaks["source"] + (" bf16 sustained x 2 (8-bit)" if fp8

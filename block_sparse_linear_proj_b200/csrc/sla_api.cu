@@ -266,26 +266,40 @@ sla_status_t launch_score(const double* qbar, const double* kbarT, const double*
     return launch_score_r<2, D, 4, 1>(qbar, kbarT, m, BH, Nq, Nk, topk, lut, st);
 }
 
-// Router: Q/K pooling (unless already pooled), W folding, fp64 score + top-k.
-sla_status_t run_router(const sla_params_t* p, const void* q, const void* k, const float* w_q,
-                        const float* w_k, int32_t* lut, void* ws, const Ws& w, bool pool_k,
-                        cudaStream_t st, cudaEvent_t kbar_ready = nullptr) {
+// Router, first part: Q (and K, unless the pre-pass pools it) pooling, W folding.
+// *m receives the folded W_q W_k^T (null without W).
+sla_status_t router_pool(const sla_params_t* p, const void* q, const void* k, const float* w_q,
+                         const float* w_k, void* ws, const Ws& w, bool pool_k, cudaStream_t st,
+                         const double** m) {
     const int BH = p->B * p->H, Nq = p->N / p->Bq, Nk = p->N / p->Bk, d = p->d;
-    double* qbar = at<double>(ws, w.qbar);
-    double* kbarT = at<double>(ws, w.kbarT);
-    launch_pool(q, p->Bq, static_cast<long long>(BH) * Nq, Nq, d, 0, qbar, st);
-    if (pool_k) launch_pool(k, p->Bk, static_cast<long long>(BH) * Nk, Nk, d, 1, kbarT, st);
-    const double* m = nullptr;
+    launch_pool(q, p->Bq, static_cast<long long>(BH) * Nq, Nq, d, 0, at<double>(ws, w.qbar), st);
+    if (pool_k) launch_pool(k, p->Bk, static_cast<long long>(BH) * Nk, Nk, d, 1, at<double>(ws, w.kbarT), st);
+    *m = nullptr;
     if (w_q || w_k) {
         Span sp(SLA_KERNEL_FOLD_W, st);
         sla::fold_w_kernel<<<d, 128, 0, st>>>(w_q, w_k, d, at<double>(ws, w.m));
-        m = at<double>(ws, w.m);
+        *m = at<double>(ws, w.m);
     }
-    if (launch_status() != SLA_OK) return SLA_ERR_CUDA;
-    // the pooled K means come from the K/V pre-pass when it runs on the side stream
+    return launch_status() == SLA_OK ? SLA_OK : SLA_ERR_CUDA;
+}
+
+// Router, second part: fp64 score + top-k (after kbar_ready, when given: the
+// pooled K means of the pre-pass on the side stream).
+sla_status_t router_score(const sla_params_t* p, int32_t* lut, void* ws, const Ws& w,
+                          const double* m, cudaStream_t st, cudaEvent_t kbar_ready = nullptr) {
+    const int BH = p->B * p->H, Nq = p->N / p->Bq, Nk = p->N / p->Bk;
     if (kbar_ready && cudaStreamWaitEvent(st, kbar_ready, 0) != cudaSuccess) return SLA_ERR_CUDA;
-    if (d == 128) return launch_score<128>(qbar, kbarT, m, BH, Nq, Nk, p->topk, lut, st);
+    const double* qbar = at<double>(ws, w.qbar);
+    const double* kbarT = at<double>(ws, w.kbarT);
+    if (p->d == 128) return launch_score<128>(qbar, kbarT, m, BH, Nq, Nk, p->topk, lut, st);
     return launch_score<64>(qbar, kbarT, m, BH, Nq, Nk, p->topk, lut, st);
+}
+
+sla_status_t run_router(const sla_params_t* p, const void* q, const void* k, const float* w_q,
+                        const float* w_k, int32_t* lut, void* ws, const Ws& w, cudaStream_t st) {
+    const double* m = nullptr;
+    const sla_status_t s = router_pool(p, q, k, w_q, w_k, ws, w, true, st, &m);
+    return s != SLA_OK ? s : router_score(p, lut, ws, w, m, st);
 }
 
 template <int D>
@@ -499,7 +513,7 @@ sla_status_t sla_route(const sla_params_t* p, const void* q, const void* k, cons
     Ws w;
     if ((s = check_ws(p, workspace, ws_bytes, w))) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    return finish(run_router(p, q, k, w_q, w_k, lut, workspace, w, true, st), st);
+    return finish(run_router(p, q, k, w_q, w_k, lut, workspace, w, st), st);
 }
 
 // ------------------------------------------------------------- side stream
@@ -510,7 +524,9 @@ sla_status_t sla_route(const sla_params_t* p, const void* q, const void* k, cons
 // writes), the attention kernel also for h_reduce.  (Pooling K a second time on the
 // caller's stream, so that the score could start before the pre-pass ends, was
 // measured slower: the extra read of K competes with the pre-pass for HBM.)  The
-// caller sees ordinary stream order.  The enqueue sequence of a call holds a
+// router's pooling and W folding are enqueued before the pre-pass, which fills the
+// GPU, so that only the score waits for it.  The caller sees ordinary stream
+// order.  The enqueue sequence of a call holds a
 // per-device lock, so concurrent host threads never cross their events.  If the
 // side stream cannot be created, everything runs on the caller's stream.
 struct SideStream {
@@ -566,9 +582,14 @@ sla_status_t sla_forward(const sla_params_t* p, const void* q, const void* k, co
     cudaStream_t sst = st;                         // the pre-pass's stream
     if (side) {
         hold = std::unique_lock<std::mutex>(side->lock);
-        if (cudaEventRecord(side->fork, st) != cudaSuccess ||
-            cudaStreamWaitEvent(side->s, side->fork, 0) != cudaSuccess)
-            return SLA_ERR_CUDA;
+        if (cudaEventRecord(side->fork, st) != cudaSuccess) return SLA_ERR_CUDA;
+    }
+    // the router's pooling and W folding go first, so that the pre-pass, which
+    // fills the GPU, does not delay them (the score needs both and the K means)
+    const double* m = nullptr;
+    if (compute && (s = router_pool(p, q, k, w_q, w_k, workspace, w, false, st, &m))) return s;
+    if (side) {
+        if (cudaStreamWaitEvent(side->s, side->fork, 0) != cudaSuccess) return SLA_ERR_CUDA;
         sst = side->s;
     }
     s = p->d == 128 ? launch_kv<128>(p, k, v, workspace, w, compute, true, false, sst, fp8, false,
@@ -585,8 +606,7 @@ sla_status_t sla_forward(const sla_params_t* p, const void* q, const void* k, co
         if (launch_status() != SLA_OK) return SLA_ERR_CUDA;
     }
     if (side && cudaEventRecord(side->stats, sst) != cudaSuccess) return SLA_ERR_CUDA;
-    if (compute && (s = run_router(p, q, k, w_q, w_k, lut_use, workspace, w, false, st,
-                                   side ? side->kbar : nullptr)))
+    if (compute && (s = router_score(p, lut_use, workspace, w, m, st, side ? side->kbar : nullptr)))
         return s;
     if (side && cudaStreamWaitEvent(st, side->stats, 0) != cudaSuccess) return SLA_ERR_CUDA;
     if (int8)
@@ -622,9 +642,14 @@ sla_status_t sla_pisa_forward(const sla_params_t* p, const void* q, const void* 
     cudaStream_t sst = st;                         // the pre-pass's stream
     if (side) {
         hold = std::unique_lock<std::mutex>(side->lock);
-        if (cudaEventRecord(side->fork, st) != cudaSuccess ||
-            cudaStreamWaitEvent(side->s, side->fork, 0) != cudaSuccess)
-            return SLA_ERR_CUDA;
+        if (cudaEventRecord(side->fork, st) != cudaSuccess) return SLA_ERR_CUDA;
+    }
+    // the router's pooling and W folding go first, so that the pre-pass, which
+    // fills the GPU, does not delay them (the score needs both and the K means)
+    const double* m = nullptr;
+    if (compute && (s = router_pool(p, q, k, w_q, w_k, workspace, w, false, st, &m))) return s;
+    if (side) {
+        if (cudaStreamWaitEvent(side->s, side->fork, 0) != cudaSuccess) return SLA_ERR_CUDA;
         sst = side->s;
     }
     s = p->d == 128 ? launch_kv<128>(p, k, v, workspace, w, compute, false, true, sst, false, fo,
@@ -633,8 +658,7 @@ sla_status_t sla_pisa_forward(const sla_params_t* p, const void* q, const void* 
                                     side ? side->kbar : nullptr);
     if (s != SLA_OK) return s;
     if (side && cudaEventRecord(side->stats, sst) != cudaSuccess) return SLA_ERR_CUDA;
-    if (compute && (s = run_router(p, q, k, w_q, w_k, lut_use, workspace, w, false, st,
-                                   side ? side->kbar : nullptr)))
+    if (compute && (s = router_score(p, lut_use, workspace, w, m, st, side ? side->kbar : nullptr)))
         return s;
     if (side && cudaStreamWaitEvent(st, side->stats, 0) != cudaSuccess) return SLA_ERR_CUDA;
     s = p->d == 128 ? launch_attn<128, sla::kModePisa>(p, q, k, v, nullptr, lut_use, out, workspace, w, st)
@@ -708,5 +732,5 @@ extern "C" sla_status_t sla_route_noalloc(const sla_params_t* p, const void* q, 
     void* scratch = nullptr;
     if ((s = route_scratch_ptr(&scratch))) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    return finish(run_router(p, q, k, w_q, w_k, lut, scratch, w, true, st), st);
+    return finish(run_router(p, q, k, w_q, w_k, lut, scratch, w, st), st);
 }
