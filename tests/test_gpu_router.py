@@ -22,6 +22,11 @@ pytestmark = pytest.mark.gpu
     (1, 2, 2048, 128, 64, 64, 32, True),      # k = Nk
     (1, 2, 2048, 128, 64, 64, 31, True),      # k = Nk - 1
     (1, 1, 1024, 128, 128, 64, 1, True),      # k = 1
+    # long rows: fewer query blocks per CTA (8, 4, 2; the MMA's 8-row tile padded)
+    (1, 1, 131072, 64, 128, 64, 37, True),    # Nk = 2048
+    (1, 1, 262144, 64, 128, 64, 100, True),   # Nk = 4096
+    (1, 1, 524288, 64, 128, 64, 300, False),  # Nk = 8192, the largest supported
+    (1, 1, 524288, 128, 128, 64, 77, True),   # the same with d = 128
 ])
 def test_route_small(B, H, N, d, Bq, Bk, k, use_w):
     inp = W.gaussian_inputs(B, H, N, d, 100 + N + k, use_w=use_w)
