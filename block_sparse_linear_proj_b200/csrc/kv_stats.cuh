@@ -11,9 +11,14 @@
 //     and (SLA) phi(K) = max(K, 0) in fp16, the A operand of its phi(K)^T V
 //     product (the conversion from bf16 is exact inside the fp16 range; values
 //     outside it are flagged).
-// phi(K)^T V uses warp-level bf16 tensor-core MMA (m16n8k16) with fp32
-// accumulation; K and V tiles of 64 tokens stream through a 3-stage cp.async
-// ring with an XOR swizzle so ldmatrix reads are conflict-free.
+// K and V tiles of 64 tokens stream through a 3-stage cp.async ring, each tile
+// stored as 64-column halves of 64 rows x 128 bytes with the 128-byte swizzle
+// (the tcgen05 operand layout).  phi(K)^T V (or, for the PISA first-order
+// term, (K - kbar_j)^T V) runs on tcgen05: after the statistics and copies
+// have read the raw K tile, it is replaced in place by phi(K) (or the centred
+// keys) in bf16, and one thread issues the block's four M = 128, K = 16
+// products (bf16 operands, both MN-major) into an fp32 accumulator in tensor
+// memory that sums the CTA's blocks.
 #pragma once
 #include "common.cuh"
 
@@ -33,31 +38,20 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
-__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1,
-                                              uint32_t& r2, uint32_t& r3) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-                 : "r"(addr));
-}
-__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4],
-                                               uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-        "{%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
 __device__ __forceinline__ uint32_t relu_bf16x2(uint32_t x) {
     __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&x);
     h = __hmax2(h, __floats2bfloat162_rn(0.f, 0.f));
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// Byte offset of element (row n, col c) in a [64][D] bf16 tile whose 16-byte
-// chunks are XOR-swizzled by (n & 7).
+// Byte offset of element (row n, col c) in a [64][D] bf16 tile stored as D/64
+// halves of 64 rows x 128 bytes, whose 16-byte chunks are XOR-swizzled by
+// (n & 7) within each 128-byte row (the 128-byte swizzle of the tensor-core
+// operand descriptors; halves are 8 KB apart).
 template <int D>
 __device__ __forceinline__ uint32_t kv_off(int n, int c) {
-    return static_cast<uint32_t>(n * D * 2 + ((((c >> 3) ^ (n & 7))) << 4) + (c & 7) * 2);
+    return static_cast<uint32_t>((c >> 6) * (kKvTok * 128) + n * 128 + ((((c >> 3) & 7) ^ (n & 7)) << 4) +
+                                 (c & 7) * 2);
 }
 
 struct KvStatsArgs {
@@ -82,6 +76,7 @@ struct KvStatsArgs {
     int center;
     // with k8: symmetric 8-bit integer K codes (absmax / 127) instead of e4m3
     int k_int8;
+    unsigned long long wait_ns;  // limit of the bounded waits on the tensor-core product
 };
 
 // grid (nchunk, BH), 256 threads.
@@ -89,11 +84,16 @@ template <int D>
 __global__ void __launch_bounds__(256, 2) kv_stats_kernel(KvStatsArgs a) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     constexpr int TILE = kKvTok * D * 2;               // bytes of one K or V tile
-    unsigned char* ring = smem_raw;                    // [stages][K tile | V tile]
-    double* kpart = reinterpret_cast<double*>(smem_raw + kKvStages * 2 * TILE);   // [256]
+    // the swizzled tiles need a 1024-byte aligned base (the launch adds 1024 bytes)
+    unsigned char* ring = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    double* kpart = reinterpret_cast<double*>(ring + kKvStages * 2 * TILE);        // [256]
     float* zpart = reinterpret_cast<float*>(kpart + 256);                          // [256]
     float* vpart = zpart + 256;                                                    // [256]
     float* amax = vpart + 256;                                                     // [2][8]
+    float* kmf = amax + 16;                                                        // [D] column means
+    uint64_t* mma_bar = reinterpret_cast<uint64_t*>(kmf + 128);                    // product done
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_bar + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const long long bh = blockIdx.y;
@@ -118,18 +118,28 @@ __global__ void __launch_bounds__(256, 2) kv_stats_kernel(KvStatsArgs a) {
         }
     };
 
-    // MMA tiling of the D x D partial: 8 warps, warp tile (D/4) x (D/2).
-    constexpr int WM = D / 4, WN = D / 2;
-    constexpr int MT = WM / 16, NT = WN / 8;
-    const int m0 = (warp & 3) * WM, n0 = (warp >> 2) * WN;
-    float acc[MT][NT][4];
-#pragma unroll
-    for (int i = 0; i < MT; ++i)
-#pragma unroll
-        for (int j = 0; j < NT; ++j)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.f;
+    // The D x D product accumulates in tensor memory: lane m = feature of the
+    // left operand, column n = feature of V.  (D = 64: an M = 128 product whose
+    // rows 64-127 repeat rows 0-63.)
     const bool do_mma = a.hpart != nullptr;
+    constexpr uint32_t TCOLS = D;                       // 64 or 128 columns
+    constexpr uint32_t ID_H = idesc_bf16(128, D, 1, 1);
+    uint32_t tmem = 0;
+    if (do_mma) {
+        if (warp == 0) {
+            tmem_alloc(tmem_slot, TCOLS);
+            tmem_relinquish();
+        }
+        if (tid == 0) {
+            mbar_init(mma_bar, 1);
+            *abort_flag = 0;
+            fence_barrier_init();
+        }
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        tmem = *tmem_slot;
+    }
 
 #pragma unroll
     for (int s = 0; s < kKvStages - 1; ++s) {
@@ -145,14 +155,8 @@ __global__ void __launch_bounds__(256, 2) kv_stats_kernel(KvStatsArgs a) {
         const int stage = blk % kKvStages;
         cp_async_wait<kKvStages - 2>();
         __syncthreads();
-        {   // prefetch the block kKvStages-1 ahead into the stage freed last iteration
-            const int nb = blk + kKvStages - 1;
-            if (nb < nblk) load_block(nb, nb % kKvStages);
-            cp_async_commit();
-        }
-        const unsigned char* kt = ring + stage * 2 * TILE;
+        unsigned char* kt = ring + stage * 2 * TILE;
         const unsigned char* vt = kt + TILE;
-        const uint32_t kt_s = smem_u32(kt), vt_s = smem_u32(vt);
 
         // column statistics of this block
         {
@@ -267,62 +271,21 @@ __global__ void __launch_bounds__(256, 2) kv_stats_kernel(KvStatsArgs a) {
             }
         }
 
-        // centred keys: this block's column means (from the column statistics
-        // above), for the two feature rows of each A fragment
-        float kb0[MT], kb1[MT];
-        if (a.center) {
-            __syncthreads();
-#pragma unroll
-            for (int i = 0; i < MT; ++i) {
-                const int c0 = m0 + i * 16 + (lane >> 2);
-                double s0 = 0.0, s1 = 0.0;
-#pragma unroll
-                for (int hh = 0; hh < HALVES; ++hh) {
-                    s0 += kpart[hh * D + c0];
-                    s1 += kpart[hh * D + c0 + 8];
-                }
-                kb0[i] = static_cast<float>(s0 * (1.0 / kKvTok));
-                kb1[i] = static_cast<float>(s1 * (1.0 / kKvTok));
-            }
-        }
-        if (do_mma) {
-#pragma unroll
-            for (int k0 = 0; k0 < kKvTok; k0 += 16) {
-                uint32_t afr[MT][4];
-#pragma unroll
-                for (int i = 0; i < MT; ++i) {
-                    // A = phi(K)^T: matrices (n k0..+7 | k0+8..+15) x (c m..m+7 | m+8..m+15)
-                    const int n = k0 + (lane & 7) + ((lane >> 4) << 3);
-                    const int c = m0 + i * 16 + (((lane >> 3) & 1) << 3);
-                    ldsm_x4_trans(kt_s + kv_off<D>(n, c), afr[i][0], afr[i][1], afr[i][2],
-                                  afr[i][3]);
-                    if (a.center) {
-                        // fragments 0, 2 hold feature row m + g, fragments 1, 3 row m + 8 + g
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float kb = (e & 1) ? kb1[i] : kb0[i];
-                            afr[i][e] = pack_bf16(bf16lo(afr[i][e]) - kb, bf16hi(afr[i][e]) - kb);
-                        }
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) afr[i][e] = relu_bf16x2(afr[i][e]);
-                    }
-                }
-#pragma unroll
-                for (int j = 0; j < NT; j += 2) {
-                    const int n = k0 + (lane & 7) + (((lane >> 3) & 1) << 3);
-                    const int e = n0 + j * 8 + ((lane >> 4) << 3);
-                    uint32_t b0, b1, b2, b3;
-                    ldsm_x4_trans(vt_s + kv_off<D>(n, e), b0, b1, b2, b3);
-#pragma unroll
-                    for (int i = 0; i < MT; ++i) {
-                        mma_bf16_16816(acc[i][j], afr[i], b0, b1);
-                        mma_bf16_16816(acc[i][j + 1], afr[i], b2, b3);
-                    }
-                }
-            }
+        // every raw read of this K tile is done, the column partials are in
+        // shared memory, and (thread 0) the previous block's product has
+        // completed, so its ring stage may be refilled
+        if (do_mma && blk > 0 && tid == 0 && !*abort_flag &&
+            !mbar_wait(mma_bar, (blk - 1) & 1, abort_flag, a.wait_ns)) {
+            report(kStatusTimeout);
+            *abort_flag = 1;
         }
         __syncthreads();
+        const bool dead = do_mma && *abort_flag;
+        {   // prefetch the block kKvStages-1 ahead into the stage of the previous block
+            const int nb = blk + kKvStages - 1;
+            if (nb < nblk && !dead) load_block(nb, nb % kKvStages);
+            cp_async_commit();
+        }
         if (tid < D) {
             double ks = 0.0;
             float zs = 0.f, vs = 0.f;
@@ -338,22 +301,76 @@ __global__ void __launch_bounds__(256, 2) kv_stats_kernel(KvStatsArgs a) {
             if (a.zj) a.zj[(bh * a.Nk + j) * D + tid] = zs;
             if (a.kc) a.kc[(bh * a.Nk + j) * D + tid] = __float2bfloat16_rn(static_cast<float>(kmean));
             if (a.vbar) a.vbar[(bh * a.Nk + j) * D + tid] = __float2half_rn(vs * (1.f / kKvTok));
+            kmf[tid] = static_cast<float>(kmean);
+        }
+        if (do_mma && a.center) __syncthreads();        // the column means, for the centring
+        if (do_mma && !dead) {
+            // the product's left operand in place: phi(K) = max(K, 0), or the keys
+            // centred by this block's column means (bf16)
+            constexpr int CPR = D / 8;
+            for (int q = tid; q < kKvTok * CPR; q += 256) {
+                const int n = q / CPR, u = q % CPR;
+                uint4* px = reinterpret_cast<uint4*>(kt + kv_off<D>(n, u * 8));
+                uint4 x = *px;
+                uint32_t w[4] = {x.x, x.y, x.z, x.w};
+                if (a.center) {
+                    const float4 m0 = *reinterpret_cast<const float4*>(kmf + u * 8);
+                    const float4 m1 = *reinterpret_cast<const float4*>(kmf + u * 8 + 4);
+                    w[0] = pack_bf16(bf16lo(w[0]) - m0.x, bf16hi(w[0]) - m0.y);
+                    w[1] = pack_bf16(bf16lo(w[1]) - m0.z, bf16hi(w[1]) - m0.w);
+                    w[2] = pack_bf16(bf16lo(w[2]) - m1.x, bf16hi(w[2]) - m1.y);
+                    w[3] = pack_bf16(bf16lo(w[3]) - m1.z, bf16hi(w[3]) - m1.w);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) w[e] = relu_bf16x2(w[e]);
+                }
+                *px = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+            fence_proxy_async_smem();
+        }
+        __syncthreads();
+        if (do_mma && !dead && tid == 0) {
+            tc_fence_after();
+            const uint32_t kt_s = smem_u32(kt), vt_s = smem_u32(vt);
+            const uint32_t lbo = D == 128 ? kKvTok * 128 : 0;     // the second 64-feature half
+#pragma unroll
+            for (int kk = 0; kk < kKvTok / 16; ++kk) {
+                const uint64_t ad = sdesc(kt_s + kk * 2048, lbo, 1024, kSwizzle128B);
+                const uint64_t bd = sdesc(vt_s + kk * 2048, kKvTok * 128, 1024, kSwizzle128B);
+                umma_f16_ss(tmem, ad, bd, ID_H, (blk > 0 || kk > 0) ? 1u : 0u);
+            }
+            umma_commit(mma_bar);
         }
     }
     cp_async_wait<0>();
 
     if (do_mma) {
-        float* hp = a.hpart + (bh * a.nchunk + chunk) * static_cast<long long>(D) * D;
-        const int g = lane >> 2, t = lane & 3;
+        // the last product, then the accumulator to this chunk's partial
+        if (tid == 0 && !*abort_flag && !mbar_wait(mma_bar, (nblk - 1) & 1, abort_flag, a.wait_ns)) {
+            report(kStatusTimeout);
+            *abort_flag = 1;
+        }
+        __syncthreads();
+        tc_fence_after();
+        if (!*abort_flag && warp < D / 32) {
+            float* hp = a.hpart + (bh * a.nchunk + chunk) * static_cast<long long>(D) * D;
+            const int r = warp * 32 + lane;                  // feature row of H
+            const uint32_t tl = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+#pragma unroll 1
+            for (int cc = 0; cc < D; cc += 32) {
+                uint32_t v[32];
+                tmem_ld32(tl + cc, v);
+                tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < MT; ++i)
-#pragma unroll
-            for (int j = 0; j < NT; ++j) {
-                const int r = m0 + i * 16 + g, c = n0 + j * 8 + 2 * t;
-                *reinterpret_cast<float2*>(hp + r * D + c) = make_float2(acc[i][j][0], acc[i][j][1]);
-                *reinterpret_cast<float2*>(hp + (r + 8) * D + c) =
-                    make_float2(acc[i][j][2], acc[i][j][3]);
+                for (int x = 0; x < 32; x += 4)
+                    *reinterpret_cast<float4*>(hp + r * D + cc + x) =
+                        make_float4(__uint_as_float(v[x]), __uint_as_float(v[x + 1]),
+                                    __uint_as_float(v[x + 2]), __uint_as_float(v[x + 3]));
             }
+        }
+        tc_fence_before();
+        __syncthreads();
+        if (warp == 0) tmem_dealloc(tmem, TCOLS);
     }
 }
 

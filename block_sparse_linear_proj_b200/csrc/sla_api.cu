@@ -328,7 +328,11 @@ sla_status_t launch_kv(const sla_params_t* p, const void* k, const void* v, void
     a.sk = fp8 ? at<float>(ws, w.sk) : nullptr;
     a.sv = fp8 ? at<float>(ws, w.sv) : nullptr;
     a.k_int8 = (fp8 && k_int8) ? 1 : 0;
-    const size_t smem = sla::kKvStages * 2 * 64 * D * 2 + 256 * 8 + 2 * 256 * 4 + 16 * 4;
+    a.wait_ns = wait_limit_ns();
+    // alignment slack, K/V ring, column partials, maxima, column means, barrier,
+    // TMEM slot, flag
+    const size_t smem = 1024 + sla::kKvStages * 2 * 64 * D * 2 + 256 * 8 + 2 * 256 * 4 + 16 * 4 +
+                        128 * 4 + 16;
     auto kern = sla::kv_stats_kernel<D>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
