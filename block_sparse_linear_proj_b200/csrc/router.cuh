@@ -137,17 +137,74 @@ __device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v)
     return v;
 }
 
+// qhat = qbar . M in place, 16 pooled rows per CTA (rows [16 b, 16 b + 16) of
+// the [nrows][D] fp64 array x), on the fp64 MMA: warp w computes output columns
+// [w D/8, (w+1) D/8) of both 8-row tiles from M fragments three k-steps ahead.
+// Each CTA reads its rows into shared memory before writing them back.
+template <int D>
+__global__ void __launch_bounds__(256) project_kernel(double* __restrict__ x, long long nrows,
+                                                      const double* __restrict__ m) {
+    constexpr int LDQ = D + 4, NT = D / 64;
+    __shared__ double xs[16 * LDQ];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    const long long r0 = static_cast<long long>(blockIdx.x) * 16;
+    const int rows = static_cast<int>(min(16LL, nrows - r0));
+    for (int a = tid; a < 16 * D; a += 256) {
+        const int r = a / D, c = a % D;
+        xs[r * LDQ + c] = r < rows ? x[(r0 + r) * D + c] : 0.0;
+    }
+    __syncthreads();
+    double acc[2][NT][2];
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) acc[mt][nt][0] = acc[mt][nt][1] = 0.0;
+    const int n0 = warp * (D / 8);
+    double bm[4][NT];
+    auto load_m = [&](double (&b)[NT], int c0) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) b[nt] = __ldg(m + (c0 + t) * D + n0 + nt * 8 + g);
+    };
+#pragma unroll
+    for (int u = 0; u < 4; ++u) load_m(bm[u], u * 4);
+#pragma unroll 1
+    for (int ks = 0; ks < D / 4; ks += 4) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            double a[2];
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt) a[mt] = xs[(mt * 8 + g) * LDQ + (ks + u) * 4 + t];
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) dmma_884(acc[mt][nt], a[mt], bm[u][nt]);
+            if (ks + u + 4 < D / 4) load_m(bm[u], (ks + u + 4) * 4);
+        }
+    }
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+        const int r = mt * 8 + g;
+        if (r >= rows) continue;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            double* dst = x + (r0 + r) * D + n0 + nt * 8 + 2 * t;
+            dst[0] = acc[mt][nt][0];
+            dst[1] = acc[mt][nt][1];
+        }
+    }
+}
+
 // One CTA: head bh = blockIdx.y, query blocks i0 = blockIdx.x * R ... i0 + R - 1.
-// Both products run on the fp64 MMA (m8n8k4, eight-row tiles; R < 8 pads the tile).
-// Shared memory: qhat [8 MT][D + 4] fp64 (rows padded so that the A-fragment
-// loads spread over the banks), hist [8][256] u32, keys [R][max(Nk, D + 4)] u64
-// (the key area doubles as the staging buffer of the pooled rows in step 1).
+// qhat = qbar M (project_kernel) or qbar itself.  The product runs on the fp64
+// MMA (m8n8k4, eight-row tiles; R < 8 pads the tile).  Shared memory: qhat
+// [8 MT][D + 4] fp64 (rows padded so that the A-fragment loads spread over the
+// banks), hist [8][256] u32, keys [R][max(Nk, D + 4)] u64.
 // DEPTH: k-steps of K fragments in flight per warp; MINB: CTAs per SM the
 // register budget is sized for.
 template <int R, int D, int DEPTH, int MINB>
-__global__ void __launch_bounds__(256, MINB) score_topk_kernel(const double* __restrict__ qbar,
-                                                         const double* __restrict__ kbarT,
-                                                         const double* __restrict__ m, int Nq,
+__global__ void __launch_bounds__(256, MINB) score_topk_kernel(const double* __restrict__ qhat_all,
+                                                         const double* __restrict__ kbarT, int Nq,
                                                          int Nk, int topk,
                                                          int32_t* __restrict__ lut) {
     constexpr int MT = R >= 8 ? R / 8 : 1;      // eight-row MMA tiles
@@ -163,60 +220,15 @@ __global__ void __launch_bounds__(256, MINB) score_topk_kernel(const double* __r
     const long long bh = blockIdx.y;
     const int i0 = blockIdx.x * R;
     const int nrows = min(R, Nq - i0);
-    const double* qb = qbar + (bh * Nq + i0) * D;
+    const double* qhat = qhat_all + (bh * Nq + i0) * D;
     const double* kt = kbarT + bh * D * static_cast<long long>(Nk);
 
-    // 1. qhat = qbar . M for the R rows (padding rows are zero).  Warp w computes
-    //    output columns [w D/8, (w+1) D/8) for every row.
-    {
-        double* stage = m ? reinterpret_cast<double*>(keys) : qh;      // [8 MT][LDQ]
-        for (int a = tid; a < 8 * MT * D; a += 256) {
-            const int r = a / D, c = a % D;
-            stage[r * LDQ + c] = r < nrows ? qb[static_cast<long long>(r) * D + c] : 0.0;
-        }
-        __syncthreads();
-        if (m) {
-            constexpr int NT = D / 64;               // 8-column tiles per warp
-            double acc[MT][NT][2];
-#pragma unroll
-            for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) acc[mt][nt][0] = acc[mt][nt][1] = 0.0;
-            const int n0 = warp * (D / 8);
-            // M fragments in a ring of 2 DEPTH k-steps, refilled right after use
-            constexpr int MD = 2 * DEPTH;
-            double bm[MD][NT];
-            auto load_m = [&](double (&b)[NT], int c0) {
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) b[nt] = __ldg(m + (c0 + t) * D + n0 + nt * 8 + g);
-            };
-#pragma unroll
-            for (int u = 0; u < MD; ++u) load_m(bm[u], u * 4);
-#pragma unroll 1
-            for (int ks = 0; ks < D / 4; ks += MD) {
-#pragma unroll
-                for (int u = 0; u < MD; ++u) {
-                    double a[MT];
-#pragma unroll
-                    for (int mt = 0; mt < MT; ++mt) a[mt] = stage[(mt * 8 + g) * LDQ + (ks + u) * 4 + t];
-#pragma unroll
-                    for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) dmma_884(acc[mt][nt], a[mt], bm[u][nt]);
-                    if (ks + u + MD < D / 4) load_m(bm[u], (ks + u + MD) * 4);
-                }
-            }
-#pragma unroll
-            for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    double* dst = qh + (mt * 8 + g) * LDQ + n0 + nt * 8 + 2 * t;
-                    dst[0] = acc[mt][nt][0];
-                    dst[1] = acc[mt][nt][1];
-                }
-            __syncthreads();
-        }
+    // 1. the R rows of qhat (padding rows are zero)
+    for (int a = tid; a < 8 * MT * D; a += 256) {
+        const int r = a / D, c = a % D;
+        qh[r * LDQ + c] = r < nrows ? qhat[static_cast<long long>(r) * D + c] : 0.0;
     }
+    __syncthreads();
 
     // 2. scores s[r][j] = qhat_r . kbar_j on the fp64 MMA.  Warp w covers 64
     //    columns (eight 8-column tiles) at a time; a ring of DEPTH k-steps of B

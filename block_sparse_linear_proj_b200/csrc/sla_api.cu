@@ -227,17 +227,16 @@ void launch_pool(const void* x, int rows, long long nblk_total, int nblk_per_hea
         sla::pool_mean_kernel<64><<<grid, 256, 0, st>>>(xb, rows, nblk_total, nblk_per_head, out_mode, out);
 }
 
-// shared memory of score_topk_kernel<R, D>: qhat tiles, histograms, keys (which
-// also stage the pooled rows)
+// shared memory of score_topk_kernel<R, D>: qhat tiles, histograms, keys
 size_t score_smem(int R, int D, int Nk) {
     const size_t mt = R >= 8 ? R / 8 : 1, ldq = D + 4;
     const size_t ldk = std::max<size_t>(Nk, ldq);
-    return 8 * mt * ldq * 8 + 8 * 256 * 4 + std::max(R * ldk, 8 * mt * ldq) * 8;
+    return 8 * mt * ldq * 8 + 8 * 256 * 4 + R * ldk * 8;
 }
 
 template <int R, int D, int DEPTH, int MINB>
-sla_status_t launch_score_r(const double* qbar, const double* kbarT, const double* m, int BH,
-                            int Nq, int Nk, int topk, int32_t* lut, cudaStream_t st) {
+sla_status_t launch_score_r(const double* qhat, const double* kbarT, int BH, int Nq, int Nk,
+                            int topk, int32_t* lut, cudaStream_t st) {
     const size_t smem = score_smem(R, D, Nk);
     auto kern = sla::score_topk_kernel<R, D, DEPTH, MINB>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -245,40 +244,48 @@ sla_status_t launch_score_r(const double* qbar, const double* kbarT, const doubl
         return SLA_ERR_CUDA;
     dim3 grid((Nq + R - 1) / R, BH);
     Span sp(SLA_KERNEL_SCORE_TOPK, st);
-    kern<<<grid, 256, smem, st>>>(qbar, kbarT, m, Nq, Nk, topk, lut);
+    kern<<<grid, 256, smem, st>>>(qhat, kbarT, Nq, Nk, topk, lut);
     return launch_status();
 }
 
 template <int D>
-sla_status_t launch_score(const double* qbar, const double* kbarT, const double* m, int BH,
-                          int Nq, int Nk, int topk, int32_t* lut, cudaStream_t st) {
+sla_status_t launch_score(const double* qhat, const double* kbarT, int BH, int Nq, int Nk,
+                          int topk, int32_t* lut, cudaStream_t st) {
     // 16 query blocks per CTA (two 8-row tiles of the fp64 MMA per K fragment).
     // Where two CTAs fit an SM's shared memory, a two-deep fragment ring keeps
     // the registers within two CTAs; otherwise one CTA per SM with a four-deep ring.
     constexpr size_t two = 113 * 1024, one = 200 * 1024;
     if (score_smem(16, D, Nk) <= two)
-        return launch_score_r<16, D, 2, 2>(qbar, kbarT, m, BH, Nq, Nk, topk, lut, st);
+        return launch_score_r<16, D, 2, 2>(qhat, kbarT, BH, Nq, Nk, topk, lut, st);
     if (score_smem(16, D, Nk) <= one)
-        return launch_score_r<16, D, 4, 1>(qbar, kbarT, m, BH, Nq, Nk, topk, lut, st);
-    if (score_smem(8, D, Nk) <= one) return launch_score_r<8, D, 4, 1>(qbar, kbarT, m, BH, Nq, Nk, topk, lut, st);
-    if (score_smem(4, D, Nk) <= one) return launch_score_r<4, D, 4, 1>(qbar, kbarT, m, BH, Nq, Nk, topk, lut, st);
+        return launch_score_r<16, D, 4, 1>(qhat, kbarT, BH, Nq, Nk, topk, lut, st);
+    if (score_smem(8, D, Nk) <= one) return launch_score_r<8, D, 4, 1>(qhat, kbarT, BH, Nq, Nk, topk, lut, st);
+    if (score_smem(4, D, Nk) <= one) return launch_score_r<4, D, 4, 1>(qhat, kbarT, BH, Nq, Nk, topk, lut, st);
     if (score_smem(2, D, Nk) > 232448) return SLA_ERR_UNSUPPORTED;   // a score row beyond shared memory
-    return launch_score_r<2, D, 4, 1>(qbar, kbarT, m, BH, Nq, Nk, topk, lut, st);
+    return launch_score_r<2, D, 4, 1>(qhat, kbarT, BH, Nq, Nk, topk, lut, st);
 }
 
-// Router, first part: Q (and K, unless the pre-pass pools it) pooling, W folding.
-// *m receives the folded W_q W_k^T (null without W).
+// Router, first part: Q (and K, unless the pre-pass pools it) pooling, W folding
+// and the projection qhat = qbar W_q W_k^T (in place).
 sla_status_t router_pool(const sla_params_t* p, const void* q, const void* k, const float* w_q,
-                         const float* w_k, void* ws, const Ws& w, bool pool_k, cudaStream_t st,
-                         const double** m) {
+                         const float* w_k, void* ws, const Ws& w, bool pool_k, cudaStream_t st) {
     const int BH = p->B * p->H, Nq = p->N / p->Bq, Nk = p->N / p->Bk, d = p->d;
-    launch_pool(q, p->Bq, static_cast<long long>(BH) * Nq, Nq, d, 0, at<double>(ws, w.qbar), st);
+    double* qbar = at<double>(ws, w.qbar);
+    launch_pool(q, p->Bq, static_cast<long long>(BH) * Nq, Nq, d, 0, qbar, st);
     if (pool_k) launch_pool(k, p->Bk, static_cast<long long>(BH) * Nk, Nk, d, 1, at<double>(ws, w.kbarT), st);
-    *m = nullptr;
     if (w_q || w_k) {
-        Span sp(SLA_KERNEL_FOLD_W, st);
-        sla::fold_w_kernel<<<d, 128, 0, st>>>(w_q, w_k, d, at<double>(ws, w.m));
-        *m = at<double>(ws, w.m);
+        double* m = at<double>(ws, w.m);
+        {
+            Span sp(SLA_KERNEL_FOLD_W, st);
+            sla::fold_w_kernel<<<d, 128, 0, st>>>(w_q, w_k, d, m);
+        }
+        const long long rows = static_cast<long long>(BH) * Nq;
+        const int grid = static_cast<int>((rows + 15) / 16);
+        Span sp(SLA_KERNEL_PROJECT, st);
+        if (d == 128)
+            sla::project_kernel<128><<<grid, 256, 0, st>>>(qbar, rows, m);
+        else
+            sla::project_kernel<64><<<grid, 256, 0, st>>>(qbar, rows, m);
     }
     return launch_status() == SLA_OK ? SLA_OK : SLA_ERR_CUDA;
 }
@@ -286,20 +293,19 @@ sla_status_t router_pool(const sla_params_t* p, const void* q, const void* k, co
 // Router, second part: fp64 score + top-k (after kbar_ready, when given: the
 // pooled K means of the pre-pass on the side stream).
 sla_status_t router_score(const sla_params_t* p, int32_t* lut, void* ws, const Ws& w,
-                          const double* m, cudaStream_t st, cudaEvent_t kbar_ready = nullptr) {
+                          cudaStream_t st, cudaEvent_t kbar_ready = nullptr) {
     const int BH = p->B * p->H, Nq = p->N / p->Bq, Nk = p->N / p->Bk;
     if (kbar_ready && cudaStreamWaitEvent(st, kbar_ready, 0) != cudaSuccess) return SLA_ERR_CUDA;
-    const double* qbar = at<double>(ws, w.qbar);
+    const double* qhat = at<double>(ws, w.qbar);
     const double* kbarT = at<double>(ws, w.kbarT);
-    if (p->d == 128) return launch_score<128>(qbar, kbarT, m, BH, Nq, Nk, p->topk, lut, st);
-    return launch_score<64>(qbar, kbarT, m, BH, Nq, Nk, p->topk, lut, st);
+    if (p->d == 128) return launch_score<128>(qhat, kbarT, BH, Nq, Nk, p->topk, lut, st);
+    return launch_score<64>(qhat, kbarT, BH, Nq, Nk, p->topk, lut, st);
 }
 
 sla_status_t run_router(const sla_params_t* p, const void* q, const void* k, const float* w_q,
                         const float* w_k, int32_t* lut, void* ws, const Ws& w, cudaStream_t st) {
-    const double* m = nullptr;
-    const sla_status_t s = router_pool(p, q, k, w_q, w_k, ws, w, true, st, &m);
-    return s != SLA_OK ? s : router_score(p, lut, ws, w, m, st);
+    const sla_status_t s = router_pool(p, q, k, w_q, w_k, ws, w, true, st);
+    return s != SLA_OK ? s : router_score(p, lut, ws, w, st);
 }
 
 template <int D>
@@ -588,10 +594,10 @@ sla_status_t sla_forward(const sla_params_t* p, const void* q, const void* k, co
         hold = std::unique_lock<std::mutex>(side->lock);
         if (cudaEventRecord(side->fork, st) != cudaSuccess) return SLA_ERR_CUDA;
     }
-    // the router's pooling and W folding go first, so that the pre-pass, which
-    // fills the GPU, does not delay them (the score needs both and the K means)
-    const double* m = nullptr;
-    if (compute && (s = router_pool(p, q, k, w_q, w_k, workspace, w, false, st, &m))) return s;
+    // the router's pooling, W folding and projection go first, so that the
+    // pre-pass, which fills the GPU, does not delay them (the score needs them
+    // and the K means)
+    if (compute && (s = router_pool(p, q, k, w_q, w_k, workspace, w, false, st))) return s;
     if (side) {
         if (cudaStreamWaitEvent(side->s, side->fork, 0) != cudaSuccess) return SLA_ERR_CUDA;
         sst = side->s;
@@ -610,7 +616,7 @@ sla_status_t sla_forward(const sla_params_t* p, const void* q, const void* k, co
         if (launch_status() != SLA_OK) return SLA_ERR_CUDA;
     }
     if (side && cudaEventRecord(side->stats, sst) != cudaSuccess) return SLA_ERR_CUDA;
-    if (compute && (s = router_score(p, lut_use, workspace, w, m, st, side ? side->kbar : nullptr)))
+    if (compute && (s = router_score(p, lut_use, workspace, w, st, side ? side->kbar : nullptr)))
         return s;
     if (side && cudaStreamWaitEvent(st, side->stats, 0) != cudaSuccess) return SLA_ERR_CUDA;
     if (int8)
@@ -648,10 +654,10 @@ sla_status_t sla_pisa_forward(const sla_params_t* p, const void* q, const void* 
         hold = std::unique_lock<std::mutex>(side->lock);
         if (cudaEventRecord(side->fork, st) != cudaSuccess) return SLA_ERR_CUDA;
     }
-    // the router's pooling and W folding go first, so that the pre-pass, which
-    // fills the GPU, does not delay them (the score needs both and the K means)
-    const double* m = nullptr;
-    if (compute && (s = router_pool(p, q, k, w_q, w_k, workspace, w, false, st, &m))) return s;
+    // the router's pooling, W folding and projection go first, so that the
+    // pre-pass, which fills the GPU, does not delay them (the score needs them
+    // and the K means)
+    if (compute && (s = router_pool(p, q, k, w_q, w_k, workspace, w, false, st))) return s;
     if (side) {
         if (cudaStreamWaitEvent(side->s, side->fork, 0) != cudaSuccess) return SLA_ERR_CUDA;
         sst = side->s;
@@ -662,7 +668,7 @@ sla_status_t sla_pisa_forward(const sla_params_t* p, const void* q, const void* 
                                     side ? side->kbar : nullptr);
     if (s != SLA_OK) return s;
     if (side && cudaEventRecord(side->stats, sst) != cudaSuccess) return SLA_ERR_CUDA;
-    if (compute && (s = router_score(p, lut_use, workspace, w, m, st, side ? side->kbar : nullptr)))
+    if (compute && (s = router_score(p, lut_use, workspace, w, st, side ? side->kbar : nullptr)))
         return s;
     if (side && cudaStreamWaitEvent(st, side->stats, 0) != cudaSuccess) return SLA_ERR_CUDA;
     s = p->d == 128 ? launch_attn<128, sla::kModePisa>(p, q, k, v, nullptr, lut_use, out, workspace, w, st)

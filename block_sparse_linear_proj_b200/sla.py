@@ -40,7 +40,7 @@ SLA_OUT_FP32 = 1
 EXPORTED = ("sla_workspace_size", "sla_route", "sla_forward", "sla_pisa_forward",
             "sla_status_string", "sla_check_device_status", "sla_version",
             "sla_profile_enable", "sla_profile_read", "sla_route_noalloc")
-KERNEL_KINDS = ("pool", "kv_stats", "h_reduce", "fold_w", "score_topk", "attn", "quant_q")
+KERNEL_KINDS = ("pool", "kv_stats", "h_reduce", "fold_w", "score_topk", "attn", "quant_q", "project")
 
 
 class SlaParams(ctypes.Structure):

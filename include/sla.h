@@ -204,8 +204,9 @@ typedef enum {
     SLA_KERNEL_FOLD_W = 3,      /* W_q W_k^T                                    */
     SLA_KERNEL_SCORE_TOPK = 4,  /* fp64 block score + top-k                     */
     SLA_KERNEL_ATTN = 5,        /* sparse / PISA attention + fused epilogue     */
-    SLA_KERNEL_QUANT_Q = 6,     /* e4m3 quantisation of Q (FP8 sparse branch)   */
-    SLA_KERNEL_KINDS = 7
+    SLA_KERNEL_QUANT_Q = 6,     /* 8-bit quantisation of Q (FP8, INT8 branch)   */
+    SLA_KERNEL_PROJECT = 7,     /* pooled Q times W_q W_k^T (router with W)      */
+    SLA_KERNEL_KINDS = 8
 } sla_kernel_kind_t;
 
 sla_status_t sla_profile_enable(int32_t on);
