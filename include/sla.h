@@ -26,7 +26,7 @@
  *    default stream).  Arguments are validated on the host before anything is
  *    enqueued; on any error nothing is launched.  sla_forward and
  *    sla_pisa_forward run their K/V pre-pass on a side stream owned by the
- *    library (one per device, created with two events on first use; no device
+ *    library (one per device, created with three events on first use; no device
  *    memory), forked from and joined back into `stream` with events, so work
  *    the caller enqueues on `stream` afterwards sees every result, and a
  *    capture of `stream` includes that work.
