@@ -157,6 +157,13 @@ __global__ void __launch_bounds__(256, 2) kv_stats_kernel(KvStatsArgs a) {
         __syncthreads();
         unsigned char* kt = ring + stage * 2 * TILE;
         const unsigned char* vt = kt + TILE;
+        // without the product, the stage of the previous block is free now:
+        // prefetch kKvStages-1 blocks ahead right away
+        if (!do_mma) {
+            const int nb = blk + kKvStages - 1;
+            if (nb < nblk) load_block(nb, nb % kKvStages);
+            cp_async_commit();
+        }
 
         // column statistics of this block
         {
@@ -281,7 +288,7 @@ __global__ void __launch_bounds__(256, 2) kv_stats_kernel(KvStatsArgs a) {
         }
         __syncthreads();
         const bool dead = do_mma && *abort_flag;
-        {   // prefetch the block kKvStages-1 ahead into the stage of the previous block
+        if (do_mma) {   // the previous block's product is done: refill its stage
             const int nb = blk + kKvStages - 1;
             if (nb < nblk && !dead) load_block(nb, nb % kKvStages);
             cp_async_commit();
