@@ -44,14 +44,17 @@ __device__ __forceinline__ uint32_t relu_bf16x2(uint32_t x) {
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// Byte offset of element (row n, col c) in a [64][D] bf16 tile stored as D/64
-// halves of 64 rows x 128 bytes, whose 16-byte chunks are XOR-swizzled by
-// (n & 7) within each 128-byte row (the 128-byte swizzle of the tensor-core
-// operand descriptors; halves are 8 KB apart).
-template <int D>
+// Byte offset of element (row n, col c) in a [64][D] bf16 tile.  TC (the tile
+// is a tensor-core operand): D/64 halves of 64 rows x 128 bytes, whose 16-byte
+// chunks are XOR-swizzled by (n & 7) within each 128-byte row (the 128-byte
+// swizzle of the operand descriptors; halves are 8 KB apart).  Otherwise rows
+// of 2D bytes whose 16-byte chunks are XOR-swizzled by (n & 7).
+template <int D, bool TC>
 __device__ __forceinline__ uint32_t kv_off(int n, int c) {
-    return static_cast<uint32_t>((c >> 6) * (kKvTok * 128) + n * 128 + ((((c >> 3) & 7) ^ (n & 7)) << 4) +
-                                 (c & 7) * 2);
+    if (TC)
+        return static_cast<uint32_t>((c >> 6) * (kKvTok * 128) + n * 128 +
+                                     ((((c >> 3) & 7) ^ (n & 7)) << 4) + (c & 7) * 2);
+    return static_cast<uint32_t>(n * D * 2 + (((c >> 3) ^ (n & 7)) << 4) + (c & 7) * 2);
 }
 
 struct KvStatsArgs {
@@ -79,8 +82,9 @@ struct KvStatsArgs {
     unsigned long long wait_ns;  // limit of the bounded waits on the tensor-core product
 };
 
-// grid (nchunk, BH), 256 threads.
-template <int D>
+// grid (nchunk, BH), 256 threads.  TC: the call wants the tensor-core product
+// (hpart non-null); without it the tiles keep a plain swizzled row layout.
+template <int D, bool TC>
 __global__ void __launch_bounds__(256, 2) kv_stats_kernel(KvStatsArgs a) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     constexpr int TILE = kKvTok * D * 2;               // bytes of one K or V tile
@@ -112,7 +116,7 @@ __global__ void __launch_bounds__(256, 2) kv_stats_kernel(KvStatsArgs a) {
         constexpr int CPR = D / 8;                      // 16-byte chunks per row
         for (int q = tid; q < kKvTok * CPR; q += 256) {
             const int n = q / CPR, u = q % CPR;
-            const uint32_t off = kv_off<D>(n, u * 8);
+            const uint32_t off = kv_off<D, TC>(n, u * 8);
             cp_async16(kd + off, kh + (row0 + n) * D + u * 8);
             if (want_v) cp_async16(vd + off, vh + (row0 + n) * D + u * 8);
         }
@@ -121,7 +125,7 @@ __global__ void __launch_bounds__(256, 2) kv_stats_kernel(KvStatsArgs a) {
     // The D x D product accumulates in tensor memory: lane m = feature of the
     // left operand, column n = feature of V.  (D = 64: an M = 128 product whose
     // rows 64-127 repeat rows 0-63.)
-    const bool do_mma = a.hpart != nullptr;
+    const bool do_mma = TC && a.hpart != nullptr;
     constexpr uint32_t TCOLS = D;                       // 64 or 128 columns
     constexpr uint32_t ID_H = idesc_bf16(128, D, 1, 1);
     uint32_t tmem = 0;
@@ -171,13 +175,13 @@ __global__ void __launch_bounds__(256, 2) kv_stats_kernel(KvStatsArgs a) {
             float zs = 0.f, vs = 0.f, kmax = 0.f;
             for (int n = half * RPH; n < (half + 1) * RPH; ++n) {
                 const float kv = __bfloat162float(
-                    *reinterpret_cast<const __nv_bfloat16*>(kt + kv_off<D>(n, col)));
+                    *reinterpret_cast<const __nv_bfloat16*>(kt + kv_off<D, TC>(n, col)));
                 ks += static_cast<double>(kv);
                 zs += fmaxf(kv, 0.f);
                 kmax = fmaxf(kmax, fabsf(kv));
                 if (want_v)
                     vs += __bfloat162float(
-                        *reinterpret_cast<const __nv_bfloat16*>(vt + kv_off<D>(n, col)));
+                        *reinterpret_cast<const __nv_bfloat16*>(vt + kv_off<D, TC>(n, col)));
             }
             kpart[tid] = ks;
             zpart[tid] = zs;
@@ -188,7 +192,7 @@ __global__ void __launch_bounds__(256, 2) kv_stats_kernel(KvStatsArgs a) {
                 float vmax = 0.f;
                 for (int n = half * RPH; n < (half + 1) * RPH; ++n)
                     vmax = fmaxf(vmax, fabsf(__bfloat162float(
-                        *reinterpret_cast<const __nv_bfloat16*>(vt + kv_off<D>(n, col)))));
+                        *reinterpret_cast<const __nv_bfloat16*>(vt + kv_off<D, TC>(n, col)))));
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) {
                     kmax = fmaxf(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
@@ -205,7 +209,7 @@ __global__ void __launch_bounds__(256, 2) kv_stats_kernel(KvStatsArgs a) {
             bool bad = false;
             for (int q = tid; q < kKvTok * CPR; q += 256) {
                 const int n = q / CPR, u = q % CPR;
-                const uint4 x = *reinterpret_cast<const uint4*>(vt + kv_off<D>(n, u * 8));
+                const uint4 x = *reinterpret_cast<const uint4*>(vt + kv_off<D, TC>(n, u * 8));
                 const uint32_t w[4] = {x.x, x.y, x.z, x.w};
                 uint32_t h[4];
 #pragma unroll
@@ -238,7 +242,7 @@ __global__ void __launch_bounds__(256, 2) kv_stats_kernel(KvStatsArgs a) {
             uint8_t* ko = a.k8 + bh * static_cast<long long>(a.N) * D;
             for (int q = tid; q < kKvTok * CPR; q += 256) {
                 const int n = q / CPR, u = q % CPR;
-                const uint4 x = *reinterpret_cast<const uint4*>(kt + kv_off<D>(n, u * 8));
+                const uint4 x = *reinterpret_cast<const uint4*>(kt + kv_off<D, TC>(n, u * 8));
                 uint32_t w0, w1;
                 if (a.k_int8) {
                     w0 = pack_s8x4(bf16lo(x.x) / s_k, bf16hi(x.x) / s_k, bf16lo(x.y) / s_k, bf16hi(x.y) / s_k);
@@ -256,7 +260,7 @@ __global__ void __launch_bounds__(256, 2) kv_stats_kernel(KvStatsArgs a) {
                 float f[8];
 #pragma unroll
                 for (int t = 0; t < 8; ++t)
-                    f[t] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(vt + kv_off<D>(n0 + t, c))) / s_v;
+                    f[t] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(vt + kv_off<D, TC>(n0 + t, c))) / s_v;
                 *reinterpret_cast<uint2*>(vo + c * kKvTok + n0) =
                     make_uint2(pack_e4m3x4(f[0], f[1], f[2], f[3]), pack_e4m3x4(f[4], f[5], f[6], f[7]));
             }
@@ -268,7 +272,7 @@ __global__ void __launch_bounds__(256, 2) kv_stats_kernel(KvStatsArgs a) {
             __half* ko = a.phik16 + bh * static_cast<long long>(a.N) * D;
             for (int q = tid; q < kKvTok * CPR; q += 256) {
                 const int n = q / CPR, u = q % CPR;
-                const uint4 x = *reinterpret_cast<const uint4*>(kt + kv_off<D>(n, u * 8));
+                const uint4 x = *reinterpret_cast<const uint4*>(kt + kv_off<D, TC>(n, u * 8));
                 const uint32_t w[4] = {x.x, x.y, x.z, x.w};
                 uint32_t h[4];
 #pragma unroll
@@ -317,7 +321,7 @@ __global__ void __launch_bounds__(256, 2) kv_stats_kernel(KvStatsArgs a) {
             constexpr int CPR = D / 8;
             for (int q = tid; q < kKvTok * CPR; q += 256) {
                 const int n = q / CPR, u = q % CPR;
-                uint4* px = reinterpret_cast<uint4*>(kt + kv_off<D>(n, u * 8));
+                uint4* px = reinterpret_cast<uint4*>(kt + kv_off<D, TC>(n, u * 8));
                 uint4 x = *px;
                 uint32_t w[4] = {x.x, x.y, x.z, x.w};
                 if (a.center) {

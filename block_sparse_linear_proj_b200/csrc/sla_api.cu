@@ -339,7 +339,7 @@ sla_status_t launch_kv(const sla_params_t* p, const void* k, const void* v, void
     // TMEM slot, flag
     const size_t smem = 1024 + sla::kKvStages * 2 * 64 * D * 2 + 256 * 8 + 2 * 256 * 4 + 16 * 4 +
                         128 * 4 + 16;
-    auto kern = sla::kv_stats_kernel<D>;
+    auto kern = a.hpart ? sla::kv_stats_kernel<D, true> : sla::kv_stats_kernel<D, false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
         return SLA_ERR_CUDA;
