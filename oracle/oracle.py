@@ -7,7 +7,10 @@ The C file is compiled here with gcc (``-O2 -fopenmp``, IEEE double, no
 fast-math) into ``oracle/liboracle.so``; numpy marshals the buffers.
 Functions:
 
-* :func:`route`        -- pooled, projected top-k block routing (SLA2 router)
+* :func:`route`        -- pooled, projected top-k block routing (SLA2 router),
+  optionally with a per-block score bias
+* :func:`block_cov_norms`, :func:`route_cov` -- PISA covariance-aware routing
+  (spectral norms of the blocks' first-order matrices about their mean)
 * :func:`sla_forward`  -- sparse branch + ReLU linear branch + alpha combine
   (``fp8=True``: the sparse branch on E4M3-quantised Q, K, P, V)
 * :func:`e4m3`         -- the E4M3 conversion (round to nearest even, saturating)
@@ -54,7 +57,7 @@ def _load():
             I = ctypes.c_int
             L = ctypes.c_int64
             D = ctypes.c_double
-            lib.oracle_route.argtypes = [I] * 7 + [P] * 6 + [I]
+            lib.oracle_route.argtypes = [I] * 7 + [P] * 7 + [I]
             lib.oracle_route.restype = I
             lib.oracle_sla_forward.argtypes = [I] * 7 + [D] + [P] * 5 + [L, P, P, P, P, I, I]
             lib.oracle_sla_forward.restype = I
@@ -102,17 +105,49 @@ def _check(rc, name):
         raise ValueError("%s: oracle rejected the arguments (code %d)" % (name, rc))
 
 
-def route(q, k, w_q, w_k, Bq, Bk, topk, threads=0):
-    """Returns (lut int32 [B,H,N/Bq,topk] ascending, gap float64 [B,H,N/Bq])."""
+def route(q, k, w_q, w_k, Bq, Bk, topk, threads=0, bias=None):
+    """Returns (lut int32 [B,H,N/Bq,topk] ascending, gap float64 [B,H,N/Bq]).
+    bias (float64 [B,H,N/Bk], optional) is added to every score of KV block j."""
     qb, kb = _bf16_bits(q), _bf16_bits(k)
     B, H, N, d = qb.shape
     wq, wk = _np(w_q, np.float32), _np(w_k, np.float32)
+    bs = None if bias is None else np.ascontiguousarray(np.asarray(bias, dtype=np.float64).reshape(B * H, N // Bk))
     lut = np.zeros((B, H, N // Bq, topk), dtype=np.int32)
     gap = np.zeros((B, H, N // Bq), dtype=np.float64)
     rc = _load().oracle_route(B, H, N, d, Bq, Bk, topk, _ptr(qb), _ptr(kb), _ptr(wq), _ptr(wk),
-                              _ptr(lut), _ptr(gap), threads)
+                              _ptr(bs), _ptr(lut), _ptr(gap), threads)
     _check(rc, "route")
     return lut, gap
+
+
+def block_cov_norms(k, v, Bk):
+    """PISA block covariance norms ([PISA] sec. 2, "Routing Consapevole della
+    Covarianza"): M_j = ||H_j - Hbar||_2, the largest singular value of the
+    block's first-order matrix H_j = sum_{n in j} (k_n - kbar_j)^T v_n minus
+    their mean over the head's blocks, Hbar = (1/Nk) sum_j H_j.  fp64 from the
+    bf16 inputs; the singular values come from numpy's SVD.  Returns [B,H,N/Bk]."""
+    kb = _bf16_bits(k)
+    B, H, N, d = kb.shape
+    Nk = N // Bk
+    kd = kb.astype(np.uint32).__lshift__(16).view(np.float32).astype(np.float64)
+    vd = _bf16_bits(v).astype(np.uint32).__lshift__(16).view(np.float32).astype(np.float64)
+    out = np.zeros((B, H, Nk), dtype=np.float64)
+    for b in range(B):
+        for h in range(H):
+            kk = kd[b, h].reshape(Nk, Bk, d)
+            vv = vd[b, h].reshape(Nk, Bk, d)
+            kc = kk - kk.mean(axis=1, keepdims=True)
+            hj = np.einsum('jnc,jne->jce', kc, vv)          # [Nk, d, d]
+            dev = hj - hj.mean(axis=0, keepdims=True)
+            out[b, h] = np.linalg.norm(dev, ord=2, axis=(1, 2))
+    return out
+
+
+def route_cov(q, k, v, Bq, Bk, topk, lam, threads=0):
+    """PISA covariance-aware routing: the top-k of s_ij + lam * M_j, with s_ij
+    the plain pooled score (no projections) and M_j from block_cov_norms."""
+    bias = lam * block_cov_norms(k, v, Bk) if lam else None
+    return route(q, k, None, None, Bq, Bk, topk, threads=threads, bias=bias)
 
 
 def _rows(rows, B, H, N):

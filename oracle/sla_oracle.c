@@ -139,6 +139,9 @@ static int lut_row_valid(const int32_t *row, int topk, int Nk)
  *   3. compressed score s_ij = Qt_i . Kt_j (V is not used);
  *   4. hard top-k per query block: the k largest s_ij, ties to the lower j,
  *      written in ascending block order.
+ * bias ([B*H][Nk], NULL = none) is added to every query block's score of KV
+ * block j before the top-k: PISA's covariance-aware selection ([PISA] sec. 2,
+ * "Routing Consapevole della Covarianza") ranks blocks by s_ij + lambda M_j.
  * gap_i = s_(k) - s_(k+1) in descending order (INFINITY when k is 0 or Nk). */
 
 typedef struct { double s; int j; } scored_t;
@@ -182,7 +185,7 @@ static void project(const double *x, int rows, int d, const float *w, double *ou
 
 int oracle_route(int B, int H, int N, int d, int Bq, int Bk, int topk,
                  const uint16_t *q, const uint16_t *k, const float *w_q, const float *w_k,
-                 int32_t *lut, double *gap, int nthreads)
+                 const double *bias, int32_t *lut, double *gap, int nthreads)
 {
     if (!check_shape(B, H, N, d, Bq, Bk, topk) || !q || !k || !lut) return ORC_EINVAL;
     set_threads(nthreads);
@@ -216,7 +219,7 @@ int oracle_route(int B, int H, int N, int d, int Bq, int Bk, int topk,
             for (int j = 0; j < Nk; ++j) {
                 double acc = 0.0;
                 for (int e = 0; e < d; ++e) acc += qt[(size_t)i * d + e] * kt[(size_t)j * d + e];
-                row[j].s = acc;
+                row[j].s = bias ? acc + bias[(size_t)bh * Nk + j] : acc;
                 row[j].j = j;
             }
             qsort(row, (size_t)Nk, sizeof(scored_t), by_score_desc);

@@ -666,3 +666,98 @@ def test_int8_mode_error_is_below_fp8():
     e8, ei = np.abs(s8 - s).mean(), np.abs(si - s).mean()
     assert 0 < ei < 0.8 * e8, (ei, e8)
     assert not np.array_equal(si, s8)
+
+
+# ------------------------------------------------ PISA covariance-aware routing
+# [PISA] sec. 2 "Routing Consapevole della Covarianza": M_j = ||H_j - Hbar||_2.
+
+def _cov_blocks(Nk, d, Bk=64):
+    """Keys and values (float32, exact in bf16) of Nk blocks with block-constant
+    keys: every first-order matrix H_j is zero."""
+    rng = np.random.default_rng(31)
+    k = np.repeat(rng.integers(-8, 9, size=(Nk, 1, d)) / 4.0, Bk, axis=1)
+    v = rng.integers(-8, 9, size=(Nk, Bk, d)) / 4.0
+    return k, v
+
+
+def _signed_pairs(Bk):
+    s = np.ones(Bk)
+    s[1::2] = -1.0                      # +1, -1, ...: zero sum in every half
+    return s
+
+
+def _as_input(x):
+    return torch.as_tensor(x.reshape(1, 1, -1, x.shape[-1]), dtype=torch.float32).to(torch.bfloat16)
+
+
+def test_cov_norms_vanish_for_block_constant_keys():
+    k, v = _cov_blocks(6, 64)
+    m = orc.block_cov_norms(_as_input(k), _as_input(v), 64)
+    assert np.array_equal(m, np.zeros((1, 1, 6)))
+
+
+def test_cov_norms_are_spectral_about_the_mean():
+    """Block 0: centred keys +-a e1 (tokens 0-31) and +-b e2 (tokens 32-63) with
+    values of the same signs along e1, e2, so H_0 = diag(32 a, 32 b); block 1
+    the same keys with negated values (H_1 = -H_0); blocks 2, 3 constant keys.
+    Hbar = 0, so M_0 = M_1 = 32 max(a, b) (the Frobenius norm would give
+    32 sqrt(a^2 + b^2)) and M_2 = M_3 = 0."""
+    d, Bk, a, b = 64, 64, 1.5, 0.75
+    k, v = _cov_blocks(4, d)
+    s = _signed_pairs(Bk)
+    for j, sign in ((0, 1.0), (1, -1.0)):
+        v[j] = 0.0
+        k[j, :32, 0] += a * s[:32]
+        k[j, 32:, 1] += b * s[32:]
+        v[j, :32, 0] = sign * s[:32]
+        v[j, 32:, 1] = sign * s[32:]
+    m = orc.block_cov_norms(_as_input(k), _as_input(v), Bk)[0, 0]
+    np.testing.assert_allclose(m, [32 * a, 32 * a, 0.0, 0.0], rtol=0, atol=1e-12)
+
+
+def test_cov_norms_subtract_the_mean_matrix():
+    """Only block 0 has a first-order matrix: its 64 centred keys are +-a e1 with
+    values of the same sign along e1, so H_0 = 64 a E_11.  Hbar = H_0 / Nk, so
+    M_0 = (1 - 1/Nk) 64 a and every other block has M = 64 a / Nk."""
+    d, Bk, a, Nk = 64, 64, 1.25, 4
+    k, v = _cov_blocks(Nk, d)
+    s = _signed_pairs(Bk)
+    k[0, :, 0] += a * s
+    v[0] = 0.0
+    v[0, :, 0] = s
+    m = orc.block_cov_norms(_as_input(k), _as_input(v), Bk)[0, 0]
+    np.testing.assert_allclose(m, [(1 - 1 / Nk) * 64 * a] + [64 * a / Nk] * (Nk - 1), rtol=0, atol=1e-12)
+
+
+def test_cov_norms_ignore_a_shift_of_a_blocks_keys():
+    rng = np.random.default_rng(32)
+    k = rng.integers(-16, 17, size=(8, 64, 64)) / 8.0
+    v = rng.integers(-16, 17, size=(8, 64, 64)) / 8.0
+    m0 = orc.block_cov_norms(_as_input(k), _as_input(v), 64)
+    k[3] += rng.integers(-8, 9, size=(1, 64)) / 8.0          # exact in bf16
+    m1 = orc.block_cov_norms(_as_input(k), _as_input(v), 64)
+    np.testing.assert_allclose(m1, m0, rtol=1e-12, atol=0)
+    assert np.all(m0 > 0)
+
+
+def test_cov_routing_lambda_zero_is_plain_routing():
+    inp = W.gaussian_inputs(1, 2, 2048, 64, 33)
+    plain, gap = orc.route(inp["q"], inp["k"], None, None, 64, 64, 7)
+    cov, gap0 = orc.route_cov(inp["q"], inp["k"], inp["v"], 64, 64, 7, 0.0)
+    assert np.array_equal(plain, cov) and np.array_equal(gap, gap0)
+
+
+def test_cov_routing_large_lambda_ranks_blocks_by_norm():
+    """With a huge weight every query block selects the top-k blocks of M (the
+    same set for all rows), written in ascending order; a moderate weight
+    changes some rows relative to plain routing."""
+    B, H, N, d, Bq, Bk, k = 1, 2, 2048, 64, 64, 64, 5
+    inp = W.gaussian_inputs(B, H, N, d, 34)
+    m = orc.block_cov_norms(inp["k"], inp["v"], Bk)
+    lut, _ = orc.route_cov(inp["q"], inp["k"], inp["v"], Bq, Bk, k, 1e12)
+    for h in range(H):
+        top = np.sort(np.argsort(-m[0, h], kind="stable")[:k])
+        assert np.array_equal(lut[0, h], np.broadcast_to(top, lut[0, h].shape))
+    plain, _ = orc.route(inp["q"], inp["k"], None, None, Bq, Bk, k)
+    some, _ = orc.route_cov(inp["q"], inp["k"], inp["v"], Bq, Bk, k, 0.5)
+    assert not np.array_equal(plain, some)
