@@ -11,9 +11,11 @@
 //     and (SLA) phi(K) = max(K, 0) in fp16, the A operand of its phi(K)^T V
 //     product (the conversion from bf16 is exact inside the fp16 range; values
 //     outside it are flagged).
-// K and V tiles of 64 tokens stream through a 3-stage cp.async ring, each tile
-// stored as 64-column halves of 64 rows x 128 bytes with the 128-byte swizzle
-// (the tcgen05 operand layout).  phi(K)^T V (or, for the PISA first-order
+// K and V tiles of 64 tokens stream through a 3-stage cp.async ring.  When the
+// call runs the product below, each tile is stored as 64-column halves of 64
+// rows x 128 bytes with the 128-byte swizzle (the tcgen05 operand layout);
+// otherwise as swizzled rows of 2d bytes, which the statistics and copy passes
+// read faster.  phi(K)^T V (or, for the PISA first-order
 // term, (K - kbar_j)^T V) runs on tcgen05: after the statistics and copies
 // have read the raw K tile, it is replaced in place by phi(K) (or the centred
 // keys) in bf16, and one thread issues the block's four M = 128, K = 16
