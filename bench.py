@@ -121,7 +121,8 @@ def _oracle_forward(w, inp, heads, rows, threads):
     hs = slice(heads[0], heads[-1] + 1)
     q, k, v = inp["q"][:, hs], inp["k"][:, hs], inp["v"][:, hs]
     t0 = time.perf_counter()
-    lut, _ = orc.route(q, k, inp["w_q"], inp["w_k"], w.Bq, w.Bk, w.topk, threads=threads)
+    bias = w.cov_lambda * orc.block_cov_norms(k, v, w.Bk) if w.cov_lambda else None
+    lut, _ = orc.route(q, k, inp["w_q"], inp["w_k"], w.Bq, w.Bk, w.topk, threads=threads, bias=bias)
     t1 = time.perf_counter()
     if w.mode == "pisa":
         orc.pisa_forward(q, k, v, lut, w.Bq, w.Bk, rows=rows, threads=threads,
@@ -203,7 +204,8 @@ SPARSE_TYPES = {W.SPARSE_BF16: "bf16", W.SPARSE_FP8_E4M3: "e4m3", W.SPARSE_INT8:
 def config_of(w, world):
     in_bytes = 3 * w.B * w.H * w.N * w.d * 2
     return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "Bq": w.Bq, "Bk": w.Bk,
-            "topk": w.topk, "mode": w.mode + ("+first_order" if w.first_order else ""),
+            "topk": w.topk, "mode": w.mode + ("+first_order" if w.first_order else "") +
+                                    ("+cov_select(lambda=%g)" % w.cov_lambda if w.cov_lambda else ""),
             "sparse_dtype": SPARSE_TYPES[w.sparse_dtype],
             "global_batch": w.B * world, "seq_len": w.N, "parallelism": "replicas%d" % world,
             "l2": "inputs exceed L2 (%d MB of Q, K, V > 126 MB)" % (in_bytes // 10**6)
@@ -271,7 +273,7 @@ def run_ours(args, w, rank, world, local_rank):
     inp = W.make_inputs(w)
     g = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
     p = S.params(w.B, w.H, w.N, w.d, w.Bq, w.Bk, w.topk, sparse_dtype=w.sparse_dtype,
-                 pisa_first_order=w.first_order)
+                 pisa_first_order=w.first_order, pisa_cov_lambda=w.cov_lambda)
     ws = S.workspace(p, device=dev)
     lut = torch.empty((w.B, w.H, w.Nq, w.topk), dtype=torch.int32, device=dev)
     out = torch.empty_like(g["q"])

@@ -196,7 +196,8 @@ __global__ void __launch_bounds__(256) project_kernel(double* __restrict__ x, lo
 }
 
 // One CTA: head bh = blockIdx.y, query blocks i0 = blockIdx.x * R ... i0 + R - 1.
-// qhat = qbar M (project_kernel) or qbar itself.  The product runs on the fp64
+// qhat = qbar M (project_kernel) or qbar itself; bias (null: none) [BH][Nk] is
+// added to every score of block j (PISA's covariance-aware selection).  The product runs on the fp64
 // MMA (m8n8k4, eight-row tiles; R < 8 pads the tile).  Shared memory: qhat
 // [8 MT][D + 4] fp64 (rows padded so that the A-fragment loads spread over the
 // banks), hist [8][256] u32, keys [R][max(Nk, D + 4)] u64.
@@ -204,7 +205,8 @@ __global__ void __launch_bounds__(256) project_kernel(double* __restrict__ x, lo
 // register budget is sized for.
 template <int R, int D, int DEPTH, int MINB>
 __global__ void __launch_bounds__(256, MINB) score_topk_kernel(const double* __restrict__ qhat_all,
-                                                         const double* __restrict__ kbarT, int Nq,
+                                                         const double* __restrict__ kbarT,
+                                                         const double* __restrict__ bias, int Nq,
                                                          int Nk, int topk,
                                                          int32_t* __restrict__ lut) {
     constexpr int MT = R >= 8 ? R / 8 : 1;      // eight-row MMA tiles
@@ -222,6 +224,7 @@ __global__ void __launch_bounds__(256, MINB) score_topk_kernel(const double* __r
     const int nrows = min(R, Nq - i0);
     const double* qhat = qhat_all + (bh * Nq + i0) * D;
     const double* kt = kbarT + bh * D * static_cast<long long>(Nk);
+    const double* brow = bias ? bias + bh * Nk : nullptr;   // per-block score term, or none
 
     // 1. the R rows of qhat (padding rows are zero)
     for (int a = tid; a < 8 * MT * D; a += 256) {
@@ -273,8 +276,11 @@ __global__ void __launch_bounds__(256, MINB) score_topk_kernel(const double* __r
 #pragma unroll
             for (int nt = 0; nt < 8; ++nt) {
                 const int j = j0 + nt * 8 + 2 * t;
-                if (j < Nk) keys[static_cast<size_t>(r) * ldk + j] = order_key(acc[mt][nt][0]);
-                if (j + 1 < Nk) keys[static_cast<size_t>(r) * ldk + j + 1] = order_key(acc[mt][nt][1]);
+                if (j < Nk)
+                    keys[static_cast<size_t>(r) * ldk + j] = order_key(brow ? acc[mt][nt][0] + brow[j] : acc[mt][nt][0]);
+                if (j + 1 < Nk)
+                    keys[static_cast<size_t>(r) * ldk + j + 1] =
+                        order_key(brow ? acc[mt][nt][1] + brow[j + 1] : acc[mt][nt][1]);
             }
         }
     }

@@ -14,6 +14,7 @@
 #include "../../include/sla.h"
 #include "attn.cuh"
 #include "common.cuh"
+#include "cov.cuh"
 #include "kv_stats.cuh"
 #include "router.cuh"
 
@@ -37,6 +38,7 @@ sla_status_t check_params(const sla_params_t* p) {
         return SLA_ERR_INVALID_ARG;
     if (p->lut_mode != SLA_LUT_COMPUTE && p->lut_mode != SLA_LUT_GIVEN) return SLA_ERR_INVALID_ARG;
     if (p->pisa_first_order != 0 && p->pisa_first_order != 1) return SLA_ERR_INVALID_ARG;
+    if (!(p->pisa_cov_lambda >= 0.f) || !std::isfinite(p->pisa_cov_lambda)) return SLA_ERR_INVALID_ARG;
     if (p->out_dtype != SLA_OUT_BF16 && p->out_dtype != SLA_OUT_FP32) return SLA_ERR_INVALID_ARG;
     if (!(std::isfinite(p->sm_scale))) return SLA_ERR_INVALID_ARG;
     if (p->d != 64 && p->d != 128) return SLA_ERR_UNSUPPORTED;
@@ -59,6 +61,7 @@ sla_status_t check_tensor(const void* t, size_t align) {
 struct Ws {
     size_t qbar, kbarT, m, lut, zj, hpart, hsum, zsum, kc, vbar, v16, phik16;
     size_t q8, k8, v8t, sq, sk, sv;       // FP8 sparse branch
+    size_t covpart, covhbar, covbias;     // covariance-aware PISA selection
     size_t total;
     int nchunk, bpc;
 };
@@ -92,6 +95,11 @@ Ws layout(const sla_params_t* p) {
         w.sq = take(BH * static_cast<size_t>(p->N) / 64 * 4);
         w.sk = take(BH * Nk * 4);
         w.sv = take(BH * Nk * 4);
+    }
+    if (p->pisa_cov_lambda > 0.f) {               // chunk sums of H_j, Hbar, lambda M_j
+        w.covpart = take(BH * static_cast<size_t>(w.nchunk) * d * d * 4);
+        w.covhbar = take(BH * d * d * 4);
+        w.covbias = take(BH * Nk * 8);
     }
     w.total = off;
     return w;
@@ -235,8 +243,8 @@ size_t score_smem(int R, int D, int Nk) {
 }
 
 template <int R, int D, int DEPTH, int MINB>
-sla_status_t launch_score_r(const double* qhat, const double* kbarT, int BH, int Nq, int Nk,
-                            int topk, int32_t* lut, cudaStream_t st) {
+sla_status_t launch_score_r(const double* qhat, const double* kbarT, const double* bias, int BH,
+                            int Nq, int Nk, int topk, int32_t* lut, cudaStream_t st) {
     const size_t smem = score_smem(R, D, Nk);
     auto kern = sla::score_topk_kernel<R, D, DEPTH, MINB>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -244,25 +252,25 @@ sla_status_t launch_score_r(const double* qhat, const double* kbarT, int BH, int
         return SLA_ERR_CUDA;
     dim3 grid((Nq + R - 1) / R, BH);
     Span sp(SLA_KERNEL_SCORE_TOPK, st);
-    kern<<<grid, 256, smem, st>>>(qhat, kbarT, Nq, Nk, topk, lut);
+    kern<<<grid, 256, smem, st>>>(qhat, kbarT, bias, Nq, Nk, topk, lut);
     return launch_status();
 }
 
 template <int D>
-sla_status_t launch_score(const double* qhat, const double* kbarT, int BH, int Nq, int Nk,
-                          int topk, int32_t* lut, cudaStream_t st) {
+sla_status_t launch_score(const double* qhat, const double* kbarT, const double* bias, int BH,
+                          int Nq, int Nk, int topk, int32_t* lut, cudaStream_t st) {
     // 16 query blocks per CTA (two 8-row tiles of the fp64 MMA per K fragment).
     // Where two CTAs fit an SM's shared memory, a two-deep fragment ring keeps
     // the registers within two CTAs; otherwise one CTA per SM with a four-deep ring.
     constexpr size_t two = 113 * 1024, one = 200 * 1024;
     if (score_smem(16, D, Nk) <= two)
-        return launch_score_r<16, D, 2, 2>(qhat, kbarT, BH, Nq, Nk, topk, lut, st);
+        return launch_score_r<16, D, 2, 2>(qhat, kbarT, bias, BH, Nq, Nk, topk, lut, st);
     if (score_smem(16, D, Nk) <= one)
-        return launch_score_r<16, D, 4, 1>(qhat, kbarT, BH, Nq, Nk, topk, lut, st);
-    if (score_smem(8, D, Nk) <= one) return launch_score_r<8, D, 4, 1>(qhat, kbarT, BH, Nq, Nk, topk, lut, st);
-    if (score_smem(4, D, Nk) <= one) return launch_score_r<4, D, 4, 1>(qhat, kbarT, BH, Nq, Nk, topk, lut, st);
+        return launch_score_r<16, D, 4, 1>(qhat, kbarT, bias, BH, Nq, Nk, topk, lut, st);
+    if (score_smem(8, D, Nk) <= one) return launch_score_r<8, D, 4, 1>(qhat, kbarT, bias, BH, Nq, Nk, topk, lut, st);
+    if (score_smem(4, D, Nk) <= one) return launch_score_r<4, D, 4, 1>(qhat, kbarT, bias, BH, Nq, Nk, topk, lut, st);
     if (score_smem(2, D, Nk) > 232448) return SLA_ERR_UNSUPPORTED;   // a score row beyond shared memory
-    return launch_score_r<2, D, 4, 1>(qhat, kbarT, BH, Nq, Nk, topk, lut, st);
+    return launch_score_r<2, D, 4, 1>(qhat, kbarT, bias, BH, Nq, Nk, topk, lut, st);
 }
 
 // Router, first part: Q (and K, unless the pre-pass pools it) pooling, W folding
@@ -293,13 +301,53 @@ sla_status_t router_pool(const sla_params_t* p, const void* q, const void* k, co
 // Router, second part: fp64 score + top-k (after kbar_ready, when given: the
 // pooled K means of the pre-pass on the side stream).
 sla_status_t router_score(const sla_params_t* p, int32_t* lut, void* ws, const Ws& w,
-                          cudaStream_t st, cudaEvent_t kbar_ready = nullptr) {
+                          cudaStream_t st, cudaEvent_t kbar_ready = nullptr,
+                          const double* bias = nullptr) {
     const int BH = p->B * p->H, Nq = p->N / p->Bq, Nk = p->N / p->Bk;
     if (kbar_ready && cudaStreamWaitEvent(st, kbar_ready, 0) != cudaSuccess) return SLA_ERR_CUDA;
     const double* qhat = at<double>(ws, w.qbar);
     const double* kbarT = at<double>(ws, w.kbarT);
-    if (p->d == 128) return launch_score<128>(qhat, kbarT, BH, Nq, Nk, p->topk, lut, st);
-    return launch_score<64>(qhat, kbarT, BH, Nq, Nk, p->topk, lut, st);
+    if (p->d == 128) return launch_score<128>(qhat, kbarT, bias, BH, Nq, Nk, p->topk, lut, st);
+    return launch_score<64>(qhat, kbarT, bias, BH, Nq, Nk, p->topk, lut, st);
+}
+
+// Covariance norms of the PISA selection: out[bh * Nk + j] = scale * M_j.
+template <int D>
+sla_status_t launch_cov_t(const sla_params_t* p, const void* k, const void* v, void* ws, const Ws& w,
+                          double scale, double* out, cudaStream_t st) {
+    const int BH = p->B * p->H, Nk = p->N / p->Bk;
+    const auto* kb = static_cast<const __nv_bfloat16*>(k);
+    const auto* vb = static_cast<const __nv_bfloat16*>(v);
+    float* part = at<float>(ws, w.covpart);
+    float* hbar = at<float>(ws, w.covhbar);
+    const size_t smem_h = 2 * sla::kCovTok * D * 4 + D * 8;
+    constexpr int R0 = (2 * sla::kCovTok * D > D * (D + 1) ? 2 * sla::kCovTok * D : D * (D + 1));
+    const size_t smem_n = R0 * 4 + D * 8 + ((sla::kLanczos + 1) * D + D + (sla::kLanczos + 1) * 8 +
+                                           sla::kLanczos + 1) * 4 + 8 + 2 * sla::kLanczos * 8;
+    auto kh = sla::cov_hsum_kernel<D>;
+    auto kn = sla::cov_norm_kernel<D>;
+    if (cudaFuncSetAttribute(kh, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_h)) != cudaSuccess ||
+        cudaFuncSetAttribute(kn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_n)) != cudaSuccess)
+        return SLA_ERR_CUDA;
+    {
+        Span sp(SLA_KERNEL_COV, st);
+        kh<<<dim3(w.nchunk, BH), 256, smem_h, st>>>(kb, vb, p->N, Nk, w.bpc, w.nchunk, part);
+    }
+    {
+        Span sp(SLA_KERNEL_COV, st);
+        sla::cov_hbar_kernel<D><<<dim3(D * D / 256, BH), 256, 0, st>>>(part, w.nchunk, Nk, hbar);
+    }
+    {
+        Span sp(SLA_KERNEL_COV, st);
+        kn<<<dim3(Nk, BH), 256, smem_n, st>>>(kb, vb, p->N, Nk, hbar, scale, out);
+    }
+    return launch_status();
+}
+
+sla_status_t launch_cov(const sla_params_t* p, const void* k, const void* v, void* ws, const Ws& w,
+                        double scale, double* out, cudaStream_t st) {
+    return p->d == 128 ? launch_cov_t<128>(p, k, v, ws, w, scale, out, st)
+                       : launch_cov_t<64>(p, k, v, ws, w, scale, out, st);
 }
 
 sla_status_t run_router(const sla_params_t* p, const void* q, const void* k, const float* w_q,
@@ -571,6 +619,7 @@ sla_status_t sla_forward(const sla_params_t* p, const void* q, const void* k, co
                          void* out, void* workspace, size_t ws_bytes, sla_stream_t stream) {
     sla_status_t s = check_params(p);
     if (s != SLA_OK) return s;
+    if (p->pisa_cov_lambda != 0.f) return SLA_ERR_INVALID_ARG;   // a PISA selection option
     if ((s = check_tensor(q, 16)) || (s = check_tensor(k, 16)) || (s = check_tensor(v, 16)) ||
         (s = check_tensor(out, 16)) || (s = check_tensor(alpha, 4)))
         return s;
@@ -668,12 +717,30 @@ sla_status_t sla_pisa_forward(const sla_params_t* p, const void* q, const void* 
                                     side ? side->kbar : nullptr);
     if (s != SLA_OK) return s;
     if (side && cudaEventRecord(side->stats, sst) != cudaSuccess) return SLA_ERR_CUDA;
-    if (compute && (s = router_score(p, lut_use, workspace, w, st, side ? side->kbar : nullptr)))
+    // covariance-aware selection: lambda M_j added to every score of block j
+    const bool cov = compute && p->pisa_cov_lambda > 0.f;
+    double* bias = cov ? at<double>(workspace, w.covbias) : nullptr;
+    if (cov && (s = launch_cov(p, k, v, workspace, w, static_cast<double>(p->pisa_cov_lambda), bias, st)))
+        return s;
+    if (compute && (s = router_score(p, lut_use, workspace, w, st, side ? side->kbar : nullptr, bias)))
         return s;
     if (side && cudaStreamWaitEvent(st, side->stats, 0) != cudaSuccess) return SLA_ERR_CUDA;
     s = p->d == 128 ? launch_attn<128, sla::kModePisa>(p, q, k, v, nullptr, lut_use, out, workspace, w, st)
                     : launch_attn<64, sla::kModePisa>(p, q, k, v, nullptr, lut_use, out, workspace, w, st);
     return finish(s, st);
+}
+
+sla_status_t sla_pisa_cov_norms(const sla_params_t* p, const void* k, const void* v, double* norms,
+                                void* workspace, size_t ws_bytes, sla_stream_t stream) {
+    sla_status_t s = check_params(p);
+    if (s != SLA_OK) return s;
+    if ((s = check_tensor(k, 16)) || (s = check_tensor(v, 16))) return s;
+    if (!norms || !aligned(norms, 8)) return SLA_ERR_INVALID_ARG;
+    if (!(p->pisa_cov_lambda > 0.f)) return SLA_ERR_INVALID_ARG;   // the workspace holds the scratch then
+    Ws w;
+    if ((s = check_ws(p, workspace, ws_bytes, w))) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return finish(launch_cov(p, k, v, workspace, w, 1.0, norms, st), st);
 }
 
 }  // extern "C"

@@ -40,7 +40,8 @@ SLA_OUT_FP32 = 1
 EXPORTED = ("sla_workspace_size", "sla_route", "sla_forward", "sla_pisa_forward",
             "sla_status_string", "sla_check_device_status", "sla_version",
             "sla_profile_enable", "sla_profile_read", "sla_route_noalloc")
-KERNEL_KINDS = ("pool", "kv_stats", "h_reduce", "fold_w", "score_topk", "attn", "quant_q", "project")
+KERNEL_KINDS = ("pool", "kv_stats", "h_reduce", "fold_w", "score_topk", "attn", "quant_q", "project",
+                "cov")
 
 
 class SlaParams(ctypes.Structure):
@@ -48,7 +49,8 @@ class SlaParams(ctypes.Structure):
                 ("d", ctypes.c_int32), ("Bq", ctypes.c_int32), ("Bk", ctypes.c_int32),
                 ("topk", ctypes.c_int32), ("sm_scale", ctypes.c_float),
                 ("sparse_dtype", ctypes.c_int32), ("lut_mode", ctypes.c_int32),
-                ("out_dtype", ctypes.c_int32), ("pisa_first_order", ctypes.c_int32)]
+                ("out_dtype", ctypes.c_int32), ("pisa_first_order", ctypes.c_int32),
+                ("pisa_cov_lambda", ctypes.c_float)]
 
 
 class SlaError(RuntimeError):
@@ -81,6 +83,8 @@ def load():
             lib.sla_forward.restype = ctypes.c_int
             lib.sla_pisa_forward.argtypes = [PP, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
             lib.sla_pisa_forward.restype = ctypes.c_int
+            lib.sla_pisa_cov_norms.argtypes = [PP, P, P, P, P, ctypes.c_size_t, P]
+            lib.sla_pisa_cov_norms.restype = ctypes.c_int
             lib.sla_status_string.argtypes = [ctypes.c_int]
             lib.sla_status_string.restype = ctypes.c_char_p
             lib.sla_check_device_status.argtypes = [P]
@@ -100,9 +104,10 @@ def status_string(code: int) -> str:
 
 
 def params(B, H, N, d, Bq, Bk, topk, sm_scale=0.0, sparse_dtype=SLA_SPARSE_BF16,
-           lut_mode=SLA_LUT_COMPUTE, out_dtype=SLA_OUT_BF16, pisa_first_order=False) -> SlaParams:
+           lut_mode=SLA_LUT_COMPUTE, out_dtype=SLA_OUT_BF16, pisa_first_order=False,
+           pisa_cov_lambda=0.0) -> SlaParams:
     return SlaParams(B, H, N, d, Bq, Bk, topk, float(sm_scale), sparse_dtype, lut_mode,
-                     out_dtype, 1 if pisa_first_order else 0)
+                     out_dtype, 1 if pisa_first_order else 0, float(pisa_cov_lambda))
 
 
 def out_torch_dtype(p: SlaParams):
@@ -189,6 +194,19 @@ def sla_forward(p, q, k, v, alpha, w_q, w_k, lut, out, ws, stream=None):
                             _stream(stream))
     _raise(rc, "sla_forward")
     return out
+
+
+def sla_pisa_cov_norms(p, k, v, norms, ws, stream=None):
+    """Block covariance norms M_j = ||H_j - Hbar||_2 into ``norms`` (fp64
+    [B,H,N/Bk]); needs p.pisa_cov_lambda > 0."""
+    B, H, N, d = p.B, p.H, p.N, p.d
+    for name, t in (("k", k), ("v", v)):
+        _check(t, torch.bfloat16, (B, H, N, d), name)
+    _check(norms, torch.float64, (B, H, N // p.Bk), "norms")
+    rc = load().sla_pisa_cov_norms(ctypes.byref(p), _ptr(k), _ptr(v), _ptr(norms), _ptr(ws),
+                                   ws.numel(), _stream(stream))
+    _raise(rc, "sla_pisa_cov_norms")
+    return norms
 
 
 def sla_pisa_forward(p, q, k, v, w_q, w_k, lut, out, ws, stream=None):

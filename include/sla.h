@@ -80,6 +80,9 @@ typedef struct sla_params {
     int32_t out_dtype;       /* sla_out_dtype_t: element type of `out`          */
     int32_t pisa_first_order;/* sla_pisa_forward: 1 adds the global first-order
                                 correction term, 0 keeps the zero-order terms  */
+    float pisa_cov_lambda;   /* sla_pisa_forward, LUT_COMPUTE: weight lambda >= 0
+                                of the covariance term of the block selection
+                                (0 = plain routing); must be 0 in sla_forward */
 } sla_params_t;
 
 /* Bytes of device workspace that sla_route, sla_forward and sla_pisa_forward
@@ -174,12 +177,31 @@ sla_status_t sla_forward(const sla_params_t *p, const void *q, const void *k, co
  * the mean over all blocks of the blocks' first-order matrices (D_t has no
  * first-order part).  S comes from the router (LUT_COMPUTE; pass
  * w_q = w_k = NULL for PISA's plain pooled score) or from `lut` (LUT_GIVEN).
+ * With LUT_COMPUTE and p->pisa_cov_lambda > 0 the selection is covariance
+ * aware ([PISA] sec. 2, "Routing Consapevole della Covarianza"): the top-k of
+ *   s_ij + lambda M_j,   M_j = || H_j - Hbar ||_2  (largest singular value),
+ *   H_j = sum_{n in j} (k_n - kbar_j)^T v_n,
+ * so heterogeneous blocks go to the exact path (M_j: see sla_pisa_cov_norms).
  * Requires Bq == Bk and sparse_dtype = BF16.
  */
 sla_status_t sla_pisa_forward(const sla_params_t *p, const void *q, const void *k,
                               const void *v, const float *w_q, const float *w_k,
                               int32_t *lut, void *out,
                               void *workspace, size_t ws_bytes, sla_stream_t stream);
+
+/*
+ * sla_pisa_cov_norms -- the block covariance norms of the covariance-aware
+ * selection: norms[(b*H + h)*Nk + j] = M_j = || H_j - Hbar ||_2 in fp64
+ * (unscaled), j < Nk = N/Bk.  H_j and Hbar are fp32 sums of exact products
+ * (keys centred in fp64, rounded once); the largest singular value comes from
+ * 24 Lanczos steps on (H_j - Hbar)^T (H_j - Hbar) (relative error ~1e-7).
+ * k, v: device bf16 [B,H,N,d]; norms: device fp64, B*H*Nk entries, 8-byte
+ * aligned, owned by the caller.  Requires Bk = 64 and p->pisa_cov_lambda > 0
+ * (the workspace then holds the norms' scratch); errors as sla_pisa_forward.
+ */
+sla_status_t sla_pisa_cov_norms(const sla_params_t *p, const void *k, const void *v,
+                                double *norms, void *workspace, size_t ws_bytes,
+                                sla_stream_t stream);
 
 /* Static text for a status code. */
 const char *sla_status_string(sla_status_t s);
@@ -206,7 +228,8 @@ typedef enum {
     SLA_KERNEL_ATTN = 5,        /* sparse / PISA attention + fused epilogue     */
     SLA_KERNEL_QUANT_Q = 6,     /* 8-bit quantisation of Q (FP8, INT8 branch)   */
     SLA_KERNEL_PROJECT = 7,     /* pooled Q times W_q W_k^T (router with W)      */
-    SLA_KERNEL_KINDS = 8
+    SLA_KERNEL_COV = 8,         /* block covariance norms (PISA selection)       */
+    SLA_KERNEL_KINDS = 9
 } sla_kernel_kind_t;
 
 sla_status_t sla_profile_enable(int32_t on);

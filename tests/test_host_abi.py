@@ -127,3 +127,24 @@ def test_workspace_size_grows_with_problem(lib):
     small = S.params(1, 2, 1024, 64, 64, 64, 4)
     big = S.params(1, 12, 32768, 128, 128, 64, 52)
     assert lib.sla_workspace_size(ctypes.byref(big)) > lib.sla_workspace_size(ctypes.byref(small))
+
+
+def test_cov_selection_arguments(lib):
+    # lambda must be finite and >= 0
+    for lam in (-1.0, float("nan"), float("inf")):
+        p = S.params(1, 2, 1024, 64, 64, 64, 4, pisa_cov_lambda=lam)
+        assert call_route(p) == S.SLA_ERR_INVALID_ARG
+        assert lib.sla_workspace_size(ctypes.byref(p)) == 0
+    # a PISA selection option: sla_forward rejects it
+    assert call_forward(S.params(1, 2, 1024, 64, 64, 64, 4, pisa_cov_lambda=0.5)) == S.SLA_ERR_INVALID_ARG
+    # the norms need lambda > 0 (the workspace holds their scratch then) and 8-byte aligned output
+    p0 = S.params(1, 2, 1024, 64, 64, 64, 4)
+    assert lib.sla_pisa_cov_norms(ctypes.byref(p0), FAKE, FAKE, FAKE, FAKE, 1 << 40, None) == \
+        S.SLA_ERR_INVALID_ARG
+    p1 = S.params(1, 2, 1024, 64, 64, 64, 4, pisa_cov_lambda=0.1)
+    assert lib.sla_pisa_cov_norms(ctypes.byref(p1), FAKE, FAKE, ctypes.c_void_p((1 << 20) + 4),
+                                  FAKE, 1 << 40, None) == S.SLA_ERR_INVALID_ARG
+    # the selection term's scratch enlarges the workspace
+    with_cov = S.params(1, 24, 32768, 128, 64, 64, 77, pisa_cov_lambda=0.1)
+    plain = S.params(1, 24, 32768, 128, 64, 64, 77)
+    assert lib.sla_workspace_size(ctypes.byref(with_cov)) > lib.sla_workspace_size(ctypes.byref(plain))

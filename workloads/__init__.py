@@ -54,6 +54,7 @@ class Workload:
     alpha_range: Optional[tuple] = (0.0, 1.0)
     use_w: bool = True
     first_order: bool = False     # PISA: add the global first-order term
+    cov_lambda: float = 0.0       # PISA: weight of the covariance-aware selection term
 
     @property
     def Nq(self) -> int:
@@ -92,8 +93,12 @@ WORKLOADS = {
     # the PISA workload with the global first-order correction
     "pisa_fo": Workload("pisa_fo", 1, 24, 32768, 128, 64, 64, 77, "pisa", SPARSE_BF16,
                         "video", 1005, (21, 30, 52), None, False, True),
+    # the PISA workload with the covariance-aware selection (lambda = 0.1 moves
+    # about 28% of the selected blocks on these inputs)
+    "pisa_cov": Workload("pisa_cov", 1, 24, 32768, 128, 64, 64, 77, "pisa", SPARSE_BF16,
+                         "video", 1005, (21, 30, 52), None, False, False, 0.1),
 }
-ORDER = ["tiny", "sla2_bf16", "sla2_long", "sla2_fp8", "sla2_int8", "pisa", "pisa_fo"]
+ORDER = ["tiny", "sla2_bf16", "sla2_long", "sla2_fp8", "sla2_int8", "pisa", "pisa_fo", "pisa_cov"]
 
 
 def _bf16(x: torch.Tensor) -> torch.Tensor:
