@@ -213,6 +213,15 @@ def config_of(w, world):
             "out_dtype": "bf16", "lut_mode": "compute"}
 
 
+def kernel_table(prof, steps):
+    """Per kernel kind: device ms per call (over `steps` calls) and per launch, the
+    launch count and the share of the summed device time.  prof: kind ->
+    (summed ms, launches), from the library's per-kernel events."""
+    total = sum(m for (m, _) in prof.values())
+    return {k: {"ms_per_call": m / max(steps, 1), "ms_per_launch": m / max(c, 1), "launches": c,
+                "share": (m / total if total else None)} for k, (m, c) in prof.items() if c}
+
+
 def kernel_code_hash():
     """sha256 of the attention kernel's code (attn.cuh + common.cuh) with comments
     and blank space removed, so that only a change of code invalidates a capture."""
@@ -389,9 +398,7 @@ def run_ours(args, w, rank, world, local_rank):
     pool_ms, pool_n = prof["pool"]
     pool_avg = pool_ms / max(pool_n, 1)
     pool_bytes = w.B * w.H * w.N * w.d * 2        # read Q
-    total_prof = sum(m for (m, _) in prof.values())
-    kernels = {k: {"ms_per_call": m / max(c, 1), "launches": c,
-                   "share": (m / total_prof if total_prof else None)} for k, (m, c) in prof.items() if c}
+    kernels = kernel_table(prof, args.steps)
     kernels["kv_stats"]["hbm"] = {"achieved_gbs": kv_bytes / (kv_avg * 1e-3) / 1e9,
                                   "peak_gbs": peaks["hbm_gbs"],
                                   "frac": kv_bytes / (kv_avg * 1e-3) / 1e9 / peaks["hbm_gbs"]}

@@ -31,3 +31,12 @@ def test_reference_arm_prints_one_contract_line():
     e = d["e2e"]
     assert e["value"] == d["value"] and e["unit"] == d["unit"]
     assert e["h2d_bytes_per_step"] == 0 and e["d2h_bytes_per_step"] == 0
+
+
+def test_kernel_table_separates_calls_and_launches():
+    import bench
+    t = bench.kernel_table({"attn": (10.0, 5), "cov": (6.0, 15), "pool": (0.0, 0)}, 5)
+    assert set(t) == {"attn", "cov"}
+    assert t["attn"]["ms_per_call"] == 2.0 and t["attn"]["ms_per_launch"] == 2.0
+    assert abs(t["cov"]["ms_per_call"] - 1.2) < 1e-12 and abs(t["cov"]["ms_per_launch"] - 0.4) < 1e-12
+    assert t["cov"]["launches"] == 15 and abs(t["attn"]["share"] + t["cov"]["share"] - 1.0) < 1e-12
