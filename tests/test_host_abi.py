@@ -148,3 +148,17 @@ def test_cov_selection_arguments(lib):
     with_cov = S.params(1, 24, 32768, 128, 64, 64, 77, pisa_cov_lambda=0.1)
     plain = S.params(1, 24, 32768, 128, 64, 64, 77)
     assert lib.sla_workspace_size(ctypes.byref(with_cov)) > lib.sla_workspace_size(ctypes.byref(plain))
+
+
+def test_cov_norms_wrapper_checks_arguments():
+    import torch
+    from block_sparse_linear_proj_b200 import sla as SL
+    p = SL.params(1, 1, 1024, 64, 64, 64, 4, pisa_cov_lambda=0.1)
+    k = torch.zeros(1, 1, 1024, 64, dtype=torch.bfloat16)
+    ws = torch.zeros(16, dtype=torch.uint8)
+    with pytest.raises(TypeError):          # norms must be fp64
+        SL.sla_pisa_cov_norms(p, k, k, torch.zeros(1, 1, 16, dtype=torch.float32), ws)
+    with pytest.raises(ValueError):         # one norm per KV block
+        SL.sla_pisa_cov_norms(p, k, k, torch.zeros(1, 1, 15, dtype=torch.float64), ws)
+    with pytest.raises(TypeError):          # bf16 keys
+        SL.sla_pisa_cov_norms(p, k.float(), k, torch.zeros(1, 1, 16, dtype=torch.float64), ws)
