@@ -85,9 +85,10 @@ typedef struct sla_params {
                                 (0 = plain routing); must be 0 in sla_forward */
 } sla_params_t;
 
-/* Bytes of device workspace that sla_route, sla_forward and sla_pisa_forward
- * need for these parameters (the maximum over the three).  Returns 0 if the
- * parameters are invalid. */
+/* Bytes of device workspace that sla_route, sla_forward, sla_pisa_forward and
+ * sla_pisa_cov_norms need for these parameters (the maximum over them; the
+ * covariance-aware selection's scratch is included when pisa_cov_lambda > 0).
+ * Returns 0 if the parameters are invalid. */
 size_t sla_workspace_size(const sla_params_t *p);
 
 /*
