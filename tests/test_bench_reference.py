@@ -40,3 +40,14 @@ def test_kernel_table_separates_calls_and_launches():
     assert t["attn"]["ms_per_call"] == 2.0 and t["attn"]["ms_per_launch"] == 2.0
     assert abs(t["cov"]["ms_per_call"] - 1.2) < 1e-12 and abs(t["cov"]["ms_per_launch"] - 0.4) < 1e-12
     assert t["cov"]["launches"] == 15 and abs(t["attn"]["share"] + t["cov"]["share"] - 1.0) < 1e-12
+
+
+def test_every_workload_has_a_config_line():
+    import bench
+    import workloads as W
+    for name in W.ORDER:
+        w = W.WORKLOADS[name]
+        c = bench.config_of(w, 1)
+        assert c["workload"] == name and c["seq_len"] == w.N and c["topk"] == w.topk
+        assert w.N % w.Bq == 0 and w.N % w.Bk == 0 and 0 <= w.topk <= w.Nk
+        assert (w.cov_lambda > 0) == ("cov_select" in c["mode"])

@@ -761,3 +761,11 @@ def test_cov_routing_large_lambda_ranks_blocks_by_norm():
     plain, _ = orc.route(inp["q"], inp["k"], None, None, Bq, Bk, k)
     some, _ = orc.route_cov(inp["q"], inp["k"], inp["v"], Bq, Bk, k, 0.5)
     assert not np.array_equal(plain, some)
+
+
+def test_route_with_zero_bias_is_plain_routing():
+    """The router's per-block bias path adds nothing when the bias is zero."""
+    inp = W.gaussian_inputs(1, 2, 2048, 64, 36)
+    plain, gap = orc.route(inp["q"], inp["k"], inp["w_q"], inp["w_k"], 64, 64, 9)
+    zero, gap0 = orc.route(inp["q"], inp["k"], inp["w_q"], inp["w_k"], 64, 64, 9, bias=np.zeros((1, 2, 32)))
+    assert np.array_equal(plain, zero) and np.array_equal(gap, gap0)
