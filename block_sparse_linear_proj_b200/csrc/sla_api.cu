@@ -214,6 +214,38 @@ struct Span {
     }
 };
 
+// A phase of a call on the caller's stream: opened at the call's entry, closed
+// by end() (when tracing is on; otherwise both are no-ops).
+struct Phase {
+    int kind; cudaStream_t st; cudaEvent_t a = nullptr;
+    Phase(int k, cudaStream_t s) : kind(k), st(s) {
+        Profiler& P = prof();
+        std::lock_guard<std::mutex> g(P.mu);
+        if (!P.on) return;
+        a = P.get();
+        if (a) cudaEventRecord(a, st);
+    }
+    void end() {
+        if (!a) return;
+        Profiler& P = prof();
+        std::lock_guard<std::mutex> g(P.mu);
+        cudaEvent_t b = P.get();
+        if (b) {
+            cudaEventRecord(b, st);
+            P.recs.push_back({kind, a, b});
+        } else {
+            P.pool.push_back(a);
+        }
+        a = nullptr;
+    }
+    ~Phase() {
+        if (!a) return;
+        Profiler& P = prof();
+        std::lock_guard<std::mutex> g(P.mu);
+        P.pool.push_back(a);   // the call failed before its attention kernel
+    }
+};
+
 // ------------------------------------------------------------- launchers
 int grid_blocks(long long n, int per_sm) {
     int dev = 0, sms = 148;
@@ -565,6 +597,7 @@ sla_status_t sla_route(const sla_params_t* p, const void* q, const void* k, cons
                        sla_stream_t stream) {
     sla_status_t s = check_params(p);
     if (s != SLA_OK) return s;
+    if (p->pisa_cov_lambda != 0.f) return SLA_ERR_INVALID_ARG;   // a sla_pisa_forward option
     if ((s = check_tensor(q, 16)) || (s = check_tensor(k, 16))) return s;
     if (p->topk > 0 && (s = check_tensor(lut, 4))) return s;
     if ((w_q && !aligned(w_q, 4)) || (w_k && !aligned(w_k, 4))) return SLA_ERR_INVALID_ARG;
@@ -636,6 +669,7 @@ sla_status_t sla_forward(const sla_params_t* p, const void* q, const void* k, co
     const bool int8 = p->sparse_dtype == SLA_SPARSE_INT8;
     const bool fp8 = p->sparse_dtype == SLA_SPARSE_FP8_E4M3 || int8;
     int32_t* lut_use = (compute && !lut) ? at<int32_t>(workspace, w.lut) : lut;
+    Phase pre(SLA_PHASE_PRE_ATTN, st);
     SideStream* side = side_stream();
     std::unique_lock<std::mutex> hold;
     cudaStream_t sst = st;                         // the pre-pass's stream
@@ -668,6 +702,7 @@ sla_status_t sla_forward(const sla_params_t* p, const void* q, const void* k, co
     if (compute && (s = router_score(p, lut_use, workspace, w, st, side ? side->kbar : nullptr)))
         return s;
     if (side && cudaStreamWaitEvent(st, side->stats, 0) != cudaSuccess) return SLA_ERR_CUDA;
+    pre.end();
     if (int8)
         s = launch_attn<128, sla::kModeSlaInt8>(p, q, k, v, alpha, lut_use, out, workspace, w, st);
     else if (fp8)
@@ -696,6 +731,7 @@ sla_status_t sla_pisa_forward(const sla_params_t* p, const void* q, const void* 
     const bool compute = p->lut_mode == SLA_LUT_COMPUTE;
     int32_t* lut_use = (compute && !lut) ? at<int32_t>(workspace, w.lut) : lut;
     const bool fo = p->pisa_first_order != 0;
+    Phase pre(SLA_PHASE_PRE_ATTN, st);
     SideStream* side = side_stream();
     std::unique_lock<std::mutex> hold;
     cudaStream_t sst = st;                         // the pre-pass's stream
@@ -725,6 +761,7 @@ sla_status_t sla_pisa_forward(const sla_params_t* p, const void* q, const void* 
     if (compute && (s = router_score(p, lut_use, workspace, w, st, side ? side->kbar : nullptr, bias)))
         return s;
     if (side && cudaStreamWaitEvent(st, side->stats, 0) != cudaSuccess) return SLA_ERR_CUDA;
+    pre.end();
     s = p->d == 128 ? launch_attn<128, sla::kModePisa>(p, q, k, v, nullptr, lut_use, out, workspace, w, st)
                     : launch_attn<64, sla::kModePisa>(p, q, k, v, nullptr, lut_use, out, workspace, w, st);
     return finish(s, st);
@@ -765,16 +802,23 @@ RouteScratch& route_scratch() {
     return r;
 }
 
-// Device address of g_route_scratch on the current device (looked up once per device).
-sla_status_t route_scratch_ptr(void** out) {
+// Device address of g_route_scratch on the current device.  Outside stream capture
+// it is looked up on every call (so a context that was reset and re-created, with
+// the module loaded again, never sees a stale address); under capture the address
+// from the last uncaptured call on this device is used, and there must be one.
+sla_status_t route_scratch_ptr(cudaStream_t st, void** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SLA_ERR_CUDA;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return SLA_ERR_CUDA;
     RouteScratch& r = route_scratch();
     std::lock_guard<std::mutex> g(r.mu);
-    if (!r.ptr[dev]) {
+    if (cs == cudaStreamCaptureStatusNone) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || !p) return SLA_ERR_CUDA;
         r.ptr[dev] = p;
+    } else if (!r.ptr[dev]) {
+        return SLA_ERR_CUDA;        // first call on this device made under capture
     }
     *out = r.ptr[dev];
     return SLA_OK;
@@ -801,13 +845,14 @@ extern "C" sla_status_t sla_route_noalloc(const sla_params_t* p, const void* q, 
                                           sla_stream_t stream) {
     sla_status_t s = check_params(p);
     if (s != SLA_OK) return s;
+    if (p->pisa_cov_lambda != 0.f) return SLA_ERR_INVALID_ARG;   // a sla_pisa_forward option
     if ((s = check_tensor(q, 16)) || (s = check_tensor(k, 16))) return s;
     if (p->topk > 0 && (s = check_tensor(lut, 4))) return s;
     if ((w_q && !aligned(w_q, 4)) || (w_k && !aligned(w_k, 4))) return SLA_ERR_INVALID_ARG;
     const Ws w = route_layout(p);
     if (w.total > kRouteScratchBytes) return SLA_ERR_WORKSPACE;
-    void* scratch = nullptr;
-    if ((s = route_scratch_ptr(&scratch))) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    void* scratch = nullptr;
+    if ((s = route_scratch_ptr(st, &scratch))) return s;
     return finish(run_router(p, q, k, w_q, w_k, lut, scratch, w, st), st);
 }

@@ -41,7 +41,9 @@ EXPORTED = ("sla_workspace_size", "sla_route", "sla_forward", "sla_pisa_forward"
             "sla_status_string", "sla_check_device_status", "sla_version",
             "sla_profile_enable", "sla_profile_read", "sla_route_noalloc")
 KERNEL_KINDS = ("pool", "kv_stats", "h_reduce", "fold_w", "score_topk", "attn", "quant_q", "project",
-                "cov")
+                "cov", "pre_attn")
+# profile entries that are phases of a call, not kernel launches
+PHASE_KINDS = ("pre_attn",)
 
 
 class SlaParams(ctypes.Structure):
@@ -233,7 +235,8 @@ def sla_profile_enable(on: bool = True) -> None:
 
 
 def sla_profile_read():
-    """{kernel kind: (total ms, launches)} since the last read (synchronises)."""
+    """{kind: (total ms, count)} since the last read (synchronises).  Kernel kinds
+    count launches; the phase kinds (PHASE_KINDS) count calls."""
     n = len(KERNEL_KINDS)
     ms = (ctypes.c_double * n)()
     cnt = (ctypes.c_int64 * n)()

@@ -101,7 +101,10 @@ size_t sla_workspace_size(const sla_params_t *p);
  *      toward the lower j, written to lut[b,h,i,:] in ascending j.
  * Pooling, projection and score are computed in fp64, so the LUT matches an
  * exact-arithmetic selection except where two scores lie within ~1e-12.
- * Ignores p->lut_mode, p->sm_scale and p->sparse_dtype.
+ * Ignores p->lut_mode, p->sm_scale, p->sparse_dtype, p->out_dtype and
+ * p->pisa_first_order.  p->pisa_cov_lambda must be 0 (SLA_ERR_INVALID_ARG
+ * otherwise): the covariance-aware selection is an option of sla_pisa_forward,
+ * and this call does not apply it.
  */
 sla_status_t sla_route(const sla_params_t *p, const void *q, const void *k,
                        const float *w_q, const float *w_k, int32_t *lut,
@@ -117,11 +120,15 @@ sla_status_t sla_route(const sla_params_t *p, const void *q, const void *k,
  * which every GPU that loads the library keeps reserved until the process
  * exits.  Calls whose scratch (8 * B*H * (N/Bq + N/Bk) * d + 8 * d*d bytes,
  * each part rounded up to 256) exceeds 32 MiB return SLA_ERR_WORKSPACE.
- * The first call on a device looks up the array's device address for that
- * device (cudaGetSymbolAddress, with that device current); make that first
- * call before any stream capture.  All calls share the one array and nothing
- * in it needs clearing between calls, but calls that overlap on the GPU (on
- * different streams, or on one device from several threads) race on it.
+ * Every call made outside stream capture looks up the array's device address
+ * for the current device (cudaGetSymbolAddress); a call made while `stream`
+ * is capturing reuses the address of the last uncaptured call on that device,
+ * so make one uncaptured call on a device before capturing one (otherwise
+ * SLA_ERR_CUDA).  Parameters are read as in sla_route (same ignored fields,
+ * same rule for pisa_cov_lambda).  All calls share the one array and nothing
+ * in it needs clearing between calls (every region is fully written before it
+ * is read), but calls that overlap on the GPU (on different streams, or on one
+ * device from several threads) race on it.
  * It allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
  */
 sla_status_t sla_route_noalloc(const sla_params_t *p, const void *q, const void *k,
@@ -215,7 +222,9 @@ sla_status_t sla_check_device_status(sla_stream_t stream);
 /*
  * Kernel tracing.  While enabled, every kernel the library launches is
  * bracketed by a pair of CUDA events recorded on its own stream (no device
- * cost; about a microsecond of host time per launch).  sla_profile_read()
+ * cost; about a microsecond of host time per launch), and each forward call
+ * records one more pair on the caller's stream, from its entry to the start
+ * of its attention kernel (SLA_PHASE_PRE_ATTN).  sla_profile_read()
  * synchronises those events and returns, per kernel kind, the summed device
  * time in milliseconds and the number of launches since the last read; it
  * then forgets them.  Host-side state only; guarded by a mutex.
@@ -230,7 +239,10 @@ typedef enum {
     SLA_KERNEL_QUANT_Q = 6,     /* 8-bit quantisation of Q (FP8, INT8 branch)   */
     SLA_KERNEL_PROJECT = 7,     /* pooled Q times W_q W_k^T (router with W)      */
     SLA_KERNEL_COV = 8,         /* block covariance norms (PISA selection)       */
-    SLA_KERNEL_KINDS = 9
+    SLA_PHASE_PRE_ATTN = 9,     /* not a kernel: from the entry of a forward call
+                                   on its stream to the start of its attention
+                                   kernel (router, pre-pass and their joins)     */
+    SLA_KERNEL_KINDS = 10
 } sla_kernel_kind_t;
 
 sla_status_t sla_profile_enable(int32_t on);

@@ -135,8 +135,12 @@ def test_cov_selection_arguments(lib):
         p = S.params(1, 2, 1024, 64, 64, 64, 4, pisa_cov_lambda=lam)
         assert call_route(p) == S.SLA_ERR_INVALID_ARG
         assert lib.sla_workspace_size(ctypes.byref(p)) == 0
-    # a PISA selection option: sla_forward rejects it
-    assert call_forward(S.params(1, 2, 1024, 64, 64, 64, 4, pisa_cov_lambda=0.5)) == S.SLA_ERR_INVALID_ARG
+    # a PISA selection option: sla_forward and the routing calls reject it
+    with_lam = S.params(1, 2, 1024, 64, 64, 64, 4, pisa_cov_lambda=0.5)
+    assert call_forward(with_lam) == S.SLA_ERR_INVALID_ARG
+    assert call_route(with_lam) == S.SLA_ERR_INVALID_ARG
+    assert lib.sla_route_noalloc(ctypes.byref(with_lam), FAKE, FAKE, None, None, FAKE, None) == \
+        S.SLA_ERR_INVALID_ARG
     # the norms need lambda > 0 (the workspace holds their scratch then) and 8-byte aligned output
     p0 = S.params(1, 2, 1024, 64, 64, 64, 4)
     assert lib.sla_pisa_cov_norms(ctypes.byref(p0), FAKE, FAKE, FAKE, FAKE, 1 << 40, None) == \

@@ -27,13 +27,18 @@ def _route_noalloc(p, g):
 
 
 def test_noalloc_route_matches_workspace_route_twice():
-    """Two calls in a row (different inputs, the second larger), each equal to
-    sla_route with a caller workspace: the LUT is integer output, compared
-    exactly."""
-    cases = [(1, 2, 1024, 64, 64, 4, 501), (1, 12, 32768, 128, 128, 52, 502)]
-    for (Bb, H, N, d, Bq, k, seed) in cases:
+    """Calls in a row, each equal to sla_route with a fresh caller workspace
+    (the LUT is integer output, compared exactly): a small call, a larger one,
+    then a small one without projections, after the larger call has filled
+    more of the shared array and its W_q W_k^T region, so that nothing left in
+    the array from an earlier call can reach the LUT."""
+    cases = [(1, 2, 1024, 64, 64, 4, 501, True), (1, 12, 32768, 128, 128, 52, 502, True),
+             (1, 2, 2048, 128, 64, 5, 503, False)]
+    for (Bb, H, N, d, Bq, k, seed, with_w) in cases:
         g = {kk: (v.cuda() if v is not None else None)
              for kk, v in W.gaussian_inputs(Bb, H, N, d, seed).items()}
+        if not with_w:
+            g["w_q"] = g["w_k"] = None
         p = S.params(Bb, H, N, d, Bq, 64, k)
         ref = _route_with_workspace(p, g)
         got = _route_noalloc(p, g)
