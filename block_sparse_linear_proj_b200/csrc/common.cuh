@@ -287,11 +287,11 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo_bytes, ui
 }
 
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 D.
-// a_mn / b_mn: operand stored MN-major (1) instead of K-major (0).
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_mn) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(a_mn) << 15) |
-           (static_cast<uint32_t>(b_mn) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
-           (static_cast<uint32_t>(M >> 4) << 24);
+// a_mn / b_mn: operand stored MN-major (1) instead of K-major (0); neg_a: D -= A B.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_mn, int neg_a = 0) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(neg_a) << 13) |
+           (static_cast<uint32_t>(a_mn) << 15) | (static_cast<uint32_t>(b_mn) << 16) |
+           (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 // Instruction descriptor, kind::f16 with fp16 A/B and fp32 D; neg_a: D -= A B.
 __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int a_mn, int b_mn, int neg_a = 0) {
@@ -314,6 +314,23 @@ __device__ __forceinline__ uint32_t pack_s8x4(float a, float b, float c, float d
     };
     return q(a) | (q(b) << 8) | (q(c) << 16) | (q(d) << 24);
 }
+// Divisor and numerator factor for the 8-bit codes of a block with maximum
+// magnitude amax: a code rounds the exact quotient top * x / amax (top = 448
+// for e4m3, 127 for the integer code).  For a bf16 x, top * x is exact in fp32,
+// and the correctly rounded fp32 quotient rounds to the same code as the exact
+// rational: that rational is either on a rounding midpoint (then representable)
+// or at least 2^-17 of its size away from every midpoint, beyond the quotient's
+// rounding error.  A block maximum above 2^64 scales both by 2^-64 (exact), so
+// top * x cannot overflow; an all-zero block divides by 1.
+struct CodeQuot {
+    float t, a;
+    __device__ __forceinline__ CodeQuot(float amax, float top) {
+        const bool big = amax > 1.8446744e19f;
+        t = big ? top * 5.421010862427522e-20f : top;
+        a = amax > 0.f ? (big ? amax * 5.421010862427522e-20f : amax) : 1.f;
+    }
+    __device__ __forceinline__ float operator()(float x) const { return __fdiv_rn(x * t, a); }
+};
 // An integer of magnitude below 2^22 as fp32, exactly: its bits added to those of
 // 1.5 * 2^23, then 1.5 * 2^23 subtracted (integer and fp32 add pipes only).
 __device__ __forceinline__ float small_int_to_float(uint32_t bits) {

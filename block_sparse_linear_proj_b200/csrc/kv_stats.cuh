@@ -230,10 +230,10 @@ __global__ void __launch_bounds__(256, 2) kv_stats_kernel(KvStatsArgs a) {
             float km = 0.f, vm = 0.f;
 #pragma unroll
             for (int w = 0; w < 8; ++w) { km = fmaxf(km, amax[w]); vm = fmaxf(vm, amax[8 + w]); }
-            // codes are picked by the correctly rounded quotient x / s (not x * (1/s),
-            // which lands on the other side of a rounding midpoint now and then)
+            // dequantisation scales; each code rounds the exact quotient top x / absmax
             const float s_k = km > 0.f ? km / (a.k_int8 ? 127.f : 448.f) : 1.f;
             const float s_v = vm > 0.f ? vm / 448.f : 1.f;
+            const CodeQuot ck(km, a.k_int8 ? 127.f : 448.f), cv(vm, 448.f);
             const int j = jb0 + blk;
             if (tid == 0) {
                 a.sk[bh * a.Nk + j] = s_k;
@@ -247,11 +247,11 @@ __global__ void __launch_bounds__(256, 2) kv_stats_kernel(KvStatsArgs a) {
                 const uint4 x = *reinterpret_cast<const uint4*>(kt + kv_off<D, TC>(n, u * 8));
                 uint32_t w0, w1;
                 if (a.k_int8) {
-                    w0 = pack_s8x4(bf16lo(x.x) / s_k, bf16hi(x.x) / s_k, bf16lo(x.y) / s_k, bf16hi(x.y) / s_k);
-                    w1 = pack_s8x4(bf16lo(x.z) / s_k, bf16hi(x.z) / s_k, bf16lo(x.w) / s_k, bf16hi(x.w) / s_k);
+                    w0 = pack_s8x4(ck(bf16lo(x.x)), ck(bf16hi(x.x)), ck(bf16lo(x.y)), ck(bf16hi(x.y)));
+                    w1 = pack_s8x4(ck(bf16lo(x.z)), ck(bf16hi(x.z)), ck(bf16lo(x.w)), ck(bf16hi(x.w)));
                 } else {
-                    w0 = pack_e4m3x4(bf16lo(x.x) / s_k, bf16hi(x.x) / s_k, bf16lo(x.y) / s_k, bf16hi(x.y) / s_k);
-                    w1 = pack_e4m3x4(bf16lo(x.z) / s_k, bf16hi(x.z) / s_k, bf16lo(x.w) / s_k, bf16hi(x.w) / s_k);
+                    w0 = pack_e4m3x4(ck(bf16lo(x.x)), ck(bf16hi(x.x)), ck(bf16lo(x.y)), ck(bf16hi(x.y)));
+                    w1 = pack_e4m3x4(ck(bf16lo(x.z)), ck(bf16hi(x.z)), ck(bf16lo(x.w)), ck(bf16hi(x.w)));
                 }
                 *reinterpret_cast<uint2*>(ko + (row0 + n) * D + u * 8) = make_uint2(w0, w1);
             }
@@ -262,7 +262,7 @@ __global__ void __launch_bounds__(256, 2) kv_stats_kernel(KvStatsArgs a) {
                 float f[8];
 #pragma unroll
                 for (int t = 0; t < 8; ++t)
-                    f[t] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(vt + kv_off<D, TC>(n0 + t, c))) / s_v;
+                    f[t] = cv(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(vt + kv_off<D, TC>(n0 + t, c))));
                 *reinterpret_cast<uint2*>(vo + c * kKvTok + n0) =
                     make_uint2(pack_e4m3x4(f[0], f[1], f[2], f[3]), pack_e4m3x4(f[4], f[5], f[6], f[7]));
             }
@@ -433,7 +433,7 @@ __global__ void __launch_bounds__(256) h_reduce_kernel(const float* __restrict__
 }
 
 // e4m3 Q (I8: symmetric 8-bit integer Q) with one absmax scale per 64-token
-// block (absmax / 448, or absmax / 127).
+// block (absmax / 448, or absmax / 127); codes round top x / absmax.
 // Grid-stride over the BH*N/64 blocks; 256 threads, 64 x D tile in registers.
 template <int D, bool I8>
 __global__ void __launch_bounds__(256) quant_q_kernel(const __nv_bfloat16* __restrict__ q,
@@ -460,8 +460,9 @@ __global__ void __launch_bounds__(256) quant_q_kernel(const __nv_bfloat16* __res
         float am = 0.f;
 #pragma unroll
         for (int w = 0; w < 8; ++w) am = fmaxf(am, part[w]);
-        // codes from the rounded quotient x / s
+        // dequantisation scale; each code rounds the exact quotient top x / absmax
         const float s = am > 0.f ? am / (I8 ? 127.f : 448.f) : 1.f;
+        const CodeQuot cq(am, I8 ? 127.f : 448.f);
         if (tid == 0) sq[blk] = s;
         uint2* dst = reinterpret_cast<uint2*>(q8 + blk * 64 * D);
         auto pack = [](float a0, float a1, float a2, float a3) {
@@ -470,8 +471,8 @@ __global__ void __launch_bounds__(256) quant_q_kernel(const __nv_bfloat16* __res
 #pragma unroll
         for (int i = 0; i < VEC; ++i)
             dst[i * 256 + tid] = make_uint2(
-                pack(bf16lo(x[i].x) / s, bf16hi(x[i].x) / s, bf16lo(x[i].y) / s, bf16hi(x[i].y) / s),
-                pack(bf16lo(x[i].z) / s, bf16hi(x[i].z) / s, bf16lo(x[i].w) / s, bf16hi(x[i].w) / s));
+                pack(cq(bf16lo(x[i].x)), cq(bf16hi(x[i].x)), cq(bf16lo(x[i].y)), cq(bf16hi(x[i].y))),
+                pack(cq(bf16lo(x[i].z)), cq(bf16hi(x[i].z)), cq(bf16lo(x[i].w)), cq(bf16hi(x[i].w))));
         __syncthreads();
     }
 }

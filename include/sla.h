@@ -151,8 +151,9 @@ sla_status_t sla_route_noalloc(const sla_params_t *p, const void *q, const void 
  * sparse_dtype FP8_E4M3 (needs d = 128, Bq = 128): the sparse branch runs on
  *      e4m3 Q, K, P and V ([SLA2] sec. 2.C; Arabic page sec. 2.j: the forward
  *      quantises Q, K, P and V).  Q, K, V: one scale per 64-token block,
- *      s = fl32(absmax / 448) (1 for an all-zero block), code = e4m3 of the
- *      rounded fp32 quotient x / s (round to nearest even, saturating).
+ *      s = absmax / 448 (1 for an all-zero block); each code is the e4m3
+ *      rounding (to nearest even, saturating) of the exact quotient
+ *      448 x / absmax, which the kernels decide exactly in fp32.
  *      Logits use the e4m3 Q.K product times s_q s_k.  P is taken against the
  *      power of two at or above the running row maximum and quantised per
  *      64-key tile as e4m3(P * 448 s_v,j / s_v,max), s_v,max the largest V
@@ -160,8 +161,8 @@ sla_status_t sla_route_noalloc(const sla_params_t *p, const void *q, const void 
  *      and divided by the row sum of the unquantised P.  The linear branch
  *      and the combine stay bf16/fp32.
  * sparse_dtype INT8 (needs d = 128, Bq = 128): as FP8_E4M3, except that Q and
- *      K take symmetric 8-bit integer codes (s = fl32(absmax / 127), code =
- *      the nearest integer to fl32(x / s), ties to even, within +-127), so
+ *      K take symmetric 8-bit integer codes (s = absmax / 127, code = the
+ *      nearest integer to the exact quotient 127 x / absmax, ties to even), so
  *      S = Q8 K8^T is an exact integer product (tcgen05 kind::i8, s32
  *      accumulation) scaled by s_q s_k; P and V keep the e4m3 rules (an
  *      integer P.V accumulator could not take the online rescale exactly).

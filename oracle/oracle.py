@@ -13,6 +13,7 @@ Functions:
   (spectral norms of the blocks' first-order matrices about their mean)
 * :func:`sla_forward`  -- sparse branch + ReLU linear branch + alpha combine
   (``fp8=True``: the sparse branch on E4M3-quantised Q, K, P, V)
+* :func:`quantise`     -- the per-block codes and scales of the 8-bit branches
 * :func:`e4m3`         -- the E4M3 conversion (round to nearest even, saturating)
 * :func:`int8`         -- the symmetric 8-bit integer code (nearest, ties to even)
 * :func:`pisa_forward` -- PISA exact-or-approximate forward (zero-order terms,
@@ -59,7 +60,7 @@ def _load():
             D = ctypes.c_double
             lib.oracle_route.argtypes = [I] * 7 + [P] * 7 + [I]
             lib.oracle_route.restype = I
-            lib.oracle_sla_forward.argtypes = [I] * 7 + [D] + [P] * 5 + [L, P, P, P, P, I, I]
+            lib.oracle_sla_forward.argtypes = [I] * 7 + [D] + [P] * 5 + [L, P, P, P, P, I, I, I]
             lib.oracle_sla_forward.restype = I
             lib.oracle_pisa_forward.argtypes = [I] * 7 + [D] + [P] * 4 + [L, P, P, I, I]
             lib.oracle_pisa_forward.restype = I
@@ -67,6 +68,8 @@ def _load():
             lib.oracle_e4m3_array.restype = None
             lib.oracle_int8_array.argtypes = [P, P, L]
             lib.oracle_int8_array.restype = None
+            lib.oracle_quantise.argtypes = [P, I, I, I, P, P]
+            lib.oracle_quantise.restype = I
             lib.oracle_max_threads.argtypes = []
             lib.oracle_max_threads.restype = I
             _lib = lib
@@ -173,13 +176,29 @@ def int8(x) -> np.ndarray:
     return out
 
 
+def quantise(x, int8=False):
+    """Codes and per-64-token-block scales of the FP8 (E4M3, top 448) or INT8
+    (top 127) sparse branch for one bf16 tensor [N, d]: each code rounds the
+    exact quotient top * x / max|x| of its block; scale = max|x| / top (1 for
+    an all-zero block).  Returns (codes float64 [N, d], scales float64 [N/64])."""
+    xb = _bf16_bits(x)
+    N, d = xb.shape
+    codes = np.zeros((N, d), dtype=np.float64)
+    scales = np.zeros(N // 64, dtype=np.float64)
+    _check(_load().oracle_quantise(_ptr(xb), N, d, 1 if int8 else 0, _ptr(codes), _ptr(scales)),
+           "quantise")
+    return codes, scales
+
+
 def sla_forward(q, k, v, alpha, lut, Bq, Bk, sm_scale=0.0, rows=None, branches=False,
-                threads=0, fp8=False, int8=False):
+                threads=0, fp8=False, int8=False, p_plain=False):
     """SLA2 forward on a given LUT.  rows=None: every row, returns [B,H,N,d];
     else flat row indices, returns [len(rows), d].  branches=True also returns
     the sparse-branch and linear-branch outputs.  fp8=True: the sparse branch
     on E4M3-quantised Q, K, P, V with per-64-token-block scales (Bk = 64).
-    int8=True: the same with 8-bit integer Q and K codes (P and V E4M3)."""
+    int8=True: the same with 8-bit integer Q and K codes (P and V E4M3).
+    p_plain (fp8 / int8): P is taken against the row maximum itself instead of
+    the power of two at or above it before its E4M3 rounding."""
     qb, kb, vb = _bf16_bits(q), _bf16_bits(k), _bf16_bits(v)
     B, H, N, d = qb.shape
     al = _np(alpha, np.float32)
@@ -192,7 +211,8 @@ def sla_forward(q, k, v, alpha, lut, Bq, Bk, sm_scale=0.0, rows=None, branches=F
     ol_ = np.zeros((n, d), dtype=np.float64) if branches else None
     rc = _load().oracle_sla_forward(B, H, N, d, Bq, Bk, topk, float(sm_scale), _ptr(qb), _ptr(kb),
                                     _ptr(vb), _ptr(al), _ptr(lt), nr, _ptr(r), _ptr(out),
-                                    _ptr(os_), _ptr(ol_), 2 if int8 else (1 if fp8 else 0), threads)
+                                    _ptr(os_), _ptr(ol_), 2 if int8 else (1 if fp8 else 0),
+                                    1 if p_plain else 0, threads)
     _check(rc, "sla_forward")
     shape = (B, H, N, d) if r is None else (n, d)
     if branches:

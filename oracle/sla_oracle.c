@@ -314,50 +314,67 @@ static rowreq_t *gather_rows(int64_t total, int64_t nrows, const int64_t *rows, 
  *   [SLA2-ar] sec. 2.j, QAT: the forward quantises Q, K, P and V), with E4M3
  *   and these scale rules (Bk must be 64):
  *     per 64-token block b of Q, K and V: s_b = max|x| / 448 (1 for an
- *     all-zero block), x8 = e4m3(x / s_b), s_b and x / s_b in fp32;
+ *     all-zero block) and x8 = e4m3(x / s_b), the code of the exact quotient
+ *     448 x / max|x| (see quantise_blocks);
  *     logits in log2 units x_tn = (q8_t . k8_n) s_q(t) s_k(j) tau log2(e);
- *     P_tn = 2^(x_tn - M_t) with M_t = ceil(max_n x_tn), l_t = sum_n P_tn;
+ *     P_tn = 2^(x_tn - M_t), l_t = sum_n P_tn, where the row reference M_t is
+ *       p_plain = 0: ceil(max_n x_tn), the power of two at or above the row
+ *                    maximum (every change of reference is then an exact power
+ *                    of two, which commutes with the E4M3 rounding of P);
+ *       p_plain = 1: max_n x_tn itself, the row maximum of the softmax;
  *     Phat_tn = e4m3(P_tn 448 s_v(j) / s_vmax), s_vmax = max over the LUT row;
  *     O_s(t) = (s_vmax / 448) sum_n Phat_tn v8_n / l_t.
  *   The linear branch and the combine are not quantised.
  *   lowbit = 2 (INT8): as above, but Q and K take 8-bit integer codes,
- *   s_b = max|x| / 127 and x8 = int8(x / s_b) (nearest, ties to even, within
- *   +-127), so q8_t . k8_n is an exact integer; P and V keep the E4M3 rules
- *   (an integer P.V accumulator could not take the online rescale exactly).
+ *   s_b = max|x| / 127 and x8 = int8(127 x / max|x|) (nearest, ties to even,
+ *   within +-127), so q8_t . k8_n is an exact integer; P and V keep the E4M3
+ *   rules (an integer P.V accumulator could not take the online rescale exactly).
  *   lowbit = 1 is the FP8 mode above; 0 is the unquantised branch.
  * rows: flat indices (b*H + h)*N + t (NULL = all rows, in order).
  * out, out_s, out_l: [nrows, d] (out_s, out_l may be NULL). */
 
-/* Per-64-token-block absmax scale and E4M3 codes of one head's [N, d] tensor.
- * The scale and the quotient that picks each code are single-precision IEEE
- * operations (correctly rounded), the precision the GPU path decides its codes
- * in; the pages fix no precision for them, and deciding a code in another
- * precision flips it whenever the quotient falls on a rounding midpoint. */
+/* Per-64-token-block absmax scale and codes of one head's [N, d] tensor.  Each
+ * code is the rounding of the exact quotient top * x / max|x| (top = 448 for
+ * E4M3, 127 for the integer code): in double, top * x is exact for a bf16 x,
+ * and the correctly rounded quotient of two exact operands rounds to the same
+ * code as the exact rational, because that rational is either on a rounding
+ * midpoint (and then exactly representable) or at least 2^-17 of its size
+ * away from every midpoint.  The scale s = max|x| / top (double) dequantises. */
 static void quantise_blocks(const uint16_t *x, int N, int d, double *x8, double *scale, int int8)
 {
-    const float top = int8 ? 127.0f : 448.0f;
+    const double top = int8 ? 127.0 : 448.0;
     for (int b = 0; b < N / 64; ++b) {
-        float amax = 0.0f;
+        double amax = 0.0;
         for (size_t e = (size_t)b * 64 * d; e < (size_t)(b + 1) * 64 * d; ++e)
-            if (fabsf((float)bf(x[e])) > amax) amax = fabsf((float)bf(x[e]));
-        const float s = amax > 0.0f ? amax / top : 1.0f;
-        scale[b] = (double)s;
+            if (fabs(bf(x[e])) > amax) amax = fabs(bf(x[e]));
+        scale[b] = amax > 0.0 ? amax / top : 1.0;
         for (size_t e = (size_t)b * 64 * d; e < (size_t)(b + 1) * 64 * d; ++e) {
-            const float quotient = (float)bf(x[e]) / s;
-            x8[e] = int8 ? oracle_int8((double)quotient) : oracle_e4m3((double)quotient);
+            const double quotient = amax > 0.0 ? (top * bf(x[e])) / amax : 0.0;
+            x8[e] = int8 ? oracle_int8(quotient) : oracle_e4m3(quotient);
         }
     }
+}
+
+/* The per-block codes and scales of quantise_blocks for one [N, d] bf16 tensor
+ * (N a multiple of 64): codes [N*d], scales [N/64].  int8 = 0: E4M3 codes
+ * (top 448); 1: 8-bit integer codes (top 127). */
+int oracle_quantise(const uint16_t *x, int N, int d, int int8, double *codes, double *scales)
+{
+    if (!x || !codes || !scales || N <= 0 || d <= 0 || N % 64) return ORC_EINVAL;
+    quantise_blocks(x, N, d, codes, scales, int8 != 0);
+    return ORC_OK;
 }
 
 int oracle_sla_forward(int B, int H, int N, int d, int Bq, int Bk, int topk, double sm_scale,
                        const uint16_t *q, const uint16_t *k, const uint16_t *v,
                        const float *alpha, const int32_t *lut,
                        int64_t nrows, const int64_t *rows,
-                       double *out, double *out_s, double *out_l, int lowbit, int nthreads)
+                       double *out, double *out_s, double *out_l, int lowbit, int p_plain,
+                       int nthreads)
 {
     if (!check_shape(B, H, N, d, Bq, Bk, topk) || !q || !k || !v || !alpha || !lut || !out)
         return ORC_EINVAL;
-    if (lowbit < 0 || lowbit > 2) return ORC_EINVAL;
+    if (lowbit < 0 || lowbit > 2 || p_plain < 0 || p_plain > 1) return ORC_EINVAL;
     const int fp8 = lowbit != 0;                   /* some quantised sparse branch */
     if (fp8 && Bk != 64) return ORC_EINVAL;
     set_threads(nthreads);
@@ -444,7 +461,9 @@ int oracle_sla_forward(int B, int H, int N, int d, int Bq, int Bk, int topk, dou
                 double ol[512];
                 for (int c = 0; c < d; ++c) { os[c] = 0.0; ol[c] = 0.0; }
                 if (fp8) {
-                    /* quantised sparse branch: log2-unit logits, power-of-two row reference */
+                    /* quantised sparse branch: log2-unit logits; the row reference is
+                     * the power of two at or above the row maximum, or (p_plain) the
+                     * row maximum itself */
                     double svmax = 0.0, mx = -INFINITY;
                     for (int s = 0; s < topk; ++s)
                         if (sv[S[s]] > svmax) svmax = sv[S[s]];
@@ -458,7 +477,7 @@ int oracle_sla_forward(int B, int H, int N, int d, int Bq, int Bk, int topk, dou
                             if (x > mx) mx = x;
                         }
                     }
-                    const double M = ceil(mx);
+                    const double M = p_plain ? mx : ceil(mx);
                     for (int s = 0; s < topk; ++s) {
                         const double qf = 448.0 * sv[S[s]] / svmax;
                         for (int r = 0; r < Bk; ++r) {

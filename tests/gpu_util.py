@@ -134,3 +134,41 @@ def random_lut(B, H, Nq, Nk, k, seed):
             for i in range(Nq):
                 lut[b, h, i] = np.sort(rng.choice(Nk, size=k, replace=False))
     return lut
+
+
+def check_lowbit(out, inp, lut, Bq, p, mode, sm_scale=0.0, rows=None, what=""):
+    """The 8-bit sparse branches (mode "fp8" or "int8") against three oracles on
+    the same rows:
+      * the quantised oracle with the kernel's reading of P's reference (the power
+        of two at or above the row maximum): the stated FP8 tolerance;
+      * the quantised oracle with P against the row maximum itself: the stated
+        tolerance plus the two oracles' own distance from each other (triangle
+        inequality: the readings round P at different points, so element by
+        element they differ by about a P-rounding error);
+      * the exact oracle: the mean error at most 1.05x the second oracle's own
+        (the CPU pins show the two readings' errors agree within 5%) plus the
+        bf16 path's mean tolerance (2e-3, for the unquantised linear branch).
+    Returns (vs pow2 oracle, vs plain oracle, gpu vs exact, plain vs exact)."""
+    o = rows_of(out, rows) if rows is not None else out.double().cpu().numpy()
+    args = (inp["q"], inp["k"], inp["v"], inp["alpha"], lut, Bq, 64)
+    kw = {mode: True}
+    ref2 = orc.sla_forward(*args, sm_scale=sm_scale, rows=rows, **kw)
+    refp = orc.sla_forward(*args, sm_scale=sm_scale, rows=rows, p_plain=True, **kw)
+    exact = orc.sla_forward(*args, sm_scale=sm_scale, rows=rows)
+    ref2, refp, exact = ref2.reshape(o.shape), refp.reshape(o.shape), exact.reshape(o.shape)
+    e2 = check(o, ref2, p, TOL_FP8, what + " vs pow2-reference oracle")
+    # triangle inequality in absolute terms: |o - refp| <= |o - ref2| + |ref2 - refp|,
+    # with |o - ref2| bounded as check() just verified (bf16 outputs: plus the
+    # format's own rounding of ref2)
+    s2 = ref2.std()
+    rnd = np.abs(bf16_round(ref2) - ref2).max() if p.out_dtype != S.SLA_OUT_FP32 else 0.0
+    d_o, d_r = np.abs(o - refp), np.abs(ref2 - refp)
+    assert d_o.max() <= TOL_FP8[0] * s2 + rnd + d_r.max(), (what, d_o.max(), d_r.max(), s2)
+    assert d_o.mean() <= TOL_FP8[1] * s2 + d_r.mean(), (what, d_o.mean(), d_r.mean(), s2)
+    dist, ep = err_units(ref2, refp), err_units(o, refp)
+    gpu_x, plain_x = err_units(o, exact), err_units(refp, exact)
+    assert gpu_x[1] <= 1.05 * plain_x[1] + 2e-3, (what, gpu_x, plain_x)
+    print("%s: vs pow2 oracle %.3g/%.3g; vs plain oracle %.3g/%.3g (oracles apart %.3g/%.3g); "
+          "vs exact: gpu %.3g/%.3g, plain oracle %.3g/%.3g" % (
+              (what,) + tuple(e2) + tuple(ep) + tuple(dist) + tuple(gpu_x) + tuple(plain_x)))
+    return e2, ep, gpu_x, plain_x
