@@ -18,6 +18,8 @@ Functions:
 * :func:`int8`         -- the symmetric 8-bit integer code (nearest, ties to even)
 * :func:`pisa_forward` -- PISA exact-or-approximate forward (zero-order terms,
   optionally the global first-order correction)
+* :func:`cocluster`    -- SVOO online bidirectional Q-K co-clustering (token
+  permutations that group tokens of one co-cluster into contiguous blocks)
 
 Inputs may be torch tensors (bf16 / fp32 / int32, on the CPU) or numpy arrays
 (bf16 given as uint16 bit patterns).
@@ -151,6 +153,70 @@ def route_cov(q, k, v, Bq, Bk, topk, lam, threads=0):
     the plain pooled score (no projections) and M_j from block_cov_norms."""
     bias = lam * block_cov_norms(k, v, Bk) if lam else None
     return route(q, k, None, None, Bq, Bk, topk, threads=threads, bias=bias)
+
+
+def cocluster(q, k, n_clusters, iters):
+    """SVOO online bidirectional Q-K co-clustering ([SVOO] sec. 2.B, "Co-Clustering
+    Bidirezionale Online"), in fp64 from the bf16 inputs.  The page gives the two
+    alternating steps; the readings taken where it is silent:
+      * C = n_clusters co-clusters; the initial query centroids are the means of
+        C contiguous chunks of N/C queries (the raster partition);
+      * step 1, keys guided by the queries: key n goes to the cluster c whose query
+        centroid has the largest affinity qbar_c . k_n (the attention score), ties
+        to the lower c; key centroids kbar_c = mean of the keys in cluster c;
+      * step 2, queries guided by the keys: query n goes to argmax_c kbar_c . q_n
+        (ties to the lower c); query centroids = means of their queries;
+      * a cluster left without tokens has no centroid and is no candidate of the
+        next assignment;
+      * iters repetitions of (step 1, step 2); the tokens are then ordered stably
+        by cluster label, so that the block-sparse path's contiguous blocks hold
+        tokens of one cluster (a block may straddle two).
+    Returns (q_perm, k_perm, q_label, k_label), int64 [B,H,N]: q_perm[b,h,i] is
+    the original index of the query at sorted position i."""
+    qb, kb = _bf16_bits(q), _bf16_bits(k)
+    B, H, N, d = qb.shape
+    C = int(n_clusters)
+    if C < 1 or N % C:
+        raise ValueError("cocluster: n_clusters must divide N")
+    to64 = lambda x: (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    qd, kd = to64(qb), to64(kb)
+    q_perm = np.zeros((B, H, N), dtype=np.int64)
+    k_perm = np.zeros((B, H, N), dtype=np.int64)
+    q_lab = np.zeros((B, H, N), dtype=np.int64)
+    k_lab = np.zeros((B, H, N), dtype=np.int64)
+
+    def assign(x, cent, valid):
+        aff = x @ cent.T                                  # [N, C] affinities
+        aff[:, ~valid] = -np.inf
+        return np.argmax(aff, axis=1)                     # first maximum: ties to the lower c
+
+    def means(x, lab, prev, prev_valid):
+        cnt = np.bincount(lab, minlength=C)
+        sums = np.zeros((C, x.shape[1]))
+        np.add.at(sums, lab, x)
+        valid = cnt > 0
+        cent = np.where(valid[:, None], sums / np.maximum(cnt, 1)[:, None], prev)
+        return cent, valid
+
+    for b in range(B):
+        for h in range(H):
+            Q, K = qd[b, h], kd[b, h]
+            qc = Q.reshape(C, N // C, d).mean(axis=1)
+            qv = np.ones(C, dtype=bool)
+            kc, kv = np.zeros((C, d)), np.zeros(C, dtype=bool)
+            ql = kl = None
+            for _ in range(iters):
+                kl = assign(K, qc, qv)
+                kc, kv = means(K, kl, kc, kv)
+                ql = assign(Q, kc, kv)
+                qc, qv = means(Q, ql, qc, qv)
+            if iters == 0:
+                ql = np.repeat(np.arange(C), N // C)
+                kl = ql.copy()
+            q_lab[b, h], k_lab[b, h] = ql, kl
+            q_perm[b, h] = np.argsort(ql, kind="stable")
+            k_perm[b, h] = np.argsort(kl, kind="stable")
+    return q_perm, k_perm, q_lab, k_lab
 
 
 def _rows(rows, B, H, N):

@@ -916,3 +916,146 @@ def test_route_with_zero_bias_is_plain_routing():
     plain, gap = orc.route(inp["q"], inp["k"], inp["w_q"], inp["w_k"], 64, 64, 9)
     zero, gap0 = orc.route(inp["q"], inp["k"], inp["w_q"], inp["w_k"], 64, 64, 9, bias=np.zeros((1, 2, 32)))
     assert np.array_equal(plain, zero) and np.array_equal(gap, gap0)
+
+
+# ------------------------------------------- SVOO online bidirectional co-clustering
+# [SVOO] sec. 2.B: keys assigned by their affinity to the query centroids, then
+# queries by their affinity to the updated key centroids, alternately; the
+# tokens are then ordered by cluster so that contiguous blocks share a cluster.
+
+def _planted(N, d, C, seed, bias=0.5, shuffle=True, scale=4.0):
+    """Tokens of C planted groups (group g: q, k near scale * u_g, with u_g
+    orthonormal).  Chunk c of the raster order (N/C tokens) holds a share `bias`
+    of group c and the rest spread over the other groups, so the initial query
+    centroid of chunk c leans toward u_c.  Returns (q, k bf16 [1,1,N,d], group)."""
+    rng = np.random.default_rng(seed)
+    u, _ = np.linalg.qr(rng.standard_normal((d, C)))
+    u = u.T                                              # [C, d] orthonormal rows
+    chunk = N // C
+    group = np.zeros(N, dtype=np.int64)
+    for c in range(C):
+        own = int(round(bias * chunk))
+        others = [g for g in range(C) if g != c]
+        lab = np.concatenate([np.full(own, c), rng.choice(others, chunk - own)])
+        if shuffle:
+            rng.shuffle(lab)
+        group[c * chunk:(c + 1) * chunk] = lab
+    q = scale * u[group] + 0.05 * rng.standard_normal((N, d))
+    k = scale * u[group] + 0.05 * rng.standard_normal((N, d))
+    to = lambda x: torch.from_numpy(x.reshape(1, 1, N, d)).float().to(torch.bfloat16)
+    return to(q), to(k), group
+
+
+def test_cocluster_single_cluster_is_identity():
+    inp = W.gaussian_inputs(1, 2, 512, 64, 81)
+    qp, kp, ql, kl = orc.cocluster(inp["q"], inp["k"], 1, 3)
+    ident = np.broadcast_to(np.arange(512), qp.shape)
+    assert np.array_equal(qp, ident) and np.array_equal(kp, ident)
+    assert (ql == 0).all() and (kl == 0).all()
+
+
+def test_cocluster_recovers_planted_groups():
+    """Every key and query of planted group g ends in cluster g, and the orders
+    are the stable sorts of the planted groups (one wrong affinity direction,
+    swapped roles of queries and keys or a missing mean breaks this)."""
+    N, d, C = 1024, 64, 4
+    q, k, group = _planted(N, d, C, 82)
+    qp, kp, ql, kl = orc.cocluster(q, k, C, 3)
+    assert np.array_equal(ql[0, 0], group) and np.array_equal(kl[0, 0], group)
+    want = np.argsort(group, kind="stable")
+    assert np.array_equal(qp[0, 0], want) and np.array_equal(kp[0, 0], want)
+
+
+def test_cocluster_block_sorted_input_is_left_in_place():
+    """Tokens already grouped in the raster chunks the iteration starts from: the
+    order does not change."""
+    N, d, C = 1024, 64, 8
+    q, k, group = _planted(N, d, C, 83, bias=1.0)
+    assert np.array_equal(group, np.repeat(np.arange(C), N // C))
+    qp, kp, ql, kl = orc.cocluster(q, k, C, 3)
+    assert np.array_equal(qp[0, 0], np.arange(N)) and np.array_equal(kp[0, 0], np.arange(N))
+
+
+def test_cocluster_labels_are_the_alternating_argmax():
+    """On video-shaped inputs: the final query labels maximise the affinity to the
+    means of the final key clusters, and the final key labels maximise it to the
+    means of the query clusters of the iteration before (empty clusters excluded,
+    ties to the lower index), computed here from the labels alone."""
+    inp = W.video_inputs(1, 2, 2048, 128, (6, 16, 21), 84)
+    C, T = 16, 3
+    _, _, ql, kl = orc.cocluster(inp["q"], inp["k"], C, T)
+    _, _, ql_prev, _ = orc.cocluster(inp["q"], inp["k"], C, T - 1)
+    Qd, Kd = f64(inp["q"]).numpy(), f64(inp["k"]).numpy()
+
+    def centroids(x, lab):
+        cnt = np.bincount(lab, minlength=C)
+        cent = np.stack([x[lab == c].mean(axis=0) if cnt[c] else np.zeros(x.shape[1]) for c in range(C)])
+        return cent, cnt > 0
+
+    for h in range(2):
+        kc, kv = centroids(Kd[0, h], kl[0, h])
+        aff = Qd[0, h] @ kc.T
+        aff[:, ~kv] = -np.inf
+        assert np.array_equal(np.argmax(aff, axis=1), ql[0, h])
+        qc, qv = centroids(Qd[0, h], ql_prev[0, h])
+        aff = Kd[0, h] @ qc.T
+        aff[:, ~qv] = -np.inf
+        assert np.array_equal(np.argmax(aff, axis=1), kl[0, h])
+        # the orders are stable sorts by label
+        assert np.array_equal(np.argsort(ql[0, h], kind="stable"), np.argsort(ql[0, h], kind="stable"))
+
+
+def test_cocluster_planted_groups_are_a_fixed_point():
+    q, k, group = _planted(1024, 64, 4, 85)
+    a = orc.cocluster(q, k, 4, 2)
+    b = orc.cocluster(q, k, 4, 5)
+    for x, y in zip(a, b):
+        assert np.array_equal(x, y)
+
+
+def _permute(inp, qp, kp):
+    """Inputs reordered by the co-clustering: queries (and alpha) by q_perm, keys
+    and values by k_perm."""
+    g = lambda x, p: torch.gather(x, 2, torch.as_tensor(p).unsqueeze(-1).expand(-1, -1, -1, x.shape[-1]))
+    out = dict(inp)
+    out["q"] = g(inp["q"], qp)
+    out["k"] = g(inp["k"], kp)
+    out["v"] = g(inp["v"], kp)
+    out["alpha"] = torch.gather(inp["alpha"], 2, torch.as_tensor(qp))
+    return out
+
+
+def test_coclustered_dense_attention_equals_unpermuted():
+    """All blocks selected with alpha = 1 is dense attention, which does not depend
+    on the order of queries or keys: routing and attending in the co-clustered
+    order, then putting the rows back, gives the unpermuted result."""
+    B, H, N, d, Bq, Bk = 1, 2, 512, 64, 64, 64
+    inp = W.gaussian_inputs(B, H, N, d, 86)
+    inp["alpha"] = torch.ones(B, H, N)
+    qp, kp, _, _ = orc.cocluster(inp["q"], inp["k"], 8, 3)
+    assert not np.array_equal(qp, np.broadcast_to(np.arange(N), qp.shape))
+    pin = _permute(inp, qp, kp)
+    Nk = N // Bk
+    lut, _ = orc.route(pin["q"], pin["k"], None, None, Bq, Bk, Nk)
+    o_perm = orc.sla_forward(pin["q"], pin["k"], pin["v"], pin["alpha"], lut, Bq, Bk)
+    back = np.zeros_like(o_perm)
+    for h in range(H):
+        back[0, h, qp[0, h]] = o_perm[0, h]
+    lut0, _ = orc.route(inp["q"], inp["k"], None, None, Bq, Bk, Nk)
+    o = orc.sla_forward(inp["q"], inp["k"], inp["v"], inp["alpha"], lut0, Bq, Bk)
+    assert np.abs(back - o).max() <= 1e-12 * np.abs(o).max()
+
+
+def test_cocluster_empty_cluster_is_no_candidate():
+    """Queries of the two raster chunks point along +u and -u, every key along +u:
+    all keys join cluster 0, cluster 1 gets no key and so no key centroid, and
+    every query must then join cluster 0 (a stale or zero centroid for cluster 1
+    would attract the -u queries)."""
+    N, d = 256, 64
+    u = np.zeros(d)
+    u[3] = 1.0
+    q = np.concatenate([np.tile(u, (N // 2, 1)), np.tile(-u, (N // 2, 1))])
+    k = np.tile(u, (N, 1)) * 0.5
+    to = lambda x: torch.from_numpy(x.reshape(1, 1, N, d)).float().to(torch.bfloat16)
+    _, _, ql, kl = orc.cocluster(to(q), to(k), 2, 2)
+    assert (kl == 0).all() and (ql == 0).all()
