@@ -122,7 +122,14 @@ def _oracle_forward(w, inp, heads, rows, threads):
     from oracle import oracle as orc
     hs = slice(heads[0], heads[-1] + 1)
     q, k, v = inp["q"][:, hs], inp["k"][:, hs], inp["v"][:, hs]
+    alpha = inp["alpha"][:, hs] if inp["alpha"] is not None else None
     t0 = time.perf_counter()
+    if w.clusters:
+        # the co-clustered order (the oracle recomputes it for every head it runs)
+        qp, kp, _, _ = orc.cocluster(q, k, w.clusters, w.cluster_iters)
+        gat = lambda x, pm: torch.gather(x, 2, torch.as_tensor(pm).unsqueeze(-1).expand(-1, -1, -1, x.shape[-1]))
+        q, k, v = gat(q, qp), gat(k, kp), gat(v, kp)
+        alpha = torch.gather(alpha, 2, torch.as_tensor(qp))
     bias = w.cov_lambda * orc.block_cov_norms(k, v, w.Bk) if w.cov_lambda else None
     lut, _ = orc.route(q, k, inp["w_q"], inp["w_k"], w.Bq, w.Bk, w.topk, threads=threads, bias=bias)
     t1 = time.perf_counter()
@@ -130,7 +137,7 @@ def _oracle_forward(w, inp, heads, rows, threads):
         orc.pisa_forward(q, k, v, lut, w.Bq, w.Bk, rows=rows, threads=threads,
                          first_order=w.first_order)
     else:
-        orc.sla_forward(q, k, v, inp["alpha"][:, hs], lut, w.Bq, w.Bk, rows=rows, threads=threads,
+        orc.sla_forward(q, k, v, alpha, lut, w.Bq, w.Bk, rows=rows, threads=threads,
                         fp8=w.sparse_dtype == W.SPARSE_FP8_E4M3, int8=w.sparse_dtype == W.SPARSE_INT8)
     return t1 - t0, time.perf_counter() - t1
 
@@ -199,7 +206,9 @@ def config_of(w, world):
     in_bytes = 3 * w.B * w.H * w.N * w.d * 2
     return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "Bq": w.Bq, "Bk": w.Bk,
             "topk": w.topk, "mode": w.mode + ("+first_order" if w.first_order else "") +
-                                    ("+cov_select(lambda=%g)" % w.cov_lambda if w.cov_lambda else ""),
+                                    ("+cov_select(lambda=%g)" % w.cov_lambda if w.cov_lambda else "") +
+                                    ("+cocluster(C=%d, iters=%d, every %d steps)" % (
+                                        w.clusters, w.cluster_iters, w.cluster_every) if w.clusters else ""),
             "sparse_dtype": SPARSE_TYPES[w.sparse_dtype],
             "global_batch": w.B * world, "seq_len": w.N, "parallelism": "replicas%d" % world,
             "l2": "inputs exceed L2 (%d MB of Q, K, V > 126 MB)" % (in_bytes // 10**6)
@@ -281,9 +290,24 @@ def run_ours(args, w, rank, world, local_rank):
     lut = torch.empty((w.B, w.H, w.Nq, w.topk), dtype=torch.int32, device=dev)
     out = torch.empty_like(g["q"])
     stream = torch.cuda.current_stream(dev)
+    if w.clusters:
+        # SVOO co-clustering: permutations recomputed every cluster_every steps,
+        # the forward in the co-clustered order every step
+        cws = S.cocluster_workspace(p, w.clusters, device=dev)
+        q_perm = torch.empty((w.B, w.H, w.N), dtype=torch.int32, device=dev)
+        k_perm = torch.empty_like(q_perm)
+        scratch = {"q": torch.empty_like(g["q"]), "k": torch.empty_like(g["k"]), "v": torch.empty_like(g["v"]),
+                   "alpha": torch.empty_like(g["alpha"]), "out": torch.empty_like(out)}
+    counter = [0]
 
     def step():
-        if w.mode == "pisa":
+        if w.clusters:
+            if counter[0] % w.cluster_every == 0:
+                S.sla_cocluster(p, g["q"], g["k"], w.clusters, w.cluster_iters, q_perm, k_perm, cws, stream)
+            counter[0] += 1
+            S.sla_forward_coclustered(p, g["q"], g["k"], g["v"], g["alpha"], g["w_q"], g["w_k"], q_perm,
+                                      k_perm, lut, out, ws, scratch, stream)
+        elif w.mode == "pisa":
             S.sla_pisa_forward(p, g["q"], g["k"], g["v"], None, None, lut, out, ws, stream)
         else:
             S.sla_forward(p, g["q"], g["k"], g["v"], g["alpha"], g["w_q"], g["w_k"], lut, out,
@@ -308,6 +332,7 @@ def run_ours(args, w, rank, world, local_rank):
     time.sleep(0.3)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
+    counter[0] = 0
     e0.record(stream)
     for _ in range(args.steps):
         step()
@@ -328,6 +353,7 @@ def run_ours(args, w, rank, world, local_rank):
     S.sla_profile_enable(True)
     e2 = torch.cuda.Event(enable_timing=True)
     e3 = torch.cuda.Event(enable_timing=True)
+    counter[0] = 0
     e2.record(stream)
     for _ in range(args.steps):
         step()

@@ -1,0 +1,219 @@
+// cocluster.cuh -- SVOO online bidirectional Q-K co-clustering ("Training-Free
+// Sparse Attention for Fast Video Generation via Offline Layer-Wise Sparsity
+// Profiling and Online Bidirectional Co-Clustering", sec. 2.B): keys are
+// assigned to the cluster whose query centroid they have the largest affinity
+// (dot product) with, then queries to the cluster of the largest affinity with
+// the updated key centroids, alternately; the tokens are then ordered stably by
+// cluster, so that the block-sparse path's contiguous blocks group tokens of one
+// cluster.  Everything is fp64 from the bf16 inputs (centroid sums of bf16
+// values are exact in fp64, so a centroid does not depend on summation order).
+//
+// Per head and per half-step:
+//   cc_assign_kernel    label[n] = argmax over non-empty clusters c of x_n . cent_c
+//                       (ties to the lower c), one token per thread, 32 centroids
+//                       at a time in shared memory;
+//   cc_count_kernel     per chunk of 1024 tokens, the tokens per label;
+//   cc_scan_kernel      each chunk's first sorted position per label;
+//   cc_scatter_kernel   perm[pos] = n, stable within a label (one warp per chunk,
+//                       tokens in order);
+//   cc_means_kernel     cent_c = mean of the label's tokens, in sorted order (a
+//                       cluster without tokens is marked empty).
+#pragma once
+#include "common.cuh"
+
+namespace sla {
+
+constexpr int kCcChunk = 1024;     // tokens per counting-sort chunk
+constexpr int kCcTile = 32;        // centroids per shared-memory tile of the assignment
+
+// Initial query centroids: means of C contiguous chunks of N/C rows.
+// grid (C, BH), D threads.
+template <int D>
+__global__ void __launch_bounds__(128) cc_chunk_mean_kernel(const __nv_bfloat16* __restrict__ x, int N, int C,
+                                                            double* __restrict__ cent, int* __restrict__ valid) {
+    const int c = blockIdx.x;
+    const long long bh = blockIdx.y;
+    const int rows = N / C;
+    const __nv_bfloat16* xr = x + (bh * N + static_cast<long long>(c) * rows) * D + threadIdx.x;
+    double s = 0.0;
+    for (int r = 0; r < rows; ++r) s += static_cast<double>(__bfloat162float(xr[static_cast<long long>(r) * D]));
+    cent[(bh * C + c) * D + threadIdx.x] = s / rows;
+    if (threadIdx.x == 0) valid[bh * C + c] = 1;
+}
+
+// label[bh][n] = argmax over valid c of x[bh][n] . cent[bh][c].
+// grid (ceil(N/128), BH), 128 threads (one token each); dynamic shared memory:
+// the CTA's tokens transposed (bf16 [D][132]), a tile of centroids (fp64
+// [kCcTile][D]) and their empty flags.
+constexpr int kCcPitch = 132;
+template <int D>
+constexpr size_t cc_assign_smem() { return static_cast<size_t>(D) * kCcPitch * 2 + kCcTile * D * 8 + kCcTile * 4; }
+
+template <int D>
+__global__ void __launch_bounds__(128) cc_assign_kernel(const __nv_bfloat16* __restrict__ x, int N, int C,
+                                                        const double* __restrict__ cent,
+                                                        const int* __restrict__ valid, int* __restrict__ label) {
+    extern __shared__ __align__(16) unsigned char cc_smem[];
+    __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(cc_smem);                       // [D][kCcPitch]
+    double* cs = reinterpret_cast<double*>(cc_smem + static_cast<size_t>(D) * kCcPitch * 2);   // [kCcTile][D]
+    int* vs = reinterpret_cast<int*>(cs + kCcTile * D);                                   // [kCcTile]
+    const long long bh = blockIdx.y;
+    const int n0 = blockIdx.x * 128;
+    const int t = threadIdx.x;
+    // stage the tile's tokens (coalesced rows), transposed so that thread t reads column t
+    for (int i = t; i < 128 * D; i += 128) {
+        const int r = i / D, dd = i % D;
+        const int n = n0 + r;
+        xs[dd * kCcPitch + r] = n < N ? x[(bh * N + n) * D + dd] : __float2bfloat16(0.f);
+    }
+    double best = -INFINITY;
+    int arg = -1;
+    for (int c0 = 0; c0 < C; c0 += kCcTile) {
+        __syncthreads();
+        const int nt = min(kCcTile, C - c0);
+        for (int i = t; i < nt * D; i += 128) cs[i] = cent[(bh * C + c0) * D + i];
+        if (t < nt) vs[t] = valid[bh * C + c0 + t];
+        __syncthreads();
+        double acc[kCcTile];
+#pragma unroll
+        for (int j = 0; j < kCcTile; ++j) acc[j] = 0.0;
+#pragma unroll 2
+        for (int dd = 0; dd < D; ++dd) {
+            const double xv = static_cast<double>(__bfloat162float(xs[dd * kCcPitch + t]));
+#pragma unroll
+            for (int j = 0; j < kCcTile; ++j) acc[j] = fma(xv, cs[j * D + dd], acc[j]);
+        }
+#pragma unroll
+        for (int j = 0; j < kCcTile; ++j)
+            if (j < nt && vs[j] && (arg < 0 || acc[j] > best)) { best = acc[j]; arg = c0 + j; }
+    }
+    if (n0 + t < N) label[bh * N + n0 + t] = arg < 0 ? 0 : arg;
+}
+
+// counts[bh][chunk][c] = tokens of the chunk with label c.  grid (nchunk, BH), 256 threads.
+__global__ void __launch_bounds__(256) cc_count_kernel(const int* __restrict__ label, int N, int C, int nchunk,
+                                                       int* __restrict__ counts) {
+    extern __shared__ int hist[];
+    const long long bh = blockIdx.y;
+    const int chunk = blockIdx.x;
+    for (int c = threadIdx.x; c < C; c += 256) hist[c] = 0;
+    __syncthreads();
+    const int n0 = chunk * kCcChunk, n1 = min(N, n0 + kCcChunk);
+    for (int n = n0 + threadIdx.x; n < n1; n += 256) {
+        const int l = label[bh * N + n];
+        if (l >= 0 && l < C) atomicAdd(&hist[l], 1);
+    }
+    __syncthreads();
+    for (int c = threadIdx.x; c < C; c += 256) counts[(bh * nchunk + chunk) * C + c] = hist[c];
+}
+
+// base[bh][chunk][c] = first sorted position of the chunk's label-c tokens;
+// start[bh][c], count[bh][c] = the label's range.  grid (BH), 1024 threads.
+__global__ void __launch_bounds__(1024) cc_scan_kernel(const int* __restrict__ counts, int C, int nchunk,
+                                                       int* __restrict__ base, int* __restrict__ start,
+                                                       int* __restrict__ count) {
+    __shared__ int tot[1024];
+    const long long bh = blockIdx.x;
+    const int c = threadIdx.x;
+    int run = 0;
+    if (c < C)
+        for (int k = 0; k < nchunk; ++k) {
+            base[(bh * nchunk + k) * C + c] = run;
+            run += counts[(bh * nchunk + k) * C + c];
+        }
+    tot[c] = c < C ? run : 0;
+    __syncthreads();
+    // exclusive scan of the totals over the labels (Hillis-Steele, 1024 entries)
+    for (int off = 1; off < 1024; off <<= 1) {
+        const int v = c >= off ? tot[c - off] : 0;
+        __syncthreads();
+        tot[c] += v;
+        __syncthreads();
+    }
+    if (c < C) {
+        const int st = tot[c] - run;
+        start[bh * C + c] = st;
+        count[bh * C + c] = run;
+        for (int k = 0; k < nchunk; ++k) base[(bh * nchunk + k) * C + c] += st;
+    }
+}
+
+// perm[bh][pos] = n for the chunk's tokens, stable within each label.
+// grid (nchunk, BH), 32 threads (one warp walks the chunk in order).
+__global__ void __launch_bounds__(32) cc_scatter_kernel(const int* __restrict__ label, int N, int C, int nchunk,
+                                                        const int* __restrict__ base, int* __restrict__ perm) {
+    extern __shared__ int run[];
+    const long long bh = blockIdx.y;
+    const int chunk = blockIdx.x;
+    const int lane = threadIdx.x;
+    for (int c = lane; c < C; c += 32) run[c] = base[(bh * nchunk + chunk) * C + c];
+    __syncwarp();
+    const int n0 = chunk * kCcChunk, n1 = min(N, n0 + kCcChunk);
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int nb = n0; nb < n1; nb += 32) {
+        const int n = nb + lane;
+        const bool in = n < n1;
+        const int l = in ? label[bh * N + n] : -1;
+        const bool ok = in && l >= 0 && l < C;
+        const uint32_t act = __ballot_sync(0xffffffffu, ok);
+        const uint32_t same = __match_any_sync(0xffffffffu, ok ? l : -1) & act;
+        if (ok) {
+            const int rank = __popc(same & lt);
+            const int pos = run[l] + rank;
+            if (pos >= 0 && pos < N) perm[bh * N + pos] = n;
+            else report(kStatusBadData);
+        }
+        __syncwarp();
+        if (ok && (same & lt) == 0) run[l] += __popc(same);   // the label's first lane advances it
+        __syncwarp();
+    }
+}
+
+// cent[bh][c] = mean of rows perm[start_c .. start_c + count_c) (in that order);
+// a label without tokens is marked empty and keeps its old centroid.
+// grid (C, BH), D threads.
+template <int D>
+__global__ void __launch_bounds__(128) cc_means_kernel(const __nv_bfloat16* __restrict__ x, int N, int C,
+                                                       const int* __restrict__ perm, const int* __restrict__ start,
+                                                       const int* __restrict__ count, double* __restrict__ cent,
+                                                       int* __restrict__ valid) {
+    const int c = blockIdx.x;
+    const long long bh = blockIdx.y;
+    const int st = start[bh * C + c], cnt = count[bh * C + c];
+    if (cnt <= 0) {
+        if (threadIdx.x == 0) valid[bh * C + c] = 0;
+        return;
+    }
+    double s = 0.0;
+    for (int i = 0; i < cnt; ++i) {
+        const int n = perm[bh * N + st + i];
+        s += static_cast<double>(__bfloat162float(x[(bh * N + n) * D + threadIdx.x]));
+    }
+    cent[(bh * C + c) * D + threadIdx.x] = s / cnt;
+    if (threadIdx.x == 0) valid[bh * C + c] = 1;
+}
+
+// dst row (bh, i) = src row (bh, perm[bh][i]) (inverse: dst row (bh, perm[bh][i])
+// = src row (bh, i)); rows of row_words 32-bit words (VEC: 16-byte words).
+// A perm entry outside [0, N) is skipped and flagged.  Grid-stride over rows.
+template <typename T>
+__global__ void __launch_bounds__(256) permute_rows_kernel(const T* __restrict__ src, const int* __restrict__ perm,
+                                                           T* __restrict__ dst, long long BH, int N, int row_words,
+                                                           int inverse) {
+    const long long rows = BH * N;
+    const int per_row = max(1, 256 / row_words);      // rows handled by one CTA pass
+    const int rr = threadIdx.x / row_words, w = threadIdx.x % row_words;
+    for (long long r0 = static_cast<long long>(blockIdx.x) * per_row; r0 < rows;
+         r0 += static_cast<long long>(gridDim.x) * per_row) {
+        const long long r = r0 + rr;
+        if (rr >= per_row || r >= rows) continue;
+        const long long bh = r / N;
+        const int p = perm[r];
+        if (p < 0 || p >= N) { if (w == 0) report(kStatusBadData); continue; }
+        const long long other = bh * N + p;
+        if (inverse) dst[other * row_words + w] = src[r * row_words + w];
+        else dst[r * row_words + w] = src[other * row_words + w];
+    }
+}
+
+}  // namespace sla

@@ -13,6 +13,7 @@
 
 #include "../../include/sla.h"
 #include "attn.cuh"
+#include "cocluster.cuh"
 #include "common.cuh"
 #include "cov.cuh"
 #include "kv_stats.cuh"
@@ -781,6 +782,155 @@ sla_status_t sla_pisa_cov_norms(const sla_params_t* p, const void* k, const void
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------ co-clustering
+namespace {
+
+struct CcWs {
+    size_t qc, kc, qv, kv, label, counts, base, start, count, total;
+    int nchunk;
+};
+
+CcWs cc_layout(const sla_params_t* p, int C) {
+    CcWs w{};
+    const size_t BH = static_cast<size_t>(p->B) * p->H, d = p->d, N = p->N;
+    w.nchunk = static_cast<int>((N + sla::kCcChunk - 1) / sla::kCcChunk);
+    size_t off = 0;
+    auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes); return o; };
+    w.qc = take(BH * C * d * 8);
+    w.kc = take(BH * C * d * 8);
+    w.qv = take(BH * C * 4);
+    w.kv = take(BH * C * 4);
+    w.label = take(BH * N * 4);
+    w.counts = take(BH * static_cast<size_t>(w.nchunk) * C * 4);
+    w.base = take(BH * static_cast<size_t>(w.nchunk) * C * 4);
+    w.start = take(BH * C * 4);
+    w.count = take(BH * C * 4);
+    w.total = off;
+    return w;
+}
+
+sla_status_t cc_check(const sla_params_t* p, int C, int iters) {
+    sla_status_t s = check_params(p);
+    if (s != SLA_OK) return s;
+    if (C < 1 || iters < 1 || iters > 64 || p->N % C != 0) return SLA_ERR_INVALID_ARG;
+    if (C > 1024) return SLA_ERR_UNSUPPORTED;
+    return SLA_OK;
+}
+
+// labels -> stable order by label -> centroids, for one half-step
+template <int D>
+sla_status_t cc_sort_means(const sla_params_t* p, int C, const __nv_bfloat16* x, void* ws, const CcWs& w,
+                           int32_t* perm, double* cent, int* valid, cudaStream_t st) {
+    const int BH = p->B * p->H, N = p->N;
+    int* label = at<int>(ws, w.label);
+    {
+        Span sp(SLA_KERNEL_COCLUSTER, st);
+        sla::cc_count_kernel<<<dim3(w.nchunk, BH), 256, C * 4, st>>>(label, N, C, w.nchunk, at<int>(ws, w.counts));
+    }
+    {
+        Span sp(SLA_KERNEL_COCLUSTER, st);
+        sla::cc_scan_kernel<<<BH, 1024, 0, st>>>(at<int>(ws, w.counts), C, w.nchunk, at<int>(ws, w.base),
+                                                 at<int>(ws, w.start), at<int>(ws, w.count));
+    }
+    {
+        Span sp(SLA_KERNEL_COCLUSTER, st);
+        sla::cc_scatter_kernel<<<dim3(w.nchunk, BH), 32, C * 4, st>>>(label, N, C, w.nchunk, at<int>(ws, w.base),
+                                                                      perm);
+    }
+    {
+        Span sp(SLA_KERNEL_COCLUSTER, st);
+        sla::cc_means_kernel<D><<<dim3(C, BH), D, 0, st>>>(x, N, C, perm, at<int>(ws, w.start),
+                                                           at<int>(ws, w.count), cent, valid);
+    }
+    return launch_status();
+}
+
+template <int D>
+sla_status_t run_cocluster(const sla_params_t* p, int C, int iters, const void* q, const void* k, int32_t* q_perm,
+                           int32_t* k_perm, void* ws, const CcWs& w, cudaStream_t st) {
+    const int BH = p->B * p->H, N = p->N;
+    const auto* qb = static_cast<const __nv_bfloat16*>(q);
+    const auto* kb = static_cast<const __nv_bfloat16*>(k);
+    double* qc = at<double>(ws, w.qc);
+    double* kc = at<double>(ws, w.kc);
+    int* qv = at<int>(ws, w.qv);
+    int* kv = at<int>(ws, w.kv);
+    int* label = at<int>(ws, w.label);
+    auto assign = sla::cc_assign_kernel<D>;
+    constexpr size_t asmem = sla::cc_assign_smem<D>();
+    if (cudaFuncSetAttribute(assign, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(asmem)) !=
+        cudaSuccess)
+        return SLA_ERR_CUDA;
+    const dim3 agrid((N + 127) / 128, BH);
+    {
+        Span sp(SLA_KERNEL_COCLUSTER, st);
+        sla::cc_chunk_mean_kernel<D><<<dim3(C, BH), D, 0, st>>>(qb, N, C, qc, qv);
+    }
+    for (int it = 0; it < iters; ++it) {
+        // keys guided by the query centroids, then queries by the updated key centroids
+        {
+            Span sp(SLA_KERNEL_COCLUSTER, st);
+            assign<<<agrid, 128, asmem, st>>>(kb, N, C, qc, qv, label);
+        }
+        sla_status_t s = cc_sort_means<D>(p, C, kb, ws, w, k_perm, kc, kv, st);
+        if (s != SLA_OK) return s;
+        {
+            Span sp(SLA_KERNEL_COCLUSTER, st);
+            assign<<<agrid, 128, asmem, st>>>(qb, N, C, kc, kv, label);
+        }
+        s = cc_sort_means<D>(p, C, qb, ws, w, q_perm, qc, qv, st);
+        if (s != SLA_OK) return s;
+    }
+    return launch_status();
+}
+
+}  // namespace
+
+extern "C" size_t sla_cocluster_workspace_size(const sla_params_t* p, int32_t n_clusters) {
+    if (cc_check(p, n_clusters, 1) != SLA_OK) return 0;
+    return cc_layout(p, n_clusters).total;
+}
+
+extern "C" sla_status_t sla_cocluster(const sla_params_t* p, const void* q, const void* k, int32_t n_clusters,
+                                      int32_t iters, int32_t* q_perm, int32_t* k_perm, void* workspace,
+                                      size_t ws_bytes, sla_stream_t stream) {
+    sla_status_t s = cc_check(p, n_clusters, iters);
+    if (s != SLA_OK) return s;
+    if ((s = check_tensor(q, 16)) || (s = check_tensor(k, 16)) || (s = check_tensor(q_perm, 4)) ||
+        (s = check_tensor(k_perm, 4)))
+        return s;
+    const CcWs w = cc_layout(p, n_clusters);
+    if (!workspace || !aligned(workspace, kAlign) || ws_bytes < w.total) return SLA_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    s = p->d == 128 ? run_cocluster<128>(p, n_clusters, iters, q, k, q_perm, k_perm, workspace, w, st)
+                    : run_cocluster<64>(p, n_clusters, iters, q, k, q_perm, k_perm, workspace, w, st);
+    return finish(s, st);
+}
+
+extern "C" sla_status_t sla_permute_rows(const void* src, const int32_t* perm, void* dst, int64_t BH, int32_t N,
+                                         int32_t row_bytes, int32_t inverse, sla_stream_t stream) {
+    if (!src || !dst || !perm || src == dst || BH < 1 || N < 1 || BH * N > 0x7fffffffLL) return SLA_ERR_INVALID_ARG;
+    if (row_bytes < 4 || row_bytes % 4 || row_bytes > 4096 || (inverse != 0 && inverse != 1))
+        return SLA_ERR_INVALID_ARG;
+    if (!aligned(perm, 4)) return SLA_ERR_INVALID_ARG;
+    const bool vec = row_bytes % 16 == 0 && aligned(src, 16) && aligned(dst, 16);
+    if (!vec && (!aligned(src, 4) || !aligned(dst, 4))) return SLA_ERR_INVALID_ARG;
+    const int words = vec ? row_bytes / 16 : row_bytes / 4;
+    if (words > 256) return SLA_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const long long rows = BH * N;
+    const int per_row = std::max(1, 256 / words);
+    const int grid = grid_blocks((rows + per_row - 1) / per_row, 8);
+    Span sp(SLA_KERNEL_PERMUTE, st);
+    if (vec)
+        sla::permute_rows_kernel<uint4><<<grid, 256, 0, st>>>(static_cast<const uint4*>(src), perm,
+                                                             static_cast<uint4*>(dst), BH, N, words, inverse);
+    else
+        sla::permute_rows_kernel<uint32_t><<<grid, 256, 0, st>>>(static_cast<const uint32_t*>(src), perm,
+                                                                static_cast<uint32_t*>(dst), BH, N, words, inverse);
+    return finish(launch_status(), st);
+}
 
 // ------------------------------------------------------------ routing without allocation
 // The scratch of sla_route_noalloc lives in this file-scope device array: the

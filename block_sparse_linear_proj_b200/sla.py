@@ -39,9 +39,10 @@ SLA_OUT_FP32 = 1
 
 EXPORTED = ("sla_workspace_size", "sla_route", "sla_forward", "sla_pisa_forward",
             "sla_status_string", "sla_check_device_status", "sla_version",
-            "sla_profile_enable", "sla_profile_read", "sla_route_noalloc")
+            "sla_profile_enable", "sla_profile_read", "sla_route_noalloc",
+            "sla_cocluster", "sla_cocluster_workspace_size", "sla_permute_rows")
 KERNEL_KINDS = ("pool", "kv_stats", "h_reduce", "fold_w", "score_topk", "attn", "quant_q", "project",
-                "cov", "pre_attn")
+                "cov", "pre_attn", "cocluster", "permute")
 # profile entries that are phases of a call, not kernel launches
 PHASE_KINDS = ("pre_attn",)
 
@@ -97,6 +98,13 @@ def load():
             lib.sla_profile_enable.restype = ctypes.c_int
             lib.sla_profile_read.argtypes = [P, P]
             lib.sla_profile_read.restype = ctypes.c_int
+            lib.sla_cocluster_workspace_size.argtypes = [PP, ctypes.c_int32]
+            lib.sla_cocluster_workspace_size.restype = ctypes.c_size_t
+            lib.sla_cocluster.argtypes = [PP, P, P, ctypes.c_int32, ctypes.c_int32, P, P, P, ctypes.c_size_t, P]
+            lib.sla_cocluster.restype = ctypes.c_int
+            lib.sla_permute_rows.argtypes = [P, P, P, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
+                                             ctypes.c_int32, P]
+            lib.sla_permute_rows.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -243,3 +251,60 @@ def sla_profile_read():
     _raise(load().sla_profile_read(ctypes.cast(ms, ctypes.c_void_p), ctypes.cast(cnt, ctypes.c_void_p)),
            "sla_profile_read")
     return {KERNEL_KINDS[i]: (ms[i], cnt[i]) for i in range(n)}
+
+
+def cocluster_workspace(p: SlaParams, n_clusters: int, device=None) -> torch.Tensor:
+    """A workspace tensor for sla_cocluster with these parameters."""
+    n = int(load().sla_cocluster_workspace_size(ctypes.byref(p), int(n_clusters)))
+    if n == 0:
+        raise SlaError(SLA_ERR_INVALID_ARG, "sla_cocluster_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def sla_cocluster(p, q, k, n_clusters, iters, q_perm, k_perm, ws, stream=None):
+    """SVOO bidirectional co-clustering: writes the stable orders of the queries
+    and keys by cluster into q_perm, k_perm (int32 [B,H,N])."""
+    B, H, N, d = p.B, p.H, p.N, p.d
+    _check(q, torch.bfloat16, (B, H, N, d), "q")
+    _check(k, torch.bfloat16, (B, H, N, d), "k")
+    _check(q_perm, torch.int32, (B, H, N), "q_perm")
+    _check(k_perm, torch.int32, (B, H, N), "k_perm")
+    rc = load().sla_cocluster(ctypes.byref(p), _ptr(q), _ptr(k), int(n_clusters), int(iters), _ptr(q_perm),
+                              _ptr(k_perm), _ptr(ws), ws.numel(), _stream(stream))
+    _raise(rc, "sla_cocluster")
+    return q_perm, k_perm
+
+
+def sla_permute_rows(src, perm, dst, inverse=False, stream=None):
+    """dst[..., i, :] = src[..., perm[..., i], :] (inverse: the scatter back).
+    src, dst: [B, H, N, ...] contiguous (a trailing row of any size, or none);
+    perm: int32 [B, H, N]."""
+    if src.shape != dst.shape or src.dtype != dst.dtype:
+        raise ValueError("src and dst must have one shape and dtype")
+    B, H, N = perm.shape
+    if tuple(src.shape[:3]) != (B, H, N) or perm.dtype != torch.int32:
+        raise ValueError("perm must be int32 [B, H, N] matching src")
+    row_bytes = src[0, 0, 0].numel() * src.element_size()
+    rc = load().sla_permute_rows(_ptr(src), _ptr(perm), _ptr(dst), B * H, N, row_bytes,
+                                 1 if inverse else 0, _stream(stream))
+    _raise(rc, "sla_permute_rows")
+    return dst
+
+
+def sla_forward_coclustered(p, q, k, v, alpha, w_q, w_k, q_perm, k_perm, lut, out, ws, scratch=None,
+                            stream=None):
+    """sla_forward in the co-clustered order: Q and alpha gathered by q_perm, K and
+    V by k_perm (into scratch, a dict of tensors shaped like q, k, v, alpha and
+    out, allocated here if not given), the forward on them, and the output rows
+    scattered back by q_perm.  Every step runs in the library's kernels."""
+    if scratch is None:
+        scratch = {"q": torch.empty_like(q), "k": torch.empty_like(k), "v": torch.empty_like(v),
+                   "alpha": torch.empty_like(alpha), "out": torch.empty_like(out)}
+    sla_permute_rows(q, q_perm, scratch["q"], stream=stream)
+    sla_permute_rows(alpha, q_perm, scratch["alpha"], stream=stream)
+    sla_permute_rows(k, k_perm, scratch["k"], stream=stream)
+    sla_permute_rows(v, k_perm, scratch["v"], stream=stream)
+    sla_forward(p, scratch["q"], scratch["k"], scratch["v"], scratch["alpha"], w_q, w_k, lut, scratch["out"], ws,
+                stream)
+    sla_permute_rows(scratch["out"], q_perm, out, inverse=True, stream=stream)
+    return out

@@ -212,6 +212,47 @@ sla_status_t sla_pisa_cov_norms(const sla_params_t *p, const void *k, const void
                                 double *norms, void *workspace, size_t ws_bytes,
                                 sla_stream_t stream);
 
+/*
+ * sla_cocluster -- online bidirectional Q-K co-clustering of "Training-Free
+ * Sparse Attention for Fast Video Generation via Offline Layer-Wise Sparsity
+ * Profiling and Online Bidirectional Co-Clustering" (SVOO), sec. 2.B.  Per head,
+ * with C = n_clusters co-clusters:
+ *   query centroids start as the means of C contiguous chunks of N/C queries;
+ *   then iters times: each key joins the cluster whose query centroid has the
+ *   largest dot product with it (ties to the lower cluster), key centroids
+ *   become the means of their keys; each query joins the cluster of the largest
+ *   dot product with the key centroids, query centroids become the means of
+ *   their queries.  A cluster left without tokens is no candidate of the next
+ *   assignment.  All in fp64 from the bf16 inputs.
+ * Outputs the stable order of the tokens by their final cluster:
+ *   q_perm[b,h,i] = the original index of the query at position i, k_perm the
+ *   same for keys (int32 [B,H,N], device memory owned by the caller).
+ * Running the block-sparse path on Q, alpha gathered by q_perm and K, V gathered
+ * by k_perm (sla_permute_rows) puts tokens of one cluster into the same blocks;
+ * the output rows go back with the inverse permutation.  The page recomputes
+ * the clusters only every few diffusion steps (e.g. 20) and reuses them.
+ * q, k: bf16 [B,H,N,d], 16-byte aligned.  Needs 1 <= n_clusters <= 1024 dividing
+ * N, 1 <= iters <= 64, and a workspace of sla_cocluster_workspace_size() bytes
+ * (256-byte aligned); other parameters as sla_route (p->Bq, p->Bk, p->topk must
+ * be valid; they are not used).  Errors as sla_route.
+ */
+size_t sla_cocluster_workspace_size(const sla_params_t *p, int32_t n_clusters);
+sla_status_t sla_cocluster(const sla_params_t *p, const void *q, const void *k,
+                           int32_t n_clusters, int32_t iters, int32_t *q_perm, int32_t *k_perm,
+                           void *workspace, size_t ws_bytes, sla_stream_t stream);
+
+/*
+ * sla_permute_rows -- reorders the rows of a [BH, N, row] tensor by a per-head
+ * permutation perm (int32 [BH, N]): inverse = 0 gathers,
+ *   dst[bh, i, :] = src[bh, perm[bh, i], :],
+ * inverse = 1 scatters back, dst[bh, perm[bh, i], :] = src[bh, i, :].
+ * row_bytes: a multiple of 4, at most 4096 (16-byte aligned pointers and a
+ * multiple of 16 take 16-byte copies); src and dst must not overlap.  A perm
+ * entry outside [0, N) is skipped and flagged SLA_ERR_DEVICE_CHECK.
+ */
+sla_status_t sla_permute_rows(const void *src, const int32_t *perm, void *dst, int64_t BH,
+                              int32_t N, int32_t row_bytes, int32_t inverse, sla_stream_t stream);
+
 /* Static text for a status code. */
 const char *sla_status_string(sla_status_t s);
 
@@ -243,7 +284,9 @@ typedef enum {
     SLA_PHASE_PRE_ATTN = 9,     /* not a kernel: from the entry of a forward call
                                    on its stream to the start of its attention
                                    kernel (router, pre-pass and their joins)     */
-    SLA_KERNEL_KINDS = 10
+    SLA_KERNEL_COCLUSTER = 10,  /* the co-clustering kernels of one call          */
+    SLA_KERNEL_PERMUTE = 11,    /* row permutation (co-clustered order)           */
+    SLA_KERNEL_KINDS = 12
 } sla_kernel_kind_t;
 
 sla_status_t sla_profile_enable(int32_t on);

@@ -166,3 +166,33 @@ def test_cov_norms_wrapper_checks_arguments():
         SL.sla_pisa_cov_norms(p, k, k, torch.zeros(1, 1, 15, dtype=torch.float64), ws)
     with pytest.raises(TypeError):          # bf16 keys
         SL.sla_pisa_cov_norms(p, k.float(), k, torch.zeros(1, 1, 16, dtype=torch.float64), ws)
+
+
+def test_cocluster_argument_checks(lib):
+    p = S.params(1, 2, 1024, 64, 64, 64, 4)
+    need = lib.sla_cocluster_workspace_size(ctypes.byref(p), 16)
+    assert need > 0
+    assert lib.sla_cocluster_workspace_size(ctypes.byref(p), 3) == 0        # must divide N
+    assert lib.sla_cocluster_workspace_size(ctypes.byref(p), 2048) == 0     # more clusters than tokens
+    call = lambda C, it, ws_bytes=1 << 40, q=FAKE, qp=FAKE: lib.sla_cocluster(
+        ctypes.byref(p), q, FAKE, C, it, qp, FAKE, FAKE, ws_bytes, None)
+    assert call(16, 0) == S.SLA_ERR_INVALID_ARG                              # at least one iteration
+    assert call(16, 65) == S.SLA_ERR_INVALID_ARG
+    assert call(5, 3) == S.SLA_ERR_INVALID_ARG
+    assert call(16, 3, q=None) == S.SLA_ERR_INVALID_ARG
+    assert call(16, 3, qp=ctypes.c_void_p((1 << 20) + 2)) == S.SLA_ERR_INVALID_ARG
+    assert call(16, 3, ws_bytes=need - 1) == S.SLA_ERR_WORKSPACE
+    big = S.params(1, 1, 4096, 64, 64, 64, 4)
+    assert lib.sla_cocluster_workspace_size(ctypes.byref(big), 2048) == 0   # more than 1024 clusters
+
+
+def test_permute_rows_argument_checks(lib):
+    f = lib.sla_permute_rows
+    A, B2 = ctypes.c_void_p(1 << 20), ctypes.c_void_p(1 << 21)
+    assert f(A, FAKE, A, 2, 64, 256, 0, None) == S.SLA_ERR_INVALID_ARG          # in place
+    assert f(A, FAKE, B2, 2, 64, 6, 0, None) == S.SLA_ERR_INVALID_ARG           # not whole words
+    assert f(A, FAKE, B2, 2, 64, 256, 2, None) == S.SLA_ERR_INVALID_ARG         # inverse is 0 or 1
+    assert f(A, None, B2, 2, 64, 256, 0, None) == S.SLA_ERR_INVALID_ARG
+    assert f(ctypes.c_void_p((1 << 20) + 2), FAKE, B2, 2, 64, 4, 0, None) == S.SLA_ERR_INVALID_ARG
+    assert f(A, FAKE, B2, 0, 64, 256, 0, None) == S.SLA_ERR_INVALID_ARG
+    assert f(A, FAKE, B2, 2, 64, 8192, 0, None) == S.SLA_ERR_INVALID_ARG

@@ -55,6 +55,9 @@ class Workload:
     use_w: bool = True
     first_order: bool = False     # PISA: add the global first-order term
     cov_lambda: float = 0.0       # PISA: weight of the covariance-aware selection term
+    clusters: int = 0             # SVOO co-clustering: co-clusters (0 = raster order)
+    cluster_iters: int = 0        # SVOO co-clustering: alternating iterations
+    cluster_every: int = 0        # SVOO co-clustering: recomputed every this many steps
 
     @property
     def Nq(self) -> int:
@@ -97,8 +100,14 @@ WORKLOADS = {
     # about 28% of the selected blocks on these inputs)
     "pisa_cov": Workload("pisa_cov", 1, 24, 32768, 128, 64, 64, 77, "pisa", SPARSE_BF16,
                          "video", 1005, (21, 30, 52), None, False, False, 0.1),
+    # the SLA2 bf16 workload in the order of SVOO's online bidirectional co-clustering
+    # (64 co-clusters, 3 iterations, recomputed every 20 steps)
+    "sla2_svoo": Workload("sla2_svoo", 1, 12, 32768, 128, 128, 64, 52, "sla", SPARSE_BF16,
+                          "video", 1002, (21, 30, 52), (0.0, 1.0), True, clusters=64, cluster_iters=3,
+                          cluster_every=20),
 }
-ORDER = ["tiny", "sla2_bf16", "sla2_long", "sla2_fp8", "sla2_int8", "pisa", "pisa_fo", "pisa_cov"]
+ORDER = ["tiny", "sla2_bf16", "sla2_long", "sla2_fp8", "sla2_int8", "pisa", "pisa_fo", "pisa_cov",
+         "sla2_svoo"]
 
 
 def _bf16(x: torch.Tensor) -> torch.Tensor:
