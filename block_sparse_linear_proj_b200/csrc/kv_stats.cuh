@@ -387,240 +387,6 @@ __global__ void __launch_bounds__(256, 2) kv_stats_kernel(KvStatsArgs a) {
     }
 }
 
-// Single-pass variant of kv_stats_kernel for the bf16 SLA and PISA calls (no
-// 8-bit codes, which need each block's maximum before any code).  Thread t owns
-// the 16-byte column group u = t % (D/8) on rows t / (D/8) + (256 / (D/8)) i of
-// each 64-token block: it reads each of its K and V chunks once from the ring,
-// accumulates the column sums there, writes the fp16 copies of V and phi(K) and
-// (for the product) rewrites its K chunk in place as the product's left operand.
-// Column sums are combined across the warp by shuffles and across the eight
-// warps in a fixed order, so every statistic is deterministic.
-template <int D, bool TC>
-__global__ void __launch_bounds__(256, 2) kv_prep_kernel(KvStatsArgs a) {
-    extern __shared__ __align__(1024) unsigned char smem_raw[];
-    constexpr int TILE = kKvTok * D * 2;
-    constexpr int CPR = D / 8;                         // 16-byte chunks per row
-    constexpr int RSTEP = 256 / CPR;                   // rows between a thread's rows
-    constexpr int RPT = kKvTok / RSTEP;                // rows per thread
-    unsigned char* ring = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    double* kp = reinterpret_cast<double*>(ring + kKvStages * 2 * TILE);           // [8][D]
-    float* zp = reinterpret_cast<float*>(kp + 8 * D);                              // [8][D]
-    float* vp = zp + 8 * D;                                                        // [8][D]
-    float* kmf = vp + 8 * D;                                                       // [D] column means
-    uint64_t* mma_bar = reinterpret_cast<uint64_t*>(kmf + D);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_bar + 1);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const long long bh = blockIdx.y;
-    const int chunk = blockIdx.x;
-    const int jb0 = chunk * a.blocks_per_chunk;
-    const int nblk = min(a.blocks_per_chunk, a.Nk - jb0);
-    if (nblk <= 0) return;
-    const __nv_bfloat16* kh = a.k + bh * static_cast<long long>(a.N) * D;
-    const __nv_bfloat16* vh = a.v + bh * static_cast<long long>(a.N) * D;
-    const int u = tid % CPR, r0 = tid / CPR;
-
-    auto load_block = [&](int blk, int stage) {
-        unsigned char* kd = ring + stage * 2 * TILE;
-        unsigned char* vd = kd + TILE;
-        const long long row0 = static_cast<long long>(jb0 + blk) * kKvTok;
-        for (int q = tid; q < kKvTok * CPR; q += 256) {
-            const int n = q / CPR, uu = q % CPR;
-            const uint32_t off = kv_off<D, TC>(n, uu * 8);
-            cp_async16(kd + off, kh + (row0 + n) * D + uu * 8);
-            cp_async16(vd + off, vh + (row0 + n) * D + uu * 8);
-        }
-    };
-
-    const bool do_mma = TC && a.hpart != nullptr;
-    constexpr uint32_t TCOLS = D;
-    constexpr uint32_t ID_H = idesc_bf16(128, D, 1, 1);
-    uint32_t tmem = 0;
-    if (do_mma) {
-        if (warp == 0) {
-            tmem_alloc(tmem_slot, TCOLS);
-            tmem_relinquish();
-        }
-        if (tid == 0) {
-            mbar_init(mma_bar, 1);
-            *abort_flag = 0;
-            fence_barrier_init();
-        }
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        tmem = *tmem_slot;
-    }
-#pragma unroll
-    for (int s = 0; s < kKvStages - 1; ++s) {
-        if (s < nblk) load_block(s, s);
-        cp_async_commit();
-    }
-
-    for (int blk = 0; blk < nblk; ++blk) {
-        const int stage = blk % kKvStages;
-        cp_async_wait<kKvStages - 2>();
-        __syncthreads();
-        unsigned char* kt = ring + stage * 2 * TILE;
-        unsigned char* vt = kt + TILE;
-        if (!do_mma) {
-            const int nb = blk + kKvStages - 1;
-            if (nb < nblk) load_block(nb, nb % kKvStages);
-            cp_async_commit();
-        }
-        const long long row0 = static_cast<long long>(jb0 + blk) * kKvTok;
-        // one pass over this thread's chunks: column sums, fp16 copies, the product's operand
-        double ks[8];
-        float zs[8], vs[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) { ks[e] = 0.0; zs[e] = 0.f; vs[e] = 0.f; }
-        bool bad = false;
-#pragma unroll
-        for (int i = 0; i < RPT; ++i) {
-            const int n = r0 + i * RSTEP;
-            const uint32_t off = kv_off<D, TC>(n, u * 8);
-            uint4 kx = *reinterpret_cast<const uint4*>(kt + off);
-            const uint4 vx = *reinterpret_cast<const uint4*>(vt + off);
-            const uint32_t kw[4] = {kx.x, kx.y, kx.z, kx.w}, vw[4] = {vx.x, vx.y, vx.z, vx.w};
-            uint32_t ph[4], vh16[4], pb[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float k0 = bf16lo(kw[e]), k1 = bf16hi(kw[e]);
-                const float v0 = bf16lo(vw[e]), v1 = bf16hi(vw[e]);
-                ks[2 * e] += static_cast<double>(k0);
-                ks[2 * e + 1] += static_cast<double>(k1);
-                const float p0 = fmaxf(k0, 0.f), p1 = fmaxf(k1, 0.f);
-                zs[2 * e] += p0;
-                zs[2 * e + 1] += p1;
-                vs[2 * e] += v0;
-                vs[2 * e + 1] += v1;
-                bad |= !(fabsf(k0) < 65504.f) || !(fabsf(k1) < 65504.f) ||
-                       !(fabsf(v0) < 65504.f) || !(fabsf(v1) < 65504.f);
-                ph[e] = pack_half2(p0, p1);
-                vh16[e] = pack_half2(v0, v1);
-                pb[e] = relu_bf16x2(kw[e]);
-            }
-            const long long g = (row0 + n) * D + u * 8;
-            if (a.v16) *reinterpret_cast<uint4*>(a.v16 + bh * static_cast<long long>(a.N) * D + g) =
-                make_uint4(vh16[0], vh16[1], vh16[2], vh16[3]);
-            if (a.phik16) *reinterpret_cast<uint4*>(a.phik16 + bh * static_cast<long long>(a.N) * D + g) =
-                make_uint4(ph[0], ph[1], ph[2], ph[3]);
-            if (do_mma && !a.center) *reinterpret_cast<uint4*>(kt + off) = make_uint4(pb[0], pb[1], pb[2], pb[3]);
-        }
-        if (bad && a.v16) report(kStatusRange);
-        // across the lanes of the warp that own the same columns
-#pragma unroll
-        for (int o = CPR; o < 32; o <<= 1) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                ks[e] += __shfl_xor_sync(0xffffffffu, ks[e], o);
-                zs[e] += __shfl_xor_sync(0xffffffffu, zs[e], o);
-                vs[e] += __shfl_xor_sync(0xffffffffu, vs[e], o);
-            }
-        }
-        if (lane < CPR) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                kp[warp * D + u * 8 + e] = ks[e];
-                zp[warp * D + u * 8 + e] = zs[e];
-                vp[warp * D + u * 8 + e] = vs[e];
-            }
-        }
-        // the previous block's product has completed: its stage may be refilled
-        if (do_mma && blk > 0 && tid == 0 && !*abort_flag &&
-            !mbar_wait(mma_bar, (blk - 1) & 1, abort_flag, a.wait_ns)) {
-            report(kStatusTimeout);
-            *abort_flag = 1;
-        }
-        if (do_mma && !a.center) fence_proxy_async_smem();     // phi(K) -> the tensor core
-        __syncthreads();
-        const bool dead = do_mma && *abort_flag;
-        if (do_mma) {
-            const int nb = blk + kKvStages - 1;
-            if (nb < nblk && !dead) load_block(nb, nb % kKvStages);
-            cp_async_commit();
-        }
-        if (tid < D) {
-            double kk = 0.0;
-            float zz = 0.f, vv = 0.f;
-#pragma unroll
-            for (int w = 0; w < 8; ++w) {
-                kk += kp[w * D + tid];
-                zz += zp[w * D + tid];
-                vv += vp[w * D + tid];
-            }
-            const int j = jb0 + blk;
-            const double kmean = kk * (1.0 / kKvTok);
-            if (a.kbarT) a.kbarT[(bh * D + tid) * a.Nk + j] = kmean;
-            if (a.zj) a.zj[(bh * a.Nk + j) * D + tid] = zz;
-            if (a.kc) a.kc[(bh * a.Nk + j) * D + tid] = __float2bfloat16_rn(static_cast<float>(kmean));
-            if (a.vbar) a.vbar[(bh * a.Nk + j) * D + tid] = __float2half_rn(vv * (1.f / kKvTok));
-            kmf[tid] = static_cast<float>(kmean);
-        }
-        if (do_mma && a.center && !dead) {
-            // the product's left operand: the keys centred by this block's column means
-            __syncthreads();
-#pragma unroll
-            for (int i = 0; i < RPT; ++i) {
-                const int n = r0 + i * RSTEP;
-                uint4* px = reinterpret_cast<uint4*>(kt + kv_off<D, TC>(n, u * 8));
-                uint4 x = *px;
-                const float4 m0 = *reinterpret_cast<const float4*>(kmf + u * 8);
-                const float4 m1 = *reinterpret_cast<const float4*>(kmf + u * 8 + 4);
-                x.x = pack_bf16(bf16lo(x.x) - m0.x, bf16hi(x.x) - m0.y);
-                x.y = pack_bf16(bf16lo(x.y) - m0.z, bf16hi(x.y) - m0.w);
-                x.z = pack_bf16(bf16lo(x.z) - m1.x, bf16hi(x.z) - m1.y);
-                x.w = pack_bf16(bf16lo(x.w) - m1.z, bf16hi(x.w) - m1.w);
-                *px = x;
-            }
-            fence_proxy_async_smem();
-            __syncthreads();
-        }
-        if (do_mma && !dead && tid == 0) {
-            tc_fence_after();
-            const uint32_t kt_s = smem_u32(kt), vt_s = smem_u32(vt);
-            const uint32_t lbo = D == 128 ? kKvTok * 128 : 0;
-#pragma unroll
-            for (int kk2 = 0; kk2 < kKvTok / 16; ++kk2) {
-                const uint64_t ad = sdesc(kt_s + kk2 * 2048, lbo, 1024, kSwizzle128B);
-                const uint64_t bd = sdesc(vt_s + kk2 * 2048, kKvTok * 128, 1024, kSwizzle128B);
-                umma_f16_ss(tmem, ad, bd, ID_H, (blk > 0 || kk2 > 0) ? 1u : 0u);
-            }
-            umma_commit(mma_bar);
-        }
-    }
-    cp_async_wait<0>();
-
-    if (do_mma) {
-        if (tid == 0 && !*abort_flag && !mbar_wait(mma_bar, (nblk - 1) & 1, abort_flag, a.wait_ns)) {
-            report(kStatusTimeout);
-            *abort_flag = 1;
-        }
-        __syncthreads();
-        tc_fence_after();
-        if (!*abort_flag && warp < D / 32) {
-            float* hp = a.hpart + (bh * a.nchunk + chunk) * static_cast<long long>(D) * D;
-            const int r = warp * 32 + lane;
-            const uint32_t tl = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-#pragma unroll 1
-            for (int cc = 0; cc < D; cc += 32) {
-                uint32_t v[32];
-                tmem_ld32(tl + cc, v);
-                tmem_ld_wait();
-#pragma unroll
-                for (int x = 0; x < 32; x += 4)
-                    *reinterpret_cast<float4*>(hp + r * D + cc + x) =
-                        make_float4(__uint_as_float(v[x]), __uint_as_float(v[x + 1]),
-                                    __uint_as_float(v[x + 2]), __uint_as_float(v[x + 3]));
-            }
-        }
-        tc_fence_before();
-        __syncthreads();
-        if (warp == 0) tmem_dealloc(tmem, TCOLS);
-    }
-}
-
 // H[bh] = sum over chunks of hpart (fixed order), stored transposed
 // (hsum[bh][e][c] = H[c][e]); Z[bh] = sum_j z_j.
 // grid (D*D/256 + 1, BH), 256 threads; the last x-block reduces Z: its eight

@@ -417,14 +417,10 @@ sla_status_t launch_kv(const sla_params_t* p, const void* k, const void* v, void
     a.k_int8 = (fp8 && k_int8) ? 1 : 0;
     a.wait_ns = wait_limit_ns();
     // alignment slack, K/V ring, column partials, maxima, column means, barrier,
-    // TMEM slot, flag.  Without 8-bit codes the single-pass variant runs (per-warp
-    // column partials [8][D] of the three sums, column means).
-    const bool single = !fp8;
-    const size_t smem = single ? 1024 + sla::kKvStages * 2 * 64 * D * 2 + 8 * D * (8 + 4 + 4) + D * 4 + 16
-                               : 1024 + sla::kKvStages * 2 * 64 * D * 2 + 256 * 8 + 2 * 256 * 4 + 16 * 4 +
-                                     128 * 4 + 16;
-    auto kern = single ? (a.hpart ? sla::kv_prep_kernel<D, true> : sla::kv_prep_kernel<D, false>)
-                       : (a.hpart ? sla::kv_stats_kernel<D, true> : sla::kv_stats_kernel<D, false>);
+    // TMEM slot, flag
+    const size_t smem = 1024 + sla::kKvStages * 2 * 64 * D * 2 + 256 * 8 + 2 * 256 * 4 + 16 * 4 +
+                        128 * 4 + 16;
+    auto kern = a.hpart ? sla::kv_stats_kernel<D, true> : sla::kv_stats_kernel<D, false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
         return SLA_ERR_CUDA;
