@@ -11,9 +11,9 @@
 // cov_hbar_kernel: Hbar, the chunk sums added in order in fp64.
 // cov_norm_kernel: per block, A = H_j - Hbar (the same fp32 H_j) in shared
 // memory, then kLanczos Lanczos steps on A^T A (products A q and A^T y, full
-// re-orthogonalisation by classical Gram-Schmidt applied twice) and the largest
-// eigenvalue of the tridiagonal matrix by bisection on its Sturm sequence in
-// fp64; M_j is its square root.  (Lanczos: the Ritz values of a Krylov space
+// re-orthogonalisation by classical Gram-Schmidt) and the largest eigenvalue of
+// the tridiagonal matrix by multisection on its Sturm sequence in fp64 (256
+// points per round, one per thread); M_j is its square root.  (Lanczos: the Ritz values of a Krylov space
 // approach the extreme eigenvalues; Sturm: the number of negative pivots of
 // T - x I counts the eigenvalues below x.)
 // Every wait is a __syncthreads; there is no spin-wait.
@@ -24,6 +24,7 @@ namespace sla {
 
 constexpr int kCovTok = 64;       // tokens per KV block
 constexpr int kLanczos = 24;      // Lanczos steps (at most)
+constexpr int kQRows = 28;        // Lanczos vector rows kept: kLanczos + 1, padded to 4 with zeros
 
 // Shared layout of one block: ks [64][D] fp32 centred keys, vs [64][D] fp32
 // values, kmean [D] fp64.  Loads block (K, V rows given) and centres the keys.
@@ -56,8 +57,13 @@ __device__ __forceinline__ void cov_load_block(const __nv_bfloat16* __restrict__
     __syncthreads();
 }
 
-// acc[i][j] += sum_n ks[n][ty RT + i] vs[n][tx RT + j]: thread (ty, tx) =
-// (tid / 16, tid % 16) owns an RT x RT tile of the D x D matrix, RT = D / 16.
+// Tile layout of a D x D matrix over 256 threads: thread (ty, tx) = (tid / 16,
+// tid % 16) owns rows cov_idx(ty, i) and columns cov_idx(tx, jj), i, jj < RT =
+// D / 16, where cov_idx(t, i) = 64 (i / 4) + 4 t + i % 4 -- runs of four, 64
+// apart, so that a half-warp's 16-byte reads of a row cover 256 contiguous bytes.
+__device__ __forceinline__ int cov_idx(int t, int i) { return (i >> 2) * 64 + t * 4 + (i & 3); }
+
+// acc[i][jj] += sum_n ks[n][cov_idx(ty, i)] vs[n][cov_idx(tx, jj)], n in order.
 template <int D>
 __device__ __forceinline__ void cov_accumulate(const float* ks, const float* vs,
                                                float (&acc)[D / 16][D / 16]) {
@@ -68,8 +74,8 @@ __device__ __forceinline__ void cov_accumulate(const float* ks, const float* vs,
         float a[RT], b[RT];
 #pragma unroll
         for (int i = 0; i < RT; i += 4) {
-            const float4 x = *reinterpret_cast<const float4*>(ks + n * D + ty * RT + i);
-            const float4 y = *reinterpret_cast<const float4*>(vs + n * D + tx * RT + i);
+            const float4 x = *reinterpret_cast<const float4*>(ks + n * D + cov_idx(ty, i));
+            const float4 y = *reinterpret_cast<const float4*>(vs + n * D + cov_idx(tx, i));
             a[i] = x.x; a[i + 1] = x.y; a[i + 2] = x.z; a[i + 3] = x.w;
             b[i] = y.x; b[i + 1] = y.y; b[i + 2] = y.z; b[i + 3] = y.w;
         }
@@ -112,7 +118,7 @@ __global__ void __launch_bounds__(256) cov_hsum_kernel(const __nv_bfloat16* __re
     for (int i = 0; i < RT; ++i)
 #pragma unroll
         for (int j = 0; j < RT; j += 4)
-            *reinterpret_cast<float4*>(dst + (ty * RT + i) * D + tx * RT + j) =
+            *reinterpret_cast<float4*>(dst + cov_idx(ty, i) * D + cov_idx(tx, j)) =
                 make_float4(acc[i][j], acc[i][j + 1], acc[i][j + 2], acc[i][j + 3]);
 }
 
@@ -142,6 +148,53 @@ __device__ __forceinline__ float cov_block_sum(float x, float* red) {
     return s;
 }
 
+// The sums over the warp's 32 lanes of R partial values per lane (R a power of
+// two, 1 < R <= 32), reduce-scattered: each step swaps half of the remaining
+// values with the lane 16, 8, ... apart and keeps the sums of the other half, so
+// after log2 R steps lane l holds the sum, over the lanes that agree with l in
+// bits log2(32 / R) and up, of row l / (32 / R); the lanes below finish it with
+// plain shuffles.  Every lane returns the full sum of its row.
+template <int R>
+__device__ __forceinline__ float cov_warp_rows(float (&p)[R], int lane) {
+#pragma unroll
+    for (int n = R, o = 16; n > 1; n >>= 1, o >>= 1) {
+        const bool up = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < n / 2; ++i) {
+            const float send = up ? p[i] : p[i + n / 2];
+            const float keep = up ? p[i + n / 2] : p[i];
+            p[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+    }
+    float s = p[0];
+#pragma unroll
+    for (int o = 16 / R; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    return s;
+}
+
+// The sums over each half-warp's 16 lanes of RT partial values per lane (RT = 4
+// or 8): a reduce-scatter within the half (offsets 8, 4, ...) leaves value i's
+// sum on lane i * 16 / RT of the half, from where every lane of the half
+// gathers all RT sums into out.
+template <int RT>
+__device__ __forceinline__ void cov_half_rows(float (&p)[RT], int lane, float (&out)[RT]) {
+#pragma unroll
+    for (int n = RT, o = 8; n > 1; n >>= 1, o >>= 1) {
+        const bool up = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < n / 2; ++i) {
+            const float send = up ? p[i] : p[i + n / 2];
+            const float keep = up ? p[i + n / 2] : p[i];
+            p[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+    }
+    float s = p[0];
+#pragma unroll
+    for (int o = 8 / RT; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+#pragma unroll
+    for (int i = 0; i < RT; ++i) out[i] = __shfl_sync(0xffffffffu, s, (lane & 16) | (i * (16 / RT)));
+}
+
 // grid (Nk, BH), 256 threads.  out[bh * Nk + j] = scale * M_j (fp64).
 template <int D>
 __global__ void __launch_bounds__(256, 2) cov_norm_kernel(const __nv_bfloat16* __restrict__ k,
@@ -150,90 +203,176 @@ __global__ void __launch_bounds__(256, 2) cov_norm_kernel(const __nv_bfloat16* _
                                                           const float* __restrict__ hbar,
                                                           double scale, double* __restrict__ out) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    constexpr int RT = D / 16, LDA = D + 1;
-    constexpr int R0 = (2 * kCovTok * D > D * LDA ? 2 * kCovTok * D : D * LDA);   // floats
-    float* ks = reinterpret_cast<float*>(smem_raw);          // block tiles, then A
-    float* vs = ks + kCovTok * D;
-    float* am = ks;                                          // A [D][D + 1]
-    double* kmean = reinterpret_cast<double*>(ks + R0);      // [D]
-    float* qv = reinterpret_cast<float*>(kmean + D);         // Lanczos vectors [kLanczos + 1][D]
-    float* yv = qv + (kLanczos + 1) * D;                     // [D]
-    float* red = yv + D;                                     // [(kLanczos + 1) * 8]
-    float* coef = red + (kLanczos + 1) * 8;                  // [kLanczos + 1]
+    constexpr int RT = D / 16;
+    float* ks = reinterpret_cast<float*>(smem_raw);          // [64][D] centred keys
+    float* vs = ks + kCovTok * D;                            // [64][D] values
+    double* kmean = reinterpret_cast<double*>(vs + kCovTok * D);   // [D]
+    float* qv = reinterpret_cast<float*>(kmean + D);         // Lanczos vectors [kQRows][D]
+    float* wv = qv + kQRows * D;                             // [D] w before re-orthogonalisation
+    float* wraw = wv + D;                                    // [D] w after it, not yet normalised
+    float* part = wraw + D;                                  // [8][D] per-warp sums of A^T y
+    float* red = part + 8 * D;                               // [16]
+    float* coef = red + 16;                                  // [32]
     double* alpha = reinterpret_cast<double*>(
-        (reinterpret_cast<uintptr_t>(coef + kLanczos + 1) + 7) & ~static_cast<uintptr_t>(7));  // [kLanczos]
+        (reinterpret_cast<uintptr_t>(coef + 32) + 7) & ~static_cast<uintptr_t>(7));  // [kLanczos]
     double* beta = alpha + kLanczos;                                  // [kLanczos]
 
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int ty = tid / 16, tx = tid % 16, half = (lane >> 4) & 1;
     const long long bh = blockIdx.y;
     const int j = blockIdx.x;
     const long long row0 = (bh * N + static_cast<long long>(j) * kCovTok) * D;
 
-    // 1. H_j, then A = H_j - Hbar over the tiles (shared memory reused)
+    // 1. H_j as this thread's RT x RT tile in registers, then A = H_j - Hbar in place
     cov_load_block<D>(k + row0, v + row0, ks, vs, kmean);
-    float acc[RT][RT];
+    float a[RT][RT];
 #pragma unroll
     for (int i = 0; i < RT; ++i)
 #pragma unroll
-        for (int jj = 0; jj < RT; ++jj) acc[i][jj] = 0.f;
-    cov_accumulate<D>(ks, vs, acc);
-    __syncthreads();
+        for (int jj = 0; jj < RT; ++jj) a[i][jj] = 0.f;
+    cov_accumulate<D>(ks, vs, a);
     {
-        const int ty = tid / 16, tx = tid % 16;
         const float* hb = hbar + bh * D * D;
 #pragma unroll
         for (int i = 0; i < RT; ++i)
 #pragma unroll
-            for (int jj = 0; jj < RT; ++jj) {
-                const int r = ty * RT + i, c = tx * RT + jj;
-                am[r * LDA + c] = acc[i][jj] - hb[r * D + c];
+            for (int jj = 0; jj < RT; jj += 4) {
+                const float4 h = __ldg(reinterpret_cast<const float4*>(hb + cov_idx(ty, i) * D + cov_idx(tx, jj)));
+                a[i][jj] -= h.x;
+                a[i][jj + 1] -= h.y;
+                a[i][jj + 2] -= h.z;
+                a[i][jj + 3] -= h.w;
             }
     }
-    // 2. Lanczos on B = A^T A from q_0 proportional to (1 + t / D)
-    const bool own = tid < D;                                 // thread t holds element t
-    const float x0 = own ? 1.f + static_cast<float>(tid) / D : 0.f;
-    const float n0 = cov_block_sum(x0 * x0, red);            // (also orders the writes of A)
-    if (own) qv[tid] = x0 / sqrtf(n0);
+    // 2. Lanczos on B = A^T A from q_0 proportional to (1 + t / D).  Thread t < D owns
+    //    element t of the vectors (q_it and q_{it-1} in registers).  A q: each thread
+    //    multiplies its tile by its columns of q, the half-warp sums the rows
+    //    (cov_half_rows), so every lane holds y = A q on its RT rows; A^T y: each
+    //    thread multiplies its tile by those, the two halves of the warp add up,
+    //    and the eight warps' sums meet in shared memory.  alpha = q . A^T A q is
+    //    |A q|^2.  w leaves each step unnormalised in wraw; the next product scales
+    //    it by 1 / beta on the way in.
+    const bool own = tid < D;
+    float qc = own ? 1.f + static_cast<float>(tid) / D : 0.f;
+    for (int i = D + tid; i < kQRows * D; i += 256) qv[i] = 0.f;
+    const float n0 = cov_block_sum(qc * qc, red);            // (also orders the writes of qv)
+    const float inv0 = 1.f / sqrtf(n0);
+    qc *= inv0;
+    if (own) {
+        qv[tid] = qc;
+        wraw[tid] = qc;
+    }
     __syncthreads();
     int m = 0;
-    float b_prev = 0.f, a_max = 0.f;      // (every thread holds the same sums)
+    float qp = 0.f, inv_b = 1.f, b_prev = 0.f, a_max = 0.f;   // (every thread holds the same sums)
     for (int it = 0; it < kLanczos; ++it) {
-        const float* q = qv + it * D;
-        if (own) {                                            // y = A q
-            float s = 0.f;
-            for (int c = 0; c < D; ++c) s = fmaf(am[tid * LDA + c], q[c], s);
-            yv[tid] = s;
+        {
+            float x[RT], p[RT], y[RT];
+#pragma unroll
+            for (int jj = 0; jj < RT; jj += 4) {
+                const float4 t4 = *reinterpret_cast<const float4*>(wraw + cov_idx(tx, jj));
+                x[jj] = t4.x * inv_b;
+                x[jj + 1] = t4.y * inv_b;
+                x[jj + 2] = t4.z * inv_b;
+                x[jj + 3] = t4.w * inv_b;
+            }
+#pragma unroll
+            for (int i = 0; i < RT; ++i) {
+                float s = a[i][0] * x[0];
+#pragma unroll
+                for (int jj = 1; jj < RT; ++jj) s = fmaf(a[i][jj], x[jj], s);
+                p[i] = s;
+            }
+            cov_half_rows<RT>(p, lane, y);
+            float y2 = 0.f;                                   // |y|^2 over the warp's rows
+            if (tx == 0) {
+#pragma unroll
+                for (int i = 0; i < RT; ++i) y2 = fmaf(y[i], y[i], y2);
+            }
+            y2 += __shfl_xor_sync(0xffffffffu, y2, 16);
+            if (lane == 0) red[warp] = y2;
+            float c[RT], r[RT / 2];
+#pragma unroll
+            for (int jj = 0; jj < RT; ++jj) {
+                float s = a[0][jj] * y[0];
+#pragma unroll
+                for (int i = 1; i < RT; ++i) s = fmaf(a[i][jj], y[i], s);
+                c[jj] = s;
+            }
+            // the halves add up; half h keeps columns cov_idx(tx, h RT/2 + kk), contiguous
+#pragma unroll
+            for (int kk = 0; kk < RT / 2; ++kk) {
+                const float send = half ? c[kk] : c[kk + RT / 2];
+                const float keep = half ? c[kk + RT / 2] : c[kk];
+                r[kk] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+            }
+            float* dst = part + warp * D + cov_idx(tx, half * (RT / 2));
+            if constexpr (RT / 2 == 4) {
+                *reinterpret_cast<float4*>(dst) = make_float4(r[0], r[1], r[2], r[3]);
+            } else {
+                *reinterpret_cast<float2*>(dst) = make_float2(r[0], r[1]);
+            }
         }
         __syncthreads();
-        float w = 0.f;
-        if (own) {                                            // w = A^T y - beta q_prev
-            float s = 0.f;
-            for (int r = 0; r < D; ++r) s = fmaf(am[r * LDA + tid], yv[r], s);
-            w = s - (it > 0 ? b_prev * qv[(it - 1) * D + tid] : 0.f);
-        }
-        const float al = cov_block_sum(own ? w * q[tid] : 0.f, red);
-        if (own) w -= al * q[tid];
-        // full re-orthogonalisation against q_0 .. q_it, twice
-#pragma unroll 1
-        for (int pass = 0; pass < 2; ++pass) {
-            for (int i = 0; i <= it; ++i) {
-                float p = own ? w * qv[i * D + tid] : 0.f;
+        float al = 0.f;
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
-                if (lane == 0) red[i * 8 + warp] = p;
-            }
-            __syncthreads();
-            if (tid <= it) {
+        for (int u = 0; u < 8; ++u) al += red[u];
+        float w = 0.f;                                        // w = A^T y - alpha q - beta q_prev
+        if (own) {
+            float s = part[tid];
+#pragma unroll
+            for (int u = 1; u < 8; ++u) s += part[u * D + tid];
+            w = s - al * qc - b_prev * qp;
+            wv[tid] = w;
+        }
+        __syncthreads();
+        // full re-orthogonalisation against q_0 .. q_it (one classical Gram-Schmidt
+        // pass: in an fp32 emulation on Gaussian and video-latent blocks a second
+        // pass changed no norm by more than 1e-9 relative): warp u forms the
+        // coefficients q_i . w of i = u, u + 8, u + 16, u + 24 together (lanes over
+        // the elements, one butterfly; zero for i > it), then every element
+        // subtracts the multiples of the q_i, rows past it being zero
+        {
+            constexpr int E = D / 32;
+            float wl[E], pc[4];
+#pragma unroll
+            for (int e = 0; e < E; ++e) wl[e] = wv[lane + 32 * e];
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                const int i = warp + 8 * kk;
                 float s = 0.f;
+                if (i <= it) {
 #pragma unroll
-                for (int w8 = 0; w8 < 8; ++w8) s += red[tid * 8 + w8];
-                coef[tid] = s;
+                    for (int e = 0; e < E; ++e) s = fmaf(qv[i * D + lane + 32 * e], wl[e], s);
+                }
+                pc[kk] = s;
             }
-            __syncthreads();
-            if (own)
-                for (int i = 0; i <= it; ++i) w -= coef[i] * qv[i * D + tid];
+            const float cs = cov_warp_rows<4>(pc, lane);
+            if ((lane & 7) == 0) coef[warp + lane] = cs;          // i = warp + 8 (lane / 8)
         }
-        const float bsq = cov_block_sum(own ? w * w : 0.f, red);
+        __syncthreads();
+        if (own) {
+            float w0 = w, w1 = 0.f;
+            for (int i = 0; i <= it; i += 4) {
+                w0 = fmaf(-coef[i], qv[i * D + tid], w0);
+                w1 = fmaf(-coef[i + 1], qv[(i + 1) * D + tid], w1);
+                w0 = fmaf(-coef[i + 2], qv[(i + 2) * D + tid], w0);
+                w1 = fmaf(-coef[i + 3], qv[(i + 3) * D + tid], w1);
+            }
+            w = w0 + w1;
+            wraw[tid] = w;
+        }
+        {                                                     // beta = |w|
+            float w2 = own ? w * w : 0.f;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) w2 += __shfl_xor_sync(0xffffffffu, w2, o);
+            if (lane == 0) red[8 + warp] = w2;
+        }
+        __syncthreads();
+        float bsq = 0.f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) bsq += red[8 + u];
         const float be = sqrtf(bsq);
         if (tid == 0) {
             alpha[it] = static_cast<double>(al);
@@ -244,34 +383,50 @@ __global__ void __launch_bounds__(256, 2) cov_norm_kernel(const __nv_bfloat16* _
         // an invariant subspace (or A = 0): the tridiagonal matrix is complete
         // (al, be and a_max are CTA-wide sums, so every thread takes the same exit)
         if (!(be > 1e-7f * a_max + 1e-30f)) break;
-        if (own) qv[(it + 1) * D + tid] = w / be;
+        inv_b = 1.f / be;
+        const float qn = w * inv_b;                           // q_{it+1}, as the next product sees it
+        if (own) qv[(it + 1) * D + tid] = qn;
+        qp = qc;
+        qc = qn;
         b_prev = be;
-        __syncthreads();
     }
     __syncthreads();
-    // 3. the largest eigenvalue of T (m x m) by bisection; M_j = sqrt of it
-    if (tid == 0) {
-        double hi = 0.0;
-        for (int i = 0; i < m; ++i) {
-            const double g = fabs(alpha[i]) + (i > 0 ? fabs(beta[i - 1]) : 0.0) +
-                             (i + 1 < m ? fabs(beta[i]) : 0.0);
-            hi = fmax(hi, g);
-        }
-        double lo = 0.0;
-        for (int s = 0; s < 200 && hi - lo > 1e-15 * hi; ++s) {
-            const double x = 0.5 * (lo + hi);
-            int below = 0;                                  // eigenvalues of T below x
-            double d = alpha[0] - x;
-            if (d < 0.0) ++below;
-            for (int i = 1; i < m; ++i) {
-                const double dd = d != 0.0 ? d : 1e-300;
-                d = alpha[i] - x - beta[i - 1] * beta[i - 1] / dd;
-                if (d < 0.0) ++below;
-            }
-            if (below == m) hi = x; else lo = x;
-        }
-        out[bh * Nk + j] = scale * sqrt(fmax(hi, 0.0));
+    // 3. the largest eigenvalue of T (m x m) by multisection: each round every thread
+    //    counts the eigenvalues of T below its own point x of the interval, as the
+    //    sign changes along p_0 .. p_{m-1}, the leading principal minors of T - x I
+    //    (Sturm sequence; three-term recurrence, no division, T scaled by 1 / hi so
+    //    no term overflows; a zero minor counts as positive, which counts one change
+    //    across it either way since its neighbours then have opposite signs), and
+    //    the interval shrinks to the two points around the largest eigenvalue, 257
+    //    times per round; M_j is the square root of the upper end
+    double hi = 0.0;
+    for (int i = 0; i < m; ++i) {
+        const double g = fabs(alpha[i]) + (i > 0 ? fabs(beta[i - 1]) : 0.0) + (i + 1 < m ? fabs(beta[i]) : 0.0);
+        hi = fmax(hi, g);
     }
+    const double inv = hi > 0.0 ? 1.0 / hi : 0.0;
+    double lo = 0.0;
+    for (int round = 0; round < 4; ++round) {
+        const double step = (hi - lo) / 257.0;
+        const double x = lo + step * (tid + 1);
+        double pm = 1.0, pc = (alpha[0] - x) * inv;
+        int below = pc < 0.0;
+        for (int i = 1; i < m; ++i) {
+            const double b = beta[i - 1] * inv;
+            const double pn = fma((alpha[i] - x) * inv, pc, -(b * b) * pm);
+            below += (pn < 0.0) != (pc < 0.0);
+            pm = pc;
+            pc = pn;
+        }
+        // points below the largest eigenvalue count fewer than m eigenvalues below them
+        const int kb = __syncthreads_count(below < m);
+        const double nlo = kb > 0 ? lo + step * kb : lo;
+        const double nhi = kb < 256 ? lo + step * (kb + 1) : hi;
+        lo = nlo;
+        hi = nhi;
+        if (!(hi - lo > 1e-15 * hi)) break;
+    }
+    if (tid == 0) out[bh * Nk + j] = scale * sqrt(fmax(hi, 0.0));
 }
 
 }  // namespace sla

@@ -354,9 +354,8 @@ sla_status_t launch_cov_t(const sla_params_t* p, const void* k, const void* v, v
     float* part = at<float>(ws, w.covpart);
     float* hbar = at<float>(ws, w.covhbar);
     const size_t smem_h = 2 * sla::kCovTok * D * 4 + D * 8;
-    constexpr int R0 = (2 * sla::kCovTok * D > D * (D + 1) ? 2 * sla::kCovTok * D : D * (D + 1));
-    const size_t smem_n = R0 * 4 + D * 8 + ((sla::kLanczos + 1) * D + D + (sla::kLanczos + 1) * 8 +
-                                           sla::kLanczos + 1) * 4 + 8 + 2 * sla::kLanczos * 8;
+    const size_t smem_n = 2 * sla::kCovTok * D * 4 + D * 8 + (sla::kQRows * D + 10 * D + 16 + 32) * 4 + 8 +
+                          2 * sla::kLanczos * 8;
     auto kh = sla::cov_hsum_kernel<D>;
     auto kn = sla::cov_norm_kernel<D>;
     if (cudaFuncSetAttribute(kh, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_h)) != cudaSuccess ||
