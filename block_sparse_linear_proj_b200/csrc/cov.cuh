@@ -9,14 +9,15 @@
 // are centred in fp64 and rounded once to fp32, so every product with a bf16
 // value is exact in fp32 and only the 64-term sums round.
 // cov_hbar_kernel: Hbar, the chunk sums added in order in fp64.
-// cov_norm_kernel: per block, A = H_j - Hbar (the same fp32 H_j) in shared
-// memory, then kLanczos Lanczos steps on A^T A (products A q and A^T y, full
-// re-orthogonalisation by classical Gram-Schmidt) and the largest eigenvalue of
-// the tridiagonal matrix by multisection on its Sturm sequence in fp64 (256
-// points per round, one per thread); M_j is its square root.  (Lanczos: the Ritz values of a Krylov space
-// approach the extreme eigenvalues; Sturm: the number of negative pivots of
-// T - x I counts the eigenvalues below x.)
-// Every wait is a __syncthreads; there is no spin-wait.
+// cov_norm_kernel: per block, A = H_j - Hbar (the same fp32 H_j) as the
+// threads' register tiles, then kLanczos Lanczos steps on A^T A (products A q
+// and A^T y from the tiles; full re-orthogonalisation by classical Gram-Schmidt);
+// writes the tridiagonal matrix T of the steps.  (Lanczos: the Ritz values of a
+// Krylov space approach the extreme eigenvalues.)
+// cov_eig_kernel: per block, the largest eigenvalue of T by multisection on its
+// Sturm sequence in fp64 (the sign changes of the leading minors of T - x I
+// count the eigenvalues below x), one warp per block; M_j is its square root.
+// Every wait is a __syncthreads or __syncwarp; there is no spin-wait.
 #pragma once
 #include "common.cuh"
 
@@ -25,35 +26,109 @@ namespace sla {
 constexpr int kCovTok = 64;       // tokens per KV block
 constexpr int kLanczos = 24;      // Lanczos steps (at most)
 constexpr int kQRows = 28;        // Lanczos vector rows kept: kLanczos + 1, padded to 4 with zeros
+constexpr int kTriStride = 2 * kLanczos + 1;   // fp64 words per block of the tridiagonal output
 
 // Shared layout of one block: ks [64][D] fp32 centred keys, vs [64][D] fp32
-// values, kmean [D] fp64.  Loads block (K, V rows given) and centres the keys.
+// values, kmean [D] fp64, kpart [8][D] fp64 scratch.  Thread t handles the
+// 16-byte chunks (rows t / CPR + c 256 / CPR, columns u * 8 .. u * 8 + 7, u =
+// t % CPR) of the block: it stores their values, sums each key column in fp64
+// (over its rows in order, then over the lanes and the warps that share its
+// columns, in order), and stores the keys centred in fp64, rounded once.  The
+// chunks come from global memory (all loads in flight together) or, kSmem, from
+// a bf16 copy of the block in shared memory that this thread's own cp.async
+// requests filled (cov_fetch_block); either way the arithmetic is the same.
 template <int D>
+__device__ __forceinline__ void cov_fetch_block(const __nv_bfloat16* __restrict__ kblk,
+                                                const __nv_bfloat16* __restrict__ vblk,
+                                                __nv_bfloat16* rk, __nv_bfloat16* rv) {
+    constexpr int CPR = D / 8, CPT = kCovTok * CPR / 256;
+    const int tid = threadIdx.x, u = tid % CPR;
+#pragma unroll 1
+    for (int c = 0; c < CPT; ++c) {
+        const int n = (tid + 256 * c) / CPR;
+        cp_async16(rk + n * D + u * 8, kblk + n * D + u * 8);
+        cp_async16(rv + n * D + u * 8, vblk + n * D + u * 8);
+    }
+    cp_async_commit();
+}
+
+template <int D, bool kSmem>
 __device__ __forceinline__ void cov_load_block(const __nv_bfloat16* __restrict__ kblk,
                                                const __nv_bfloat16* __restrict__ vblk, float* ks,
-                                               float* vs, double* kmean) {
-    const int tid = threadIdx.x;
+                                               float* vs, double* kmean, double* kpart) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     constexpr int CPR = D / 8;                         // 16-byte chunks per row
-    for (int q = tid; q < kCovTok * CPR; q += 256) {
-        const int n = q / CPR, u = q % CPR;
-        const uint4 x = __ldg(reinterpret_cast<const uint4*>(kblk + n * D + u * 8));
-        const uint4 y = __ldg(reinterpret_cast<const uint4*>(vblk + n * D + u * 8));
-        float4* kd = reinterpret_cast<float4*>(ks + n * D + u * 8);
+    constexpr int CPT = kCovTok * CPR / 256;           // chunks per thread
+    const int u = tid % CPR;
+    uint4 xk[CPT], xv[CPT];
+    if constexpr (!kSmem) {
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) {
+            const int n = (tid + 256 * c) / CPR;
+            xk[c] = __ldg(reinterpret_cast<const uint4*>(kblk + n * D + u * 8));
+            xv[c] = __ldg(reinterpret_cast<const uint4*>(vblk + n * D + u * 8));
+        }
+    } else {
+        cp_async_wait<0>();                            // this thread's own copies
+    }
+    auto chunk = [&](const __nv_bfloat16* base, const uint4* held, int c) -> uint4 {
+        if constexpr (kSmem) {
+            const int n = (tid + 256 * c) / CPR;
+            return *reinterpret_cast<const uint4*>(base + n * D + u * 8);
+        } else {
+            return held[c];
+        }
+    };
+    double cs[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) cs[e] = 0.0;
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) {
+        const int n = (tid + 256 * c) / CPR;
+        const uint4 y = chunk(vblk, xv, c);
         float4* vd = reinterpret_cast<float4*>(vs + n * D + u * 8);
-        kd[0] = make_float4(bf16lo(x.x), bf16hi(x.x), bf16lo(x.y), bf16hi(x.y));
-        kd[1] = make_float4(bf16lo(x.z), bf16hi(x.z), bf16lo(x.w), bf16hi(x.w));
         vd[0] = make_float4(bf16lo(y.x), bf16hi(y.x), bf16lo(y.y), bf16hi(y.y));
         vd[1] = make_float4(bf16lo(y.z), bf16hi(y.z), bf16lo(y.w), bf16hi(y.w));
+        const uint4 x = chunk(kblk, xk, c);
+        const uint32_t wk[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            cs[2 * e] += static_cast<double>(bf16lo(wk[e]));
+            cs[2 * e + 1] += static_cast<double>(bf16hi(wk[e]));
+        }
+    }
+#pragma unroll
+    for (int o = CPR; o < 32; o <<= 1)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) cs[e] += __shfl_xor_sync(0xffffffffu, cs[e], o);
+    if (lane < CPR) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) kpart[warp * D + u * 8 + e] = cs[e];
     }
     __syncthreads();
     if (tid < D) {
-        double s = 0.0;
-        for (int n = 0; n < kCovTok; ++n) s += static_cast<double>(ks[n * D + tid]);
-        kmean[tid] = s * (1.0 / kCovTok);
+        double sm = kpart[tid];
+#pragma unroll
+        for (int w = 1; w < 8; ++w) sm += kpart[w * D + tid];
+        kmean[tid] = sm * (1.0 / kCovTok);
     }
     __syncthreads();
-    for (int q = tid; q < kCovTok * D; q += 256)
-        ks[q] = static_cast<float>(static_cast<double>(ks[q]) - kmean[q % D]);
+    const double* mu = kmean + u * 8;
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) {
+        const int n = (tid + 256 * c) / CPR;
+        const uint4 x = chunk(kblk, xk, c);
+        const uint32_t wk[4] = {x.x, x.y, x.z, x.w};
+        float f[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            f[2 * e] = static_cast<float>(static_cast<double>(bf16lo(wk[e])) - mu[2 * e]);
+            f[2 * e + 1] = static_cast<float>(static_cast<double>(bf16hi(wk[e])) - mu[2 * e + 1]);
+        }
+        float4* kd = reinterpret_cast<float4*>(ks + n * D + u * 8);
+        kd[0] = make_float4(f[0], f[1], f[2], f[3]);
+        kd[1] = make_float4(f[4], f[5], f[6], f[7]);
+    }
     __syncthreads();
 }
 
@@ -87,15 +162,19 @@ __device__ __forceinline__ void cov_accumulate(const float* ks, const float* vs,
 }
 
 // grid (nchunk, BH), 256 threads; part [BH][nchunk][D][D] fp32 (empty chunks: zeros).
+// The next block's bf16 copy is in flight (cp.async) while this one accumulates.
 template <int D>
-__global__ void __launch_bounds__(256) cov_hsum_kernel(const __nv_bfloat16* __restrict__ k,
-                                                       const __nv_bfloat16* __restrict__ v, int N,
-                                                       int Nk, int bpc, int nchunk,
-                                                       float* __restrict__ part) {
+__global__ void __launch_bounds__(256, 2) cov_hsum_kernel(const __nv_bfloat16* __restrict__ k,
+                                                          const __nv_bfloat16* __restrict__ v, int N,
+                                                          int Nk, int bpc, int nchunk,
+                                                          float* __restrict__ part) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     float* ks = reinterpret_cast<float*>(smem_raw);
     float* vs = ks + kCovTok * D;
     double* kmean = reinterpret_cast<double*>(vs + kCovTok * D);
+    double* kpart = kmean + D;                         // [8][D]
+    __nv_bfloat16* rk = reinterpret_cast<__nv_bfloat16*>(kpart + 8 * D);   // [64][D] bf16 copies
+    __nv_bfloat16* rv = rk + kCovTok * D;
     constexpr int RT = D / 16;
     const long long bh = blockIdx.y;
     const int chunk = blockIdx.x;
@@ -106,11 +185,13 @@ __global__ void __launch_bounds__(256) cov_hsum_kernel(const __nv_bfloat16* __re
     for (int i = 0; i < RT; ++i)
 #pragma unroll
         for (int j = 0; j < RT; ++j) acc[i][j] = 0.f;
+    auto row0 = [&](int b) { return (bh * N + static_cast<long long>(jb0 + b) * kCovTok) * D; };
+    if (nb > 0) cov_fetch_block<D>(k + row0(0), v + row0(0), rk, rv);
     for (int b = 0; b < nb; ++b) {
-        const long long row0 = (bh * N + static_cast<long long>(jb0 + b) * kCovTok) * D;
-        cov_load_block<D>(k + row0, v + row0, ks, vs, kmean);
+        cov_load_block<D, true>(rk, rv, ks, vs, kmean, kpart);   // (ends with a barrier)
+        if (b + 1 < nb) cov_fetch_block<D>(k + row0(b + 1), v + row0(b + 1), rk, rv);
         cov_accumulate<D>(ks, vs, acc);
-        __syncthreads();                               // before the next block's load
+        __syncthreads();                               // before the next block's stores
     }
     float* dst = part + (bh * nchunk + chunk) * static_cast<long long>(D) * D;
     const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
@@ -195,19 +276,22 @@ __device__ __forceinline__ void cov_half_rows(float (&p)[RT], int lane, float (&
     for (int i = 0; i < RT; ++i) out[i] = __shfl_sync(0xffffffffu, s, (lane & 16) | (i * (16 / RT)));
 }
 
-// grid (Nk, BH), 256 threads.  out[bh * Nk + j] = scale * M_j (fp64).
+// grid (Nk, BH), 256 threads.  tri[(bh * Nk + j) * kTriStride ..]: the Lanczos
+// tridiagonal matrix T of block j -- alpha_0 .. alpha_{m-1}, beta_0 .. beta_{m-2}
+// (beta_{m-1} and the unused entries are zero) and m, all fp64.
 template <int D>
 __global__ void __launch_bounds__(256, 2) cov_norm_kernel(const __nv_bfloat16* __restrict__ k,
                                                           const __nv_bfloat16* __restrict__ v,
                                                           int N, int Nk,
                                                           const float* __restrict__ hbar,
-                                                          double scale, double* __restrict__ out) {
+                                                          double* __restrict__ tri) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     constexpr int RT = D / 16;
     float* ks = reinterpret_cast<float*>(smem_raw);          // [64][D] centred keys
     float* vs = ks + kCovTok * D;                            // [64][D] values
     double* kmean = reinterpret_cast<double*>(vs + kCovTok * D);   // [D]
-    float* qv = reinterpret_cast<float*>(kmean + D);         // Lanczos vectors [kQRows][D]
+    double* kpart = kmean + D;                               // [8][D]
+    float* qv = reinterpret_cast<float*>(kpart + 8 * D);     // Lanczos vectors [kQRows][D]
     float* wv = qv + kQRows * D;                             // [D] w before re-orthogonalisation
     float* wraw = wv + D;                                    // [D] w after it, not yet normalised
     float* part = wraw + D;                                  // [8][D] per-warp sums of A^T y
@@ -225,7 +309,7 @@ __global__ void __launch_bounds__(256, 2) cov_norm_kernel(const __nv_bfloat16* _
     const long long row0 = (bh * N + static_cast<long long>(j) * kCovTok) * D;
 
     // 1. H_j as this thread's RT x RT tile in registers, then A = H_j - Hbar in place
-    cov_load_block<D>(k + row0, v + row0, ks, vs, kmean);
+    cov_load_block<D, false>(k + row0, v + row0, ks, vs, kmean, kpart);
     float a[RT][RT];
 #pragma unroll
     for (int i = 0; i < RT; ++i)
@@ -391,42 +475,72 @@ __global__ void __launch_bounds__(256, 2) cov_norm_kernel(const __nv_bfloat16* _
         b_prev = be;
     }
     __syncthreads();
-    // 3. the largest eigenvalue of T (m x m) by multisection: each round every thread
-    //    counts the eigenvalues of T below its own point x of the interval, as the
-    //    sign changes along p_0 .. p_{m-1}, the leading principal minors of T - x I
-    //    (Sturm sequence; three-term recurrence, no division, T scaled by 1 / hi so
-    //    no term overflows; a zero minor counts as positive, which counts one change
-    //    across it either way since its neighbours then have opposite signs), and
-    //    the interval shrinks to the two points around the largest eigenvalue, 257
-    //    times per round; M_j is the square root of the upper end
-    double hi = 0.0;
-    for (int i = 0; i < m; ++i) {
-        const double g = fabs(alpha[i]) + (i > 0 ? fabs(beta[i - 1]) : 0.0) + (i + 1 < m ? fabs(beta[i]) : 0.0);
-        hi = fmax(hi, g);
+    // 3. T out, for cov_eig_kernel
+    double* t = tri + (bh * Nk + j) * kTriStride;
+    if (tid < kLanczos) {
+        t[tid] = tid < m ? alpha[tid] : 0.0;
+        t[kLanczos + tid] = tid + 1 < m ? beta[tid] : 0.0;
     }
-    const double inv = hi > 0.0 ? 1.0 / hi : 0.0;
-    double lo = 0.0;
-    for (int round = 0; round < 4; ++round) {
-        const double step = (hi - lo) / 257.0;
-        const double x = lo + step * (tid + 1);
-        double pm = 1.0, pc = (alpha[0] - x) * inv;
-        int below = pc < 0.0;
-        for (int i = 1; i < m; ++i) {
-            const double b = beta[i - 1] * inv;
-            const double pn = fma((alpha[i] - x) * inv, pc, -(b * b) * pm);
-            below += (pn < 0.0) != (pc < 0.0);
+    if (tid == 0) t[2 * kLanczos] = static_cast<double>(m);
+}
+
+// The largest eigenvalue of each block's T by multisection, one warp per block:
+// grid ceil(nblk / 8), 256 threads; out[blk] = scale * M_j.  The lanes scale T by
+// 2^-e, the power of two that brings its largest Gershgorin bound g into [1/2, 1)
+// (exact, no division), and pad it to kLanczos rows with decoupled diagonal
+// entries 2 (above every point tried, so they change no count).  Each round every
+// lane counts the eigenvalues of T below its own point x of the interval, as the
+// sign changes along the leading principal minors of T - x I (Sturm sequence;
+// three-term recurrence, no division; a zero minor may take either sign, since
+// its neighbours then have opposite signs and one change is counted across it
+// either way), and the interval shrinks to the two points around the largest
+// eigenvalue, 33 times per round; seven rounds narrow it by 33^7 = 4.3e10.  M_j
+// is the square root of 2^e times the upper end.
+__global__ void __launch_bounds__(256) cov_eig_kernel(const double* __restrict__ tri, long long nblk,
+                                                      double scale, double* __restrict__ out) {
+    __shared__ double sa[8][kLanczos], sb[8][kLanczos];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long blk = static_cast<long long>(blockIdx.x) * 8 + warp;
+    if (blk >= nblk) return;                               // (whole warps; no barrier below)
+    const double* t = tri + blk * kTriStride;
+    const int m = static_cast<int>(t[2 * kLanczos]);
+    const double al = lane < kLanczos ? t[lane] : 0.0;
+    const double be = lane < kLanczos ? t[kLanczos + lane] : 0.0;          // beta_lane (zero from m - 1 on)
+    const double bp = __shfl_up_sync(0xffffffffu, be, 1);                 // beta_{lane-1}
+    double g = lane < m ? fabs(al) + (lane > 0 ? fabs(bp) : 0.0) + fabs(be) : 0.0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) g = fmax(g, __shfl_xor_sync(0xffffffffu, g, o));
+    int e = 0;
+    const double gs = g > 0.0 ? frexp(g, &e) : 0.0;                      // g = gs 2^e, gs in [1/2, 1)
+    if (lane < kLanczos) {
+        const double b = ldexp(be, -e);
+        sa[warp][lane] = lane < m ? ldexp(al, -e) : 2.0;
+        sb[warp][lane] = b * b;
+    }
+    __syncwarp();
+    const double* A = sa[warp];
+    const double* B2 = sb[warp];
+    double lo = 0.0, hi = gs;
+    for (int round = 0; round < 7; ++round) {
+        const double step = (hi - lo) * (1.0 / 33.0);
+        const double x = lo + step * (lane + 1);
+        double pm = 1.0, pc = A[0] - x;
+        int below = __double2hiint(pc) < 0;
+#pragma unroll
+        for (int i = 1; i < kLanczos; ++i) {
+            const double pn = fma(A[i] - x, pc, -B2[i - 1] * pm);
+            below += (__double2hiint(pn) ^ __double2hiint(pc)) < 0;
             pm = pc;
             pc = pn;
         }
         // points below the largest eigenvalue count fewer than m eigenvalues below them
-        const int kb = __syncthreads_count(below < m);
+        const int kb = __popc(__ballot_sync(0xffffffffu, below < m));
         const double nlo = kb > 0 ? lo + step * kb : lo;
-        const double nhi = kb < 256 ? lo + step * (kb + 1) : hi;
+        const double nhi = kb < 32 ? lo + step * (kb + 1) : hi;
         lo = nlo;
         hi = nhi;
-        if (!(hi - lo > 1e-15 * hi)) break;
     }
-    if (tid == 0) out[bh * Nk + j] = scale * sqrt(fmax(hi, 0.0));
+    if (lane == 0) out[blk] = scale * sqrt(fmax(ldexp(hi, e), 0.0));
 }
 
 }  // namespace sla

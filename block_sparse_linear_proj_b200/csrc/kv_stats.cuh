@@ -29,17 +29,6 @@ namespace sla {
 constexpr int kKvTok = 64;     // tokens per KV block (Bk)
 constexpr int kKvStages = 3;
 
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-    asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
 __device__ __forceinline__ uint32_t relu_bf16x2(uint32_t x) {
     __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&x);
     h = __hmax2(h, __floats2bfloat162_rn(0.f, 0.f));

@@ -62,7 +62,7 @@ sla_status_t check_tensor(const void* t, size_t align) {
 struct Ws {
     size_t qbar, kbarT, m, lut, zj, hpart, hsum, zsum, kc, vbar, v16, phik16;
     size_t q8, k8, v8t, sq, sk, sv;       // FP8 sparse branch
-    size_t covpart, covhbar, covbias;     // covariance-aware PISA selection
+    size_t covpart, covhbar, covbias, covtri;   // covariance-aware PISA selection
     size_t total;
     int nchunk, bpc;
 };
@@ -101,6 +101,7 @@ Ws layout(const sla_params_t* p) {
         w.covpart = take(BH * static_cast<size_t>(w.nchunk) * d * d * 4);
         w.covhbar = take(BH * d * d * 4);
         w.covbias = take(BH * Nk * 8);
+        w.covtri = take(BH * Nk * sla::kTriStride * 8);
     }
     w.total = off;
     return w;
@@ -353,9 +354,10 @@ sla_status_t launch_cov_t(const sla_params_t* p, const void* k, const void* v, v
     const auto* vb = static_cast<const __nv_bfloat16*>(v);
     float* part = at<float>(ws, w.covpart);
     float* hbar = at<float>(ws, w.covhbar);
-    const size_t smem_h = 2 * sla::kCovTok * D * 4 + D * 8;
-    const size_t smem_n = 2 * sla::kCovTok * D * 4 + D * 8 + (sla::kQRows * D + 10 * D + 16 + 32) * 4 + 8 +
+    const size_t smem_h = 2 * sla::kCovTok * D * 4 + 9 * D * 8 + 2 * sla::kCovTok * D * 2;
+    const size_t smem_n = 2 * sla::kCovTok * D * 4 + 9 * D * 8 + (sla::kQRows * D + 10 * D + 16 + 32) * 4 + 8 +
                           2 * sla::kLanczos * 8;
+    double* tri = at<double>(ws, w.covtri);
     auto kh = sla::cov_hsum_kernel<D>;
     auto kn = sla::cov_norm_kernel<D>;
     if (cudaFuncSetAttribute(kh, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_h)) != cudaSuccess ||
@@ -371,7 +373,12 @@ sla_status_t launch_cov_t(const sla_params_t* p, const void* k, const void* v, v
     }
     {
         Span sp(SLA_KERNEL_COV, st);
-        kn<<<dim3(Nk, BH), 256, smem_n, st>>>(kb, vb, p->N, Nk, hbar, scale, out);
+        kn<<<dim3(Nk, BH), 256, smem_n, st>>>(kb, vb, p->N, Nk, hbar, tri);
+    }
+    {
+        Span sp(SLA_KERNEL_COV, st);
+        const long long nblk = static_cast<long long>(BH) * Nk;
+        sla::cov_eig_kernel<<<static_cast<unsigned>((nblk + 7) / 8), 256, 0, st>>>(tri, nblk, scale, out);
     }
     return launch_status();
 }
