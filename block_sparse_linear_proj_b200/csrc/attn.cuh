@@ -227,12 +227,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     constexpr int NBOX = D / 64;
     constexpr int KS = L::KS, VS = L::VS;
     // tensor memory columns: S_0 | S_1 | O_0 | O_1 | G_0 (| G_1 when d = 64).
-    // P(e) is written over the first columns of its S buffer (packed fp16 pairs,
-    // or e4m3 quads in FP8 mode).
+    // SLA: P(e) is written over the first columns of its S buffer (packed fp16
+    // pairs, or e4m3 quads in FP8 mode).  PISA (no G): P(e) has buffers of its own,
+    // P_0 | P_1 after O_1, so S(e+2) may overwrite S buffer h as soon as the
+    // softmax has read S(e), while P.V(e) still reads P(e).
     constexpr uint32_t NCOLS = 512;
     constexpr uint32_t COL_O = 128;                   // + h * D
     constexpr uint32_t COL_G0 = 128 + 2 * D;          // + g * D
+    constexpr uint32_t COL_P = 128 + 2 * D;           // PISA: + h * 32
     static_assert(PISA || COL_G0 + L::GRMAX * D <= NCOLS, "tensor memory budget");
+    static_assert(!PISA || COL_P + 64 <= NCOLS, "tensor memory budget");
 
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -249,7 +253,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     uint64_t* s_full = v_empty + VS;              // [2] S(e) in buffer e & 1
     uint64_t* p_full = s_full + 2;                // [2] P(e) written (4 warps)
     uint64_t* pv_done = p_full + 2;               // [2] P.V(e) complete: buffer free, O_{e&1} current
-    uint64_t* final_bar = pv_done + 2;
+    uint64_t* s_free = pv_done + 2;               // [2] PISA: S(e) read by the softmax (4 warps)
+    uint64_t* final_bar = s_free + 2;
     uint64_t* epi_ready = final_bar + 1;
     uint64_t* lin_done = epi_ready + 1;
     uint64_t* drain_bar = lin_done + 1;
@@ -294,6 +299,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             mbar_init(&s_full[b], 1);
             mbar_init(&p_full[b], 4);
             mbar_init(&pv_done[b], 1);
+            mbar_init(&s_free[b], 4);
         }
         mbar_init(final_bar, 1);
         mbar_init(epi_ready, 9);
@@ -502,11 +508,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             constexpr uint32_t ID_S = I8 ? idesc_s8(128, 64) : FP8 ? idesc_e4m3(128, 64) : idesc_bf16(128, 64, 0, 0);
             bool ok = mbar_wait(q_full, 0, abort_flag, lim);
             for (int e = 0; ok && e < n_total; ++e) {
-                // S(e) needs its K tile and its buffer back: P(e-2), written over
-                // S(e-2), has been consumed once P.V(e-2) completed
+                // S(e) needs its K tile and its buffer back: SLA, P(e-2), written over
+                // S(e-2), has been consumed once P.V(e-2) completed; PISA, the softmax
+                // has read S(e-2)
                 const int s = e % KS, b = e & 1;
                 if (!mbar_wait(&k_full[s], (e / KS) & 1, abort_flag, lim) ||
-                    (e >= 2 && !mbar_wait(&pv_done[b], ((e >> 1) - 1) & 1, abort_flag, lim))) { ok = false; break; }
+                    (e >= 2 && !mbar_wait(PISA ? &s_free[b] : &pv_done[b], ((e >> 1) - 1) & 1, abort_flag, lim))) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
                 if (FP8) {
                     // e4m3 (or s8, exact s32 sums): 32 elements (32 bytes) per instruction
@@ -548,8 +558,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 if (!mbar_wait(&v_full[s], (e / VS) & 1, abort_flag, lim) ||
                     !mbar_wait(&p_full[b], u & 1, abort_flag, lim)) { ok = false; break; }
                 tc_fence_after();
-                // O_b += P(e) V_e, P read from the first columns of S buffer b
+                // O_b += P(e) V_e, P read from the first columns of S buffer b (PISA:
+                // from P buffer b)
                 const uint32_t o_col = tmem + COL_O + b * D;
+                const uint32_t p_col = tmem + (PISA ? COL_P + b * 32 : b * 64);
                 if (FP8) {
                     // B = V^T (e4m3, K-major: 64 tokens = 64 bytes per row, 64-byte swizzle)
 #pragma unroll
@@ -561,7 +573,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
                         const uint64_t bd = sdesc(sV(s) + kk * 2048, L::KBOX, 1024, kSwizzle128B);
-                        umma_f16_ts(o_col, tmem + b * 64 + kk * 8, bd, ID_PV, (u > 0 || kk > 0) ? 1u : 0u);
+                        umma_f16_ts(o_col, p_col + kk * 8, bd, ID_PV, (u > 0 || kk > 0) ? 1u : 0u);
                     }
                 }
                 umma_commit(&pv_done[b]);
@@ -716,9 +728,48 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const int u = e >> 1;
             if (!wwait(&s_full[h], u & 1)) { ok = false; break; }
             tc_fence_after();
+            // PISA: P(e) goes to P buffer h once P.V(e-2) has read P(e-2) (and O_h
+            // may be rescaled only then); SLA: S(e) was issued after P.V(e-2)
+            // completed, so both hold already
+            bool pv_ok = !PISA || e < 2;
+            auto wait_pv = [&]() {
+                if (!pv_ok) {
+                    if (!wwait(&pv_done[h], (u - 1) & 1)) return false;
+                    tc_fence_after();
+                    pv_ok = true;
+                }
+                return true;
+            };
+            const uint32_t p_dst = tl + (PISA ? COL_P + h * 32 : h * 64);
+            if (e < n_exact && !__any_sync(0xffffffffu, (sched[e] >> (16 + g)) & 1)) {
+                // no row of this warp selected the block (the other group did): its P
+                // is zero, with nothing to load, exponentiate or rescale
+                if (PISA) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&s_free[h]);
+                }
+                if (!wait_pv()) { ok = false; break; }
+                uint32_t z[16];
+#pragma unroll
+                for (int x = 0; x < 16; ++x) z[x] = 0u;
+                tmem_st16(p_dst, z);
+                if (!FP8) tmem_st16(p_dst + 16, z);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&p_full[h]);
+                continue;
+            }
             tmem_ld32(tl + h * 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
             tmem_ld32(tl + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
             tmem_ld_wait();
+            if (PISA) {
+                // S buffer h is free for S(e+2)
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s_free[h]);
+            }
             if (I8) {
                 // s32 scores, |S| <= 128 * 127^2 < 2^22: exact in fp32
 #pragma unroll
@@ -757,8 +808,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const float m_new = need ? (FP8 ? ceilf(mx) : mx) : m_run;
             const bool rescale_o = need && m_run != -INFINITY;
             if (__any_sync(0xffffffffu, rescale_o)) {
-                // O_h holds P.V of this warpgroup's entries up to e-2, all complete:
-                // S(e) was issued only after P.V(e-2) finished
+                // O_h holds P.V of this warpgroup's entries up to e-2, all complete
+                if (!wait_pv()) { ok = false; break; }
                 const float f = rescale_o ? (FP8 ? exp2_int(m_run - m_new) : fast_exp2(m_run - m_new)) : 1.f;
 #pragma unroll 1
                 for (int cc = 0; cc < D; cc += 32) {
@@ -790,10 +841,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 const bool exact = e < n_exact;
                 ls = exact ? softmax_half<0, true, PISA>(sv, c, m_run, live, pwa)
                            : softmax_half<0, false, PISA>(sv, c, m_run, live, pwa);
-                tmem_st16(tl + h * 64, pwa);
                 ls += exact ? softmax_half<32, true, PISA>(sv, c, m_run, live, pwb)
                             : softmax_half<32, false, PISA>(sv, c, m_run, live, pwb);
-                tmem_st16(tl + h * 64 + 16, pwb);
+                if (!wait_pv()) { ok = false; break; }
+                tmem_st16(p_dst, pwa);
+                tmem_st16(p_dst + 16, pwb);
             }
             tmem_st_wait();
             l_run += ls;
