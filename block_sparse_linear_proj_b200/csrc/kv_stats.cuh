@@ -21,6 +21,12 @@
 // keys) in bf16, and one thread issues the block's four M = 128, K = 16
 // products (bf16 operands, both MN-major) into an fp32 accumulator in tensor
 // memory that sums the CTA's blocks.
+// X3 (the covariance norms' H_j, exactly): the keys are centred in fp64 by the
+// block's column means and rounded once to fp32, as the covariance kernels do,
+// and that fp32 value is split exactly into three bf16 parts (hi, then the
+// rounded remainder, then the rest: 8 + 8 + 8 bits of the 24); each part's
+// product with V is exact in fp32 and the three (twelve K = 16 MMAs) add into
+// the accumulator.  Two ring stages leave room for the two extra parts' tiles.
 #pragma once
 #include "common.cuh"
 
@@ -48,6 +54,15 @@ __device__ __forceinline__ uint32_t kv_off(int n, int c) {
     return static_cast<uint32_t>(n * D * 2 + (((c >> 3) ^ (n & 7)) << 4) + (c & 7) * 2);
 }
 
+// the three bf16 parts of x: hi + mid + lo == x exactly (x fp32; each
+// remainder is exact in fp32 and the last has at most 8 significant bits)
+__device__ __forceinline__ void split3_bf16(float x, float& hi, float& mid, float& lo) {
+    hi = __bfloat162float(__float2bfloat16_rn(x));
+    const float r1 = x - hi;
+    mid = __bfloat162float(__float2bfloat16_rn(r1));
+    lo = __bfloat162float(__float2bfloat16_rn(r1 - mid));
+}
+
 struct KvStatsArgs {
     const __nv_bfloat16* k;     // [BH][N][D]
     const __nv_bfloat16* v;     // [BH][N][D] (may be null when only kbarT is wanted)
@@ -66,7 +81,8 @@ struct KvStatsArgs {
     float* sk;                  // [BH][Nk]
     float* sv;                  // [BH][Nk]
     // PISA first-order term: the product uses K centred by its block mean,
-    // (k_n - kbar_j), instead of phi(K), so hpart sums the blocks' H_j
+    // (k_n - kbar_j), instead of phi(K), so hpart sums the blocks' H_j (in the
+    // X3 kernel exactly, from fp64-centred keys split into three bf16 parts)
     int center;
     // with k8: symmetric 8-bit integer K codes (absmax / 127) instead of e4m3
     int k_int8;
@@ -75,18 +91,22 @@ struct KvStatsArgs {
 
 // grid (nchunk, BH), 256 threads.  TC: the call wants the tensor-core product
 // (hpart non-null); without it the tiles keep a plain swizzled row layout.
-template <int D, bool TC>
+// X3 (with TC and center): the exact three-part product, two ring stages.
+template <int D, bool TC, bool X3 = false>
 __global__ void __launch_bounds__(256, 2) kv_stats_kernel(KvStatsArgs a) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     constexpr int TILE = kKvTok * D * 2;               // bytes of one K or V tile
+    constexpr int kKvStages = X3 ? 2 : ::sla::kKvStages;
     // the swizzled tiles need a 1024-byte aligned base (the launch adds 1024 bytes)
     unsigned char* ring = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    double* kpart = reinterpret_cast<double*>(ring + kKvStages * 2 * TILE);        // [256]
+    unsigned char* xpart = ring + kKvStages * 2 * TILE;                            // X3: [2] tiles
+    double* kpart = reinterpret_cast<double*>(xpart + (X3 ? 2 * TILE : 0));         // [256]
     float* zpart = reinterpret_cast<float*>(kpart + 256);                          // [256]
     float* vpart = zpart + 256;                                                    // [256]
     float* amax = vpart + 256;                                                     // [2][8]
     float* kmf = amax + 16;                                                        // [D] column means
-    uint64_t* mma_bar = reinterpret_cast<uint64_t*>(kmf + 128);                    // product done
+    double* kmd = reinterpret_cast<double*>(kmf + 128);                            // X3: [D] fp64 means
+    uint64_t* mma_bar = reinterpret_cast<uint64_t*>(kmd + (X3 ? D : 0));           // product done
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_bar + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -304,6 +324,7 @@ __global__ void __launch_bounds__(256, 2) kv_stats_kernel(KvStatsArgs a) {
             if (a.kc) a.kc[(bh * a.Nk + j) * D + tid] = __float2bfloat16_rn(static_cast<float>(kmean));
             if (a.vbar) a.vbar[(bh * a.Nk + j) * D + tid] = __float2half_rn(vs * (1.f / kKvTok));
             kmf[tid] = static_cast<float>(kmean);
+            if (X3) kmd[tid] = kmean;
         }
         if (do_mma && a.center) __syncthreads();        // the column means, for the centring
         if (do_mma && !dead) {
@@ -315,7 +336,22 @@ __global__ void __launch_bounds__(256, 2) kv_stats_kernel(KvStatsArgs a) {
                 uint4* px = reinterpret_cast<uint4*>(kt + kv_off<D, TC>(n, u * 8));
                 uint4 x = *px;
                 uint32_t w[4] = {x.x, x.y, x.z, x.w};
-                if (a.center) {
+                if (X3) {
+                    // fp64-centred keys, rounded once to fp32, as three bf16 parts
+                    uint32_t wm[4], wl[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        float h0, m0, l0, h1, m1, l1;
+                        split3_bf16(static_cast<float>(static_cast<double>(bf16lo(w[e])) - kmd[u * 8 + 2 * e]), h0, m0, l0);
+                        split3_bf16(static_cast<float>(static_cast<double>(bf16hi(w[e])) - kmd[u * 8 + 2 * e + 1]), h1, m1, l1);
+                        w[e] = pack_bf16(h0, h1);
+                        wm[e] = pack_bf16(m0, m1);
+                        wl[e] = pack_bf16(l0, l1);
+                    }
+                    const uint32_t off = kv_off<D, TC>(n, u * 8);
+                    *reinterpret_cast<uint4*>(xpart + off) = make_uint4(wm[0], wm[1], wm[2], wm[3]);
+                    *reinterpret_cast<uint4*>(xpart + TILE + off) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+                } else if (a.center) {
                     const float4 m0 = *reinterpret_cast<const float4*>(kmf + u * 8);
                     const float4 m1 = *reinterpret_cast<const float4*>(kmf + u * 8 + 4);
                     w[0] = pack_bf16(bf16lo(w[0]) - m0.x, bf16hi(w[0]) - m0.y);
@@ -333,13 +369,17 @@ __global__ void __launch_bounds__(256, 2) kv_stats_kernel(KvStatsArgs a) {
         __syncthreads();
         if (do_mma && !dead && tid == 0) {
             tc_fence_after();
-            const uint32_t kt_s = smem_u32(kt), vt_s = smem_u32(vt);
+            const uint32_t kt_s = smem_u32(kt), vt_s = smem_u32(vt), xp_s = smem_u32(xpart);
             const uint32_t lbo = D == 128 ? kKvTok * 128 : 0;     // the second 64-feature half
 #pragma unroll
-            for (int kk = 0; kk < kKvTok / 16; ++kk) {
-                const uint64_t ad = sdesc(kt_s + kk * 2048, lbo, 1024, kSwizzle128B);
-                const uint64_t bd = sdesc(vt_s + kk * 2048, kKvTok * 128, 1024, kSwizzle128B);
-                umma_f16_ss(tmem, ad, bd, ID_H, (blk > 0 || kk > 0) ? 1u : 0u);
+            for (int part = 0; part < (X3 ? 3 : 1); ++part) {
+                const uint32_t a_s = part == 0 ? kt_s : xp_s + (part - 1) * TILE;
+#pragma unroll
+                for (int kk = 0; kk < kKvTok / 16; ++kk) {
+                    const uint64_t ad = sdesc(a_s + kk * 2048, lbo, 1024, kSwizzle128B);
+                    const uint64_t bd = sdesc(vt_s + kk * 2048, kKvTok * 128, 1024, kSwizzle128B);
+                    umma_f16_ss(tmem, ad, bd, ID_H, (blk > 0 || part > 0 || kk > 0) ? 1u : 0u);
+                }
             }
             umma_commit(mma_bar);
         }

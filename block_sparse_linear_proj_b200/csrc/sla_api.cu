@@ -346,13 +346,15 @@ sla_status_t router_score(const sla_params_t* p, int32_t* lut, void* ws, const W
 }
 
 // Covariance norms of the PISA selection: out[bh * Nk + j] = scale * M_j.
+// part_ready: the K/V pre-pass has left the chunk sums of H_j in w.hpart (its
+// exact three-part product), so cov_hsum_kernel does not run.
 template <int D>
 sla_status_t launch_cov_t(const sla_params_t* p, const void* k, const void* v, void* ws, const Ws& w,
-                          double scale, double* out, cudaStream_t st) {
+                          double scale, double* out, cudaStream_t st, bool part_ready = false) {
     const int BH = p->B * p->H, Nk = p->N / p->Bk;
     const auto* kb = static_cast<const __nv_bfloat16*>(k);
     const auto* vb = static_cast<const __nv_bfloat16*>(v);
-    float* part = at<float>(ws, w.covpart);
+    float* part = part_ready ? at<float>(ws, w.hpart) : at<float>(ws, w.covpart);
     float* hbar = at<float>(ws, w.covhbar);
     const size_t smem_h = 2 * sla::kCovTok * D * 4 + 9 * D * 8 + 2 * sla::kCovTok * D * 2;
     const size_t smem_n = 2 * sla::kCovTok * D * 4 + 9 * D * 8 + (sla::kQRows * D + 10 * D + 16 + 32) * 4 + 8 +
@@ -363,7 +365,7 @@ sla_status_t launch_cov_t(const sla_params_t* p, const void* k, const void* v, v
     if (cudaFuncSetAttribute(kh, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_h)) != cudaSuccess ||
         cudaFuncSetAttribute(kn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_n)) != cudaSuccess)
         return SLA_ERR_CUDA;
-    {
+    if (!part_ready) {
         Span sp(SLA_KERNEL_COV, st);
         kh<<<dim3(w.nchunk, BH), 256, smem_h, st>>>(kb, vb, p->N, Nk, w.bpc, w.nchunk, part);
     }
@@ -384,9 +386,9 @@ sla_status_t launch_cov_t(const sla_params_t* p, const void* k, const void* v, v
 }
 
 sla_status_t launch_cov(const sla_params_t* p, const void* k, const void* v, void* ws, const Ws& w,
-                        double scale, double* out, cudaStream_t st) {
-    return p->d == 128 ? launch_cov_t<128>(p, k, v, ws, w, scale, out, st)
-                       : launch_cov_t<64>(p, k, v, ws, w, scale, out, st);
+                        double scale, double* out, cudaStream_t st, bool part_ready = false) {
+    return p->d == 128 ? launch_cov_t<128>(p, k, v, ws, w, scale, out, st, part_ready)
+                       : launch_cov_t<64>(p, k, v, ws, w, scale, out, st, part_ready);
 }
 
 sla_status_t run_router(const sla_params_t* p, const void* q, const void* k, const float* w_q,
@@ -399,7 +401,7 @@ template <int D>
 sla_status_t launch_kv(const sla_params_t* p, const void* k, const void* v, void* ws, const Ws& w,
                        bool want_kbar, bool sla_stats, bool pisa_stats, cudaStream_t st,
                        bool fp8 = false, bool first_order = false, cudaEvent_t after_stats = nullptr,
-                       bool k_int8 = false) {
+                       bool k_int8 = false, bool cov_exact = false) {
     const int BH = p->B * p->H, Nk = p->N / p->Bk;
     sla::KvStatsArgs a{};
     a.k = static_cast<const __nv_bfloat16*>(k);
@@ -410,8 +412,10 @@ sla_status_t launch_kv(const sla_params_t* p, const void* k, const void* v, void
     a.nchunk = w.nchunk;
     a.kbarT = want_kbar ? at<double>(ws, w.kbarT) : nullptr;
     a.zj = sla_stats ? at<float>(ws, w.zj) : nullptr;
-    a.hpart = (sla_stats || first_order) ? at<float>(ws, w.hpart) : nullptr;
-    a.center = first_order ? 1 : 0;
+    // cov_exact: the product sums the blocks' H_j exactly (three-part keys), for
+    // the covariance norms and, with first_order, for the first-order term too
+    a.hpart = (sla_stats || first_order || cov_exact) ? at<float>(ws, w.hpart) : nullptr;
+    a.center = (first_order || cov_exact) ? 1 : 0;
     a.kc = pisa_stats ? at<__nv_bfloat16>(ws, w.kc) : nullptr;
     a.vbar = pisa_stats ? at<__half>(ws, w.vbar) : nullptr;
     a.v16 = at<__half>(ws, w.v16);
@@ -424,9 +428,11 @@ sla_status_t launch_kv(const sla_params_t* p, const void* k, const void* v, void
     a.wait_ns = wait_limit_ns();
     // alignment slack, K/V ring, column partials, maxima, column means, barrier,
     // TMEM slot, flag
-    const size_t smem = 1024 + sla::kKvStages * 2 * 64 * D * 2 + 256 * 8 + 2 * 256 * 4 + 16 * 4 +
-                        128 * 4 + 16;
-    auto kern = a.hpart ? sla::kv_stats_kernel<D, true> : sla::kv_stats_kernel<D, false>;
+    // (X3: two ring stages and two more tiles, and the fp64 column means)
+    const size_t smem = 1024 + (cov_exact ? 6 : sla::kKvStages * 2) * 64 * D * 2 + 256 * 8 + 2 * 256 * 4 +
+                        16 * 4 + 128 * 4 + (cov_exact ? D * 8 : 0) + 16;
+    auto kern = cov_exact ? sla::kv_stats_kernel<D, true, true>
+                          : a.hpart ? sla::kv_stats_kernel<D, true> : sla::kv_stats_kernel<D, false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
         return SLA_ERR_CUDA;
@@ -754,17 +760,21 @@ sla_status_t sla_pisa_forward(const sla_params_t* p, const void* q, const void* 
         if (cudaStreamWaitEvent(side->s, side->fork, 0) != cudaSuccess) return SLA_ERR_CUDA;
         sst = side->s;
     }
+    // covariance-aware selection: lambda M_j added to every score of block j; the
+    // pre-pass forms the chunk sums of H_j on its way through K and V
+    const bool cov = compute && p->pisa_cov_lambda > 0.f;
     s = p->d == 128 ? launch_kv<128>(p, k, v, workspace, w, compute, false, true, sst, false, fo,
-                                     side ? side->kbar : nullptr)
+                                     side ? side->kbar : nullptr, false, cov)
                     : launch_kv<64>(p, k, v, workspace, w, compute, false, true, sst, false, fo,
-                                    side ? side->kbar : nullptr);
+                                    side ? side->kbar : nullptr, false, cov);
     if (s != SLA_OK) return s;
     if (side && cudaEventRecord(side->stats, sst) != cudaSuccess) return SLA_ERR_CUDA;
-    // covariance-aware selection: lambda M_j added to every score of block j
-    const bool cov = compute && p->pisa_cov_lambda > 0.f;
     double* bias = cov ? at<double>(workspace, w.covbias) : nullptr;
-    if (cov && (s = launch_cov(p, k, v, workspace, w, static_cast<double>(p->pisa_cov_lambda), bias, st)))
-        return s;
+    if (cov) {
+        if (side && cudaStreamWaitEvent(st, side->kbar, 0) != cudaSuccess) return SLA_ERR_CUDA;
+        if ((s = launch_cov(p, k, v, workspace, w, static_cast<double>(p->pisa_cov_lambda), bias, st, true)))
+            return s;
+    }
     if (compute && (s = router_score(p, lut_use, workspace, w, st, side ? side->kbar : nullptr, bias)))
         return s;
     if (side && cudaStreamWaitEvent(st, side->stats, 0) != cudaSuccess) return SLA_ERR_CUDA;
