@@ -5,21 +5,24 @@
 //   H_j = sum_{n in j} (k_n - kbar_j)^T v_n,   Hbar = (1/Nk) sum_j H_j,
 // and ||.||_2 is the largest singular value.
 //
-// cov_hsum_kernel: per chunk of blocks, the sum of their H_j (fp32).  The keys
-// are centred in fp64 and rounded once to fp32, so every product with a bf16
-// value is exact in fp32 and only the 64-term sums round.
+// The chunk sums of the H_j come from the K/V pre-pass (kv_stats_kernel, its
+// exact mode): keys centred in fp64 by the block's column means, rounded once to
+// fp32 and split exactly into three bf16 parts, so every product with a bf16
+// value is exact in fp32; the tensor core accumulates them in fp32.
 // cov_hbar_kernel: Hbar, the chunk sums added in order in fp64.
-// cov_norm_kernel: per block, A = H_j - Hbar (the same fp32 H_j) as the
-// threads' register tiles, then kLanczos Lanczos steps on A^T A (products A q
-// and A^T y from the tiles; full re-orthogonalisation by classical Gram-Schmidt);
-// writes the tridiagonal matrix T of the steps.  (Lanczos: the Ritz values of a
-// Krylov space approach the extreme eigenvalues.)
+// cov_norm_kernel: per block, H_j again on the tensor core (the same centring,
+// split and products), A = H_j - Hbar as the threads' register tiles, then
+// kLanczos Lanczos steps on A^T A (products A q and A^T y from the tiles; full
+// re-orthogonalisation by classical Gram-Schmidt); writes the tridiagonal matrix
+// T of the steps.  (Lanczos: the Ritz values of a Krylov space approach the
+// extreme eigenvalues.)
 // cov_eig_kernel: per block, the largest eigenvalue of T by multisection on its
 // Sturm sequence in fp64 (the sign changes of the leading minors of T - x I
 // count the eigenvalues below x), one warp per block; M_j is its square root.
-// Every wait is a __syncthreads or __syncwarp; there is no spin-wait.
+// Every wait is a __syncthreads, a __syncwarp or the bounded wait on the product.
 #pragma once
 #include "common.cuh"
+#include "kv_stats.cuh"
 
 namespace sla {
 
@@ -28,180 +31,11 @@ constexpr int kLanczos = 24;      // Lanczos steps (at most)
 constexpr int kQRows = 28;        // Lanczos vector rows kept: kLanczos + 1, padded to 4 with zeros
 constexpr int kTriStride = 2 * kLanczos + 1;   // fp64 words per block of the tridiagonal output
 
-// Shared layout of one block: ks [64][D] fp32 centred keys, vs [64][D] fp32
-// values, kmean [D] fp64, kpart [8][D] fp64 scratch.  Thread t handles the
-// 16-byte chunks (rows t / CPR + c 256 / CPR, columns u * 8 .. u * 8 + 7, u =
-// t % CPR) of the block: it stores their values, sums each key column in fp64
-// (over its rows in order, then over the lanes and the warps that share its
-// columns, in order), and stores the keys centred in fp64, rounded once.  The
-// chunks come from global memory (all loads in flight together) or, kSmem, from
-// a bf16 copy of the block in shared memory that this thread's own cp.async
-// requests filled (cov_fetch_block); either way the arithmetic is the same.
-template <int D>
-__device__ __forceinline__ void cov_fetch_block(const __nv_bfloat16* __restrict__ kblk,
-                                                const __nv_bfloat16* __restrict__ vblk,
-                                                __nv_bfloat16* rk, __nv_bfloat16* rv) {
-    constexpr int CPR = D / 8, CPT = kCovTok * CPR / 256;
-    const int tid = threadIdx.x, u = tid % CPR;
-#pragma unroll 1
-    for (int c = 0; c < CPT; ++c) {
-        const int n = (tid + 256 * c) / CPR;
-        cp_async16(rk + n * D + u * 8, kblk + n * D + u * 8);
-        cp_async16(rv + n * D + u * 8, vblk + n * D + u * 8);
-    }
-    cp_async_commit();
-}
-
-template <int D, bool kSmem>
-__device__ __forceinline__ void cov_load_block(const __nv_bfloat16* __restrict__ kblk,
-                                               const __nv_bfloat16* __restrict__ vblk, float* ks,
-                                               float* vs, double* kmean, double* kpart) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    constexpr int CPR = D / 8;                         // 16-byte chunks per row
-    constexpr int CPT = kCovTok * CPR / 256;           // chunks per thread
-    const int u = tid % CPR;
-    uint4 xk[CPT], xv[CPT];
-    if constexpr (!kSmem) {
-#pragma unroll
-        for (int c = 0; c < CPT; ++c) {
-            const int n = (tid + 256 * c) / CPR;
-            xk[c] = __ldg(reinterpret_cast<const uint4*>(kblk + n * D + u * 8));
-            xv[c] = __ldg(reinterpret_cast<const uint4*>(vblk + n * D + u * 8));
-        }
-    } else {
-        cp_async_wait<0>();                            // this thread's own copies
-    }
-    auto chunk = [&](const __nv_bfloat16* base, const uint4* held, int c) -> uint4 {
-        if constexpr (kSmem) {
-            const int n = (tid + 256 * c) / CPR;
-            return *reinterpret_cast<const uint4*>(base + n * D + u * 8);
-        } else {
-            return held[c];
-        }
-    };
-    double cs[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) cs[e] = 0.0;
-#pragma unroll
-    for (int c = 0; c < CPT; ++c) {
-        const int n = (tid + 256 * c) / CPR;
-        const uint4 y = chunk(vblk, xv, c);
-        float4* vd = reinterpret_cast<float4*>(vs + n * D + u * 8);
-        vd[0] = make_float4(bf16lo(y.x), bf16hi(y.x), bf16lo(y.y), bf16hi(y.y));
-        vd[1] = make_float4(bf16lo(y.z), bf16hi(y.z), bf16lo(y.w), bf16hi(y.w));
-        const uint4 x = chunk(kblk, xk, c);
-        const uint32_t wk[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            cs[2 * e] += static_cast<double>(bf16lo(wk[e]));
-            cs[2 * e + 1] += static_cast<double>(bf16hi(wk[e]));
-        }
-    }
-#pragma unroll
-    for (int o = CPR; o < 32; o <<= 1)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) cs[e] += __shfl_xor_sync(0xffffffffu, cs[e], o);
-    if (lane < CPR) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) kpart[warp * D + u * 8 + e] = cs[e];
-    }
-    __syncthreads();
-    if (tid < D) {
-        double sm = kpart[tid];
-#pragma unroll
-        for (int w = 1; w < 8; ++w) sm += kpart[w * D + tid];
-        kmean[tid] = sm * (1.0 / kCovTok);
-    }
-    __syncthreads();
-    const double* mu = kmean + u * 8;
-#pragma unroll
-    for (int c = 0; c < CPT; ++c) {
-        const int n = (tid + 256 * c) / CPR;
-        const uint4 x = chunk(kblk, xk, c);
-        const uint32_t wk[4] = {x.x, x.y, x.z, x.w};
-        float f[8];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            f[2 * e] = static_cast<float>(static_cast<double>(bf16lo(wk[e])) - mu[2 * e]);
-            f[2 * e + 1] = static_cast<float>(static_cast<double>(bf16hi(wk[e])) - mu[2 * e + 1]);
-        }
-        float4* kd = reinterpret_cast<float4*>(ks + n * D + u * 8);
-        kd[0] = make_float4(f[0], f[1], f[2], f[3]);
-        kd[1] = make_float4(f[4], f[5], f[6], f[7]);
-    }
-    __syncthreads();
-}
-
 // Tile layout of a D x D matrix over 256 threads: thread (ty, tx) = (tid / 16,
 // tid % 16) owns rows cov_idx(ty, i) and columns cov_idx(tx, jj), i, jj < RT =
 // D / 16, where cov_idx(t, i) = 64 (i / 4) + 4 t + i % 4 -- runs of four, 64
 // apart, so that a half-warp's 16-byte reads of a row cover 256 contiguous bytes.
 __device__ __forceinline__ int cov_idx(int t, int i) { return (i >> 2) * 64 + t * 4 + (i & 3); }
-
-// acc[i][jj] += sum_n ks[n][cov_idx(ty, i)] vs[n][cov_idx(tx, jj)], n in order.
-template <int D>
-__device__ __forceinline__ void cov_accumulate(const float* ks, const float* vs,
-                                               float (&acc)[D / 16][D / 16]) {
-    constexpr int RT = D / 16;
-    const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
-#pragma unroll 4
-    for (int n = 0; n < kCovTok; ++n) {
-        float a[RT], b[RT];
-#pragma unroll
-        for (int i = 0; i < RT; i += 4) {
-            const float4 x = *reinterpret_cast<const float4*>(ks + n * D + cov_idx(ty, i));
-            const float4 y = *reinterpret_cast<const float4*>(vs + n * D + cov_idx(tx, i));
-            a[i] = x.x; a[i + 1] = x.y; a[i + 2] = x.z; a[i + 3] = x.w;
-            b[i] = y.x; b[i + 1] = y.y; b[i + 2] = y.z; b[i + 3] = y.w;
-        }
-#pragma unroll
-        for (int i = 0; i < RT; ++i)
-#pragma unroll
-            for (int j = 0; j < RT; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
-    }
-}
-
-// grid (nchunk, BH), 256 threads; part [BH][nchunk][D][D] fp32 (empty chunks: zeros).
-// The next block's bf16 copy is in flight (cp.async) while this one accumulates.
-template <int D>
-__global__ void __launch_bounds__(256, 2) cov_hsum_kernel(const __nv_bfloat16* __restrict__ k,
-                                                          const __nv_bfloat16* __restrict__ v, int N,
-                                                          int Nk, int bpc, int nchunk,
-                                                          float* __restrict__ part) {
-    extern __shared__ __align__(1024) unsigned char smem_raw[];
-    float* ks = reinterpret_cast<float*>(smem_raw);
-    float* vs = ks + kCovTok * D;
-    double* kmean = reinterpret_cast<double*>(vs + kCovTok * D);
-    double* kpart = kmean + D;                         // [8][D]
-    __nv_bfloat16* rk = reinterpret_cast<__nv_bfloat16*>(kpart + 8 * D);   // [64][D] bf16 copies
-    __nv_bfloat16* rv = rk + kCovTok * D;
-    constexpr int RT = D / 16;
-    const long long bh = blockIdx.y;
-    const int chunk = blockIdx.x;
-    const int jb0 = chunk * bpc;
-    const int nb = min(bpc, Nk - jb0);
-    float acc[RT][RT];
-#pragma unroll
-    for (int i = 0; i < RT; ++i)
-#pragma unroll
-        for (int j = 0; j < RT; ++j) acc[i][j] = 0.f;
-    auto row0 = [&](int b) { return (bh * N + static_cast<long long>(jb0 + b) * kCovTok) * D; };
-    if (nb > 0) cov_fetch_block<D>(k + row0(0), v + row0(0), rk, rv);
-    for (int b = 0; b < nb; ++b) {
-        cov_load_block<D, true>(rk, rv, ks, vs, kmean, kpart);   // (ends with a barrier)
-        if (b + 1 < nb) cov_fetch_block<D>(k + row0(b + 1), v + row0(b + 1), rk, rv);
-        cov_accumulate<D>(ks, vs, acc);
-        __syncthreads();                               // before the next block's stores
-    }
-    float* dst = part + (bh * nchunk + chunk) * static_cast<long long>(D) * D;
-    const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
-#pragma unroll
-    for (int i = 0; i < RT; ++i)
-#pragma unroll
-        for (int j = 0; j < RT; j += 4)
-            *reinterpret_cast<float4*>(dst + cov_idx(ty, i) * D + cov_idx(tx, j)) =
-                make_float4(acc[i][j], acc[i][j + 1], acc[i][j + 2], acc[i][j + 3]);
-}
 
 // grid (D*D/256, BH), 256 threads: hbar[bh] = (sum over chunks of part) / Nk.
 template <int D>
@@ -279,17 +113,33 @@ __device__ __forceinline__ void cov_half_rows(float (&p)[RT], int lane, float (&
 // grid (Nk, BH), 256 threads.  tri[(bh * Nk + j) * kTriStride ..]: the Lanczos
 // tridiagonal matrix T of block j -- alpha_0 .. alpha_{m-1}, beta_0 .. beta_{m-2}
 // (beta_{m-1} and the unused entries are zero) and m, all fp64.
+// H_j runs on tcgen05: the block's K and V rows land (cp.async) in the operand
+// layout of the K/V pre-pass (64-column halves, 128-byte swizzle), the keys are
+// centred by fp64 column means, rounded once to fp32 and split exactly into three
+// bf16 parts (split3_bf16), and one thread issues the twelve M = 128, K = 16
+// products of the parts with V into a D-column fp32 accumulator in tensor memory.
+// The accumulator passes through shared memory (rows of 16-byte chunks XOR-
+// swizzled by the row) into each thread's register tile.  The product waits on
+// one mbarrier, bounded (wait_ns): on expiry the status word is set and the block
+// continues on a zero matrix.
 template <int D>
 __global__ void __launch_bounds__(256, 2) cov_norm_kernel(const __nv_bfloat16* __restrict__ k,
                                                           const __nv_bfloat16* __restrict__ v,
                                                           int N, int Nk,
                                                           const float* __restrict__ hbar,
-                                                          double* __restrict__ tri) {
+                                                          double* __restrict__ tri,
+                                                          unsigned long long wait_ns) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     constexpr int RT = D / 16;
-    float* ks = reinterpret_cast<float*>(smem_raw);          // [64][D] centred keys
-    float* vs = ks + kCovTok * D;                            // [64][D] values
-    double* kmean = reinterpret_cast<double*>(vs + kCovTok * D);   // [D]
+    constexpr int TILE = kCovTok * D * 2;                    // one bf16 operand tile
+    // the swizzled tiles need a 1024-byte aligned base (the launch adds 1024 bytes)
+    unsigned char* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    unsigned char* tK = base;                                // K, then the parts' hi
+    unsigned char* tV = base + TILE;                         // V (the B operand)
+    unsigned char* tM = base + 2 * TILE;                     // mid parts
+    unsigned char* tL = base + 3 * TILE;                     // lo parts
+    float* hs = reinterpret_cast<float*>(base);              // then H_j [D][D], after the product
+    double* kmean = reinterpret_cast<double*>(base + 4 * TILE);   // [D]
     double* kpart = kmean + D;                               // [8][D]
     float* qv = reinterpret_cast<float*>(kpart + 8 * D);     // Lanczos vectors [kQRows][D]
     float* wv = qv + kQRows * D;                             // [D] w before re-orthogonalisation
@@ -300,6 +150,9 @@ __global__ void __launch_bounds__(256, 2) cov_norm_kernel(const __nv_bfloat16* _
     double* alpha = reinterpret_cast<double*>(
         (reinterpret_cast<uintptr_t>(coef + 32) + 7) & ~static_cast<uintptr_t>(7));  // [kLanczos]
     double* beta = alpha + kLanczos;                                  // [kLanczos]
+    uint64_t* mma_bar = reinterpret_cast<uint64_t*>(beta + kLanczos);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_bar + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -308,26 +161,135 @@ __global__ void __launch_bounds__(256, 2) cov_norm_kernel(const __nv_bfloat16* _
     const int j = blockIdx.x;
     const long long row0 = (bh * N + static_cast<long long>(j) * kCovTok) * D;
 
-    // 1. H_j as this thread's RT x RT tile in registers, then A = H_j - Hbar in place
-    cov_load_block<D, false>(k + row0, v + row0, ks, vs, kmean, kpart);
+    // 1. H_j on the tensor core, then A = H_j - Hbar as this thread's RT x RT tile
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, D);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        mbar_init(mma_bar, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    {
+        constexpr int CPR = D / 8;                           // 16-byte chunks per row
+        for (int q = tid; q < kCovTok * CPR; q += 256) {
+            const int n = q / CPR, u = q % CPR;
+            const uint32_t off = kv_off<D, true>(n, u * 8);
+            cp_async16(tK + off, k + row0 + n * D + u * 8);
+            cp_async16(tV + off, v + row0 + n * D + u * 8);
+        }
+        cp_async_commit();
+        cp_async_wait<0>();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    {                                                         // fp64 column means of the keys
+        constexpr int HALVES = 256 / D, RPH = kCovTok / HALVES;
+        const int col = tid % D, hf = tid / D;
+        double sm = 0.0;
+        for (int n = hf * RPH; n < (hf + 1) * RPH; ++n)
+            sm += static_cast<double>(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(tK + kv_off<D, true>(n, col))));
+        kpart[tid] = sm;
+        __syncthreads();
+        if (tid < D) {
+            double t = kpart[tid];
+#pragma unroll
+            for (int h = 1; h < HALVES; ++h) t += kpart[h * D + tid];
+            kmean[tid] = t * (1.0 / kCovTok);
+        }
+        __syncthreads();
+    }
+    {                                                         // the keys' three bf16 parts
+        constexpr int CPR = D / 8;
+        for (int q = tid; q < kCovTok * CPR; q += 256) {
+            const int n = q / CPR, u = q % CPR;
+            const uint32_t off = kv_off<D, true>(n, u * 8);
+            const uint4 x = *reinterpret_cast<const uint4*>(tK + off);
+            const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+            uint32_t wh[4], wm[4], wl[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                float h0, m0, l0, h1, m1, l1;
+                split3_bf16(static_cast<float>(static_cast<double>(bf16lo(w[e])) - kmean[u * 8 + 2 * e]), h0, m0, l0);
+                split3_bf16(static_cast<float>(static_cast<double>(bf16hi(w[e])) - kmean[u * 8 + 2 * e + 1]), h1, m1, l1);
+                wh[e] = pack_bf16(h0, h1);
+                wm[e] = pack_bf16(m0, m1);
+                wl[e] = pack_bf16(l0, l1);
+            }
+            *reinterpret_cast<uint4*>(tK + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+            *reinterpret_cast<uint4*>(tM + off) = make_uint4(wm[0], wm[1], wm[2], wm[3]);
+            *reinterpret_cast<uint4*>(tL + off) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+        }
+        fence_proxy_async_smem();
+    }
+    __syncthreads();
+    if (tid == 0) {
+        tc_fence_after();
+        constexpr uint32_t ID_H = idesc_bf16(128, D, 1, 1);
+        const uint32_t lbo = D == 128 ? kCovTok * 128 : 0;   // the second 64-feature half (D = 64: rows repeat)
+        const uint32_t vt_s = smem_u32(tV);
+#pragma unroll
+        for (int p3 = 0; p3 < 3; ++p3) {
+            const uint32_t a_s = smem_u32(p3 == 0 ? tK : p3 == 1 ? tM : tL);
+#pragma unroll
+            for (int kk = 0; kk < kCovTok / 16; ++kk) {
+                const uint64_t ad = sdesc(a_s + kk * 2048, lbo, 1024, kSwizzle128B);
+                const uint64_t bd = sdesc(vt_s + kk * 2048, kCovTok * 128, 1024, kSwizzle128B);
+                umma_f16_ss(tmem, ad, bd, ID_H, (p3 > 0 || kk > 0) ? 1u : 0u);
+            }
+        }
+        umma_commit(mma_bar);
+        if (!mbar_wait(mma_bar, 0, abort_flag, wait_ns)) {
+            report(kStatusTimeout);
+            *abort_flag = 1;
+        }
+    }
+    __syncthreads();
+    tc_fence_after();
+    const bool dead = *abort_flag != 0;
+    constexpr int C4 = D / 4;                                // 16-byte chunks per row of H_j
+    if (!dead && 32 * (warp & 3) < D) {
+        // warp w: rows 32 (w % 4) + lane (its tensor-memory lanes), columns of half w / 4
+        const int r = 32 * (warp & 3) + lane;
+        const uint32_t tl = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
+#pragma unroll 1
+        for (int cc = (warp >> 2) * (D / 2); cc < (warp >> 2) * (D / 2) + D / 2; cc += 32) {
+            uint32_t vv[32];
+            tmem_ld32(tl + cc, vv);
+            tmem_ld_wait();
+#pragma unroll
+            for (int x = 0; x < 32; x += 4) {
+                const int c4 = ((cc + x) >> 2) ^ (r & (C4 - 1));
+                *reinterpret_cast<float4*>(hs + r * D + c4 * 4) =
+                    make_float4(__uint_as_float(vv[x]), __uint_as_float(vv[x + 1]), __uint_as_float(vv[x + 2]),
+                                __uint_as_float(vv[x + 3]));
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, D);
     float a[RT][RT];
-#pragma unroll
-    for (int i = 0; i < RT; ++i)
-#pragma unroll
-        for (int jj = 0; jj < RT; ++jj) a[i][jj] = 0.f;
-    cov_accumulate<D>(ks, vs, a);
     {
         const float* hb = hbar + bh * D * D;
 #pragma unroll
-        for (int i = 0; i < RT; ++i)
+        for (int i = 0; i < RT; ++i) {
+            const int r = cov_idx(ty, i);
 #pragma unroll
             for (int jj = 0; jj < RT; jj += 4) {
-                const float4 h = __ldg(reinterpret_cast<const float4*>(hb + cov_idx(ty, i) * D + cov_idx(tx, jj)));
-                a[i][jj] -= h.x;
-                a[i][jj + 1] -= h.y;
-                a[i][jj + 2] -= h.z;
-                a[i][jj + 3] -= h.w;
+                const int c = cov_idx(tx, jj);
+                const float4 h = __ldg(reinterpret_cast<const float4*>(hb + r * D + c));
+                const float4 x = dead ? make_float4(h.x, h.y, h.z, h.w)
+                                      : *reinterpret_cast<const float4*>(hs + r * D + (((c >> 2) ^ (r & (C4 - 1))) << 2));
+                a[i][jj] = x.x - h.x;
+                a[i][jj + 1] = x.y - h.y;
+                a[i][jj + 2] = x.z - h.z;
+                a[i][jj + 3] = x.w - h.w;
             }
+        }
     }
     // 2. Lanczos on B = A^T A from q_0 proportional to (1 + t / D).  Thread t < D owns
     //    element t of the vectors (q_it and q_{it-1} in registers).  A q: each thread

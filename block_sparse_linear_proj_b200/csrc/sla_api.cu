@@ -62,7 +62,7 @@ sla_status_t check_tensor(const void* t, size_t align) {
 struct Ws {
     size_t qbar, kbarT, m, lut, zj, hpart, hsum, zsum, kc, vbar, v16, phik16;
     size_t q8, k8, v8t, sq, sk, sv;       // FP8 sparse branch
-    size_t covpart, covhbar, covbias, covtri;   // covariance-aware PISA selection
+    size_t covhbar, covbias, covtri;   // covariance-aware PISA selection (chunk sums: hpart)
     size_t total;
     int nchunk, bpc;
 };
@@ -98,7 +98,6 @@ Ws layout(const sla_params_t* p) {
         w.sv = take(BH * Nk * 4);
     }
     if (p->pisa_cov_lambda > 0.f) {               // chunk sums of H_j, Hbar, lambda M_j
-        w.covpart = take(BH * static_cast<size_t>(w.nchunk) * d * d * 4);
         w.covhbar = take(BH * d * d * 4);
         w.covbias = take(BH * Nk * 8);
         w.covtri = take(BH * Nk * sla::kTriStride * 8);
@@ -346,36 +345,31 @@ sla_status_t router_score(const sla_params_t* p, int32_t* lut, void* ws, const W
 }
 
 // Covariance norms of the PISA selection: out[bh * Nk + j] = scale * M_j.
-// part_ready: the K/V pre-pass has left the chunk sums of H_j in w.hpart (its
-// exact three-part product), so cov_hsum_kernel does not run.
+// The K/V pre-pass has left the chunk sums of H_j in w.hpart (its exact
+// three-part product, kv_stats_kernel<D, true, true>).
 template <int D>
 sla_status_t launch_cov_t(const sla_params_t* p, const void* k, const void* v, void* ws, const Ws& w,
-                          double scale, double* out, cudaStream_t st, bool part_ready = false) {
+                          double scale, double* out, cudaStream_t st) {
     const int BH = p->B * p->H, Nk = p->N / p->Bk;
     const auto* kb = static_cast<const __nv_bfloat16*>(k);
     const auto* vb = static_cast<const __nv_bfloat16*>(v);
-    float* part = part_ready ? at<float>(ws, w.hpart) : at<float>(ws, w.covpart);
+    float* part = at<float>(ws, w.hpart);
     float* hbar = at<float>(ws, w.covhbar);
-    const size_t smem_h = 2 * sla::kCovTok * D * 4 + 9 * D * 8 + 2 * sla::kCovTok * D * 2;
-    const size_t smem_n = 2 * sla::kCovTok * D * 4 + 9 * D * 8 + (sla::kQRows * D + 10 * D + 16 + 32) * 4 + 8 +
-                          2 * sla::kLanczos * 8;
+    // (alignment slack; the four operand tiles, later H_j, take the first 2 * 64 * D * 4 bytes;
+    // barrier, TMEM slot and flag after the tridiagonal matrix)
+    const size_t smem_n = 1024 + 2 * sla::kCovTok * D * 4 + 9 * D * 8 +
+                          (sla::kQRows * D + 10 * D + 16 + 32) * 4 + 8 + 2 * sla::kLanczos * 8 + 16;
     double* tri = at<double>(ws, w.covtri);
-    auto kh = sla::cov_hsum_kernel<D>;
     auto kn = sla::cov_norm_kernel<D>;
-    if (cudaFuncSetAttribute(kh, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_h)) != cudaSuccess ||
-        cudaFuncSetAttribute(kn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_n)) != cudaSuccess)
+    if (cudaFuncSetAttribute(kn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_n)) != cudaSuccess)
         return SLA_ERR_CUDA;
-    if (!part_ready) {
-        Span sp(SLA_KERNEL_COV, st);
-        kh<<<dim3(w.nchunk, BH), 256, smem_h, st>>>(kb, vb, p->N, Nk, w.bpc, w.nchunk, part);
-    }
     {
         Span sp(SLA_KERNEL_COV, st);
         sla::cov_hbar_kernel<D><<<dim3(D * D / 256, BH), 256, 0, st>>>(part, w.nchunk, Nk, hbar);
     }
     {
         Span sp(SLA_KERNEL_COV, st);
-        kn<<<dim3(Nk, BH), 256, smem_n, st>>>(kb, vb, p->N, Nk, hbar, tri);
+        kn<<<dim3(Nk, BH), 256, smem_n, st>>>(kb, vb, p->N, Nk, hbar, tri, wait_limit_ns());
     }
     {
         Span sp(SLA_KERNEL_COV, st);
@@ -386,9 +380,9 @@ sla_status_t launch_cov_t(const sla_params_t* p, const void* k, const void* v, v
 }
 
 sla_status_t launch_cov(const sla_params_t* p, const void* k, const void* v, void* ws, const Ws& w,
-                        double scale, double* out, cudaStream_t st, bool part_ready = false) {
-    return p->d == 128 ? launch_cov_t<128>(p, k, v, ws, w, scale, out, st, part_ready)
-                       : launch_cov_t<64>(p, k, v, ws, w, scale, out, st, part_ready);
+                        double scale, double* out, cudaStream_t st) {
+    return p->d == 128 ? launch_cov_t<128>(p, k, v, ws, w, scale, out, st)
+                       : launch_cov_t<64>(p, k, v, ws, w, scale, out, st);
 }
 
 sla_status_t run_router(const sla_params_t* p, const void* q, const void* k, const float* w_q,
@@ -418,7 +412,9 @@ sla_status_t launch_kv(const sla_params_t* p, const void* k, const void* v, void
     a.center = (first_order || cov_exact) ? 1 : 0;
     a.kc = pisa_stats ? at<__nv_bfloat16>(ws, w.kc) : nullptr;
     a.vbar = pisa_stats ? at<__half>(ws, w.vbar) : nullptr;
-    a.v16 = at<__half>(ws, w.v16);
+    // (the forward's fp16 V copy; a call that only wants the covariance sums makes none)
+    const bool cov_only = cov_exact && !want_kbar && !sla_stats && !pisa_stats && !first_order;
+    a.v16 = cov_only ? nullptr : at<__half>(ws, w.v16);
     a.phik16 = sla_stats ? at<__half>(ws, w.phik16) : nullptr;
     a.k8 = fp8 ? at<uint8_t>(ws, w.k8) : nullptr;
     a.v8t = fp8 ? at<uint8_t>(ws, w.v8t) : nullptr;
@@ -772,7 +768,7 @@ sla_status_t sla_pisa_forward(const sla_params_t* p, const void* q, const void* 
     double* bias = cov ? at<double>(workspace, w.covbias) : nullptr;
     if (cov) {
         if (side && cudaStreamWaitEvent(st, side->kbar, 0) != cudaSuccess) return SLA_ERR_CUDA;
-        if ((s = launch_cov(p, k, v, workspace, w, static_cast<double>(p->pisa_cov_lambda), bias, st, true)))
+        if ((s = launch_cov(p, k, v, workspace, w, static_cast<double>(p->pisa_cov_lambda), bias, st)))
             return s;
     }
     if (compute && (s = router_score(p, lut_use, workspace, w, st, side ? side->kbar : nullptr, bias)))
@@ -794,6 +790,12 @@ sla_status_t sla_pisa_cov_norms(const sla_params_t* p, const void* k, const void
     Ws w;
     if ((s = check_ws(p, workspace, ws_bytes, w))) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // the chunk sums of H_j from the K/V pre-pass's exact product, then the norms
+    s = p->d == 128 ? launch_kv<128>(p, k, v, workspace, w, false, false, false, st, false, false, nullptr,
+                                     false, true)
+                    : launch_kv<64>(p, k, v, workspace, w, false, false, false, st, false, false, nullptr,
+                                    false, true);
+    if (s != SLA_OK) return s;
     return finish(launch_cov(p, k, v, workspace, w, 1.0, norms, st), st);
 }
 

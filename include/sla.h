@@ -201,9 +201,10 @@ sla_status_t sla_pisa_forward(const sla_params_t *p, const void *q, const void *
 /*
  * sla_pisa_cov_norms -- the block covariance norms of the covariance-aware
  * selection: norms[(b*H + h)*Nk + j] = M_j = || H_j - Hbar ||_2 in fp64
- * (unscaled), j < Nk = N/Bk.  H_j and Hbar are fp32 sums of exact products
- * (keys centred in fp64, rounded once); the largest singular value comes from
- * 24 Lanczos steps on (H_j - Hbar)^T (H_j - Hbar) (relative error ~1e-7).
+ * (unscaled), j < Nk = N/Bk.  H_j and Hbar are fp32 tensor-core sums of exact
+ * products (keys centred in fp64, rounded once to fp32 and split exactly into
+ * three bf16 parts); the largest singular value comes from 24 Lanczos steps on
+ * (H_j - Hbar)^T (H_j - Hbar) (relative error a few 1e-7).
  * k, v: device bf16 [B,H,N,d]; norms: device fp64, B*H*Nk entries, 8-byte
  * aligned, owned by the caller.  Requires Bk = 64 and p->pisa_cov_lambda > 0
  * (the workspace then holds the norms' scratch); errors as sla_pisa_forward.
