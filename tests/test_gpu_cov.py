@@ -1,9 +1,9 @@
 """PISA covariance-aware selection on the GPU: the block norms
 M_j = ||H_j - Hbar||_2 against the oracle (numpy SVD in fp64), and the LUT of
 a covariance-aware sla_pisa_forward against the oracle's routing with the
-bias lambda M_j.  GPU norms carry a relative error of order 1e-7 (fp32 sums of
-exact products, fp32 Lanczos), so LUT rows whose k-th and (k+1)-th biased
-scores lie closer than 1e-5 + 4e-6 lambda max M may differ."""
+bias lambda M_j.  GPU norms carry a relative error of a few 1e-7 (the tensor
+core's fp32 sums of exact products, fp32 Lanczos), so LUT rows whose k-th and
+(k+1)-th biased scores lie closer than 1e-5 + 4e-6 lambda max M may differ."""
 import numpy as np
 import pytest
 import torch
@@ -12,7 +12,7 @@ import block_sparse_linear_proj_b200 as S
 import workloads as W
 from oracle import oracle as orc
 
-from gpu_util import dev, new_out
+from gpu_util import check, dev, new_out
 
 pytestmark = pytest.mark.gpu
 
@@ -122,3 +122,24 @@ def test_cov_workload_lut():
     ref, gap = orc.route(inp["q"], inp["k"], None, None, w.Bq, w.Bk, w.topk, bias=w.cov_lambda * m)
     excl = _check_cov_lut(lut.cpu().numpy(), ref, gap, m, w.cov_lambda)
     print("pisa_cov: %d of %d rows excluded by the gap rule" % (excl.sum(), excl.size))
+
+
+def test_cov_routing_with_first_order_term():
+    """Both PISA options at once: the covariance-aware LUT (the pre-pass then
+    forms the blocks' H_j sums exactly, for Hbar and for the first-order term)
+    and the first-order output on that LUT, against the oracle."""
+    B, H, N, d, k, lam = 1, 2, 4096, 128, 8, 0.5
+    inp = W.gaussian_inputs(B, H, N, d, 91, use_w=False, with_alpha=False)
+    g = dev(inp)
+    p = S.params(B, H, N, d, 64, 64, k, pisa_cov_lambda=lam, pisa_first_order=True,
+                 out_dtype=S.SLA_OUT_FP32)
+    lut = torch.full((B, H, N // 64, k), -1, dtype=torch.int32, device="cuda")
+    out = new_out(p, g["q"])
+    S.sla_pisa_forward(p, g["q"], g["k"], g["v"], None, None, lut, out, S.workspace(p))
+    assert S.sla_check_device_status() == 0
+    m = orc.block_cov_norms(inp["k"], inp["v"], 64)
+    ref, gap = orc.route_cov(inp["q"], inp["k"], inp["v"], 64, 64, k, lam)
+    _check_cov_lut(lut.cpu().numpy(), ref, gap, m, lam)
+    lut_np = lut.cpu().numpy()
+    want = orc.pisa_forward(inp["q"], inp["k"], inp["v"], lut_np, 64, 64, first_order=True)
+    check(out, want, p)
