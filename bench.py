@@ -9,9 +9,10 @@ resident in HBM.  Default workload: SLA2 bf16, B=1 H=12 N=32768 d=128,
 Bq=128 Bk=64, keep 52 of 512 KV blocks (90% sparse), bf16 output.
 
 Printed (rank 0, one JSON line): dense-equivalent TFLOPS (4 B H N^2 d / t) as
-`value`, ms per call, the end-to-end number through the same C ABI with host
-buffers (host->device copies of the inputs and the device->host copy of the
-output inside the timed region), the attention kernel's roofline (live CUDA
+`value`, ms per call, the end-to-end number through the C ABI's host-buffer
+calls (sla_forward_host, sla_pisa_forward_host: the host->device copies of the
+inputs and the device->host copy of the output inside the timed region,
+pipelined with the computation head chunk by head chunk), the attention kernel's roofline (live CUDA
 events around each launch on its stream, against the burst bf16 peak), the
 HBM fractions of the pre-passes on their algorithmic bytes and of the span
 before attention (one read of Q, K and V), the CPU oracle's throughput on
@@ -369,16 +370,27 @@ def run_ours(args, w, rank, world, local_rank):
     # ---- end-to-end through the C ABI with host buffers
     hosts = {k: (v.pin_memory() if v is not None else None) for k, v in inp.items()}
     out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    h2d = sum(v.numel() * v.element_size() for v in hosts.values() if v is not None)
+    copied = (list(hosts) if w.clusters else ["q", "k", "v"] if w.mode == "pisa" else ["q", "k", "v", "alpha"])
+    h2d = sum(hosts[k].numel() * hosts[k].element_size() for k in copied if hosts.get(k) is not None)
     d2h = out_h.numel() * out_h.element_size()
     e2e_steps = max(3, min(args.steps, 20))
 
+    # the library's host-buffer calls pipeline the copies with the computation
+    # head chunk by head chunk; the co-clustered call (a composition in Python)
+    # copies its inputs in, runs, and copies the output back
     def e2e_step():
-        for k, v in hosts.items():
-            if v is not None:
-                g[k].copy_(v, non_blocking=True)
-        step()
-        out_h.copy_(out, non_blocking=True)
+        if w.clusters:
+            for k, v in hosts.items():
+                if v is not None:
+                    g[k].copy_(v, non_blocking=True)
+            step()
+            out_h.copy_(out, non_blocking=True)
+        elif w.mode == "pisa":
+            S.sla_pisa_forward_host(p, hosts["q"], hosts["k"], hosts["v"], out_h, g["q"], g["k"], g["v"],
+                                    out, None, None, lut, ws, stream=stream)
+        else:
+            S.sla_forward_host(p, hosts["q"], hosts["k"], hosts["v"], hosts["alpha"], out_h, g["q"], g["k"],
+                               g["v"], g["alpha"], out, g["w_q"], g["w_k"], lut, ws, stream=stream)
 
     e2e_step()
     torch.cuda.synchronize(dev)

@@ -780,6 +780,124 @@ sla_status_t sla_pisa_forward(const sla_params_t* p, const void* q, const void* 
     return finish(s, st);
 }
 
+}  // extern "C"
+
+// ------------------------------------------------- host-buffer forward calls
+namespace {
+
+// Two library streams per device (host-to-device and device-to-host copies) and
+// their events, created on first use; a lock covers each call's enqueue sequence.
+struct HostPipe {
+    cudaStream_t h2d = nullptr, d2h = nullptr;
+    cudaEvent_t fork = nullptr, in = nullptr, done = nullptr, join = nullptr;
+    bool ok = false;
+    std::mutex lock;
+};
+
+HostPipe* host_pipe() {
+    static HostPipe pipes[64];
+    static std::mutex create;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    HostPipe& x = pipes[dev];
+    std::lock_guard<std::mutex> g(create);
+    if (!x.ok) {
+        if (cudaStreamCreateWithFlags(&x.h2d, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaStreamCreateWithFlags(&x.d2h, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaEventCreateWithFlags(&x.fork, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&x.in, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&x.done, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&x.join, cudaEventDisableTiming) != cudaSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        x.ok = true;
+    }
+    return &x;
+}
+
+// The (batch, head) problems of a call are independent and contiguous in every
+// tensor, so heads [h0, h0 + n) are a call with B = 1, H = n at offset h0.  Each
+// chunk's inputs are copied on the h2d stream; its forward runs on the caller's
+// stream once they have landed; its output goes back on the d2h stream while
+// later chunks arrive and compute.  fwd runs one chunk (device pointers).
+template <typename Fwd>
+sla_status_t run_host(const sla_params_t* p, const void* q_h, const void* k_h, const void* v_h,
+                      const float* alpha_h, void* out_h, void* q, void* k, void* v, float* alpha, void* out,
+                      int32_t* lut, int heads_per_chunk, cudaStream_t st, Fwd fwd) {
+    sla_status_t s = check_params(p);
+    if (s != SLA_OK) return s;
+    if (!q_h || !k_h || !v_h || !out_h || !q || !k || !v || !out || (alpha_h && !alpha) || heads_per_chunk < 0)
+        return SLA_ERR_INVALID_ARG;
+    const long long BH = static_cast<long long>(p->B) * p->H;
+    const size_t tok = static_cast<size_t>(p->N);
+    const size_t qkv_head = tok * p->d * 2;
+    const size_t out_head = tok * p->d * (p->out_dtype == SLA_OUT_FP32 ? 4 : 2);
+    const size_t lut_head = static_cast<size_t>(p->N / p->Bq) * p->topk;
+    const long long hc = heads_per_chunk > 0 ? heads_per_chunk : std::max<long long>(1, (BH + 7) / 8);
+    HostPipe* hp = host_pipe();
+    if (!hp) return SLA_ERR_CUDA;
+    std::lock_guard<std::mutex> g(hp->lock);
+    if (cudaEventRecord(hp->fork, st) != cudaSuccess || cudaStreamWaitEvent(hp->h2d, hp->fork, 0) != cudaSuccess)
+        return SLA_ERR_CUDA;
+    auto off = [](const void* b, size_t bytes) { return static_cast<const char*>(b) + bytes; };
+    auto offw = [](void* b, size_t bytes) { return static_cast<char*>(b) + bytes; };
+    for (long long h0 = 0; h0 < BH; h0 += hc) {
+        const long long n = std::min(hc, BH - h0);
+        const size_t o = static_cast<size_t>(h0) * qkv_head, nb = static_cast<size_t>(n) * qkv_head;
+        if (cudaMemcpyAsync(offw(q, o), off(q_h, o), nb, cudaMemcpyHostToDevice, hp->h2d) != cudaSuccess ||
+            cudaMemcpyAsync(offw(k, o), off(k_h, o), nb, cudaMemcpyHostToDevice, hp->h2d) != cudaSuccess ||
+            cudaMemcpyAsync(offw(v, o), off(v_h, o), nb, cudaMemcpyHostToDevice, hp->h2d) != cudaSuccess)
+            return SLA_ERR_CUDA;
+        if (alpha_h && cudaMemcpyAsync(alpha + h0 * static_cast<long long>(tok), alpha_h + h0 * static_cast<long long>(tok),
+                                       static_cast<size_t>(n) * tok * 4, cudaMemcpyHostToDevice, hp->h2d) != cudaSuccess)
+            return SLA_ERR_CUDA;
+        if (cudaEventRecord(hp->in, hp->h2d) != cudaSuccess || cudaStreamWaitEvent(st, hp->in, 0) != cudaSuccess)
+            return SLA_ERR_CUDA;
+        sla_params_t pc = *p;
+        pc.B = 1;
+        pc.H = static_cast<int32_t>(n);
+        s = fwd(&pc, offw(q, o), offw(k, o), offw(v, o), alpha ? alpha + h0 * static_cast<long long>(tok) : nullptr,
+                lut ? lut + h0 * static_cast<long long>(lut_head) : nullptr,
+                offw(out, static_cast<size_t>(h0) * out_head));
+        if (s != SLA_OK) return s;
+        if (cudaEventRecord(hp->done, st) != cudaSuccess || cudaStreamWaitEvent(hp->d2h, hp->done, 0) != cudaSuccess ||
+            cudaMemcpyAsync(offw(out_h, static_cast<size_t>(h0) * out_head), off(out, static_cast<size_t>(h0) * out_head),
+                            static_cast<size_t>(n) * out_head, cudaMemcpyDeviceToHost, hp->d2h) != cudaSuccess)
+            return SLA_ERR_CUDA;
+    }
+    if (cudaEventRecord(hp->join, hp->d2h) != cudaSuccess || cudaStreamWaitEvent(st, hp->join, 0) != cudaSuccess)
+        return SLA_ERR_CUDA;
+    return SLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+sla_status_t sla_forward_host(const sla_params_t* p, const void* q_h, const void* k_h, const void* v_h,
+                              const float* alpha_h, void* out_h, void* q, void* k, void* v, float* alpha,
+                              void* out, const float* w_q, const float* w_k, int32_t* lut,
+                              int32_t heads_per_chunk, void* workspace, size_t ws_bytes, sla_stream_t stream) {
+    if (!alpha_h || !alpha) return SLA_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return run_host(p, q_h, k_h, v_h, alpha_h, out_h, q, k, v, alpha, out, lut, heads_per_chunk, st,
+                    [&](const sla_params_t* pc, void* qc, void* kc, void* vc, float* ac, int32_t* lc, void* oc) {
+                        return sla_forward(pc, qc, kc, vc, ac, w_q, w_k, lc, oc, workspace, ws_bytes, stream);
+                    });
+}
+
+sla_status_t sla_pisa_forward_host(const sla_params_t* p, const void* q_h, const void* k_h, const void* v_h,
+                                   void* out_h, void* q, void* k, void* v, void* out, const float* w_q,
+                                   const float* w_k, int32_t* lut, int32_t heads_per_chunk, void* workspace,
+                                   size_t ws_bytes, sla_stream_t stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return run_host(p, q_h, k_h, v_h, nullptr, out_h, q, k, v, nullptr, out, lut, heads_per_chunk, st,
+                    [&](const sla_params_t* pc, void* qc, void* kc, void* vc, float*, int32_t* lc, void* oc) {
+                        return sla_pisa_forward(pc, qc, kc, vc, w_q, w_k, lc, oc, workspace, ws_bytes, stream);
+                    });
+}
+
 sla_status_t sla_pisa_cov_norms(const sla_params_t* p, const void* k, const void* v, double* norms,
                                 void* workspace, size_t ws_bytes, sla_stream_t stream) {
     sla_status_t s = check_params(p);

@@ -40,7 +40,8 @@ SLA_OUT_FP32 = 1
 EXPORTED = ("sla_workspace_size", "sla_route", "sla_forward", "sla_pisa_forward",
             "sla_status_string", "sla_check_device_status", "sla_version",
             "sla_profile_enable", "sla_profile_read", "sla_route_noalloc",
-            "sla_cocluster", "sla_cocluster_workspace_size", "sla_permute_rows")
+            "sla_cocluster", "sla_cocluster_workspace_size", "sla_permute_rows",
+            "sla_forward_host", "sla_pisa_forward_host")
 KERNEL_KINDS = ("pool", "kv_stats", "h_reduce", "fold_w", "score_topk", "attn", "quant_q", "project",
                 "cov", "pre_attn", "cocluster", "permute")
 # profile entries that are phases of a call, not kernel launches
@@ -105,6 +106,12 @@ def load():
             lib.sla_permute_rows.argtypes = [P, P, P, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
                                              ctypes.c_int32, P]
             lib.sla_permute_rows.restype = ctypes.c_int
+            lib.sla_forward_host.argtypes = [PP, P, P, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_int32, P,
+                                             ctypes.c_size_t, P]
+            lib.sla_forward_host.restype = ctypes.c_int
+            lib.sla_pisa_forward_host.argtypes = [PP, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_int32, P,
+                                                  ctypes.c_size_t, P]
+            lib.sla_pisa_forward_host.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -204,6 +211,57 @@ def sla_forward(p, q, k, v, alpha, w_q, w_k, lut, out, ws, stream=None):
                             _stream(stream))
     _raise(rc, "sla_forward")
     return out
+
+
+def _hptr(t):
+    """A host (CPU) tensor's address; pinned memory lets the copies overlap."""
+    if t is None or t.numel() == 0:
+        return None
+    if t.is_cuda:
+        raise ValueError("tensor must be in host memory")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def sla_forward_host(p, q_h, k_h, v_h, alpha_h, out_h, q, k, v, alpha, out, w_q, w_k, lut, ws,
+                     heads_per_chunk=0, stream=None):
+    """sla_forward with host inputs and output: chunks of heads are copied into
+    the device buffers q, k, v, alpha, computed into ``out`` and copied back into
+    ``out_h``, the copies overlapping the computation."""
+    B, H, N, d = p.B, p.H, p.N, p.d
+    for name, t in (("q_h", q_h), ("k_h", k_h), ("v_h", v_h), ("q", q), ("k", k), ("v", v)):
+        _check(t, torch.bfloat16, (B, H, N, d), name)
+    for name, t in (("alpha_h", alpha_h), ("alpha", alpha)):
+        _check(t, torch.float32, (B, H, N), name)
+    for name, t in (("out_h", out_h), ("out", out)):
+        _check(t, out_torch_dtype(p), (B, H, N, d), name)
+    if lut is not None:
+        _check(lut, torch.int32, (B, H, N // p.Bq, p.topk), "lut")
+    rc = load().sla_forward_host(ctypes.byref(p), _hptr(q_h), _hptr(k_h), _hptr(v_h), _hptr(alpha_h),
+                                 _hptr(out_h), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(out),
+                                 _ptr(w_q), _ptr(w_k), _ptr(lut), int(heads_per_chunk), _ptr(ws),
+                                 ws.numel(), _stream(stream))
+    _raise(rc, "sla_forward_host")
+    return out_h
+
+
+def sla_pisa_forward_host(p, q_h, k_h, v_h, out_h, q, k, v, out, w_q, w_k, lut, ws,
+                          heads_per_chunk=0, stream=None):
+    """sla_pisa_forward with host inputs and output (see sla_forward_host)."""
+    B, H, N, d = p.B, p.H, p.N, p.d
+    for name, t in (("q_h", q_h), ("k_h", k_h), ("v_h", v_h), ("q", q), ("k", k), ("v", v)):
+        _check(t, torch.bfloat16, (B, H, N, d), name)
+    for name, t in (("out_h", out_h), ("out", out)):
+        _check(t, out_torch_dtype(p), (B, H, N, d), name)
+    if lut is not None:
+        _check(lut, torch.int32, (B, H, N // p.Bq, p.topk), "lut")
+    rc = load().sla_pisa_forward_host(ctypes.byref(p), _hptr(q_h), _hptr(k_h), _hptr(v_h), _hptr(out_h),
+                                      _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(w_q), _ptr(w_k),
+                                      _ptr(lut), int(heads_per_chunk), _ptr(ws), ws.numel(),
+                                      _stream(stream))
+    _raise(rc, "sla_pisa_forward_host")
+    return out_h
 
 
 def sla_pisa_cov_norms(p, k, v, norms, ws, stream=None):

@@ -199,6 +199,42 @@ sla_status_t sla_pisa_forward(const sla_params_t *p, const void *q, const void *
                               void *workspace, size_t ws_bytes, sla_stream_t stream);
 
 /*
+ * sla_forward_host / sla_pisa_forward_host -- sla_forward and sla_pisa_forward
+ * with the inputs and the output in host memory.  The (batch, head) problems of
+ * a call are independent ([SLA2] sec. 2, [PISA] sec. 2: attention, routing and
+ * every statistic are per head), so the call works through chunks of
+ * heads_per_chunk consecutive heads (0: about an eighth of B*H): each chunk's
+ * Q, K, V (and alpha) are copied to the caller's device buffers on a library
+ * stream, its forward runs on `stream` as soon as they have landed, and its
+ * output is copied back on a second library stream while later chunks arrive
+ * and compute.  The result equals that of one sla_forward (sla_pisa_forward) call
+ * on the whole problem.
+ *   q_h, k_h, v_h: host bf16 [B,H,N,d]; alpha_h: host fp32 [B,H,N] (sla_forward_host
+ *   only); out_h: host [B,H,N,d] in the type p->out_dtype selects.  Page-locked
+ *   (pinned) host memory lets the copies overlap; pageable memory is correct but
+ *   serialises them.
+ *   q, k, v, alpha, out: the caller's device buffers of those shapes (16-byte
+ *   aligned; alpha 4-byte), overwritten by the call.
+ *   w_q, w_k, lut, workspace, ws_bytes: as for sla_forward / sla_pisa_forward (the
+ *   workspace sized for the whole problem serves every chunk; lut, if given,
+ *   is the whole problem's).
+ * Asynchronous on stream: it starts after the work queued on stream before it,
+ * and work queued on stream after it waits for its last copy.  Errors as
+ * sla_forward; a NULL buffer or heads_per_chunk < 0 is SLA_ERR_INVALID_ARG.  An
+ * error in a later chunk leaves the earlier chunks' work queued.
+ */
+sla_status_t sla_forward_host(const sla_params_t *p, const void *q_h, const void *k_h,
+                              const void *v_h, const float *alpha_h, void *out_h, void *q,
+                              void *k, void *v, float *alpha, void *out, const float *w_q,
+                              const float *w_k, int32_t *lut, int32_t heads_per_chunk,
+                              void *workspace, size_t ws_bytes, sla_stream_t stream);
+sla_status_t sla_pisa_forward_host(const sla_params_t *p, const void *q_h, const void *k_h,
+                                   const void *v_h, void *out_h, void *q, void *k, void *v,
+                                   void *out, const float *w_q, const float *w_k, int32_t *lut,
+                                   int32_t heads_per_chunk, void *workspace, size_t ws_bytes,
+                                   sla_stream_t stream);
+
+/*
  * sla_pisa_cov_norms -- the block covariance norms of the covariance-aware
  * selection: norms[(b*H + h)*Nk + j] = M_j = || H_j - Hbar ||_2 in fp64
  * (unscaled), j < Nk = N/Bk.  H_j and Hbar are fp32 tensor-core sums of exact
