@@ -100,3 +100,25 @@ def test_forward_host_pageable_memory_and_arguments():
         S.sla_forward_host(p, _pinned(inp)["q"], inp["k"], inp["v"], inp["alpha"], outs[0], g["q"], g["k"],
                            g["v"], g["alpha"], out, g["w_q"], g["w_k"], None, S.workspace(p), heads_per_chunk=-1)
     assert ei.value.code == S.sla.SLA_ERR_INVALID_ARG
+
+
+def test_forward_host_given_lut():
+    """LUT_GIVEN: each chunk reads its own rows of the caller's LUT."""
+    B, H, N, d, Bq, k = 1, 5, 2048, 128, 128, 7
+    inp = W.gaussian_inputs(B, H, N, d, 80)
+    g = dev(inp)
+    rng = np.random.default_rng(3)
+    lut_np = np.sort(np.stack([[[rng.choice(N // 64, k, replace=False) for _ in range(N // Bq)]
+                                for _ in range(H)] for _ in range(B)]), axis=-1).astype(np.int32)
+    p = params(B, H, N, d, Bq, 64, k, given=True, f32=True)
+    h = _pinned(inp)
+    out_h = torch.full(inp["q"].shape, float("nan"), dtype=torch.float32).pin_memory()
+    bufs = {n: torch.empty_like(g[n]) for n in ("q", "k", "v", "alpha")}
+    out = torch.empty(g["q"].shape, dtype=torch.float32, device="cuda")
+    lut = torch.as_tensor(lut_np).cuda()
+    S.sla_forward_host(p, h["q"], h["k"], h["v"], h["alpha"], out_h, bufs["q"], bufs["k"], bufs["v"],
+                       bufs["alpha"], out, g["w_q"], g["w_k"], lut, S.workspace(p), heads_per_chunk=2)
+    torch.cuda.synchronize()
+    assert S.sla_check_device_status() == 0
+    ref = orc.sla_forward(inp["q"], inp["k"], inp["v"], inp["alpha"], lut_np, Bq, 64)
+    check(out_h, ref, p)
