@@ -10,7 +10,7 @@
 //
 // Per head and per half-step:
 //   cc_assign_kernel    label[n] = argmax over non-empty clusters c of x_n . cent_c
-//                       (ties to the lower c), one token per thread, 32 centroids
+//                       (ties to the lower c), two tokens per thread, 16 centroids
 //                       at a time in shared memory;
 //   cc_count_kernel     per chunk of 1024 tokens, the tokens per label;
 //   cc_scan_kernel      each chunk's first sorted position per label;
@@ -24,7 +24,7 @@
 namespace sla {
 
 constexpr int kCcChunk = 1024;     // tokens per counting-sort chunk
-constexpr int kCcTile = 32;        // centroids per shared-memory tile of the assignment
+constexpr int kCcTile = 16;        // centroids per shared-memory tile of the assignment
 
 // Initial query centroids: means of C contiguous chunks of N/C rows.
 // grid (C, BH), D threads.
@@ -42,10 +42,14 @@ __global__ void __launch_bounds__(128) cc_chunk_mean_kernel(const __nv_bfloat16*
 }
 
 // label[bh][n] = argmax over valid c of x[bh][n] . cent[bh][c].
-// grid (ceil(N/128), BH), 128 threads (one token each); dynamic shared memory:
-// the CTA's tokens transposed (bf16 [D][132]), a tile of centroids (fp64
-// [kCcTile][D]) and their empty flags.
-constexpr int kCcPitch = 132;
+// grid (ceil(N/256), BH), 128 threads, each with two tokens (t and t + 128 of
+// the CTA's 256), so that every centroid coordinate read from shared memory
+// serves two FMAs; dynamic shared memory: the CTA's tokens transposed (bf16
+// [D][kCcPitch]), a tile of kCcTile centroids transposed (fp64 [D][kCcTile]: one
+// 16-byte read gives two centroids' coordinate) and their empty flags.  Each dot
+// product is summed over the coordinates in order.
+constexpr int kCcPitch = 260;
+constexpr int kCcTok = 256;        // tokens per CTA
 template <int D>
 constexpr size_t cc_assign_smem() { return static_cast<size_t>(D) * kCcPitch * 2 + kCcTile * D * 8 + kCcTile * 4; }
 
@@ -55,39 +59,55 @@ __global__ void __launch_bounds__(128) cc_assign_kernel(const __nv_bfloat16* __r
                                                         const int* __restrict__ valid, int* __restrict__ label) {
     extern __shared__ __align__(16) unsigned char cc_smem[];
     __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(cc_smem);                       // [D][kCcPitch]
-    double* cs = reinterpret_cast<double*>(cc_smem + static_cast<size_t>(D) * kCcPitch * 2);   // [kCcTile][D]
+    double* cs = reinterpret_cast<double*>(cc_smem + static_cast<size_t>(D) * kCcPitch * 2);   // [D][kCcTile]
     int* vs = reinterpret_cast<int*>(cs + kCcTile * D);                                   // [kCcTile]
     const long long bh = blockIdx.y;
-    const int n0 = blockIdx.x * 128;
+    const int n0 = blockIdx.x * kCcTok;
     const int t = threadIdx.x;
-    // stage the tile's tokens (coalesced rows), transposed so that thread t reads column t
-    for (int i = t; i < 128 * D; i += 128) {
+    // stage the CTA's tokens (coalesced rows), transposed so that thread t reads columns t and t + 128
+    for (int i = t; i < kCcTok * D; i += 128) {
         const int r = i / D, dd = i % D;
         const int n = n0 + r;
         xs[dd * kCcPitch + r] = n < N ? x[(bh * N + n) * D + dd] : __float2bfloat16(0.f);
     }
-    double best = -INFINITY;
-    int arg = -1;
+    double best[2] = {-INFINITY, -INFINITY};
+    int arg[2] = {-1, -1};
     for (int c0 = 0; c0 < C; c0 += kCcTile) {
         __syncthreads();
         const int nt = min(kCcTile, C - c0);
-        for (int i = t; i < nt * D; i += 128) cs[i] = cent[(bh * C + c0) * D + i];
+        for (int i = t; i < kCcTile * D; i += 128) {            // (consecutive threads: consecutive centroids)
+            const int jc = i % kCcTile, dd = i / kCcTile;
+            cs[i] = jc < nt ? cent[(bh * C + c0 + jc) * D + dd] : 0.0;
+        }
         if (t < nt) vs[t] = valid[bh * C + c0 + t];
         __syncthreads();
-        double acc[kCcTile];
+        double a0[kCcTile], a1[kCcTile];
 #pragma unroll
-        for (int j = 0; j < kCcTile; ++j) acc[j] = 0.0;
+        for (int j = 0; j < kCcTile; ++j) a0[j] = a1[j] = 0.0;
 #pragma unroll 2
         for (int dd = 0; dd < D; ++dd) {
-            const double xv = static_cast<double>(__bfloat162float(xs[dd * kCcPitch + t]));
+            const double x0 = static_cast<double>(__bfloat162float(xs[dd * kCcPitch + t]));
+            const double x1 = static_cast<double>(__bfloat162float(xs[dd * kCcPitch + t + 128]));
+            const double2* c2 = reinterpret_cast<const double2*>(cs + dd * kCcTile);
 #pragma unroll
-            for (int j = 0; j < kCcTile; ++j) acc[j] = fma(xv, cs[j * D + dd], acc[j]);
+            for (int j = 0; j < kCcTile / 2; ++j) {
+                const double2 cc = c2[j];
+                a0[2 * j] = fma(x0, cc.x, a0[2 * j]);
+                a0[2 * j + 1] = fma(x0, cc.y, a0[2 * j + 1]);
+                a1[2 * j] = fma(x1, cc.x, a1[2 * j]);
+                a1[2 * j + 1] = fma(x1, cc.y, a1[2 * j + 1]);
+            }
         }
 #pragma unroll
-        for (int j = 0; j < kCcTile; ++j)
-            if (j < nt && vs[j] && (arg < 0 || acc[j] > best)) { best = acc[j]; arg = c0 + j; }
+        for (int j = 0; j < kCcTile; ++j) {
+            if (j < nt && vs[j]) {
+                if (arg[0] < 0 || a0[j] > best[0]) { best[0] = a0[j]; arg[0] = c0 + j; }
+                if (arg[1] < 0 || a1[j] > best[1]) { best[1] = a1[j]; arg[1] = c0 + j; }
+            }
+        }
     }
-    if (n0 + t < N) label[bh * N + n0 + t] = arg < 0 ? 0 : arg;
+    if (n0 + t < N) label[bh * N + n0 + t] = arg[0] < 0 ? 0 : arg[0];
+    if (n0 + t + 128 < N) label[bh * N + n0 + t + 128] = arg[1] < 0 ? 0 : arg[1];
 }
 
 // counts[bh][chunk][c] = tokens of the chunk with label c.  grid (nchunk, BH), 256 threads.
@@ -169,28 +189,43 @@ __global__ void __launch_bounds__(32) cc_scatter_kernel(const int* __restrict__ 
     }
 }
 
-// cent[bh][c] = mean of rows perm[start_c .. start_c + count_c) (in that order);
-// a label without tokens is marked empty and keeps its old centroid.
-// grid (C, BH), D threads.
+// cent[bh][c] = mean of rows perm[start_c .. start_c + count_c); a label
+// without tokens is marked empty and keeps its old centroid.  The sums of bf16
+// values are exact in fp64, so the kCcMeanGroups row groups (rows i, i + G, ...)
+// and their combination in a fixed order give the value of any order.
+// grid (C, BH), kCcMeanGroups * D threads.
+constexpr int kCcMeanGroups = 4;
 template <int D>
-__global__ void __launch_bounds__(128) cc_means_kernel(const __nv_bfloat16* __restrict__ x, int N, int C,
-                                                       const int* __restrict__ perm, const int* __restrict__ start,
-                                                       const int* __restrict__ count, double* __restrict__ cent,
-                                                       int* __restrict__ valid) {
+__global__ void __launch_bounds__(kCcMeanGroups * 128) cc_means_kernel(const __nv_bfloat16* __restrict__ x, int N,
+                                                                       int C, const int* __restrict__ perm,
+                                                                       const int* __restrict__ start,
+                                                                       const int* __restrict__ count,
+                                                                       double* __restrict__ cent,
+                                                                       int* __restrict__ valid) {
+    __shared__ double part[kCcMeanGroups][D];
     const int c = blockIdx.x;
     const long long bh = blockIdx.y;
+    const int col = threadIdx.x % D, grp = threadIdx.x / D;
     const int st = start[bh * C + c], cnt = count[bh * C + c];
     if (cnt <= 0) {
         if (threadIdx.x == 0) valid[bh * C + c] = 0;
         return;
     }
     double s = 0.0;
-    for (int i = 0; i < cnt; ++i) {
+#pragma unroll 4
+    for (int i = grp; i < cnt; i += kCcMeanGroups) {
         const int n = perm[bh * N + st + i];
-        s += static_cast<double>(__bfloat162float(x[(bh * N + n) * D + threadIdx.x]));
+        s += static_cast<double>(__bfloat162float(x[(bh * N + n) * D + col]));
     }
-    cent[(bh * C + c) * D + threadIdx.x] = s / cnt;
-    if (threadIdx.x == 0) valid[bh * C + c] = 1;
+    part[grp][col] = s;
+    __syncthreads();
+    if (grp == 0) {
+        double t = part[0][col];
+#pragma unroll
+        for (int g2 = 1; g2 < kCcMeanGroups; ++g2) t += part[g2][col];
+        cent[(bh * C + c) * D + col] = t / cnt;
+        if (col == 0) valid[bh * C + c] = 1;
+    }
 }
 
 // dst row (bh, i) = src row (bh, perm[bh][i]) (inverse: dst row (bh, perm[bh][i])

@@ -976,7 +976,7 @@ sla_status_t cc_sort_means(const sla_params_t* p, int C, const __nv_bfloat16* x,
     }
     {
         Span sp(SLA_KERNEL_COCLUSTER, st);
-        sla::cc_means_kernel<D><<<dim3(C, BH), D, 0, st>>>(x, N, C, perm, at<int>(ws, w.start),
+        sla::cc_means_kernel<D><<<dim3(C, BH), sla::kCcMeanGroups * D, 0, st>>>(x, N, C, perm, at<int>(ws, w.start),
                                                            at<int>(ws, w.count), cent, valid);
     }
     return launch_status();
@@ -998,7 +998,7 @@ sla_status_t run_cocluster(const sla_params_t* p, int C, int iters, const void* 
     if (cudaFuncSetAttribute(assign, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(asmem)) !=
         cudaSuccess)
         return SLA_ERR_CUDA;
-    const dim3 agrid((N + 127) / 128, BH);
+    const dim3 agrid((N + sla::kCcTok - 1) / sla::kCcTok, BH);
     {
         Span sp(SLA_KERNEL_COCLUSTER, st);
         sla::cc_chunk_mean_kernel<D><<<dim3(C, BH), D, 0, st>>>(qb, N, C, qc, qv);
