@@ -46,7 +46,9 @@ __global__ void __launch_bounds__(128) cc_chunk_mean_kernel(const __nv_bfloat16*
 // the CTA's 256), so that every centroid coordinate read from shared memory
 // serves two FMAs; dynamic shared memory: the CTA's tokens transposed (bf16
 // [D][kCcPitch]), a tile of kCcTile centroids transposed (fp64 [D][kCcTile]: one
-// 16-byte read gives two centroids' coordinate) and their empty flags.  Each dot
+// 16-byte read gives two centroids' coordinate) and their empty flags.  The
+// tokens arrive in 16-byte loads, eight in flight per thread; the next centroid
+// tile is loaded into registers while the current one is in use.  Each dot
 // product is summed over the coordinates in order.
 constexpr int kCcPitch = 260;
 constexpr int kCcTok = 256;        // tokens per CTA
@@ -61,26 +63,57 @@ __global__ void __launch_bounds__(128) cc_assign_kernel(const __nv_bfloat16* __r
     __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(cc_smem);                       // [D][kCcPitch]
     double* cs = reinterpret_cast<double*>(cc_smem + static_cast<size_t>(D) * kCcPitch * 2);   // [D][kCcTile]
     int* vs = reinterpret_cast<int*>(cs + kCcTile * D);                                   // [kCcTile]
+    constexpr int kPer = kCcTile * D / 128;                                                // tile values per thread
     const long long bh = blockIdx.y;
     const int n0 = blockIdx.x * kCcTok;
     const int t = threadIdx.x;
-    // stage the CTA's tokens (coalesced rows), transposed so that thread t reads columns t and t + 128
-    for (int i = t; i < kCcTok * D; i += 128) {
-        const int r = i / D, dd = i % D;
-        const int n = n0 + r;
-        xs[dd * kCcPitch + r] = n < N ? x[(bh * N + n) * D + dd] : __float2bfloat16(0.f);
+    // the first centroid tile into registers (consecutive threads: consecutive centroids)
+    double pre[kPer];
+    int pre_v = 0;
+    auto fetch = [&](int c0) {
+        const int nt = min(kCcTile, C - c0);
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+            const int i = t + 128 * u;
+            const int jc = i % kCcTile, dd = i / kCcTile;
+            pre[u] = jc < nt ? cent[(bh * C + c0 + jc) * D + dd] : 0.0;
+        }
+        pre_v = t < nt ? valid[bh * C + c0 + t] : 0;
+    };
+    fetch(0);
+    // stage the CTA's tokens, transposed so that thread t reads columns t and t + 128:
+    // unit u of 16 bytes is row r = u % 256, coordinates 8 (u / 256) .. + 7
+    constexpr int kUnits = kCcTok * D / 8 / 128;                                           // per thread
+    static_assert(kUnits % 8 == 0, "eight loads in flight");
+#pragma unroll 1
+    for (int u0 = 0; u0 < kUnits; u0 += 8) {
+        uint4 buf[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int u = t + 128 * (u0 + j);
+            const int r = u % kCcTok, n = n0 + r;
+            buf[j] = n < N ? *reinterpret_cast<const uint4*>(x + (bh * N + n) * D + (u / kCcTok) * 8)
+                           : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int u = t + 128 * (u0 + j);
+            const int r = u % kCcTok, d0 = (u / kCcTok) * 8;
+            const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&buf[j]);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) xs[(d0 + q) * kCcPitch + r] = e[q];
+        }
     }
     double best[2] = {-INFINITY, -INFINITY};
     int arg[2] = {-1, -1};
     for (int c0 = 0; c0 < C; c0 += kCcTile) {
         __syncthreads();
         const int nt = min(kCcTile, C - c0);
-        for (int i = t; i < kCcTile * D; i += 128) {            // (consecutive threads: consecutive centroids)
-            const int jc = i % kCcTile, dd = i / kCcTile;
-            cs[i] = jc < nt ? cent[(bh * C + c0 + jc) * D + dd] : 0.0;
-        }
-        if (t < nt) vs[t] = valid[bh * C + c0 + t];
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) cs[t + 128 * u] = pre[u];
+        if (t < kCcTile) vs[t] = pre_v;
         __syncthreads();
+        if (c0 + kCcTile < C) fetch(c0 + kCcTile);
         double a0[kCcTile], a1[kCcTile];
 #pragma unroll
         for (int j = 0; j < kCcTile; ++j) a0[j] = a1[j] = 0.0;
