@@ -223,39 +223,55 @@ __global__ void __launch_bounds__(32) cc_scatter_kernel(const int* __restrict__ 
 }
 
 // cent[bh][c] = mean of rows perm[start_c .. start_c + count_c); a label
-// without tokens is marked empty and keeps its old centroid.  The sums of bf16
-// values are exact in fp64, so the kCcMeanGroups row groups (rows i, i + G, ...)
-// and their combination in a fixed order give the value of any order.
-// grid (C, BH), kCcMeanGroups * D threads.
-constexpr int kCcMeanGroups = 4;
+// without tokens is marked empty and keeps its old centroid.  D/8 threads share
+// a row (16-byte loads of eight coordinates), so kCcMeanThreads*8/D rows are
+// read at a time, four per thread in flight.  Sums of bf16 values in fp64 are
+// exact while the values' binary exponents span less than 53 - 8 - log2(rows)
+// bits, so the row groups and their combination in a fixed order give the
+// value of any order.  grid (C, BH), kCcMeanThreads threads.
+constexpr int kCcMeanThreads = 512;
 template <int D>
-__global__ void __launch_bounds__(kCcMeanGroups * 128) cc_means_kernel(const __nv_bfloat16* __restrict__ x, int N,
-                                                                       int C, const int* __restrict__ perm,
-                                                                       const int* __restrict__ start,
-                                                                       const int* __restrict__ count,
-                                                                       double* __restrict__ cent,
-                                                                       int* __restrict__ valid) {
-    __shared__ double part[kCcMeanGroups][D];
+__global__ void __launch_bounds__(kCcMeanThreads) cc_means_kernel(const __nv_bfloat16* __restrict__ x, int N, int C,
+                                                                 const int* __restrict__ perm,
+                                                                 const int* __restrict__ start,
+                                                                 const int* __restrict__ count,
+                                                                 double* __restrict__ cent,
+                                                                 int* __restrict__ valid) {
+    constexpr int L = D / 8, R = kCcMeanThreads / L;      // threads per row, rows at a time
+    __shared__ double part[R][D];
     const int c = blockIdx.x;
     const long long bh = blockIdx.y;
-    const int col = threadIdx.x % D, grp = threadIdx.x / D;
+    const int k8 = (threadIdx.x % L) * 8, grp = threadIdx.x / L;
     const int st = start[bh * C + c], cnt = count[bh * C + c];
     if (cnt <= 0) {
         if (threadIdx.x == 0) valid[bh * C + c] = 0;
         return;
     }
-    double s = 0.0;
-#pragma unroll 4
-    for (int i = grp; i < cnt; i += kCcMeanGroups) {
-        const int n = perm[bh * N + st + i];
-        s += static_cast<double>(__bfloat162float(x[(bh * N + n) * D + col]));
-    }
-    part[grp][col] = s;
-    __syncthreads();
-    if (grp == 0) {
-        double t = part[0][col];
+    double s[8];
 #pragma unroll
-        for (int g2 = 1; g2 < kCcMeanGroups; ++g2) t += part[g2][col];
+    for (int q = 0; q < 8; ++q) s[q] = 0.0;
+    for (int i0 = grp; i0 < cnt; i0 += 4 * R) {
+        int n[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) n[u] = i0 + u * R < cnt ? perm[bh * N + st + i0 + u * R] : -1;
+        uint4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            v[u] = n[u] >= 0 ? *reinterpret_cast<const uint4*>(x + (bh * N + n[u]) * D + k8) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&v[u]);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) s[q] += static_cast<double>(__bfloat162float(e[q]));
+        }
+    }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) part[grp][k8 + q] = s[q];
+    __syncthreads();
+    if (threadIdx.x < D) {
+        const int col = threadIdx.x;
+        double t = part[0][col];
+        for (int g2 = 1; g2 < R; ++g2) t += part[g2][col];
         cent[(bh * C + c) * D + col] = t / cnt;
         if (col == 0) valid[bh * C + c] = 1;
     }

@@ -976,7 +976,7 @@ sla_status_t cc_sort_means(const sla_params_t* p, int C, const __nv_bfloat16* x,
     }
     {
         Span sp(SLA_KERNEL_COCLUSTER, st);
-        sla::cc_means_kernel<D><<<dim3(C, BH), sla::kCcMeanGroups * D, 0, st>>>(x, N, C, perm, at<int>(ws, w.start),
+        sla::cc_means_kernel<D><<<dim3(C, BH), sla::kCcMeanThreads, 0, st>>>(x, N, C, perm, at<int>(ws, w.start),
                                                            at<int>(ws, w.count), cent, valid);
     }
     return launch_status();
