@@ -279,7 +279,10 @@ __global__ void __launch_bounds__(kCcMeanThreads) cc_means_kernel(const __nv_bfl
 
 // dst row (bh, i) = src row (bh, perm[bh][i]) (inverse: dst row (bh, perm[bh][i])
 // = src row (bh, i)); rows of row_words 32-bit words (VEC: 16-byte words).
-// A perm entry outside [0, N) is skipped and flagged.  Grid-stride over rows.
+// A perm entry outside [0, N) is skipped and flagged.  Grid-stride over rows,
+// kPermRows rows per thread at a time (their perm entries first, then their
+// loads), so that several loads are in flight behind each index load.
+constexpr int kPermRows = 4;
 template <typename T>
 __global__ void __launch_bounds__(256) permute_rows_kernel(const T* __restrict__ src, const int* __restrict__ perm,
                                                            T* __restrict__ dst, long long BH, int N, int row_words,
@@ -287,16 +290,29 @@ __global__ void __launch_bounds__(256) permute_rows_kernel(const T* __restrict__
     const long long rows = BH * N;
     const int per_row = max(1, 256 / row_words);      // rows handled by one CTA pass
     const int rr = threadIdx.x / row_words, w = threadIdx.x % row_words;
-    for (long long r0 = static_cast<long long>(blockIdx.x) * per_row; r0 < rows;
-         r0 += static_cast<long long>(gridDim.x) * per_row) {
-        const long long r = r0 + rr;
-        if (rr >= per_row || r >= rows) continue;
-        const long long bh = r / N;
-        const int p = perm[r];
-        if (p < 0 || p >= N) { if (w == 0) report(kStatusBadData); continue; }
-        const long long other = bh * N + p;
-        if (inverse) dst[other * row_words + w] = src[r * row_words + w];
-        else dst[r * row_words + w] = src[other * row_words + w];
+    if (rr >= per_row) return;
+    const long long step = static_cast<long long>(gridDim.x) * per_row;
+    for (long long r0 = static_cast<long long>(blockIdx.x) * per_row + rr; r0 < rows; r0 += kPermRows * step) {
+        int p[kPermRows];
+#pragma unroll
+        for (int u = 0; u < kPermRows; ++u) {
+            const long long r = r0 + u * step;
+            p[u] = r < rows ? perm[r] : -1;
+        }
+        T v[kPermRows] = {};
+#pragma unroll
+        for (int u = 0; u < kPermRows; ++u) {
+            const long long r = r0 + u * step;
+            if (r < rows && p[u] >= 0 && p[u] < N)
+                v[u] = src[(inverse ? r : (r / N) * N + p[u]) * row_words + w];
+        }
+#pragma unroll
+        for (int u = 0; u < kPermRows; ++u) {
+            const long long r = r0 + u * step;
+            if (r >= rows) continue;
+            if (p[u] < 0 || p[u] >= N) { if (w == 0) report(kStatusBadData); continue; }
+            dst[(inverse ? (r / N) * N + p[u] : r) * row_words + w] = v[u];
+        }
     }
 }
 

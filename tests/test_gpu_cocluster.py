@@ -82,7 +82,10 @@ def test_cocluster_video_workload():
 
 
 @pytest.mark.parametrize("shape,dtype", [((2, 3, 512, 128), torch.bfloat16), ((1, 2, 256, 64), torch.bfloat16),
-                                         ((2, 3, 512), torch.float32), ((1, 2, 128, 128), torch.float32)])
+                                         ((2, 3, 512), torch.float32), ((1, 2, 128, 128), torch.float32),
+                                         ((1, 3, 1000, 64), torch.bfloat16),       # rows not a multiple of a pass
+                                         ((1, 4, 32768, 128), torch.bfloat16),     # several grid strides a thread
+                                         ((4, 8, 65536), torch.float32)])
 def test_permute_rows_gather_and_scatter(shape, dtype):
     g = torch.Generator().manual_seed(93)
     x = torch.randn(shape, generator=g).to(dtype).cuda()
