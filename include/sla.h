@@ -207,8 +207,10 @@ sla_status_t sla_pisa_forward(const sla_params_t *p, const void *q, const void *
  * Q, K, V (and alpha) are copied to the caller's device buffers on a library
  * stream, its forward runs on `stream` as soon as they have landed, and its
  * output is copied back on a second library stream while later chunks arrive
- * and compute.  The result equals that of one sla_forward (sla_pisa_forward) call
- * on the whole problem.
+ * and compute.  The result is that of one sla_forward (sla_pisa_forward) call
+ * on the whole problem up to summation order: the LUT is identical, and the
+ * linear branch's per-head sums are split over a number of partial sums that
+ * depends on the heads in a chunk.
  *   q_h, k_h, v_h: host bf16 [B,H,N,d]; alpha_h: host fp32 [B,H,N] (sla_forward_host
  *   only); out_h: host [B,H,N,d] in the type p->out_dtype selects.  Page-locked
  *   (pinned) host memory lets the copies overlap; pageable memory is correct but
