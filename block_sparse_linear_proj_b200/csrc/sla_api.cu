@@ -67,14 +67,29 @@ struct Ws {
     int nchunk, bpc;
 };
 
+// K/V pre-pass chunking for bh heads: ~4 waves of CTAs over the heads, >= 8
+// blocks per chunk.
+void kv_chunking(long long bh, long long Nk, int& bpc, int& nchunk) {
+    const long long target = std::max<long long>(1, 592 / bh);
+    bpc = std::max<int>(8, static_cast<int>((Nk + target - 1) / target));
+    nchunk = static_cast<int>((Nk + bpc - 1) / bpc);
+}
+
 Ws layout(const sla_params_t* p) {
     Ws w{};
     const size_t BH = static_cast<size_t>(p->B) * p->H;
     const size_t d = p->d, Nq = p->N / p->Bq, Nk = p->N / p->Bk;
-    // K/V pre-pass chunking: ~4 waves of CTAs over the heads, >= 8 blocks per chunk
-    const long long target = std::max<long long>(1, 592 / static_cast<long long>(BH));
-    w.bpc = std::max<int>(8, static_cast<int>((Nk + target - 1) / target));
-    w.nchunk = static_cast<int>((Nk + w.bpc - 1) / w.bpc);
+    kv_chunking(static_cast<long long>(BH), static_cast<long long>(Nk), w.bpc, w.nchunk);
+    // The chunk partials are sized for the most that any call over at most BH
+    // heads (same N, d, blocks and modes) uses, so that the workspace size never
+    // falls as heads are added and a workspace for BH heads serves a call over a
+    // subset of them.  Above 592 heads a head is one chunk.
+    size_t parts = BH * static_cast<size_t>(w.nchunk);
+    for (long long h = 1; h < std::min<long long>(static_cast<long long>(BH), 593); ++h) {
+        int b_ = 0, n_ = 0;
+        kv_chunking(h, static_cast<long long>(Nk), b_, n_);
+        parts = std::max(parts, static_cast<size_t>(h) * n_);
+    }
     size_t off = 0;
     auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes); return o; };
     w.qbar = take(BH * Nq * d * 8);
@@ -82,7 +97,7 @@ Ws layout(const sla_params_t* p) {
     w.m = take(d * d * 8);
     w.lut = take(BH * Nq * static_cast<size_t>(p->topk) * 4 + 4);
     w.zj = take(BH * Nk * d * 4);
-    w.hpart = take(BH * static_cast<size_t>(w.nchunk) * d * d * 4);
+    w.hpart = take(parts * d * d * 4);
     w.hsum = take(BH * d * d * 4);
     w.zsum = take(BH * d * 4);
     w.kc = take(BH * Nk * d * 2);
@@ -535,6 +550,41 @@ sla_status_t finish(sla_status_t s, cudaStream_t st) {
     return SLA_OK;
 }
 
+
+// Argument checks of sla_forward and sla_pisa_forward, before anything is
+// enqueued (also run by the host-buffer calls on the whole problem).
+sla_status_t forward_args(const sla_params_t* p, const void* q, const void* k, const void* v, const float* alpha,
+                          const float* w_q, const float* w_k, const int32_t* lut, const void* out,
+                          void* workspace, size_t ws_bytes, Ws& w) {
+    sla_status_t s = check_params(p);
+    if (s != SLA_OK) return s;
+    if (p->pisa_cov_lambda != 0.f) return SLA_ERR_INVALID_ARG;   // a PISA selection option
+    if ((s = check_tensor(q, 16)) || (s = check_tensor(k, 16)) || (s = check_tensor(v, 16)) ||
+        (s = check_tensor(out, 16)) || (s = check_tensor(alpha, 4)))
+        return s;
+    if ((w_q && !aligned(w_q, 4)) || (w_k && !aligned(w_k, 4))) return SLA_ERR_INVALID_ARG;
+    if (p->lut_mode == SLA_LUT_GIVEN && !lut && p->topk > 0) return SLA_ERR_INVALID_ARG;
+    if (lut && !aligned(lut, 4)) return SLA_ERR_INVALID_ARG;
+    if (p->sparse_dtype != SLA_SPARSE_BF16 && (p->d != 128 || p->Bq != 128))
+        return SLA_ERR_UNSUPPORTED;
+    return check_ws(p, workspace, ws_bytes, w);
+}
+
+sla_status_t pisa_args(const sla_params_t* p, const void* q, const void* k, const void* v, const float* w_q,
+                       const float* w_k, const int32_t* lut, const void* out, void* workspace, size_t ws_bytes,
+                       Ws& w) {
+    sla_status_t s = check_params(p);
+    if (s != SLA_OK) return s;
+    if ((s = check_tensor(q, 16)) || (s = check_tensor(k, 16)) || (s = check_tensor(v, 16)) ||
+        (s = check_tensor(out, 16)))
+        return s;
+    if ((w_q && !aligned(w_q, 4)) || (w_k && !aligned(w_k, 4))) return SLA_ERR_INVALID_ARG;
+    if (p->lut_mode == SLA_LUT_GIVEN && !lut && p->topk > 0) return SLA_ERR_INVALID_ARG;
+    if (lut && !aligned(lut, 4)) return SLA_ERR_INVALID_ARG;
+    if (p->Bq != p->Bk || p->sparse_dtype != SLA_SPARSE_BF16) return SLA_ERR_UNSUPPORTED;
+    return check_ws(p, workspace, ws_bytes, w);
+}
+
 }  // namespace
 
 extern "C" {
@@ -659,19 +709,9 @@ SideStream* side_stream() {
 sla_status_t sla_forward(const sla_params_t* p, const void* q, const void* k, const void* v,
                          const float* alpha, const float* w_q, const float* w_k, int32_t* lut,
                          void* out, void* workspace, size_t ws_bytes, sla_stream_t stream) {
-    sla_status_t s = check_params(p);
-    if (s != SLA_OK) return s;
-    if (p->pisa_cov_lambda != 0.f) return SLA_ERR_INVALID_ARG;   // a PISA selection option
-    if ((s = check_tensor(q, 16)) || (s = check_tensor(k, 16)) || (s = check_tensor(v, 16)) ||
-        (s = check_tensor(out, 16)) || (s = check_tensor(alpha, 4)))
-        return s;
-    if ((w_q && !aligned(w_q, 4)) || (w_k && !aligned(w_k, 4))) return SLA_ERR_INVALID_ARG;
-    if (p->lut_mode == SLA_LUT_GIVEN && !lut && p->topk > 0) return SLA_ERR_INVALID_ARG;
-    if (lut && !aligned(lut, 4)) return SLA_ERR_INVALID_ARG;
-    if (p->sparse_dtype != SLA_SPARSE_BF16 && (p->d != 128 || p->Bq != 128))
-        return SLA_ERR_UNSUPPORTED;
     Ws w;
-    if ((s = check_ws(p, workspace, ws_bytes, w))) return s;
+    sla_status_t s = forward_args(p, q, k, v, alpha, w_q, w_k, lut, out, workspace, ws_bytes, w);
+    if (s != SLA_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const bool compute = p->lut_mode == SLA_LUT_COMPUTE;
     // fp8: the 8-bit sparse branch (e4m3 P and V); int8: with integer Q and K codes
@@ -725,17 +765,9 @@ sla_status_t sla_forward(const sla_params_t* p, const void* q, const void* k, co
 sla_status_t sla_pisa_forward(const sla_params_t* p, const void* q, const void* k, const void* v,
                               const float* w_q, const float* w_k, int32_t* lut, void* out,
                               void* workspace, size_t ws_bytes, sla_stream_t stream) {
-    sla_status_t s = check_params(p);
-    if (s != SLA_OK) return s;
-    if ((s = check_tensor(q, 16)) || (s = check_tensor(k, 16)) || (s = check_tensor(v, 16)) ||
-        (s = check_tensor(out, 16)))
-        return s;
-    if ((w_q && !aligned(w_q, 4)) || (w_k && !aligned(w_k, 4))) return SLA_ERR_INVALID_ARG;
-    if (p->lut_mode == SLA_LUT_GIVEN && !lut && p->topk > 0) return SLA_ERR_INVALID_ARG;
-    if (lut && !aligned(lut, 4)) return SLA_ERR_INVALID_ARG;
-    if (p->Bq != p->Bk || p->sparse_dtype != SLA_SPARSE_BF16) return SLA_ERR_UNSUPPORTED;
     Ws w;
-    if ((s = check_ws(p, workspace, ws_bytes, w))) return s;
+    sla_status_t s = pisa_args(p, q, k, v, w_q, w_k, lut, out, workspace, ws_bytes, w);
+    if (s != SLA_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const bool compute = p->lut_mode == SLA_LUT_COMPUTE;
     int32_t* lut_use = (compute && !lut) ? at<int32_t>(workspace, w.lut) : lut;
@@ -879,7 +911,10 @@ sla_status_t sla_forward_host(const sla_params_t* p, const void* q_h, const void
                               const float* alpha_h, void* out_h, void* q, void* k, void* v, float* alpha,
                               void* out, const float* w_q, const float* w_k, int32_t* lut,
                               int32_t heads_per_chunk, void* workspace, size_t ws_bytes, sla_stream_t stream) {
-    if (!alpha_h || !alpha) return SLA_ERR_INVALID_ARG;
+    Ws w;
+    sla_status_t s = forward_args(p, q, k, v, alpha, w_q, w_k, lut, out, workspace, ws_bytes, w);
+    if (s != SLA_OK) return s;
+    if (!alpha_h) return SLA_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     return run_host(p, q_h, k_h, v_h, alpha_h, out_h, q, k, v, alpha, out, lut, heads_per_chunk, st,
                     [&](const sla_params_t* pc, void* qc, void* kc, void* vc, float* ac, int32_t* lc, void* oc) {
@@ -891,6 +926,9 @@ sla_status_t sla_pisa_forward_host(const sla_params_t* p, const void* q_h, const
                                    void* out_h, void* q, void* k, void* v, void* out, const float* w_q,
                                    const float* w_k, int32_t* lut, int32_t heads_per_chunk, void* workspace,
                                    size_t ws_bytes, sla_stream_t stream) {
+    Ws w;
+    sla_status_t s = pisa_args(p, q, k, v, w_q, w_k, lut, out, workspace, ws_bytes, w);
+    if (s != SLA_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     return run_host(p, q_h, k_h, v_h, nullptr, out_h, q, k, v, nullptr, out, lut, heads_per_chunk, st,
                     [&](const sla_params_t* pc, void* qc, void* kc, void* vc, float*, int32_t* lc, void* oc) {

@@ -88,7 +88,9 @@ typedef struct sla_params {
 /* Bytes of device workspace that sla_route, sla_forward, sla_pisa_forward and
  * sla_pisa_cov_norms need for these parameters (the maximum over them; the
  * covariance-aware selection's scratch is included when pisa_cov_lambda > 0).
- * Returns 0 if the parameters are invalid. */
+ * It never decreases as B*H grows with the other fields fixed, so a workspace
+ * for B*H heads serves a call over any subset of them.  Returns 0 if the
+ * parameters are invalid. */
 size_t sla_workspace_size(const sla_params_t *p);
 
 /*
@@ -221,9 +223,11 @@ sla_status_t sla_pisa_forward(const sla_params_t *p, const void *q, const void *
  *   workspace sized for the whole problem serves every chunk; lut, if given,
  *   is the whole problem's).
  * Asynchronous on stream: it starts after the work queued on stream before it,
- * and work queued on stream after it waits for its last copy.  Errors as
- * sla_forward; a NULL buffer or heads_per_chunk < 0 is SLA_ERR_INVALID_ARG.  An
- * error in a later chunk leaves the earlier chunks' work queued.
+ * and work queued on stream after it waits for its last copy.  The arguments
+ * are checked as sla_forward (sla_pisa_forward) checks them, for the whole
+ * problem, before anything is enqueued; a NULL host buffer or heads_per_chunk < 0
+ * is SLA_ERR_INVALID_ARG.  A CUDA error in a later chunk leaves the earlier
+ * chunks' work queued.
  */
 sla_status_t sla_forward_host(const sla_params_t *p, const void *q_h, const void *k_h,
                               const void *v_h, const float *alpha_h, void *out_h, void *q,

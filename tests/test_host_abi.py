@@ -196,3 +196,53 @@ def test_permute_rows_argument_checks(lib):
     assert f(ctypes.c_void_p((1 << 20) + 2), FAKE, B2, 2, 64, 4, 0, None) == S.SLA_ERR_INVALID_ARG
     assert f(A, FAKE, B2, 0, 64, 256, 0, None) == S.SLA_ERR_INVALID_ARG
     assert f(A, FAKE, B2, 2, 64, 8192, 0, None) == S.SLA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("N,d,Bq,topk", [(32768, 128, 128, 52), (8192, 64, 64, 16), (1024, 128, 64, 4)])
+def test_workspace_size_never_falls_as_heads_grow(lib, N, d, Bq, topk):
+    """A workspace for B*H heads serves a call over a subset of them (the
+    host-buffer calls run chunks of heads in the whole problem's workspace).
+    The pre-pass's chunks per head shrink as heads are added, so the partial
+    sums are sized for the most that any smaller head count uses."""
+    prev = 0
+    for H in list(range(1, 40)) + [147, 148, 149, 295, 296, 297, 298, 591, 592, 593, 700]:
+        need = lib.sla_workspace_size(ctypes.byref(S.params(1, H, N, d, Bq, 64, topk)))
+        assert need >= prev, H
+        prev = need
+    # B and H enter only through B*H
+    a = lib.sla_workspace_size(ctypes.byref(S.params(3, 99, N, d, Bq, 64, topk)))
+    b = lib.sla_workspace_size(ctypes.byref(S.params(1, 297, N, d, Bq, 64, topk)))
+    assert a == b
+
+
+def call_forward_host(p, hpc=0, q_h=FAKE, alpha_h=FAKE, q=FAKE, lut=FAKE, ws=FAKE, ws_bytes=1 << 40):
+    return S.load().sla_forward_host(ctypes.byref(p), q_h, FAKE, FAKE, alpha_h, FAKE, q, FAKE, FAKE, FAKE,
+                                     FAKE, None, None, lut, hpc, ws, ws_bytes, None)
+
+
+def call_pisa_host(p, hpc=0, out_h=FAKE, out=FAKE, ws_bytes=1 << 40):
+    return S.load().sla_pisa_forward_host(ctypes.byref(p), FAKE, FAKE, FAKE, out_h, FAKE, FAKE, FAKE, out,
+                                          None, None, FAKE, hpc, FAKE, ws_bytes, None)
+
+
+def test_host_buffer_calls_check_arguments_before_enqueueing(lib):
+    """Every rejection here returns before a stream, an event or a copy is
+    touched: the whole problem is checked as the device call checks it."""
+    p = S.params(1, 2, 1024, 64, 64, 64, 4)
+    need = lib.sla_workspace_size(ctypes.byref(p))
+    assert call_forward_host(S.params(1, 2, 1000, 64, 64, 64, 4)) == S.SLA_ERR_INVALID_ARG
+    assert call_forward_host(p, q=ctypes.c_void_p((1 << 20) + 8)) == S.SLA_ERR_INVALID_ARG
+    assert call_forward_host(p, ws_bytes=need - 1) == S.SLA_ERR_WORKSPACE
+    assert call_forward_host(p, ws=None) == S.SLA_ERR_WORKSPACE
+    assert call_forward_host(p, q_h=None) == S.SLA_ERR_INVALID_ARG
+    assert call_forward_host(p, alpha_h=None) == S.SLA_ERR_INVALID_ARG
+    assert call_forward_host(p, hpc=-1) == S.SLA_ERR_INVALID_ARG
+    pg = S.params(1, 2, 1024, 64, 64, 64, 4, lut_mode=S.SLA_LUT_GIVEN)
+    assert call_forward_host(pg, lut=None) == S.SLA_ERR_INVALID_ARG
+    assert call_forward_host(S.params(1, 2, 1024, 64, 64, 64, 4, sparse_dtype=1)) == S.SLA_ERR_UNSUPPORTED
+    pp = S.params(1, 2, 1024, 64, 64, 64, 4)
+    assert call_pisa_host(S.params(1, 2, 1024, 64, 128, 64, 4)) == S.SLA_ERR_UNSUPPORTED
+    assert call_pisa_host(pp, out=ctypes.c_void_p((1 << 20) + 4)) == S.SLA_ERR_INVALID_ARG
+    assert call_pisa_host(pp, out_h=None) == S.SLA_ERR_INVALID_ARG
+    assert call_pisa_host(pp, hpc=-3) == S.SLA_ERR_INVALID_ARG
+    assert call_pisa_host(pp, ws_bytes=lib.sla_workspace_size(ctypes.byref(pp)) - 1) == S.SLA_ERR_WORKSPACE
