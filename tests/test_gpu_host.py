@@ -122,3 +122,32 @@ def test_forward_host_given_lut():
     assert S.sla_check_device_status() == 0
     ref = orc.sla_forward(inp["q"], inp["k"], inp["v"], inp["alpha"], lut_np, Bq, 64)
     check(out_h, ref, p)
+
+
+def test_forward_host_many_heads_in_the_whole_problems_workspace():
+    """297 heads of 64 KV blocks in chunks of 296 and 1: the whole problem's
+    pre-pass keeps a head in one chunk (297 partial sums), while the 296-head
+    chunk splits each head in two (592).  The workspace sized for the whole
+    problem must still serve that chunk."""
+    B, H, N, d, Bq, k = 1, 297, 4096, 64, 64, 4
+    inp = W.gaussian_inputs(B, H, N, d, 81)
+    g = dev(inp)
+    p = params(B, H, N, d, Bq, 64, k, f32=False)
+    ws = S.workspace(p)
+    lut_d = torch.full((B, H, N // Bq, k), -1, dtype=torch.int32, device="cuda")
+    out_d = torch.empty(g["q"].shape, dtype=S.sla.out_torch_dtype(p), device="cuda")
+    S.sla_forward(p, g["q"], g["k"], g["v"], g["alpha"], g["w_q"], g["w_k"], lut_d, out_d, ws)
+    h = _pinned(inp)
+    out_h = torch.full(inp["q"].shape, float("nan"), dtype=S.sla.out_torch_dtype(p)).pin_memory()
+    bufs = {n: torch.empty_like(g[n]) for n in ("q", "k", "v", "alpha")}
+    out = torch.empty_like(out_d)
+    lut = torch.full_like(lut_d, -1)
+    S.sla_forward_host(p, h["q"], h["k"], h["v"], h["alpha"], out_h, bufs["q"], bufs["k"], bufs["v"],
+                       bufs["alpha"], out, g["w_q"], g["w_k"], lut, ws, heads_per_chunk=296)
+    torch.cuda.synchronize()
+    assert S.sla_check_device_status() == 0
+    assert torch.equal(lut, lut_d)
+    o_h = out_h.float()
+    o_d = out_d.float().cpu()
+    assert torch.isfinite(o_h).all()
+    assert (o_h - o_d).abs().max() <= 1e-3 * o_d.abs().max()
