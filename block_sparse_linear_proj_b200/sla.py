@@ -136,9 +136,17 @@ def _ptr(t):
         return None
     if not t.is_cuda:
         raise ValueError("tensor must be on a CUDA device")
+    if t.device.index != torch.cuda.current_device():
+        # the kernels run on the current device and would dereference another GPU's address
+        raise ValueError("tensor is on %s but the current device is cuda:%d"
+                         % (t.device, torch.cuda.current_device()))
     if not t.is_contiguous():
         raise ValueError("tensor must be contiguous")
     return ctypes.c_void_p(t.data_ptr())
+
+
+def _nbytes(t):
+    return t.numel() * t.element_size()
 
 
 def _check(t, dtype, shape, name):
@@ -151,6 +159,9 @@ def _check(t, dtype, shape, name):
 def _stream(stream):
     if stream is None:
         stream = torch.cuda.current_stream()
+    elif stream.device.index != torch.cuda.current_device():
+        raise ValueError("stream is on %s but the current device is cuda:%d"
+                         % (stream.device, torch.cuda.current_device()))
     return ctypes.c_void_p(stream.cuda_stream)
 
 
@@ -178,7 +189,7 @@ def sla_route(p, q, k, w_q, w_k, lut, ws, stream=None):
     _check(k, torch.bfloat16, (B, H, N, d), "k")
     _check(lut, torch.int32, (B, H, N // p.Bq, p.topk), "lut")
     rc = load().sla_route(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(w_q), _ptr(w_k), _ptr(lut),
-                          _ptr(ws), ws.numel(), _stream(stream))
+                          _ptr(ws), _nbytes(ws), _stream(stream))
     _raise(rc, "sla_route")
     return lut
 
@@ -207,7 +218,7 @@ def sla_forward(p, q, k, v, alpha, w_q, w_k, lut, out, ws, stream=None):
     if lut is not None:
         _check(lut, torch.int32, (B, H, N // p.Bq, p.topk), "lut")
     rc = load().sla_forward(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(w_q),
-                            _ptr(w_k), _ptr(lut), _ptr(out), _ptr(ws), ws.numel(),
+                            _ptr(w_k), _ptr(lut), _ptr(out), _ptr(ws), _nbytes(ws),
                             _stream(stream))
     _raise(rc, "sla_forward")
     return out
@@ -241,7 +252,7 @@ def sla_forward_host(p, q_h, k_h, v_h, alpha_h, out_h, q, k, v, alpha, out, w_q,
     rc = load().sla_forward_host(ctypes.byref(p), _hptr(q_h), _hptr(k_h), _hptr(v_h), _hptr(alpha_h),
                                  _hptr(out_h), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(out),
                                  _ptr(w_q), _ptr(w_k), _ptr(lut), int(heads_per_chunk), _ptr(ws),
-                                 ws.numel(), _stream(stream))
+                                 _nbytes(ws), _stream(stream))
     _raise(rc, "sla_forward_host")
     return out_h
 
@@ -258,7 +269,7 @@ def sla_pisa_forward_host(p, q_h, k_h, v_h, out_h, q, k, v, out, w_q, w_k, lut, 
         _check(lut, torch.int32, (B, H, N // p.Bq, p.topk), "lut")
     rc = load().sla_pisa_forward_host(ctypes.byref(p), _hptr(q_h), _hptr(k_h), _hptr(v_h), _hptr(out_h),
                                       _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(w_q), _ptr(w_k),
-                                      _ptr(lut), int(heads_per_chunk), _ptr(ws), ws.numel(),
+                                      _ptr(lut), int(heads_per_chunk), _ptr(ws), _nbytes(ws),
                                       _stream(stream))
     _raise(rc, "sla_pisa_forward_host")
     return out_h
@@ -272,7 +283,7 @@ def sla_pisa_cov_norms(p, k, v, norms, ws, stream=None):
         _check(t, torch.bfloat16, (B, H, N, d), name)
     _check(norms, torch.float64, (B, H, N // p.Bk), "norms")
     rc = load().sla_pisa_cov_norms(ctypes.byref(p), _ptr(k), _ptr(v), _ptr(norms), _ptr(ws),
-                                   ws.numel(), _stream(stream))
+                                   _nbytes(ws), _stream(stream))
     _raise(rc, "sla_pisa_cov_norms")
     return norms
 
@@ -286,7 +297,7 @@ def sla_pisa_forward(p, q, k, v, w_q, w_k, lut, out, ws, stream=None):
     if lut is not None:
         _check(lut, torch.int32, (B, H, N // p.Bq, p.topk), "lut")
     rc = load().sla_pisa_forward(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(w_q),
-                                 _ptr(w_k), _ptr(lut), _ptr(out), _ptr(ws), ws.numel(),
+                                 _ptr(w_k), _ptr(lut), _ptr(out), _ptr(ws), _nbytes(ws),
                                  _stream(stream))
     _raise(rc, "sla_pisa_forward")
     return out
@@ -328,7 +339,7 @@ def sla_cocluster(p, q, k, n_clusters, iters, q_perm, k_perm, ws, stream=None):
     _check(q_perm, torch.int32, (B, H, N), "q_perm")
     _check(k_perm, torch.int32, (B, H, N), "k_perm")
     rc = load().sla_cocluster(ctypes.byref(p), _ptr(q), _ptr(k), int(n_clusters), int(iters), _ptr(q_perm),
-                              _ptr(k_perm), _ptr(ws), ws.numel(), _stream(stream))
+                              _ptr(k_perm), _ptr(ws), _nbytes(ws), _stream(stream))
     _raise(rc, "sla_cocluster")
     return q_perm, k_perm
 
